@@ -1,0 +1,397 @@
+"""Pins for the oracle: each check ties it to something other than itself.
+
+Library routines (torch's rms_norm, gelu, softmax, topk, linear), closed forms,
+brute force on tiny inputs and the identities the model pages state.  Every test here
+runs on the CPU.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import synth
+from tests import cases
+
+RNG = np.random.default_rng(7)
+
+
+def _rand(*s, scale=1.0):
+    return RNG.standard_normal(s) * scale
+
+
+# ------------------------------------------------------------------ pieces vs library
+
+def test_rms_norm_matches_torch():
+    v = _rand(5, 48, scale=3.0)
+    g = RNG.uniform(0.5, 1.5, 48)
+    eps = 1e-6
+    ref = F.rms_norm(torch.from_numpy(v), (48,), torch.from_numpy(g), eps).numpy()
+    np.testing.assert_allclose(oracle.rms_norm(v, g, eps), ref, rtol=1e-13, atol=0)
+    ref0 = F.rms_norm(torch.from_numpy(v), (48,), None, eps).numpy()
+    np.testing.assert_allclose(oracle.rms_norm(v, None, eps), ref0, rtol=1e-13, atol=0)
+
+
+def test_rms_norm_closed_form():
+    # A constant row c has mean square c^2, so the norm is c / sqrt(c^2 + eps).
+    c, eps = -2.5, 1e-6
+    got = oracle.rms_norm(np.full((1, 7), c), None, eps)
+    np.testing.assert_allclose(got, np.full((1, 7), c / math.sqrt(c * c + eps)), rtol=1e-15)
+
+
+def test_gelu_tanh_matches_torch_and_limits():
+    a = np.linspace(-9, 9, 1001)
+    ref = F.gelu(torch.from_numpy(a), approximate="tanh").numpy()
+    np.testing.assert_allclose(oracle.gelu_tanh(a), ref, rtol=1e-13, atol=1e-15)
+    assert oracle.gelu_tanh(np.array([0.0]))[0] == 0.0
+    assert abs(oracle.gelu_tanh(np.array([30.0]))[0] - 30.0) < 1e-12
+    assert abs(oracle.gelu_tanh(np.array([-30.0]))[0]) < 1e-12
+
+
+def test_softmax_matches_torch():
+    l = _rand(4, 128, scale=0.05)
+    ref = torch.softmax(torch.from_numpy(l), dim=-1).numpy()
+    np.testing.assert_allclose(oracle.softmax(l), ref, rtol=1e-14)
+
+
+# ------------------------------------------------------------------ router
+
+def _tiny_router_inputs(T=6, H=16, E=7):
+    x = _rand(T, H)
+    rs = RNG.uniform(0.5, 1.5, H)
+    wr = _rand(E, H, scale=0.3)
+    pes = RNG.uniform(0.5, 1.5, E)
+    return x, rs, wr, pes
+
+
+def test_router_topk_brute_force():
+    """P4: the top-k set is the k-subset with the largest logit sum (ties: smallest indices)."""
+    for k in (1, 2, 3, 7):
+        x, rs, wr, pes = _tiny_router_inputs()
+        r = oracle.router(x, rs, wr, None, pes, k, 1e-6)
+        for t in range(x.shape[0]):
+            l = r["logits"][t]
+            best = max(itertools.combinations(range(len(l)), k),
+                       key=lambda S: (sum(l[i] for i in S), [-i for i in S]))
+            assert sorted(best) == sorted(r["topk_idx"][t].tolist())
+            # ordered by logit descending
+            sel = l[r["topk_idx"][t]]
+            assert np.all(np.diff(sel) <= 0)
+
+
+def test_router_ties_go_to_lower_index():
+    # Equal rows of W_r give equal logits: the lower expert index must come first.
+    x, rs, wr, pes = _tiny_router_inputs(T=3, E=6)
+    wr[4] = wr[1]
+    wr[5] = wr[1]
+    r = oracle.router(x, rs, wr, np.array([0, 9.0, 0, 0, 9.0, 9.0]), pes, 3, 1e-6)
+    assert r["topk_idx"].tolist() == [[1, 4, 5]] * 3
+
+
+def test_router_matches_torch_topk():
+    x, rs, wr, pes = _tiny_router_inputs(T=20, H=32, E=16)
+    r = oracle.router(x, rs, wr, None, pes, 4, 1e-6)
+    v, i = torch.topk(torch.from_numpy(r["logits"]), 4, dim=-1, sorted=True)
+    assert np.array_equal(i.numpy(), r["topk_idx"])
+
+
+def test_router_closed_form_logits():
+    """A constant x, a constant learned scale s and constant W_r rows a_e give
+    logit_e = a_e * s * sqrt(H) * sign(c) / sqrt(1 + eps / c^2)."""
+    H, E, c, s, eps = 64, 5, -1.7, 1.25, 1e-6
+    a = np.array([0.3, -0.2, 0.1, 0.5, -0.05])
+    x = np.full((1, H), c)
+    r = oracle.router(x, np.full(H, s), np.repeat(a[:, None], H, axis=1), None, np.ones(E), 2, eps)
+    want = a * s * math.sqrt(H) * math.copysign(1.0, c) / math.sqrt(1 + eps / (c * c))
+    np.testing.assert_allclose(r["logits"][0], want, rtol=1e-13)
+    # the bias is added to the logits
+    b = np.arange(E, dtype=np.float64)
+    rb = oracle.router(x, np.full(H, s), np.repeat(a[:, None], H, axis=1), b, np.ones(E), 2, eps)
+    np.testing.assert_allclose(rb["logits"][0], want + b, rtol=1e-13)
+
+
+def test_routing_weights_renormalised():
+    """P2: the weights sum to 1 before per_expert_scale, are positive, and
+    per_expert_scale multiplies each selected expert's weight."""
+    x, rs, wr, pes = _tiny_router_inputs(T=30, H=24, E=9)
+    r = oracle.router(x, rs, wr, None, pes, 3, 1e-6)
+    np.testing.assert_allclose(r["topk_w_renorm"].sum(1), 1.0, atol=1e-15)
+    assert np.all(r["topk_w_renorm"] > 0)
+    np.testing.assert_allclose(r["topk_w"], r["topk_w_renorm"] * pes[r["topk_idx"]], rtol=1e-15)
+    # renormalised softmax = exp(l_j) / sum over the selected of exp(l_i)
+    l = np.take_along_axis(r["logits"], r["topk_idx"].astype(np.int64), 1)
+    e = np.exp(l - l.max(1, keepdims=True))
+    np.testing.assert_allclose(r["topk_w_renorm"], e / e.sum(1, keepdims=True), rtol=1e-13)
+
+
+# ------------------------------------------------------------------ permutation
+
+def _permute_brute(idx, E):
+    pairs = [(int(e), p) for p, e in enumerate(np.asarray(idx).reshape(-1))]
+    src = [p for e in range(E) for (ee, p) in pairs if ee == e]
+    counts = [sum(1 for (ee, _) in pairs if ee == e) for e in range(E)]
+    offs = [0]
+    for c in counts:
+        offs.append(offs[-1] + c)
+    inv = [0] * len(src)
+    for q, p in enumerate(src):
+        inv[p] = q
+    return offs, src, inv
+
+
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (5, 2, 4), (33, 4, 16), (64, 8, 128), (0, 8, 128)])
+def test_permute_brute_force(T, k, E):
+    """P6: counting sort by expert, stable by flat index t*k+j."""
+    idx = RNG.integers(0, E, size=(T, k)).astype(np.int32)
+    offs, src, inv = oracle.permute(idx, E)
+    bo, bs, bi = _permute_brute(idx, E)
+    assert offs.tolist() == bo and src.tolist() == bs and inv.tolist() == bi
+
+
+# ------------------------------------------------------------------ expert MLP
+
+def test_gated_mlp_matches_torch_linear():
+    H, I = 24, 10
+    u = _rand(3, H)
+    wgu = _rand(2 * I, H, scale=0.2)
+    wd = _rand(H, I, scale=0.2)
+    tu = torch.from_numpy(u)
+    g = F.linear(tu, torch.from_numpy(wgu[:I]))
+    v = F.linear(tu, torch.from_numpy(wgu[I:]))
+    ref = F.linear(F.gelu(g, approximate="tanh") * v, torch.from_numpy(wd)).numpy()
+    np.testing.assert_allclose(oracle.gated_mlp(u, wgu, wd), ref, rtol=1e-12, atol=1e-14)
+
+
+def test_gated_mlp_permutation_closed_form():
+    """With permutation matrices P (gate), Q (up), R (down):
+    y = R (gelu(P u) * (Q u)); a transposed operand would use P^T, Q^T or R^T."""
+    n = 6
+    P = np.eye(n)[[1, 2, 3, 4, 5, 0]]
+    Q = np.eye(n)[[3, 0, 4, 1, 5, 2]]
+    R = np.eye(n)[[2, 5, 1, 0, 3, 4]]
+    u = np.arange(1.0, n + 1.0) * np.array([1, -1, 1, -1, 1, -1]) * 0.7
+    want = np.empty(n)
+    for i in range(n):
+        gi = u[[1, 2, 3, 4, 5, 0][i]]
+        vi = u[[3, 0, 4, 1, 5, 2][i]]
+        want[i] = 0.5 * gi * (1 + math.tanh(math.sqrt(2 / math.pi) * (gi + 0.044715 * gi ** 3))) * vi
+    want = want[[2, 5, 1, 0, 3, 4]]
+    got = oracle.gated_mlp(u[None], np.vstack([P, Q]), R)[0]
+    np.testing.assert_allclose(got, want, rtol=1e-14)
+
+
+# ------------------------------------------------------------------ block identities
+
+def _tiny_block(T=6, H=16, E=6, k=2, I=4, D=8, seed=3, bias=None):
+    shape = synth.Shape(T=T, H=H, E=E, k=k, I=I, D=D)
+    p = synth.make_layer(seed, shape, std=0.3)
+    x = synth.x_rows(seed + 1, H, T)
+    return shape, p, x
+
+
+def test_all_experts_dense_equals_sparse():
+    """P1: the all-experts-dense form (weight 0 for unselected experts) equals sparse top-k."""
+    shape, p, x = _tiny_block(T=9, H=32, E=8, k=3, I=8, D=8)
+    ex = cases.bf16_experts(p)
+    a = oracle.block_forward(x, p, ex, shape.k, shape.eps)
+    b = oracle.block_forward(x, p, ex, shape.k, shape.eps, all_experts_dense=True)
+    np.testing.assert_allclose(a["moe"], b["moe"], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(a["out"], b["out"], rtol=1e-12, atol=1e-15)
+
+
+def test_k_equals_E_is_dense_softmax_mixture():
+    """P3: with k = E the renormalisation is the full softmax, so
+    moe = sum_e p_e * pes_e * MLP_e(xn)."""
+    shape, p, x = _tiny_block(T=5, H=16, E=5, k=5, I=4, D=4)
+    ex = cases.bf16_experts(p)
+    o = oracle.block_forward(x, p, ex, shape.k, shape.eps)
+    pes = oracle.bf16(p["per_expert_scale"])
+    want = np.zeros_like(o["moe"])
+    for e in range(shape.E):
+        want += (o["probs"][:, e] * pes[e])[:, None] * oracle.gated_mlp(o["xn_moe"], ex.gate_up(e), ex.down(e))
+    np.testing.assert_allclose(o["moe"], want, rtol=1e-12, atol=1e-15)
+
+
+def test_single_expert_is_plain_gated_mlp():
+    """P5: E = k = 1 gives moe = per_expert_scale * MLP(xn_moe); a zero down projection
+    gives moe = 0 and out = x + post_ff(post_dense(dense))."""
+    shape, p, x = _tiny_block(T=4, H=16, E=1, k=1, I=4, D=4)
+    ex = cases.bf16_experts(p)
+    o = oracle.block_forward(x, p, ex, 1, shape.eps)
+    pes = oracle.bf16(p["per_expert_scale"])[0]
+    np.testing.assert_allclose(o["topk_w"], pes, rtol=1e-15)
+    np.testing.assert_allclose(o["moe"], pes * oracle.gated_mlp(o["xn_moe"], ex.gate_up(0), ex.down(0)),
+                               rtol=1e-13)
+    p0 = dict(p, w_down=np.zeros_like(p["w_down"]))
+    o0 = oracle.block_forward(x, p0, cases.bf16_experts(p0), 1, shape.eps)
+    assert np.all(o0["moe"] == 0)
+    eps = shape.eps
+    want = oracle.bf16(x) + oracle.rms_norm(oracle.rms_norm(o0["dense"], oracle.bf16(p["g_post_dense"]), eps),
+                                            oracle.bf16(p["g_post_ff"]), eps)
+    np.testing.assert_allclose(o0["out"], want, rtol=1e-13)
+
+
+def test_rows_are_independent():
+    """P7: permuting the tokens permutes the outputs (no capacity limit, no cross-token term)."""
+    shape, p, x = _tiny_block(T=7, H=16, E=6, k=2, I=4, D=4)
+    ex = cases.bf16_experts(p)
+    perm = np.array([3, 0, 6, 1, 5, 2, 4])
+    a = oracle.block_forward(x, p, ex, shape.k, shape.eps)
+    b = oracle.block_forward(x[perm], p, ex, shape.k, shape.eps)
+    np.testing.assert_allclose(b["out"], a["out"][perm], rtol=1e-14)
+    assert np.array_equal(b["topk_idx"], a["topk_idx"][perm])
+
+
+def _block_brute(x, p, k, eps):
+    """The block with plain Python loops and math.* only, from the definitions."""
+    X = oracle.bf16(x)
+    T, H = X.shape
+    E = p["w_router"].shape[0]
+    f = {n: oracle.bf16(p[n]) for n in p if p[n] is not None}
+    I = f["w_gate_up"].shape[1] // 2
+    D = f["w_dense_gate_up"].shape[0] // 2
+
+    def gelu(a):
+        return 0.5 * a * (1 + math.tanh(math.sqrt(2 / math.pi) * (a + 0.044715 * a ** 3)))
+
+    def norm(v, g):
+        r = math.sqrt(sum(t * t for t in v) / len(v) + eps)
+        return [v[i] / r * (1.0 if g is None else g[i]) for i in range(len(v))]
+
+    def mlp(u, wgu, wd, n):
+        h = []
+        for i in range(n):
+            g = sum(u[c] * wgu[i][c] for c in range(H))
+            v = sum(u[c] * wgu[n + i][c] for c in range(H))
+            h.append(gelu(g) * v)
+        return [sum(h[i] * wd[o][i] for i in range(n)) for o in range(H)]
+
+    outs = []
+    for t in range(T):
+        xh = norm(list(X[t]), None)
+        z = [xh[c] * f["router_scale"][c] / math.sqrt(H) for c in range(H)]
+        l = [sum(z[c] * f["w_router"][e][c] for c in range(H)) for e in range(E)]
+        S = max(itertools.combinations(range(E), k), key=lambda S: (sum(l[i] for i in S), [-i for i in S]))
+        m = max(l)
+        ex = [math.exp(v - m) for v in l]
+        tot = sum(ex)
+        pr = [v / tot for v in ex]
+        ssum = sum(pr[i] for i in S)
+        moe = [0.0] * H
+        um = [xh[c] * f["g_pre_moe"][c] for c in range(H)]
+        for e in S:
+            y = mlp(um, f["w_gate_up"][e], f["w_down"][e], I)
+            w = pr[e] / ssum * f["per_expert_scale"][e]
+            moe = [moe[c] + w * y[c] for c in range(H)]
+        ud = [xh[c] * f["g_pre_dense"][c] for c in range(H)]
+        dense = mlp(ud, f["w_dense_gate_up"], f["w_dense_down"], D)
+        a = norm(dense, f["g_post_dense"])
+        b = norm(moe, f["g_post_moe"])
+        c = norm([a[i] + b[i] for i in range(H)], f["g_post_ff"])
+        outs.append([X[t][i] + c[i] for i in range(H)])
+    return np.array(outs)
+
+
+def test_block_brute_force_tiny():
+    """P4: the whole block against plain loops (subset search for the top-k)."""
+    shape, p, x = _tiny_block(T=3, H=8, E=5, k=2, I=3, D=4)
+    got = oracle.block_forward(x, p, cases.bf16_experts(p), shape.k, shape.eps)["out"]
+    np.testing.assert_allclose(got, _block_brute(x, p, shape.k, shape.eps), rtol=1e-11, atol=1e-13)
+
+
+# ------------------------------------------------------------------ int8
+
+def test_int8_quantiser_pins():
+    """P8 and R9: |q s - w| <= s/2, the largest |q| of a non-zero row is 127, an
+    all-zero row takes s = 1 and q = 0, and halves round to even."""
+    w = synth.normal_bf16(5, (99,), (6, 40), 0.02)
+    w[3] = 0
+    q, s = oracle.quantize_int8_per_channel(w)
+    wf = synth.bf16_bits_to_f32(w).astype(np.float64)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert np.all(np.abs(q.astype(np.float64) * s[:, None] - wf) <= s[:, None] / 2 * (1 + 1e-6))
+    nz = [i for i in range(6) if i != 3]
+    assert np.all(np.abs(q[nz]).max(1) == 127)
+    assert s[3] == 1.0 and np.all(q[3] == 0)
+    # amax = 127/128 makes s = 2^-7 exactly; 2.5 s, 3.5 s, -2.5 s, -0.5 s -> 2, 4, -2, 0
+    row = np.array([127 / 128, 2.5 / 128, 3.5 / 128, -2.5 / 128, -0.5 / 128], dtype=np.float32)
+    qq, ss = oracle.quantize_int8_per_channel(synth.f32_to_bf16_bits(row)[None])
+    assert ss[0] == np.float32(2.0 ** -7)
+    assert qq[0].tolist() == [127, 2, 4, -2, 0]
+
+
+# ------------------------------------------------------------------ the bar discriminates
+
+def test_fp16_accumulation_fails_the_bar():
+    """P9 (negative control): expert GEMMs that accumulate in fp16 at H = 2816 miss the
+    bar (on these synthetic weights by the max-abs term; the page's cosine ~0.97 was
+    seen on the real checkpoint and is not asserted), while fp32 accumulation with bf16 storage of xn and h meets it
+    (ONNX export card, "MoE dispatch": fp16-accumulated expert GEMMs lose accuracy at
+    this hidden size)."""
+    H, I, n = 2816, 704, 6
+    wgu = synth.normal_bf16(11, (1,), (2 * I, H), 0.02)
+    wd = synth.normal_bf16(11, (2,), (H, I), 0.02)
+    u = oracle.bf16(synth.x_rows(12, H, n))
+    W1, W2 = oracle.bf16(wgu), oracle.bf16(wd)
+    ref = oracle.gated_mlp(u, W1, W2)
+
+    def dot_fp16(a, B):  # sequential fp16 accumulation of fp16-rounded products
+        prod = (a[:, None, :] * B[None, :, :]).astype(np.float16)
+        return np.cumsum(prod, axis=-1, dtype=np.float16)[..., -1].astype(np.float64)
+
+    u16 = u.astype(np.float16).astype(np.float64)
+    g = dot_fp16(u16, W1[:I])
+    v = dot_fp16(u16, W1[I:])
+    h = (oracle.gelu_tanh(g) * v).astype(np.float16).astype(np.float64)
+    y16 = dot_fp16(h, W2)
+    with pytest.raises(AssertionError, match="max-abs"):
+        cases.check_bar(y16, ref, cases.FRAC_BF16, "fp16-accumulate model")
+
+    def to_bf16(a):
+        return synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(a.astype(np.float32))).astype(np.float64)
+
+    ub = to_bf16(u)
+    g32 = (ub.astype(np.float32) @ W1[:I].T.astype(np.float32)).astype(np.float64)
+    v32 = (ub.astype(np.float32) @ W1[I:].T.astype(np.float32)).astype(np.float64)
+    h32 = to_bf16(oracle.gelu_tanh(g32) * v32)
+    y32 = (h32.astype(np.float32) @ W2.T.astype(np.float32)).astype(np.float64)
+    cases.check_bar(to_bf16(y32), ref, cases.FRAC_BF16, "fp32-accumulate model")
+
+
+# ------------------------------------------------------------------ workloads
+
+def test_layer_shape_matches_the_pages():
+    with open(os.path.join(cases.GOLDEN, "gemma4_26b_a4b_moe.json")) as f:
+        g = json.load(f)
+    s = synth.DECODE
+    assert (s.H, s.E, s.k, s.I, s.D) == (g["hidden_size"], g["num_experts"], g["top_k"],
+                                         g["moe_intermediate_size"], g["intermediate_size"])
+    assert synth.STACK_LAYERS == g["num_layers"]
+    assert synth.PREFILL.H == s.H and synth.PREFILL.T == 2048
+
+
+def test_gap_filter_gives_unique_topk():
+    c = cases.make_case(synth.TINY, seed=42)
+    r = oracle.router(oracle.bf16(c.x), oracle.bf16(c.p["router_scale"]), oracle.bf16(c.p["w_router"]),
+                      None, oracle.bf16(c.p["per_expert_scale"]), c.shape.k, c.shape.eps)
+    assert oracle.topk_gaps(r["logits"], c.shape.k).min() >= cases.MIN_GAP
+
+
+def test_zipf_workload_is_skewed():
+    """The calibrated offset leaves some experts near or above ten times the mean load
+    and at least one expert empty."""
+    shape = synth.PREFILL
+    p = synth.make_router(1234, shape)
+    x = synth.x_rows(1235, shape.H, shape.T)
+    b = synth.zipf_bias(1234, shape.E, cases.zipf_alpha())
+    r = oracle.router(oracle.bf16(x), oracle.bf16(p["router_scale"]), oracle.bf16(p["w_router"]),
+                      b, oracle.bf16(p["per_expert_scale"]), shape.k, shape.eps)
+    c = np.bincount(r["topk_idx"].reshape(-1), minlength=shape.E)
+    mean = shape.T * shape.k / shape.E
+    assert (c == 0).sum() >= 1
+    assert (c >= 8 * mean).sum() >= 2
