@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid MoE feed-forward block (Gemma-4-26B-A4B shape) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill]
+
+A step is one moe_block_forward (router -> permute -> experts + dense MLP -> combine,
+post norms, residual) over one batch of synthetic tokens.  The default workload is the
+decode layer: T=8 tokens, H=2816, E=128, top-8, expert intermediate 704, dense
+intermediate 2112, bf16 weights N(0, 0.02), activations N(0, 1), gains U(0.5, 1.5).
+Steps rotate over distinct layer copies (and distinct inputs) so that no step finds
+its weights in L2.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (numpy, fp64) on the same workload instead, on a
+bounded sample per step; it is the baseline arm, not a GPU path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = ("MoE-FFN tokens/s (1 B200) at T=8..16K; % HBM roofline (decode) / "
+          "% TC peak (prefill)")
+UNIT = "tokens/s"
+
+WORKLOADS = {
+    "decode": dict(shape=synth.DECODE, layers=8, zipf=False, steps=3000, warmup=100,
+                   name="Gemma-4-26B-A4B-shaped MoE-FFN layer, decode T=8 (bf16 experts)"),
+    "prefill": dict(shape=synth.PREFILL, layers=4, zipf=True, steps=200, warmup=10,
+                    name="Gemma-4-26B-A4B-shaped MoE-FFN layer, prefill T=2048, Zipf-skewed router"),
+}
+ZIPF_ALPHA_FILE = os.path.join(ROOT, "tests", "golden", "zipf_alpha.json")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={ident}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            return None
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------- work model
+
+def algorithmic(shape, used_experts: int):
+    """Bytes that must move and FLOPs that must run for one block call.
+
+    Bytes: the weights of the experts that received a token, the dense MLP, the router
+    and the norm vectors, plus x in and out.  Intermediates are implementation traffic.
+    """
+    H, E, k, I, D, T = shape.H, shape.E, shape.k, shape.I, shape.D, shape.T
+    b_experts = used_experts * 3 * I * H * 2
+    b_dense = 3 * D * H * 2
+    b = b_experts + b_dense + E * H * 2 + 6 * H * 2 + E * 2 + 2 * T * H * 2
+    flops = T * (2 * k * 3 * I * H + 2 * 3 * D * H + 2 * E * H)
+    # the gate_up launch alone: its weights, its token rows in, h out
+    b_gate_up = used_experts * 2 * I * H * 2 + 2 * D * H * 2 + (T * k + T) * H * 2 + (T * k * I + T * D) * 2
+    f_gate_up = T * (2 * k * 2 * I * H + 2 * 2 * D * H)
+    return {"bytes": b, "flops": flops, "gate_up_bytes": b_gate_up, "gate_up_flops": f_gate_up}
+
+
+# ---------------------------------------------------------------------------- our arm
+
+def run_ours(args, wl, rank, world, device):
+    import mixture_experts_ffn_05_b200 as mf
+    mf.lib()  # fails loudly without the built CUDA library
+    shape = wl["shape"]
+    T = shape.T
+    cfg = mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps)
+    seed = 1234 + 7919 * rank
+    alpha = None
+    layers = []
+    for l in range(wl["layers"]):
+        t = synth.torch_layer(shape, seed, l, device)
+        if wl["zipf"]:
+            with open(ZIPF_ALPHA_FILE) as f:
+                alpha = float(json.load(f)["alpha"])
+            t["logit_bias"] = torch.from_numpy(synth.zipf_bias(seed, shape.E, alpha)).to(device)
+        layers.append(t)
+    bws = [mf.BlockWeights(cfg, t) for t in layers]
+    W, K = args.warmup, args.steps
+    xs = [synth.torch_x(shape, seed, i, device) for i in range(W + K)]
+    out = torch.empty(T, shape.H, dtype=torch.bfloat16, device=device)
+    ws = mf.workspace(cfg, T, device)
+    stream = torch.cuda.current_stream(device)
+
+    # routing of each timed step (outside the timed region): experts that receive tokens
+    used = []
+    ti = torch.empty(T, shape.k, dtype=torch.int32, device=device)
+    tw = torch.empty(T, shape.k, dtype=torch.float32, device=device)
+    xa = torch.empty(T, shape.H, dtype=torch.bfloat16, device=device)
+    xb = torch.empty_like(xa)
+    for i in range(K):
+        L = layers[(W + i) % len(layers)]
+        mf.moe_router(cfg, xs[W + i], L["router_scale"], L["w_router"], L.get("logit_bias"),
+                      L["per_expert_scale"], L["g_pre_moe"], L["g_pre_dense"], ti, tw, xa, xb, ws)
+        used.append(int(torch.unique(ti).numel()))
+
+    def step(i, ev=None):
+        mf.moe_block_forward(cfg, xs[i], bws[i % len(bws)], out, ws, stream=stream, stage_events=ev)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(mf.MOE_BLOCK_EVENTS)]
+                for _ in range(K)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(device)
+    time.sleep(0.15)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for i in range(K):
+        step(W + i, stage_ev[i])
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    st = mf.moe_check_device_status(ws)
+    if st != mf.MOE_OK:
+        raise RuntimeError(f"device status after the timed region: {mf.status_string(st)}")
+    t_ms = e0.elapsed_time(e1)
+    stages = {n: [] for n in ("router", "permute", "gather", "clear", "gate_up", "down", "combine")}
+    for ev in stage_ev:
+        for j, n in enumerate(stages):
+            stages[n].append(ev[j].elapsed_time(ev[j + 1]))
+    t_max = t_ms
+    if world > 1:
+        tt = torch.tensor([t_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        t_max = float(tt.item())
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region
+    x_host = torch.empty(W + K, T, shape.H, dtype=torch.bfloat16, pin_memory=True)
+    for i in range(W + K):
+        x_host[i].copy_(xs[i])
+    out_host = torch.empty(K, T, shape.H, dtype=torch.bfloat16, pin_memory=True)
+    x_dev = torch.empty(T, shape.H, dtype=torch.bfloat16, device=device)
+
+    def e2e_step(i, j):
+        x_dev.copy_(x_host[i], non_blocking=True)
+        mf.moe_block_forward(cfg, x_dev, bws[i % len(bws)], out, ws, stream=stream)
+        out_host[j].copy_(out, non_blocking=True)
+
+    for i in range(min(W, 10)):
+        e2e_step(i, 0)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(K):
+        e2e_step(W + i, i)
+    f1.record(stream)
+    torch.cuda.synchronize(device)
+    te = f0.elapsed_time(f1)
+    if world > 1:
+        tt = torch.tensor([te], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        te = float(tt.item())
+    if mf.moe_check_device_status(ws) != mf.MOE_OK:
+        raise RuntimeError("device status after the end-to-end region")
+
+    # ---- roofline of the dominant kernel (the gate_up grouped GEMM) and of the block
+    pk = peaks()
+    alg = [algorithmic(shape, u) for u in used]
+    gu_bytes = sum(a["gate_up_bytes"] for a in alg)
+    gu_ms = sum(stages["gate_up"])
+    gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
+    blk_bytes = sum(a["bytes"] for a in alg) / K
+    blk_flops = sum(a["flops"] for a in alg) / K
+    ms_step = t_max / K
+    prefill = T >= 1024
+    if prefill:
+        gu_tf = sum(a["gate_up_flops"] for a in alg) / (gu_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(gu_tf, 2), "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(gu_tf / pk["bf16_tflops"], 4), "traffic": None,
+                "kernel": "grouped_gemm_kernel (gate_up launch)",
+                "peak_source": f"bf16_tflops of {pk['source']} peaks"}
+    else:
+        roof = {"bound": "hbm", "achieved": round(gu_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gu_gbs / pk["hbm_gbs"], 4), "traffic": None,
+                "kernel": "grouped_gemm_kernel (gate_up launch)",
+                "peak_source": f"hbm_gbs of {pk['source']} peaks"}
+    t_hbm = blk_bytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = blk_flops / (pk["bf16_tflops"] * 1e12)
+    block_roof = {"bytes_per_step": int(blk_bytes), "flops_per_step": int(blk_flops),
+                  "hbm_frac": round(t_hbm / (ms_step * 1e-3), 4),
+                  "tc_frac": round(t_tc / (ms_step * 1e-3), 4),
+                  "binding_frac": round(max(t_hbm, t_tc) / (ms_step * 1e-3), 4),
+                  "mean_used_experts": round(sum(used) / K, 2)}
+    launches_per_step = 2 + (1 if T * shape.k <= 8192 else 3) + 1 + 2 + 1
+    res = {
+        "metric": METRIC, "value": round(world * T * K / (t_max * 1e-3), 1), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights of the layer's shape)",
+        "config": {"workload": wl["name"], "T": T, "H": shape.H, "E": shape.E, "top_k": shape.k,
+                   "expert_inter": shape.I, "dense_inter": shape.D, "expert_weights": "bf16",
+                   "router_bias": ("zipf s=1.1, alpha=%.5f" % alpha) if wl["zipf"] else "none",
+                   "layers_rotated": len(layers),
+                   "l2": "steps rotate over %d distinct layers (%.1f GB of weights) and distinct "
+                         "inputs; no step's weights are L2-resident" %
+                         (len(layers), len(layers) * 3 * shape.E * shape.I * shape.H * 2 / 1e9),
+                   "parallelism": f"dp{world} (replicas, no collective)"},
+        "roofline": roof,
+        "block_roofline": block_roof,
+        "stages_ms": {n: round(statistics.mean(v), 5) for n, v in stages.items()},
+        "e2e": {"value": round(world * T * K / (te * 1e-3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(shape, layers[0], xs[W], wl, alpha)
+    return res
+
+
+# ---------------------------------------------------------------------------- the oracle
+
+def _host_layer(layer):
+    out = {}
+    for n, t in layer.items():
+        if t.dtype == torch.bfloat16:
+            out[n] = t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        else:
+            out[n] = t.cpu().numpy()
+    return out
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def _oracle_rows(shape):
+    return shape.T if shape.T <= 64 else 64
+
+
+def cpu_baseline(shape, layer, x, wl, alpha, budget_s=15.0):
+    """The oracle, as it stands, on the host cores: tokens/s over a bounded sample."""
+    import oracle
+    p = _host_layer(layer)
+    bias = p.pop("logit_bias", None)
+    ex = oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
+    rows = _oracle_rows(shape)
+    xh = x[:rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.block_forward(xh, p, ex, shape.k, shape.eps, bias)
+        n += 1
+        el = time.perf_counter() - t0
+        if el > budget_s or n >= 200:
+            break
+    return {"value": round(n * rows / el, 3), "unit": UNIT, "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} oracle block calls of {rows} tokens of the {wl['name']} workload "
+                      f"(layer 0), {el:.1f} s"}
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    shape = wl["shape"]
+    layer = synth.torch_layer(shape, 1234, 0, "cpu")
+    alpha = None
+    if wl["zipf"]:
+        with open(ZIPF_ALPHA_FILE) as f:
+            alpha = float(json.load(f)["alpha"])
+    p = _host_layer(layer)
+    bias = synth.zipf_bias(1234, shape.E, alpha) if wl["zipf"] else None
+    ex = oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
+    rows = _oracle_rows(shape)
+    xs = [synth.torch_x(shape, 1234, i, "cpu")[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+          for i in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        oracle.block_forward(xs[i], p, ex, shape.k, shape.eps, bias)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.block_forward(xs[args.warmup + i], p, ex, shape.k, shape.eps, bias)
+    el = time.perf_counter() - t0
+    v = round(args.steps * rows / el, 3)
+    sample = f"{args.steps} timed oracle block calls of {rows} tokens each ({wl['name']})"
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": wl["name"], "T": shape.T, "rows_per_step": rows},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        args.steps = args.steps if args.steps is not None else 10
+        args.warmup = args.warmup if args.warmup is not None else 3
+    else:
+        args.steps = args.steps if args.steps is not None else wl["steps"]
+        args.warmup = args.warmup if args.warmup is not None else wl["warmup"]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, wl, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        res = run_ours(args, wl, rank, world, device)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+/*
+ * moe_ffn.h - C interface of the hybrid mixture-of-experts feed-forward block
+ * (Gemma-4-26B-A4B shape) on NVIDIA B200 (sm_100a).
+ *
+ * The block, per token x (one row of H values):
+ *
+ *   xhat       = x / sqrt(mean(x^2) + eps)                      scale-free RMSNorm
+ *   router     : z = xhat * router_scale * H^-0.5, logits = z W_r^T (+ bias),
+ *                softmax (fp32) -> top-k -> renormalise -> * per_expert_scale
+ *   experts    : for each selected expert e with weight w:
+ *                g, u = xn_moe W_gate_up[e]^T (gate rows, then up rows),
+ *                h = gelu_tanh(g) * u,  y = h W_down[e]^T,  moe += w * y
+ *   dense MLP  : the same gated-GELU MLP with intermediate D on xn_dense
+ *   out        = x + N_post_ff( N_post_dense(dense) + N_post_moe(moe) )
+ *
+ * where xn_moe = xhat * g_pre_moe, xn_dense = xhat * g_pre_dense and
+ * N_g(v) = v / sqrt(mean(v^2) + eps) * g.
+ *
+ * Sources: "Gemma-4 26B-A4B-it - ONNX MoE text decoder", table "Truthful graph
+ * contracts" (rows "Mixture of Experts", "MoE topology", "Router");
+ * "Gemma-4 26B-A4B (MoE) on AWS Inferentia2", sections "The architecture (a
+ * dual-path FFN)" and "How it works (the recipe)"; "Gemma-4 26B-A4B (MoE, int8
+ * experts) on AWS Inferentia2" for the per-channel int8 expert weights.
+ *
+ * Conventions for every entry point
+ *   - bf16 values are passed as their 16-bit patterns (moe_bf16_t).
+ *   - All tensors are row-major with the reduction (K) dimension contiguous.
+ *   - Every pointer is device memory owned by the caller, 16-byte aligned, unless
+ *     marked "host".  The library never allocates or frees memory in these calls;
+ *     scratch comes from the caller's workspace `ws` of `ws_bytes` bytes, which must
+ *     be at least moe_workspace_size(cfg, T) and 256-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
+ *     only enqueues work on that stream and returns; results are ready when the
+ *     stream reaches that point.  Calls on different streams must not share `ws`.
+ *   - Size limits: H a multiple of 128 (128..6144), I and D multiples of 64
+ *     (64..16384), 1 <= E <= 256, 1 <= k <= min(E, 16), 0 <= T, T*k < 2^31.
+ *     T = 0 returns MOE_OK and launches nothing.
+ *   - Argument errors are found on the host before anything is launched and
+ *     return MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED or MOE_ERR_WORKSPACE.  A failed
+ *     launch returns MOE_ERR_CUDA.  Nothing throws across this interface.
+ *   - The GPU kernels bound every wait they make.  A wait that runs out records
+ *     MOE_ERR_DEVICE_TIMEOUT in a status word inside `ws`, and the kernel returns;
+ *     moe_check_device_status() reads and clears it.
+ *   - Results are deterministic: the same inputs give the same bits on every run.
+ */
+#ifndef MOE_FFN_H
+#define MOE_FFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t; /* bf16 bit pattern */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* a pointer, size or layout argument is invalid */
+  MOE_ERR_UNSUPPORTED = 2,    /* sizes outside the limits above */
+  MOE_ERR_WORKSPACE = 3,      /* ws NULL, misaligned or smaller than required */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime or driver call failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5  /* a bounded device wait ran out (see above) */
+} moe_status_t;
+
+typedef enum {
+  MOE_W_BF16 = 0, /* expert weights in bf16 */
+  MOE_W_INT8 = 1  /* expert weights int8, one fp32 scale per output row */
+} moe_wdtype_t;
+
+/* Sizes of one layer. */
+typedef struct {
+  int32_t hidden;        /* H */
+  int32_t num_experts;   /* E */
+  int32_t top_k;         /* k */
+  int32_t expert_inter;  /* I: intermediate size of each expert */
+  int32_t dense_inter;   /* D: intermediate size of the shared dense MLP */
+  float eps;             /* RMSNorm epsilon, > 0 */
+  int32_t expert_wdtype; /* moe_wdtype_t */
+} moe_config_t;
+
+/* Expert weights, read-only; may be shared by concurrent calls.
+ *   w_gate_up [E][2I][H]  rows 0..I-1 are the gate projection, rows I..2I-1 the up
+ *                         projection (the pages' fused gate_up weight);
+ *   w_down    [E][H][I];
+ *   bf16 (MOE_W_BF16): s_gate_up and s_down must be NULL.
+ *   int8 (MOE_W_INT8): the weight is q * s, with s_gate_up [E][2I] and s_down [E][H]
+ *                      fp32 per-output-row scales (see moe_quantize_int8). */
+typedef struct {
+  const void* w_gate_up;
+  const void* w_down;
+  const float* s_gate_up;
+  const float* s_down;
+} moe_expert_weights_t;
+
+/* All weights of one block. */
+typedef struct {
+  const moe_bf16_t* router_scale;     /* [H] learned router scale */
+  const moe_bf16_t* w_router;         /* [E][H] */
+  const float* logit_bias;            /* [E] fp32 added to the logits, or NULL */
+  const moe_bf16_t* per_expert_scale; /* [E] */
+  const moe_bf16_t* g_pre_moe;        /* [H] gain of the MoE branch's pre norm */
+  const moe_bf16_t* g_pre_dense;      /* [H] gain of the dense branch's pre norm */
+  const moe_bf16_t* g_post_moe;       /* [H] or NULL: post norm of the MoE branch skipped */
+  const moe_bf16_t* g_post_dense;     /* [H] or NULL: post norm of the dense branch skipped */
+  const moe_bf16_t* g_post_ff;        /* [H] gain of the final post_ff norm */
+  moe_expert_weights_t experts;
+  const moe_bf16_t* w_dense_gate_up;  /* [2D][H] gate rows then up rows */
+  const moe_bf16_t* w_dense_down;     /* [H][D] */
+} moe_block_weights_t;
+
+/* Bytes of workspace every call below needs for T tokens (0 if cfg is invalid).
+ * Host function; launches nothing. */
+size_t moe_workspace_size(const moe_config_t* cfg, int32_t T);
+
+/* Router and pre norms (ONNX export card, "Truthful graph contracts", Router row;
+ * Inferentia2 card, "The architecture").
+ *   x [T][H] bf16 (the un-normed block input).
+ *   Outputs: topk_idx [T][k] int32 expert ids, ordered by logit descending and, for
+ *   equal logits, by expert id ascending; topk_w [T][k] fp32 routing weights
+ *   (renormalised over the k selected, then times per_expert_scale);
+ *   xn_moe, xn_dense [T][H] bf16 = xhat * g_pre_moe, xhat * g_pre_dense.
+ *   logit_bias may be NULL. */
+moe_status_t moe_router(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
+                        const moe_bf16_t* router_scale, const moe_bf16_t* w_router,
+                        const float* logit_bias, const moe_bf16_t* per_expert_scale,
+                        const moe_bf16_t* g_pre_moe, const moe_bf16_t* g_pre_dense,
+                        int32_t* topk_idx, float* topk_w, moe_bf16_t* xn_moe,
+                        moe_bf16_t* xn_dense, void* ws, size_t ws_bytes, void* stream);
+
+/* Token-to-expert permutation (a counting sort; the gathered-per-expert dispatch of
+ * the Tenstorrent card's "gathered expert prefill", computed exactly).
+ *   topk_idx [T][k] int32 in [0, E).  The flat pair index is p = t*k + j.
+ *   expert_offsets [E+1]: expert e's pairs occupy [offsets[e], offsets[e+1]).
+ *   sorted_src [T*k]: the pairs grouped by expert, in increasing p within a group.
+ *   inv_pos [T*k]: inv_pos[p] is the position of pair p in sorted_src.
+ *   An id outside [0, E) returns nothing useful; the kernel does not read or write
+ *   out of bounds for it (such pairs are dropped and the offsets count the rest). */
+moe_status_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx,
+                         int32_t* expert_offsets, int32_t* sorted_src, int32_t* inv_pos,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Routed experts (ONNX export card, "Mixture of Experts" row; Inferentia2 card,
+ * "How it works": outputs weighted by the routing weights and summed).
+ *   xn_moe [T][H] bf16; topk_w [T][k] fp32; expert_offsets, sorted_src, inv_pos as
+ *   produced by moe_permute.
+ *   moe_out [T][H] bf16 = sum_j topk_w[t][j] * MLP_{e(t,j)}(xn_moe[t]), the branch
+ *   output before its post norm.  Accumulation is fp32; h and the weighted expert
+ *   outputs are stored as bf16 between the two GEMMs. */
+moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* xn_moe,
+                             const float* topk_w, const int32_t* expert_offsets,
+                             const int32_t* sorted_src, const int32_t* inv_pos,
+                             const moe_expert_weights_t* experts, moe_bf16_t* moe_out,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Shared dense MLP (ONNX export card, "MoE topology" row).
+ *   xn_dense [T][H]; w_gate_up [2D][H] (gate rows, then up rows); w_down [H][D].
+ *   dense_out [T][H] bf16 = gelu_tanh(xn g^T) * (xn u^T) W_down^T, fp32 accumulation. */
+moe_status_t dense_mlp_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* xn_dense,
+                               const moe_bf16_t* w_gate_up, const moe_bf16_t* w_down,
+                               moe_bf16_t* dense_out, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole block: router -> permute -> experts and dense MLP -> combine, post norms
+ * and residual (ONNX export card, "MoE topology" row).
+ *   x [T][H] bf16 input; out [T][H] bf16.  moe_out [T][H] bf16 may be NULL; when given
+ *   it receives the MoE branch output before its post norm.
+ *   stage_events: NULL, or a host array of MOE_BLOCK_EVENTS cudaEvent_t that the call
+ *   records on `stream` at its stage boundaries, for timing each stage:
+ *     [0] start  [1] router done  [2] permutation done  [3] row gather done
+ *     [4] counters cleared  [5] gate_up GEMMs done  [6] down GEMMs done  [7] combine done */
+#define MOE_BLOCK_EVENTS 8
+moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
+                               const moe_block_weights_t* w, moe_bf16_t* out,
+                               moe_bf16_t* moe_out, void* ws, size_t ws_bytes, void* stream,
+                               void* const* stage_events);
+
+/* Per-output-row symmetric int8 quantisation ("Gemma-4 26B-A4B (MoE, int8 experts)",
+ * "How it works": per-channel symmetric INT8 expert weights).
+ *   w [rows][cols] bf16 -> q [rows][cols] int8, scales [rows] fp32, computed in fp32:
+ *   s = max|w| / 127 (s = 1 for an all-zero row), q = round-half-even(w / s) clamped to
+ *   [-127, 127].  cols a multiple of 8 (1..65536), rows >= 0. */
+moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, int8_t* q,
+                               float* scales, void* stream);
+
+/* Waits for `stream`, then reads and clears the device status word in `ws`.
+ * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, or MOE_ERR_CUDA if the stream failed. */
+moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream);
+
+/* A short constant English description of a status code. */
+const char* moe_status_string(moe_status_t status);
+
+/* Version of this interface (increases when a signature changes). */
+int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_FFN_H */

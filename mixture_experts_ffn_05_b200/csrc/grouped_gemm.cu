@@ -1,0 +1,442 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// Used for both halves of every expert MLP and of the shared dense MLP:
+//   gate_up (kind 0): h[pos][i] = gelu_tanh(g) * u, g/u = xn[pos] . W_gate_up[e][i or I+i]
+//   down    (kind 1): Y[row][o] = w(row) * (h[pos] . W_down[e][o])
+// (ONNX export card, "Truthful graph contracts", "Mixture of Experts" and "MoE topology"
+// rows; Inferentia2 card, "How it works": expert outputs weighted by the routing weight).
+//
+// Orientation: the weights are the M operand (128 rows per tile, streamed once from
+// HBM by TMA), the tokens of one expert are the N operand (BN columns).  A decode
+// batch puts a handful of tokens on each expert, so N is small and the kernel is a
+// weight stream; a prefill batch fills N up to 256.  For gate_up, each 128-row tile is
+// 64 gate rows followed by the 64 matching up rows, so one accumulator holds both
+// halves and the epilogue pairs them.
+//
+// Work list: for each problem (experts, then the optional dense MLP), for each group,
+// for each M tile, for each N tile of BN tokens, `split` pieces along K.  Pieces are
+// dealt round-robin to a persistent grid (one CTA per SM).  When split > 1 each piece
+// stores its fp32 partial tile; the last piece to arrive (an atomic counter) sums all
+// partials in piece order, so the result does not depend on arrival order.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads into a ring of shared-memory
+// stages, warp 1 issues tcgen05.mma into one of two TMEM accumulators, warps 2-5 read
+// the accumulator back (tcgen05.ld) and run the epilogue while the next tile is being
+// multiplied.  Every wait is bounded; a wait that runs out records a timeout in the
+// status word and the CTA winds down.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+constexpr int kGemmThreads = 192;
+constexpr int kMaxEntries = 258;  // groups of problem 0 (<= 256) + problem 1 (1) + 1
+
+template <int BN>
+struct Cfg {
+  static constexpr int kABytes = 128 * 64 * 2;  // 128 weight rows x 64 K (bf16)
+  static constexpr int kBBytes = BN * 64 * 2;   // BN token rows x 64 K
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kStages = BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4));
+  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+  // after the stages: barriers, bookkeeping, the gate/up exchange buffer
+  static constexpr int kBarOff = kStages * kStage;
+  static constexpr int kNumBars = 2 * kStages + 5;  // full, empty, acc_full x2, acc_empty x2, drain
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kMiscInts = 8;               // tmem slot, abort, bcast, ...
+  static constexpr int kPreOff = kMiscOff + kMiscInts * 4;
+  static constexpr int kTabInts = 4 * kMaxEntries;  // pre, cnt, b0, ng
+  static constexpr int kXchgOff = ((kPreOff + kTabInts * 4) + 15) & ~15;
+  static constexpr int kXchgBytes = 16 * 64 * 4;
+  static constexpr int kSmem = kXchgOff + kXchgBytes + 1024;  // + alignment slack
+  static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment");
+};
+
+struct Piece {
+  int p, g, m, n, s;
+  int k0, k1;
+  int b_row0, n_valid;
+  int first_piece;
+};
+
+__device__ __forceinline__ int find_entry(const int* pre, int nent, int piece) {
+  int lo = 0, hi = nent - 1;  // largest i with pre[i] <= piece
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= piece) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int BN>
+__device__ __forceinline__ Piece decode_piece(int piece, const GemmParams& P, const int* pre,
+                                              const int* b0, const int* ng, int nent) {
+  Piece pc;
+  const int i = find_entry(pre, nent, piece);
+  const int G0 = P.prob[0].groups;
+  pc.p = i < G0 ? 0 : 1;
+  pc.g = i < G0 ? i : i - G0;
+  const GemmProblem& pr = P.prob[pc.p];
+  const int ntl = (ng[i] + BN - 1) / BN;
+  const int local = piece - pre[i];
+  pc.s = local % pr.split;
+  const int tl = local / pr.split;
+  pc.n = tl % ntl;
+  pc.m = tl / ntl;
+  pc.k0 = pc.s * pr.k_steps / pr.split;
+  pc.k1 = (pc.s + 1) * pr.k_steps / pr.split;
+  pc.b_row0 = b0[i];
+  pc.n_valid = min(BN, ng[i] - pc.n * BN);
+  pc.first_piece = piece - pc.s;
+  return pc;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams P) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* acc_full = empty + C::kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  int* misc = reinterpret_cast<int*>(smem + C::kMiscOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 0);
+  volatile int* abort_flag = misc + 1;
+  volatile int* bcast = misc + 2;
+  int* pre = reinterpret_cast<int*>(smem + C::kPreOff);
+  int* cnt = pre + kMaxEntries;
+  int* b0 = cnt + kMaxEntries;
+  int* ng = b0 + kMaxEntries;
+  float* xchg = reinterpret_cast<float*>(smem + C::kXchgOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nent = P.prob[0].groups + (P.nprob > 1 ? P.prob[1].groups : 0);
+
+  // ---- setup: barriers, TMEM, the piece table
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    mbar_init(drain, 1);
+    mbar_fence_init();
+    *abort_flag = 0;
+    tma_prefetch_map(&maps.a[0]);
+    tma_prefetch_map(&maps.b[0]);
+    if (P.nprob > 1) {
+      tma_prefetch_map(&maps.a[1]);
+      tma_prefetch_map(&maps.b[1]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < nent; i += kGemmThreads) {
+    const int p = i < P.prob[0].groups ? 0 : 1;
+    const int g = p == 0 ? i : i - P.prob[0].groups;
+    const GemmProblem& pr = P.prob[p];
+    int s0, n;
+    if (pr.offsets) {
+      // Segments are clamped to [0, b_rows) so a bad offsets table cannot move any
+      // access out of the B operand or the outputs.
+      const int brows = pr.n_tokens;
+      int a = pr.offsets[g], b = pr.offsets[g + 1];
+      a = max(0, min(a, brows));
+      b = max(a, min(b, brows));
+      s0 = a;
+      n = b - a;
+    } else {
+      s0 = 0;
+      n = pr.n_tokens;
+    }
+    b0[i] = s0;
+    ng[i] = n;
+    cnt[i] = pr.m_tiles * ((n + BN - 1) / BN) * pr.split;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < nent; base += 32) {
+      const int i = base + lane;
+      const int v = i < nent ? cnt[i] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (i < nent) pre[i] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) pre[nent] = carry;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = pre[nent];
+  const uint64_t tmo = P.timeout_ns;
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();  // weights: read once
+      const uint64_t pol_b = policy_evict_last();   // tokens: reused by every M tile
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed[C::kStages];
+      for (int i = 0; i < C::kStages; ++i) armed[i] = -1;
+      bool ok = true;
+      for (int piece = blockIdx.x; piece < total && ok; piece += gridDim.x) {
+        const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
+        const GemmProblem& pr = P.prob[pc.p];
+        const CUtensorMap* ma = &maps.a[pr.map];
+        const CUtensorMap* mb = &maps.b[pr.map];
+        const int arow = pc.g * pr.w_rows_per_group + pc.m * (pr.kind == 0 ? 64 : 128);
+        const int brow = pc.b_row0 + pc.n * BN;
+        for (int ks = pc.k0; ks < pc.k1; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::kStage;
+          mbar_arrive_expect_tx(&full[stage], C::kStage);
+          if (pr.kind == 0) {
+            tma_load_2d(sa, ma, &full[stage], ks * 64, arow, pol_w);
+            tma_load_2d(sa + C::kABytes / 2, ma, &full[stage], ks * 64, arow + pr.nw, pol_w);
+          } else {
+            tma_load_2d(sa, ma, &full[stage], ks * 64, arow, pol_w);
+          }
+          tma_load_2d(sa + C::kABytes, mb, &full[stage], ks * 64, brow, pol_b);
+          armed[stage] = static_cast<int>(phase);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        record_status(P.status, kStatusTimeout);
+        *abort_flag = 1;
+        // Let every copy already issued land before the CTA winds down.
+        for (int i = 0; i < C::kStages; ++i)
+          if (armed[i] >= 0) mbar_wait(&full[i], static_cast<uint32_t>(armed[i]), tmo, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int ab = 0;
+      uint32_t aph = 0;
+      bool ok = true, issued = false;
+      for (int piece = blockIdx.x; piece < total && ok; piece += gridDim.x) {
+        const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
+        const uint32_t idesc = idesc_bf16_f32(128, (pc.n_valid + 15) & ~15);
+        if (!mbar_wait(&acc_empty[ab], aph ^ 1u, tmo, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(ab * BN);
+        for (int ks = pc.k0; ks < pc.k1; ++ks) {
+          if (!mbar_wait(&full[stage], phase, tmo, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::kStage);
+          const uint64_t ad = sdesc_k_sw128(sa);
+          const uint64_t bd = sdesc_k_sw128(sa + C::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (ks > pc.k0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          issued = true;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[ab]);
+        ab ^= 1;
+        if (ab == 0) aph ^= 1u;
+      }
+      if (!ok) {
+        record_status(P.status, kStatusTimeout);
+        *abort_flag = 1;
+        if (issued) {  // wait for the MMAs in flight before TMEM is released
+          umma_commit(drain);
+          mbar_wait(drain, 0, tmo, nullptr);
+        }
+      }
+    }
+  } else {
+    // ================= epilogue (warps 2..5, TMEM lanes by warp % 4) =================
+    const int q = warp & 3;
+    const int row = q * 32 + lane;  // accumulator row = TMEM lane
+    const int et = threadIdx.x - 64;
+    int ab = 0;
+    uint32_t aph = 0;
+    for (int piece = blockIdx.x; piece < total; piece += gridDim.x) {
+      const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
+      const GemmProblem& pr = P.prob[pc.p];
+      if (et == 0) *bcast = mbar_wait(&acc_full[ab], aph, tmo, abort_flag) ? 1 : 0;
+      named_sync(1, 128);
+      if (!*bcast) {
+        if (et == 0) {
+          record_status(P.status, kStatusTimeout);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(ab * BN);
+      const int ncols = (pc.n_valid + 15) & ~15;
+      bool last = true;
+      if (pr.split > 1) {
+        float* part = P.partials + static_cast<size_t>(piece) * BN * 128;
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + c0, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) __stcg(part + (c0 + i) * 128 + row, v[i]);
+        }
+        __threadfence();
+        named_sync(1, 128);
+        if (et == 0) {
+          const unsigned old = atomicAdd(P.counters + pc.first_piece, 1u);
+          const int l = (old == static_cast<unsigned>(pr.split - 1)) ? 1 : 0;
+          if (l) P.counters[pc.first_piece] = 0u;  // ready for the next launch
+          *bcast = l;
+        }
+        named_sync(1, 128);
+        last = *bcast != 0;
+        if (last) __threadfence();
+      }
+      if (last) {
+        const int out_col0 = pc.m * (pr.kind == 0 ? 64 : 128);
+        float sc = 1.f;
+        if (pr.wscale) {
+          const int wr = pr.kind == 0 ? (row < 64 ? out_col0 + row : pr.nw + out_col0 + row - 64)
+                                      : out_col0 + row;
+          sc = pr.wscale[static_cast<size_t>(pc.g) * pr.w_rows_per_group + wr];
+        }
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + c0, v);
+          if (pr.split > 1) {
+            float acc[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+            for (int s2 = 0; s2 < pr.split; ++s2) {
+              if (s2 == pc.s) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] += v[i];
+              } else {
+                const float* qp = P.partials + static_cast<size_t>(pc.first_piece + s2) * BN * 128;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] += __ldcg(qp + (c0 + i) * 128 + row);
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = acc[i];
+          }
+          if (pr.kind == 0) {
+            if (row >= 64) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) xchg[i * 64 + (row - 64)] = v[i] * sc;
+            }
+            named_sync(1, 128);
+            if (row < 64) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int col = c0 + i;
+                if (col < pc.n_valid) {
+                  const float h = gelu_tanh(v[i] * sc) * xchg[i * 64 + row];
+                  const size_t orow = static_cast<size_t>(pc.b_row0 + pc.n * BN + col);
+                  pr.out[orow * pr.out_ld + out_col0 + row] = bf16_bits(h);
+                }
+              }
+            }
+            named_sync(1, 128);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int col = c0 + i;
+              if (col < pc.n_valid) {
+                const int pos = pc.b_row0 + pc.n * BN + col;
+                const int orow = pr.out_rows ? pr.out_rows[pos] : pos;
+                if (orow >= 0 && orow < pr.n_tokens) {
+                  const float w = pr.route_w ? pr.route_w[orow] : 1.f;
+                  pr.out[static_cast<size_t>(orow) * pr.out_ld + out_col0 + row] =
+                      bf16_bits(v[i] * sc * w);
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      named_sync(1, 128);  // every flag of this piece is read before the next is written
+      mbar_arrive(&acc_empty[ab]);
+      ab ^= 1;
+      if (ab == 0) aph ^= 1u;
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <int BN>
+static cudaError_t launch_bn(const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s) {
+  const int smem = Cfg<BN>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  grouped_gemm_kernel<BN><<<grid, kGemmThreads, smem, s>>>(maps, p);
+  return cudaGetLastError();
+}
+
+size_t grouped_gemm_smem_bytes(int bn) {
+  switch (bn) {
+    case 16: return Cfg<16>::kSmem;
+    case 32: return Cfg<32>::kSmem;
+    case 64: return Cfg<64>::kSmem;
+    case 128: return Cfg<128>::kSmem;
+    case 256: return Cfg<256>::kSmem;
+  }
+  return 0;
+}
+
+cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
+                                cudaStream_t s) {
+  switch (bn) {
+    case 16: return launch_bn<16>(maps, p, grid, s);
+    case 32: return launch_bn<32>(maps, p, grid, s);
+    case 64: return launch_bn<64>(maps, p, grid, s);
+    case 128: return launch_bn<128>(maps, p, grid, s);
+    case 256: return launch_bn<256>(maps, p, grid, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,78 @@
+// Host-side declarations shared by the kernel files and the C interface (moe_ffn.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// One GEMM problem of a grouped launch.  The weights are the M operand (rows of a
+// K-major matrix streamed by TMA), the tokens the N operand.
+//   kind 0 (gate_up): each M tile is 64 gate rows + the 64 matching up rows of one
+//     group; the epilogue writes h = gelu_tanh(gate) * up as bf16.
+//   kind 1 (down): each M tile is 128 rows of the output; the epilogue scales by the
+//     int8 row scale (if any) and the routing weight (if any) and writes bf16.
+struct GemmProblem {
+  int kind;              // 0 gate_up, 1 down
+  int groups;            // experts, or 1 for the dense MLP
+  const int* offsets;    // [groups+1] token segments in the B operand; NULL = one group
+  int n_tokens;          // rows of the B operand and of the output (segments are
+                         // clamped to it); the single group's tokens if offsets == NULL
+  int k_steps;           // K / 64
+  int m_tiles;           // gate_up: Nw / 64;  down: rows / 128
+  int w_rows_per_group;  // gate_up: 2 * Nw;   down: rows
+  int nw;                // gate_up: Nw (first up row); down: unused
+  int split;             // pieces per tile along K (>= 1)
+  int map;               // tensor-map pair: 0 or 1
+  uint16_t* out;         // bf16 output
+  int out_ld;            // elements per output row
+  const int* out_rows;   // down: output row of B row pos (sorted_src); NULL = pos
+  const float* route_w;  // down: weight per output row (topk_w flattened); NULL = 1
+  const float* wscale;   // int8 row scales [groups][w_rows_per_group]; NULL for bf16
+};
+
+struct GemmParams {
+  GemmProblem prob[2];
+  int nprob;
+  int int8_weights;     // A operand stored as int8 (converted in shared memory)
+  float* partials;      // split-K partial tiles, [piece][BN][128] fp32
+  unsigned* counters;   // split-K arrival counters, zero between launches
+  unsigned* status;     // device status word
+  uint64_t timeout_ns;  // bound of every wait
+};
+
+struct GemmMaps {
+  CUtensorMap a[2];  // weights of problem map 0 / 1
+  CUtensorMap b[2];  // tokens of problem map 0 / 1
+};
+
+// kernels/*.cu launchers.  All return cudaSuccess or the launch error.
+cudaError_t launch_router_logits(int T, int H, int E, float eps, float inv_sqrt_h,
+                                 const uint16_t* x, const uint16_t* router_scale,
+                                 const uint16_t* w_router, const float* bias,
+                                 const uint16_t* g_pre_moe, const uint16_t* g_pre_dense,
+                                 uint16_t* xn_moe, uint16_t* xn_dense, float* logits,
+                                 cudaStream_t s);
+cudaError_t launch_router_topk(int T, int E, int k, const float* logits,
+                               const uint16_t* per_expert_scale, int* topk_idx, float* topk_w,
+                               cudaStream_t s);
+cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int* sorted_src,
+                           int* inv_pos, int* block_hist, int* block_base, cudaStream_t s);
+int permute_blocks(int n);  // blocks of the multi-block path (0 = single-block path)
+cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
+                               const uint16_t* src, uint16_t* dst, cudaStream_t s);
+cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
+                                cudaStream_t s);
+size_t grouped_gemm_smem_bytes(int bn);
+cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
+                                 const uint16_t* y, const uint16_t* dense,
+                                 const uint16_t* g_post_moe, const uint16_t* g_post_dense,
+                                 const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
+                                 cudaStream_t s);
+cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, uint16_t* moe_out,
+                               cudaStream_t s);
+cudaError_t launch_quantize_int8(const uint16_t* w, int64_t rows, int cols, int8_t* q,
+                                 float* scales, cudaStream_t s);
+
+}  // namespace moe

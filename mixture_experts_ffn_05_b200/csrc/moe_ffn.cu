@@ -1,0 +1,529 @@
+// C interface of the hybrid MoE feed-forward block: argument checks, workspace layout,
+// TMA tensor maps and the launch sequence.  See include/moe_ffn.h for the contract.
+#include <cudaTypedefs.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "moe_ffn.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bound of every device wait: 2 s
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- sizes and checks
+
+struct Dims {
+  int T, H, E, k, I, D;
+  float eps;
+  int int8;
+};
+
+moe_status_t check_cfg(const moe_config_t* c, int32_t T, Dims* d) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (!(c->eps > 0.f) || !(c->eps < 1e30f)) return MOE_ERR_INVALID_ARG;
+  if (c->expert_wdtype != MOE_W_BF16 && c->expert_wdtype != MOE_W_INT8) return MOE_ERR_INVALID_ARG;
+  if (c->hidden < 128 || c->hidden > 6144 || c->hidden % 128) return MOE_ERR_UNSUPPORTED;
+  if (c->expert_inter < 64 || c->expert_inter > 16384 || c->expert_inter % 64) return MOE_ERR_UNSUPPORTED;
+  if (c->dense_inter < 64 || c->dense_inter > 16384 || c->dense_inter % 64) return MOE_ERR_UNSUPPORTED;
+  if (c->num_experts < 1 || c->num_experts > 256) return MOE_ERR_UNSUPPORTED;
+  if (c->top_k < 1 || c->top_k > 16 || c->top_k > c->num_experts) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(T) * c->top_k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  // every weight tensor must be addressable by a 32-bit TMA row coordinate
+  if (static_cast<int64_t>(c->num_experts) * 2 * c->expert_inter >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(c->num_experts) * c->hidden >= (int64_t(1) << 31))
+    return MOE_ERR_UNSUPPORTED;
+  d->T = T;
+  d->H = c->hidden;
+  d->E = c->num_experts;
+  d->k = c->top_k;
+  d->I = c->expert_inter;
+  d->D = c->dense_inter;
+  d->eps = c->eps;
+  d->int8 = c->expert_wdtype == MOE_W_INT8;
+  return MOE_OK;
+}
+
+// Token-tile width of the GEMMs: about twice the mean number of tokens per expert.
+int choose_bn(const Dims& d) {
+  const double avg = static_cast<double>(d.T) * d.k / d.E;
+  int bn = 16;
+  while (bn < 256 && bn < 2.0 * avg) bn *= 2;
+  return bn;
+}
+
+// K pieces per tile: only for the narrowest token tiles (weight-streaming batches),
+// so that the tile list is fine enough to keep every SM streaming to the end.
+int choose_split(int k_steps, int bn) {
+  if (bn != 16) return 1;
+  return std::max(1, std::min(k_steps, (k_steps + 10) / 11));
+}
+
+struct Layout {
+  size_t status, counters, logits, bhist, bbase, topk_idx, topk_w, offsets, sorted, inv;
+  size_t xn_moe, xn_dense, aperm, h, y, hd, dense, partials, total;
+  size_t counters_bytes;
+  int bn, split_gu, split_dgu, split_d, split_dd;
+};
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+Layout layout_of(const Dims& d) {
+  Layout L{};
+  const int64_t T = d.T, Tk = static_cast<int64_t>(d.T) * d.k;
+  L.bn = choose_bn(d);
+  L.split_gu = choose_split(d.H / 64, L.bn);
+  L.split_dgu = choose_split(d.H / 64, L.bn);
+  L.split_d = choose_split(d.I / 64, L.bn);
+  L.split_dd = choose_split(d.D / 64, L.bn);
+  // Upper bound of the N tiles: every non-empty expert has a partial tile.
+  const int64_t ntl_e = std::min<int64_t>(d.E, Tk) + ceil_div(Tk, L.bn);
+  const int64_t ntl_d = ceil_div(T, L.bn);
+  const int64_t pieces_gu = (d.I / 64) * ntl_e * L.split_gu + (d.D / 64) * ntl_d * L.split_dgu;
+  const int64_t pieces_dn = (d.H / 128) * ntl_e * L.split_d + (d.H / 128) * ntl_d * L.split_dd;
+  const int64_t pieces = std::max(pieces_gu, pieces_dn);
+  const bool any_split = L.split_gu > 1 || L.split_dgu > 1 || L.split_d > 1 || L.split_dd > 1;
+  const int nb = permute_blocks(static_cast<int>(Tk));
+
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + std::max<size_t>(bytes, 1), kAlign);
+    return at;
+  };
+  L.status = take(256);
+  L.counters_bytes = static_cast<size_t>(pieces) * 4;
+  L.counters = take(L.counters_bytes);
+  L.logits = take(static_cast<size_t>(T) * d.E * 4);
+  L.bhist = take(static_cast<size_t>(nb) * d.E * 4);
+  L.bbase = take(static_cast<size_t>(nb) * d.E * 4);
+  L.topk_idx = take(Tk * 4);
+  L.topk_w = take(Tk * 4);
+  L.offsets = take((d.E + 1) * 4);
+  L.sorted = take(Tk * 4);
+  L.inv = take(Tk * 4);
+  L.xn_moe = take(T * d.H * 2);
+  L.xn_dense = take(T * d.H * 2);
+  L.aperm = take(Tk * d.H * 2);
+  L.h = take(Tk * d.I * 2);
+  L.y = take(Tk * d.H * 2);
+  L.hd = take(T * d.D * 2);
+  L.dense = take(T * d.H * 2);
+  L.partials = take(any_split ? static_cast<size_t>(pieces) * L.bn * 128 * 4 : 0);
+  L.total = off;
+  return L;
+}
+
+moe_status_t check_ws(const Dims& d, void* ws, size_t ws_bytes, Layout* L) {
+  *L = layout_of(d);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < L->total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// ---------------------------------------------------------------- devices and TMA
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+int g_sm_count[64] = {0};
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+// K-major 2-D map: rows x cols elements, box 64 (K) x box_rows, 128-byte swizzle.
+bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
+               CUtensorMapDataType dt, int elem_bytes) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  return encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2);
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ---------------------------------------------------------------- the expert / dense GEMMs
+
+struct GemmJob {
+  // experts (problem 0), may be absent
+  bool experts;
+  const uint16_t* a_rows;    // gathered xn_moe rows, [Tk][H]
+  const void* w_gate_up;
+  const void* w_down;
+  const float* s_gate_up;
+  const float* s_down;
+  const int* offsets;
+  const int* sorted_src;
+  const float* topk_w;
+  uint16_t* y;               // [Tk][H] weighted expert outputs
+  // dense MLP (problem 1 when experts are present, else problem 0), may be absent
+  bool dense;
+  const uint16_t* xn_dense;  // [T][H]
+  const uint16_t* w_dgu;     // [2D][H]
+  const uint16_t* w_dd;      // [H][D]
+  uint16_t* dense_out;       // [T][H]
+};
+
+// Records ev[i] on s when a stage-event array was given.
+bool mark(void* const* ev, int i, cudaStream_t s) {
+  return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
+}
+
+moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& j,
+                       cudaStream_t s, void* const* ev = nullptr) {
+  const int64_t Tk = static_cast<int64_t>(d.T) * d.k;
+  const int grid = sm_count();
+  if (grid <= 0) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(at<uint8_t>(ws, L.status), 0, L.counters - L.status + L.counters_bytes, s) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (!mark(ev, 4, s)) return MOE_ERR_CUDA;
+  uint16_t* h = at<uint16_t>(ws, L.h);
+  uint16_t* hd = at<uint16_t>(ws, L.hd);
+
+  GemmParams gu{}, dn{};
+  GemmMaps mgu{}, mdn{};
+  for (GemmParams* P : {&gu, &dn}) {
+    P->partials = at<float>(ws, L.partials);
+    P->counters = at<unsigned>(ws, L.counters);
+    P->status = at<unsigned>(ws, L.status);
+    P->timeout_ns = kWaitTimeoutNs;
+    P->int8_weights = 0;
+  }
+  int np = 0;
+  if (j.experts) {
+    GemmProblem& a = gu.prob[np];
+    a = GemmProblem{};
+    a.kind = 0; a.groups = d.E; a.offsets = j.offsets; a.n_tokens = static_cast<int>(Tk);
+    a.k_steps = d.H / 64; a.m_tiles = d.I / 64; a.w_rows_per_group = 2 * d.I; a.nw = d.I;
+    a.split = L.split_gu; a.map = np; a.out = h; a.out_ld = d.I; a.wscale = j.s_gate_up;
+    GemmProblem& b = dn.prob[np];
+    b = GemmProblem{};
+    b.kind = 1; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = static_cast<int>(Tk);
+    b.k_steps = d.I / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H; b.nw = 0;
+    b.split = L.split_d; b.map = np; b.out = j.y; b.out_ld = d.H; b.out_rows = j.sorted_src;
+    b.route_w = j.topk_w; b.wscale = j.s_down;
+    if (!encode_bf16(&mgu.a[np], j.w_gate_up, static_cast<int64_t>(d.E) * 2 * d.I, d.H, 64) ||
+        !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, L.bn) ||
+        !encode_bf16(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128) ||
+        !encode_bf16(&mdn.b[np], h, Tk, d.I, L.bn))
+      return MOE_ERR_CUDA;
+    ++np;
+  }
+  if (j.dense) {
+    GemmProblem& a = gu.prob[np];
+    a = GemmProblem{};
+    a.kind = 0; a.groups = 1; a.offsets = nullptr; a.n_tokens = d.T;
+    a.k_steps = d.H / 64; a.m_tiles = d.D / 64; a.w_rows_per_group = 2 * d.D; a.nw = d.D;
+    a.split = L.split_dgu; a.map = np; a.out = hd; a.out_ld = d.D;
+    GemmProblem& b = dn.prob[np];
+    b = GemmProblem{};
+    b.kind = 1; b.groups = 1; b.offsets = nullptr; b.n_tokens = d.T;
+    b.k_steps = d.D / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H;
+    b.split = L.split_dd; b.map = np; b.out = j.dense_out; b.out_ld = d.H;
+    if (!encode_bf16(&mgu.a[np], j.w_dgu, 2 * static_cast<int64_t>(d.D), d.H, 64) ||
+        !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, L.bn) ||
+        !encode_bf16(&mdn.a[np], j.w_dd, d.H, d.D, 128) ||
+        !encode_bf16(&mdn.b[np], hd, d.T, d.D, L.bn))
+      return MOE_ERR_CUDA;
+    ++np;
+  }
+  gu.nprob = dn.nprob = np;
+  if (np == 1) {  // unused second pair: a valid copy of the first
+    mgu.a[1] = mgu.a[0]; mgu.b[1] = mgu.b[0];
+    mdn.a[1] = mdn.a[0]; mdn.b[1] = mdn.b[0];
+  }
+  moe_status_t st = cuda_status(launch_grouped_gemm(L.bn, mgu, gu, grid, s));
+  if (st != MOE_OK) return st;
+  if (!mark(ev, 5, s)) return MOE_ERR_CUDA;
+  st = cuda_status(launch_grouped_gemm(L.bn, mdn, dn, grid, s));
+  if (st != MOE_OK) return st;
+  return mark(ev, 6, s) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool w_ok(const moe_expert_weights_t* w, bool int8) {
+  if (w == nullptr || w->w_gate_up == nullptr || w->w_down == nullptr) return false;
+  if (!aligned16(w->w_gate_up) || !aligned16(w->w_down)) return false;
+  if (int8) return w->s_gate_up != nullptr && w->s_down != nullptr;
+  return w->s_gate_up == nullptr && w->s_down == nullptr;
+}
+
+}  // namespace
+
+// ================================================================ the C interface
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return 1; }
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported size";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device wait ran out";
+  }
+  return "unknown status";
+}
+
+size_t moe_workspace_size(const moe_config_t* cfg, int32_t T) {
+  Dims d;
+  if (check_cfg(cfg, T, &d) != MOE_OK) return 0;
+  return layout_of(d).total;
+}
+
+moe_status_t moe_router(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
+                        const moe_bf16_t* router_scale, const moe_bf16_t* w_router,
+                        const float* logit_bias, const moe_bf16_t* per_expert_scale,
+                        const moe_bf16_t* g_pre_moe, const moe_bf16_t* g_pre_dense,
+                        int32_t* topk_idx, float* topk_w, moe_bf16_t* xn_moe,
+                        moe_bf16_t* xn_dense, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  moe_status_t st = check_cfg(cfg, T, &d);
+  if (st != MOE_OK) return st;
+  for (const void* p : {(const void*)x, (const void*)router_scale, (const void*)w_router,
+                        (const void*)per_expert_scale, (const void*)g_pre_moe,
+                        (const void*)g_pre_dense, (const void*)topk_idx, (const void*)topk_w,
+                        (const void*)xn_moe, (const void*)xn_dense})
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (logit_bias != nullptr && !aligned16(logit_bias)) return MOE_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* logits = at<float>(ws, L.logits);
+  st = cuda_status(launch_router_logits(d.T, d.H, d.E, d.eps, 1.0f / sqrtf(static_cast<float>(d.H)),
+                                        x, router_scale, w_router, logit_bias, g_pre_moe,
+                                        g_pre_dense, xn_moe, xn_dense, logits, s));
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_router_topk(d.T, d.E, d.k, logits, per_expert_scale, topk_idx, topk_w, s));
+}
+
+moe_status_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx,
+                         int32_t* expert_offsets, int32_t* sorted_src, int32_t* inv_pos,
+                         void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  moe_status_t st = check_cfg(cfg, T, &d);
+  if (st != MOE_OK) return st;
+  for (const void* p : {(const void*)topk_idx, (const void*)expert_offsets,
+                        (const void*)sorted_src, (const void*)inv_pos})
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  return cuda_status(launch_permute(d.T * d.k, d.E, topk_idx, expert_offsets, sorted_src, inv_pos,
+                                    at<int>(ws, L.bhist), at<int>(ws, L.bbase),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* xn_moe,
+                             const float* topk_w, const int32_t* expert_offsets,
+                             const int32_t* sorted_src, const int32_t* inv_pos,
+                             const moe_expert_weights_t* experts, moe_bf16_t* moe_out,
+                             void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  moe_status_t st = check_cfg(cfg, T, &d);
+  if (st != MOE_OK) return st;
+  for (const void* p : {(const void*)xn_moe, (const void*)topk_w, (const void*)expert_offsets,
+                        (const void*)sorted_src, (const void*)inv_pos, (const void*)moe_out})
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (!w_ok(experts, d.int8)) return MOE_ERR_INVALID_ARG;
+  if (d.int8) return MOE_ERR_UNSUPPORTED;
+  Layout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int Tk = d.T * d.k;
+  uint16_t* aperm = at<uint16_t>(ws, L.aperm);
+  uint16_t* y = at<uint16_t>(ws, L.y);
+  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted_src, xn_moe, aperm, s))) != MOE_OK)
+    return st;
+  GemmJob j{};
+  j.experts = true;
+  j.a_rows = aperm;
+  j.w_gate_up = experts->w_gate_up;
+  j.w_down = experts->w_down;
+  j.s_gate_up = experts->s_gate_up;
+  j.s_down = experts->s_down;
+  j.offsets = expert_offsets;
+  j.sorted_src = sorted_src;
+  j.topk_w = topk_w;
+  j.y = y;
+  if ((st = run_gemms(d, L, ws, j, s)) != MOE_OK) return st;
+  return cuda_status(launch_combine_moe(d.T, d.H, d.k, y, moe_out, s));
+}
+
+moe_status_t dense_mlp_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* xn_dense,
+                               const moe_bf16_t* w_gate_up, const moe_bf16_t* w_down,
+                               moe_bf16_t* dense_out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  moe_status_t st = check_cfg(cfg, T, &d);
+  if (st != MOE_OK) return st;
+  for (const void* p : {(const void*)xn_dense, (const void*)w_gate_up, (const void*)w_down,
+                        (const void*)dense_out})
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  Layout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  GemmJob j{};
+  j.dense = true;
+  j.xn_dense = xn_dense;
+  j.w_dgu = w_gate_up;
+  j.w_dd = w_down;
+  j.dense_out = dense_out;
+  return run_gemms(d, L, ws, j, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
+                               const moe_block_weights_t* w, moe_bf16_t* out,
+                               moe_bf16_t* moe_out, void* ws, size_t ws_bytes, void* stream,
+                               void* const* ev) {
+  Dims d;
+  moe_status_t st = check_cfg(cfg, T, &d);
+  if (st != MOE_OK) return st;
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)x, (const void*)out, (const void*)w->router_scale,
+                        (const void*)w->w_router, (const void*)w->per_expert_scale,
+                        (const void*)w->g_pre_moe, (const void*)w->g_pre_dense,
+                        (const void*)w->g_post_ff, (const void*)w->w_dense_gate_up,
+                        (const void*)w->w_dense_down})
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)moe_out, (const void*)w->logit_bias,
+                        (const void*)w->g_post_moe, (const void*)w->g_post_dense})
+    if (p != nullptr && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (!w_ok(&w->experts, d.int8)) return MOE_ERR_INVALID_ARG;
+  if (d.int8) return MOE_ERR_UNSUPPORTED;
+  Layout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int Tk = d.T * d.k;
+  int* topk_idx = at<int>(ws, L.topk_idx);
+  float* topk_w = at<float>(ws, L.topk_w);
+  int* offsets = at<int>(ws, L.offsets);
+  int* sorted = at<int>(ws, L.sorted);
+  int* inv = at<int>(ws, L.inv);
+  uint16_t* xn_moe = at<uint16_t>(ws, L.xn_moe);
+  uint16_t* xn_dense = at<uint16_t>(ws, L.xn_dense);
+  uint16_t* aperm = at<uint16_t>(ws, L.aperm);
+  uint16_t* y = at<uint16_t>(ws, L.y);
+  uint16_t* dense = at<uint16_t>(ws, L.dense);
+  float* logits = at<float>(ws, L.logits);
+
+  if (ev != nullptr)
+    for (int i = 0; i < MOE_BLOCK_EVENTS; ++i)
+      if (ev[i] == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!mark(ev, 0, s)) return MOE_ERR_CUDA;
+  if ((st = cuda_status(launch_router_logits(
+           d.T, d.H, d.E, d.eps, 1.0f / sqrtf(static_cast<float>(d.H)), x, w->router_scale,
+           w->w_router, w->logit_bias, w->g_pre_moe, w->g_pre_dense, xn_moe, xn_dense, logits,
+           s))) != MOE_OK)
+    return st;
+  if ((st = cuda_status(launch_router_topk(d.T, d.E, d.k, logits, w->per_expert_scale, topk_idx,
+                                           topk_w, s))) != MOE_OK)
+    return st;
+  if (!mark(ev, 1, s)) return MOE_ERR_CUDA;
+  if ((st = cuda_status(launch_permute(Tk, d.E, topk_idx, offsets, sorted, inv, at<int>(ws, L.bhist),
+                                       at<int>(ws, L.bbase), s))) != MOE_OK)
+    return st;
+  if (!mark(ev, 2, s)) return MOE_ERR_CUDA;
+  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe, aperm, s))) != MOE_OK)
+    return st;
+  if (!mark(ev, 3, s)) return MOE_ERR_CUDA;
+  GemmJob j{};
+  j.experts = true;
+  j.a_rows = aperm;
+  j.w_gate_up = w->experts.w_gate_up;
+  j.w_down = w->experts.w_down;
+  j.s_gate_up = w->experts.s_gate_up;
+  j.s_down = w->experts.s_down;
+  j.offsets = offsets;
+  j.sorted_src = sorted;
+  j.topk_w = topk_w;
+  j.y = y;
+  j.dense = true;
+  j.xn_dense = xn_dense;
+  j.w_dgu = w->w_dense_gate_up;
+  j.w_dd = w->w_dense_down;
+  j.dense_out = dense;
+  if ((st = run_gemms(d, L, ws, j, s, ev)) != MOE_OK) return st;
+  if ((st = cuda_status(launch_combine_block(d.T, d.H, d.k, d.eps, x, y, dense, w->g_post_moe,
+                                             w->g_post_dense, w->g_post_ff, out, moe_out, s))) !=
+      MOE_OK)
+    return st;
+  return mark(ev, 7, s) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, int8_t* q,
+                               float* scales, void* stream) {
+  if (rows < 0 || cols < 8 || cols > 65536 || cols % 8) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (rows > (int64_t(1) << 34)) return MOE_ERR_UNSUPPORTED;
+  if (w == nullptr || q == nullptr || scales == nullptr || !aligned16(w) || !aligned16(q))
+    return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scales) & 3u) != 0) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_int8(w, rows, cols, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned host = 0;
+  if (cudaMemcpyAsync(&host, ws, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (host == 0) return MOE_OK;
+  if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  return host == static_cast<unsigned>(MOE_ERR_DEVICE_TIMEOUT) ? MOE_ERR_DEVICE_TIMEOUT : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

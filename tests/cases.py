@@ -64,7 +64,7 @@ def zipf_alpha() -> float:
 
 
 def gap_filtered_x(seed: int, shape: synth.Shape, p: dict, bias, min_gap: float = MIN_GAP,
-                   max_attempts: int = 400, layer: int = 0) -> np.ndarray:
+                   max_attempts: int = 20000, layer: int = 0) -> np.ndarray:
     """Draw x row by row, redrawing a row until its oracle logits have top-(k+1)
     adjacent gaps >= min_gap.  Returns bf16 bits [T][H]."""
     T, H = shape.T, shape.H
@@ -88,22 +88,38 @@ def gap_filtered_x(seed: int, shape: synth.Shape, p: dict, bias, min_gap: float 
     return x
 
 
-_LAYER_CACHE: dict = {}
+class _Lru(dict):
+    def __init__(self, n):
+        super().__init__()
+        self.n = n
+
+    def put(self, key, value):
+        if key in self:
+            del self[key]
+        while len(self) >= self.n:
+            del self[next(iter(self))]
+        self[key] = value
+        return value
+
+
+_LAYER_CACHE = _Lru(3)
+_CASE_CACHE = _Lru(16)
 
 
 def make_case(shape: synth.Shape, seed: int = 1234, zipf: bool = False, layer: int = 0,
               gap: bool = True) -> Case:
+    ckey = (shape, seed, zipf, layer, gap)
+    if ckey in _CASE_CACHE:
+        return _CASE_CACHE[ckey]
     key = (shape.H, shape.E, shape.I, shape.D, seed, layer)
-    if key not in _LAYER_CACHE:
-        _LAYER_CACHE.clear()
-        _LAYER_CACHE[key] = synth.make_layer(seed, shape, layer)
-    p = _LAYER_CACHE[key]
+    p = _LAYER_CACHE[key] if key in _LAYER_CACHE else _LAYER_CACHE.put(
+        key, synth.make_layer(seed, shape, layer))
     bias = synth.zipf_bias(seed, shape.E, zipf_alpha()) if zipf else None
     if gap:
         x = gap_filtered_x(seed + 1, shape, p, bias, layer=layer)
     else:
         x = synth.x_rows(seed + 1, shape.H, shape.T, layer=layer)
-    return Case(shape, x, p, bias, seed)
+    return _CASE_CACHE.put(ckey, Case(shape, x, p, bias, seed))
 
 
 def bf16_experts(p: dict) -> oracle.Experts:

@@ -1,0 +1,92 @@
+"""Helpers of the GPU tests: move seeded inputs to the device, call the library through
+its binding, and fetch results back as numpy."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import mixture_experts_ffn_05_b200 as mf
+import oracle
+import synth
+from tests import cases
+
+
+def to_dev(a: np.ndarray, dtype=torch.bfloat16) -> torch.Tensor:
+    if dtype is torch.bfloat16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dtype).cuda()
+
+
+def bf16_np(t: torch.Tensor) -> np.ndarray:
+    """A bf16 device tensor as float64 numpy values."""
+    return oracle.bf16(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def config(shape: synth.Shape, int8: bool = False) -> mf.Config:
+    return mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps, int8)
+
+
+_DEV_CACHE = cases._Lru(3)
+
+
+def device_layer(case: cases.Case) -> dict:
+    key = id(case.p)
+    if key not in _DEV_CACHE or _DEV_CACHE[key][0] is not case.p:
+        _DEV_CACHE.put(key, (case.p, {n: to_dev(v) for n, v in case.p.items()}))
+    d = dict(_DEV_CACHE[key][1])
+    if case.bias is not None:
+        d["logit_bias"] = to_dev(case.bias, torch.float32)
+    return d
+
+
+_ORACLE_CACHE = cases._Lru(12)
+
+
+def oracle_block(case: cases.Case) -> dict:
+    key = (id(case.p), hash(case.x.tobytes()), None if case.bias is None else case.bias.tobytes())
+    if key not in _ORACLE_CACHE or _ORACLE_CACHE[key][0] is not case.p:
+        _ORACLE_CACHE.put(key, (case.p, oracle.block_forward(
+            case.x, case.p, cases.bf16_experts(case.p), case.shape.k, case.shape.eps, case.bias)))
+    return _ORACLE_CACHE[key][1]
+
+
+def run_router(cfg, case, layer, x=None):
+    T = case.shape.T
+    x = to_dev(case.x) if x is None else x
+    r = {
+        "topk_idx": torch.empty(T, cfg.top_k, dtype=torch.int32, device="cuda"),
+        "topk_w": torch.empty(T, cfg.top_k, dtype=torch.float32, device="cuda"),
+        "xn_moe": torch.empty(T, cfg.hidden, dtype=torch.bfloat16, device="cuda"),
+        "xn_dense": torch.empty(T, cfg.hidden, dtype=torch.bfloat16, device="cuda"),
+    }
+    ws = mf.workspace(cfg, T)
+    mf.moe_router(cfg, x, layer["router_scale"], layer["w_router"], layer.get("logit_bias"),
+                  layer["per_expert_scale"], layer["g_pre_moe"], layer["g_pre_dense"],
+                  r["topk_idx"], r["topk_w"], r["xn_moe"], r["xn_dense"], ws)
+    return r
+
+
+def run_permute(cfg, topk_idx: torch.Tensor):
+    T, k = topk_idx.shape
+    n = T * k
+    p = {
+        "offsets": torch.empty(cfg.num_experts + 1, dtype=torch.int32, device="cuda"),
+        "sorted_src": torch.empty(max(n, 1), dtype=torch.int32, device="cuda"),
+        "inv_pos": torch.empty(max(n, 1), dtype=torch.int32, device="cuda"),
+    }
+    ws = mf.workspace(cfg, T)
+    mf.moe_permute(cfg, topk_idx, p["offsets"], p["sorted_src"], p["inv_pos"], ws)
+    return p
+
+
+def run_block(cfg, case, layer, want_moe=True, ws=None, x=None):
+    T = case.shape.T
+    x = to_dev(case.x) if x is None else x
+    out = torch.empty(T, cfg.hidden, dtype=torch.bfloat16, device="cuda")
+    moe = torch.empty(T, cfg.hidden, dtype=torch.bfloat16, device="cuda") if want_moe else None
+    ws = mf.workspace(cfg, T) if ws is None else ws
+    bw = mf.BlockWeights(cfg, layer)
+    mf.moe_block_forward(cfg, x, bw, out, ws, moe_out=moe)
+    st = mf.moe_check_device_status(ws)
+    assert st == mf.MOE_OK, mf.status_string(st)
+    return out, moe

@@ -1,0 +1,133 @@
+"""The C interface on the CPU: the library loads, exports what include/moe_ffn.h
+declares, sizes its workspace, and rejects bad arguments before launching anything.
+No test here runs a kernel."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mixture_experts_ffn_05_b200 as mf
+from mixture_experts_ffn_05_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_ffn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mbuild.build()
+    return mf.lib()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    assert _declared_functions() == sorted(mf.ENTRY_POINTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", mf.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if l.strip()}
+    for name in _declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_version_and_status_strings(lib):
+    assert lib.moe_abi_version() == 1
+    for s in range(6):
+        assert mf.status_string(s)
+    assert mf.status_string(99) == "unknown status"
+
+
+CFG = mf.Config(hidden=2816, num_experts=128, top_k=8, expert_inter=704, dense_inter=2112)
+TINY = mf.Config(hidden=512, num_experts=16, top_k=4, expert_inter=128, dense_inter=384)
+
+
+def test_workspace_size(lib):
+    assert mf.workspace_size(CFG, 8) > 0
+    assert mf.workspace_size(CFG, 2048) > mf.workspace_size(CFG, 8)
+    assert mf.workspace_size(CFG, 0) > 0
+    bad = [dict(hidden=100), dict(hidden=6272), dict(top_k=129), dict(top_k=17),
+           dict(num_experts=257), dict(expert_inter=96), dict(dense_inter=0), dict(eps=0.0)]
+    for b in bad:
+        c = mf.Config(**{**CFG.__dict__, **b})
+        assert mf.workspace_size(c, 8) == 0, b
+    assert lib.moe_workspace_size(None, 8) == 0
+    assert mf.workspace_size(CFG, -1) == 0
+
+
+FAKE = 1 << 20  # an aligned address that is never dereferenced
+
+
+def _router(lib, cfg, T, ptrs, ws, ws_bytes):
+    return lib.moe_router(ctypes.byref(cfg.c()), T, *ptrs, ws, ws_bytes, None)
+
+
+def test_arguments_rejected_before_launch(lib):
+    n = mf.workspace_size(CFG, 8)
+    p = [FAKE] * 11
+    # a required pointer missing
+    q = list(p); q[0] = None
+    assert _router(lib, CFG, 8, q, FAKE, n) == mf.MOE_ERR_INVALID_ARG
+    # a misaligned pointer
+    q = list(p); q[1] = FAKE + 2
+    assert _router(lib, CFG, 8, q, FAKE, n) == mf.MOE_ERR_INVALID_ARG
+    # workspace too small, missing or misaligned
+    assert _router(lib, CFG, 8, p, FAKE, n - 1) == mf.MOE_ERR_WORKSPACE
+    assert _router(lib, CFG, 8, p, None, n) == mf.MOE_ERR_WORKSPACE
+    assert _router(lib, CFG, 8, p, FAKE + 16, n) == mf.MOE_ERR_WORKSPACE
+    # unsupported sizes, negative T
+    bad = mf.Config(**{**CFG.__dict__, "top_k": 200})
+    assert _router(lib, bad, 8, p, FAKE, n) == mf.MOE_ERR_UNSUPPORTED
+    assert _router(lib, CFG, -3, p, FAKE, n) == mf.MOE_ERR_INVALID_ARG
+    # T = 0 is a no-op that succeeds without touching memory
+    assert _router(lib, CFG, 0, p, FAKE, mf.workspace_size(CFG, 0)) == mf.MOE_OK
+
+
+def test_every_entry_point_validates(lib):
+    c = ctypes.byref(CFG.c())
+    n = mf.workspace_size(CFG, 8)
+    assert lib.moe_permute(c, 8, None, FAKE, FAKE, FAKE, FAKE, n, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute(c, 8, FAKE, FAKE, FAKE, FAKE, FAKE, 1, None) == mf.MOE_ERR_WORKSPACE
+    ew = mf.CExpertWeights(FAKE, FAKE, None, None)
+    assert lib.moe_ffn_forward(c, 8, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, n,
+                               None) == mf.MOE_ERR_INVALID_ARG
+    ew_bad = mf.CExpertWeights(FAKE, FAKE, FAKE, None)  # scales given for bf16 weights
+    assert lib.moe_ffn_forward(c, 8, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(ew_bad), FAKE,
+                               FAKE, n, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_ffn_forward(c, 0, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(ew), FAKE, FAKE,
+                               n, None) == mf.MOE_OK
+    assert lib.dense_mlp_forward(c, 8, FAKE, None, FAKE, FAKE, FAKE, n, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.dense_mlp_forward(c, 0, FAKE, FAKE, FAKE, FAKE, FAKE, n, None) == mf.MOE_OK
+    bw = mf.CBlockWeights(*([FAKE] * 9), ew, FAKE, FAKE)
+    assert lib.moe_block_forward(c, 8, FAKE, None, FAKE, None, FAKE, n, None, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_block_forward(c, 8, FAKE, ctypes.byref(bw), FAKE, None, FAKE, n - 1,
+                                 None, None) == mf.MOE_ERR_WORKSPACE
+    assert lib.moe_block_forward(c, 0, FAKE, ctypes.byref(bw), FAKE, None, FAKE, n,
+                                 None, None) == mf.MOE_OK
+    ev = (ctypes.c_void_p * 8)(*([FAKE] * 7 + [None]))  # an event missing
+    assert lib.moe_block_forward(c, 8, FAKE, ctypes.byref(bw), FAKE, None, FAKE, n,
+                                 None, ev) == mf.MOE_ERR_INVALID_ARG
+    bw.g_post_moe = FAKE + 4
+    assert lib.moe_block_forward(c, 8, FAKE, ctypes.byref(bw), FAKE, None, FAKE, n,
+                                 None, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_int8(FAKE, 4, 12, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_int8(None, 4, 16, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_int8(FAKE, 0, 16, FAKE, FAKE, None) == mf.MOE_OK
+    assert lib.moe_check_device_status(None, 256, None) == mf.MOE_ERR_WORKSPACE
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(8, 512, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        mf.dense_mlp_forward(TINY, x, x, x, x, torch.zeros(16, dtype=torch.uint8))

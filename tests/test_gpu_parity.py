@@ -1,0 +1,204 @@
+"""Parity of the CUDA path with the oracle, through the C interface, on a B200.
+
+Indices and the permutation are compared bit for bit; floating-point outputs at the
+accuracy bar (per-row cosine >= 0.9999, max-abs error <= 2e-2 * rms of the oracle row,
+plus half a bf16 ulp for the bf16 output format).
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_ffn_05_b200 as mf
+import oracle
+import synth
+from tests import cases
+from tests.gpu_util import (bf16_np, config, device_layer, oracle_block, run_block, run_permute,
+                            run_router, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+# name -> (shape, zipf offset)
+SHAPES = {
+    "tiny": (synth.TINY, False),
+    "tiny_T37": (synth.Shape(T=37, H=512, E=16, k=4, I=128, D=384), False),
+    "tiny_T1": (synth.Shape(T=1, H=512, E=16, k=4, I=128, D=384), False),
+    "decode_T8": (synth.DECODE, False),
+    "decode_T1": (synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112), False),
+    "decode_T64": (synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112), False),
+    "prefill_T2048_zipf": (synth.PREFILL, True),
+    "limits": (synth.Shape(T=5, H=6144, E=256, k=16, I=64, D=64), False),
+}
+FAST = ["tiny", "tiny_T37", "tiny_T1", "decode_T8", "decode_T1", "decode_T64"]
+
+
+def _case(name):
+    shape, zipf = SHAPES[name]
+    return cases.make_case(shape, seed=1234, zipf=zipf)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    mf.lib()
+
+
+# ------------------------------------------------------------------ router
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_router(name):
+    c = _case(name)
+    cfg = config(c.shape)
+    layer = device_layer(c)
+    r = run_router(cfg, c, layer)
+    o = oracle_block(c)
+    assert np.array_equal(r["topk_idx"].cpu().numpy(), o["topk_idx"])
+    np.testing.assert_allclose(r["topk_w"].cpu().numpy(), o["topk_w"], rtol=2e-6, atol=0)
+    for nm in ("xn_moe", "xn_dense"):
+        got = bf16_np(r[nm])
+        ref = o[nm]
+        allow = cases.half_ulp_bf16(ref) * (1 + 1e-5) + 2e-6 * np.abs(ref)
+        assert np.all(np.abs(got - ref) <= allow), nm
+
+
+# ------------------------------------------------------------------ permutation
+
+@pytest.mark.parametrize("T,k,E", [(8, 4, 16), (37, 8, 128), (1, 8, 128), (2048, 8, 128),
+                                   (1025, 8, 128), (3000, 16, 256), (16384, 8, 128)])
+def test_permute_bit_exact(T, k, E):
+    rng = np.random.default_rng(T * 131 + k)
+    # skewed ids: some experts empty, some hot
+    p = rng.zipf(1.3, size=(T, k)) % E
+    idx = p.astype(np.int32)
+    cfg = mf.Config(512, E, k, 64, 64)
+    got = run_permute(cfg, to_dev(idx, torch.int32))
+    offs, src, inv = oracle.permute(idx, E)
+    n = T * k
+    assert np.array_equal(got["offsets"].cpu().numpy(), offs)
+    assert np.array_equal(got["sorted_src"].cpu().numpy()[:n], src)
+    assert np.array_equal(got["inv_pos"].cpu().numpy()[:n], inv)
+
+
+def test_permute_drops_invalid_ids():
+    idx = np.array([[3, -1], [16, 3], [0, 2]], dtype=np.int32)  # E = 16: -1 and 16 invalid
+    cfg = mf.Config(512, 16, 2, 64, 64)
+    got = run_permute(cfg, to_dev(idx, torch.int32))
+    flat = idx.reshape(-1)
+    valid = np.nonzero((flat >= 0) & (flat < 16))[0]
+    order = valid[np.argsort(flat[valid], kind="stable")]
+    offs = got["offsets"].cpu().numpy()
+    assert offs[-1] == len(valid)
+    assert np.array_equal(got["sorted_src"].cpu().numpy()[:len(valid)], order)
+
+
+# ------------------------------------------------------------------ branches
+
+@pytest.mark.parametrize("name", FAST + ["prefill_T2048_zipf", "limits"])
+def test_expert_branch(name):
+    """moe_ffn_forward: the routed experts before their post norm."""
+    c = _case(name)
+    cfg = config(c.shape)
+    layer = device_layer(c)
+    r = run_router(cfg, c, layer)
+    p = run_permute(cfg, r["topk_idx"])
+    moe = torch.empty(c.shape.T, cfg.hidden, dtype=torch.bfloat16, device="cuda")
+    ws = mf.workspace(cfg, c.shape.T)
+    mf.moe_ffn_forward(cfg, r["xn_moe"], r["topk_w"], p["offsets"], p["sorted_src"], p["inv_pos"],
+                       layer, moe, ws)
+    assert mf.moe_check_device_status(ws) == mf.MOE_OK
+    cases.check_bar(bf16_np(moe), oracle_block(c)["moe"], cases.FRAC_BF16, f"moe {name}")
+
+
+@pytest.mark.parametrize("name", FAST + ["prefill_T2048_zipf", "limits"])
+def test_dense_branch(name):
+    c = _case(name)
+    cfg = config(c.shape)
+    layer = device_layer(c)
+    r = run_router(cfg, c, layer)
+    out = torch.empty(c.shape.T, cfg.hidden, dtype=torch.bfloat16, device="cuda")
+    ws = mf.workspace(cfg, c.shape.T)
+    mf.dense_mlp_forward(cfg, r["xn_dense"], layer["w_dense_gate_up"], layer["w_dense_down"], out, ws)
+    assert mf.moe_check_device_status(ws) == mf.MOE_OK
+    cases.check_bar(bf16_np(out), oracle_block(c)["dense"], cases.FRAC_BF16, f"dense {name}")
+
+
+# ------------------------------------------------------------------ the block
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_block(name):
+    c = _case(name)
+    cfg = config(c.shape)
+    out, moe = run_block(cfg, c, device_layer(c))
+    o = oracle_block(c)
+    cases.check_bar(bf16_np(out), o["out"], cases.FRAC_BF16, f"out {name}")
+    cases.check_bar(bf16_np(moe), o["moe"], cases.FRAC_BF16, f"moe_out {name}")
+
+
+def test_block_without_branch_post_norms():
+    """g_post_moe / g_post_dense given as NULL skip those norms."""
+    c = _case("tiny_T37")
+    cfg = config(c.shape)
+    layer = device_layer(c)
+    layer.pop("g_post_moe")
+    layer.pop("g_post_dense")
+    out, _ = run_block(cfg, c, layer)
+    p = dict(c.p, g_post_moe=None, g_post_dense=None)
+    o = oracle.block_forward(c.x, p, cases.bf16_experts(c.p), c.shape.k, c.shape.eps, c.bias)
+    cases.check_bar(bf16_np(out), o["out"], cases.FRAC_BF16, "out without branch post norms")
+
+
+@pytest.mark.parametrize("name", ["decode_T8", "prefill_T2048_zipf"])
+def test_block_is_deterministic(name):
+    c = _case(name)
+    cfg = config(c.shape)
+    layer = device_layer(c)
+    a, ma = run_block(cfg, c, layer)
+    b, mb = run_block(cfg, c, layer)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(ma.view(torch.int16), mb.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["tiny_T37", "decode_T64"])
+def test_block_rows_are_independent(name):
+    """Shuffling the tokens shuffles the outputs the same way, bit for bit."""
+    c = _case(name)
+    cfg = config(c.shape)
+    layer = device_layer(c)
+    a, _ = run_block(cfg, c, layer)
+    perm = np.random.default_rng(5).permutation(c.shape.T)
+    c2 = cases.Case(c.shape, c.x[perm], c.p, c.bias, c.seed)
+    b, _ = run_block(cfg, c2, layer)
+    assert torch.equal(b.view(torch.int16), a[torch.from_numpy(perm).cuda()].view(torch.int16))
+
+
+def test_block_zero_tokens():
+    c = _case("tiny")
+    cfg = config(c.shape)
+    bw = mf.BlockWeights(cfg, device_layer(c))
+    x = torch.empty(0, cfg.hidden, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(0, cfg.hidden, dtype=torch.bfloat16, device="cuda")
+    ws = mf.workspace(cfg, 0)
+    mf.moe_block_forward(cfg, x, bw, out, ws)
+
+
+def test_zipf_case_has_empty_and_hot_experts():
+    c = _case("prefill_T2048_zipf")
+    idx = oracle_block(c)["topk_idx"]
+    cnt = np.bincount(idx.reshape(-1), minlength=c.shape.E)
+    assert (cnt == 0).sum() >= 1 and cnt.max() >= 8 * c.shape.T * c.shape.k / c.shape.E
+
+
+# ------------------------------------------------------------------ int8 quantiser
+
+def test_quantize_int8_bit_exact():
+    w = synth.normal_bf16(77, (1,), (300, 2816), 0.02)
+    w[5] = 0                                              # all-zero row
+    row = np.zeros(2816, dtype=np.float32)
+    row[:5] = [127 / 128, 2.5 / 128, 3.5 / 128, -2.5 / 128, -0.5 / 128]   # halves to even
+    w[7] = synth.f32_to_bf16_bits(row)
+    q = torch.empty(w.shape, dtype=torch.int8, device="cuda")
+    s = torch.empty(w.shape[0], dtype=torch.float32, device="cuda")
+    mf.moe_quantize_int8(to_dev(w), q, s)
+    qo, so = oracle.quantize_int8_per_channel(w)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
