@@ -133,7 +133,7 @@ def run_ours(args, wl, rank, world, device):
     seed = 1234 + 7919 * rank
     alpha = None
     layers = []
-    for l in range(wl["layers"]):
+    for l in range(args.layers or wl["layers"]):
         t = synth.torch_layer(shape, seed, l, device)
         if wl["zipf"]:
             with open(ZIPF_ALPHA_FILE) as f:
@@ -169,6 +169,9 @@ def run_ours(args, wl, rank, world, device):
         torch.distributed.barrier()
     stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(mf.MOE_BLOCK_EVENTS)]
                 for _ in range(K)]
+    for evs in stage_ev:  # create the CUDA events before the timed region
+        for e in evs:
+            e.record(stream)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     clocks = Clocks(device)
@@ -375,6 +378,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None, help="layer copies to rotate over")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":

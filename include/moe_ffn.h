@@ -34,7 +34,8 @@
  *     stream reaches that point.  Calls on different streams must not share `ws`.
  *   - Size limits: H a multiple of 128 (128..6144), I and D multiples of 64
  *     (64..16384), 1 <= E <= 256, 1 <= k <= min(E, 16), 0 <= T, T*k < 2^31.
- *     T = 0 returns MOE_OK and launches nothing.
+ *     T = 0 returns MOE_OK at once (before any pointer is checked) and launches
+ *     nothing.
  *   - Argument errors are found on the host before anything is launched and
  *     return MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED or MOE_ERR_WORKSPACE.  A failed
  *     launch returns MOE_ERR_CUDA.  Nothing throws across this interface.
@@ -167,8 +168,9 @@ moe_status_t dense_mlp_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
  *   it receives the MoE branch output before its post norm.
  *   stage_events: NULL, or a host array of MOE_BLOCK_EVENTS cudaEvent_t that the call
  *   records on `stream` at its stage boundaries, for timing each stage:
- *     [0] start  [1] router done  [2] permutation done  [3] row gather done
- *     [4] counters cleared  [5] gate_up GEMMs done  [6] down GEMMs done  [7] combine done */
+ *     [0] start  [1] router done (with the permutation for small batches)
+ *     [2] permutation done  [3] row gather done  [4] GEMMs start
+ *     [5] gate_up GEMMs done  [6] down GEMMs done  [7] combine done */
 #define MOE_BLOCK_EVENTS 8
 moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
                                const moe_block_weights_t* w, moe_bf16_t* out,

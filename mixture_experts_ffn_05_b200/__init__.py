@@ -244,6 +244,9 @@ def moe_block_forward(cfg, x, weights: BlockWeights, out, ws, moe_out=None, stre
     if stage_events is not None:
         if len(stage_events) != MOE_BLOCK_EVENTS:
             raise ValueError(f"stage_events needs {MOE_BLOCK_EVENTS} events")
+        for e in stage_events:
+            if e.cuda_event == 0:  # torch creates the CUDA event on its first record
+                e.record(torch.cuda.current_stream() if stream is None else stream)
         ev = (_P * MOE_BLOCK_EVENTS)(*[e.cuda_event for e in stage_events])
     st = lib().moe_block_forward(ctypes.byref(cfg.c()), T, _ptr(x, BF16, "x"),
                                  ctypes.byref(weights.c), _ptr(out, BF16, "out"),

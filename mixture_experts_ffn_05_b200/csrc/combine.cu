@@ -5,16 +5,15 @@
 // layernorms" add a post norm on each branch:
 //   m   = sum_{j=0..k-1} Y[t*k + j]          (weights already applied, fixed slot order)
 //   out = x + N_post_ff( N_post_dense(d) + N_post_moe(m) ),  N_g(v) = v / rms(v) * g
-// All sums in fp32; the output is rounded to bf16 once.  One CTA of 128 threads per
-// token; each thread owns chunks of 8 columns.
+// All sums in fp32; the output is rounded to bf16 once.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
-constexpr int kCombThreads = 128;
-constexpr int kCombMaxChunks = 6;  // H <= 6144: 768 chunks of 8 over 128 threads
+constexpr int kCombMaxThreads = 768;  // H <= 6144: one 8-column chunk per thread
 
+// Block reduction in a fixed order (deterministic).  nthreads is a multiple of 32.
 __device__ __forceinline__ float block_sum(float v, float* red) {
   v = warp_sum(v);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -22,82 +21,81 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   if (lane == 0) red[warp] = v;
   __syncthreads();
   float s = 0.f;
-#pragma unroll
-  for (int w = 0; w < kCombThreads / 32; ++w) s += red[w];  // fixed order
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) s += red[w];
   return s;
 }
 
-__global__ void __launch_bounds__(kCombThreads) combine_block_kernel(
+// One CTA per token, one 8-column chunk per thread.
+__global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
     int H, int k, float eps, const uint16_t* __restrict__ x, const uint16_t* __restrict__ y,
     const uint16_t* __restrict__ dense, const uint16_t* __restrict__ g_pm,
     const uint16_t* __restrict__ g_pd, const uint16_t* __restrict__ g_ff,
     uint16_t* __restrict__ out, uint16_t* __restrict__ moe_out) {
-  __shared__ float red[kCombThreads / 32];
+  __shared__ float red[kCombMaxThreads / 32];
   const int t = blockIdx.x;
-  const int nch = H >> 3;
-  float m[kCombMaxChunks][8], d[kCombMaxChunks][8];
+  const int c = threadIdx.x;
+  const bool on = c < (H >> 3);
+  float m[8], d[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = d[i] = 0.f;
+  if (on) {
+    const uint4* yr = reinterpret_cast<const uint4*>(y + static_cast<size_t>(t) * k * H) + c;
+    uint4 buf[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k) buf[j] = __ldg(yr + static_cast<size_t>(j) * (H >> 3));
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k) {  // slot order j = 0..k-1
+        float f[8];
+        unpack8(buf[j], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] += f[i];
+      }
+    unpack8(__ldg(reinterpret_cast<const uint4*>(dense + static_cast<size_t>(t) * H) + c), d);
+    if (moe_out) reinterpret_cast<uint4*>(moe_out + static_cast<size_t>(t) * H)[c] = pack8(m);
+  }
   float ssm = 0.f, ssd = 0.f;
 #pragma unroll
-  for (int u = 0; u < kCombMaxChunks; ++u) {
-    const int c = threadIdx.x + u * kCombThreads;
-    if (c < nch) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m[u][i] = 0.f;
-      for (int j = 0; j < k; ++j) {
-        float f[8];
-        unpack8(__ldg(reinterpret_cast<const uint4*>(y + (static_cast<size_t>(t) * k + j) * H) + c), f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m[u][i] += f[i];
-      }
-      unpack8(__ldg(reinterpret_cast<const uint4*>(dense + static_cast<size_t>(t) * H) + c), d[u]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        ssm = fmaf(m[u][i], m[u][i], ssm);
-        ssd = fmaf(d[u][i], d[u][i], ssd);
-      }
-      if (moe_out) reinterpret_cast<uint4*>(moe_out + static_cast<size_t>(t) * H)[c] = pack8(m[u]);
-    }
+  for (int i = 0; i < 8; ++i) {
+    ssm = fmaf(m[i], m[i], ssm);
+    ssd = fmaf(d[i], d[i], ssd);
   }
   const float rm = g_pm ? 1.0f / sqrtf(block_sum(ssm, red) / H + eps) : 1.f;
   const float rd = g_pd ? 1.0f / sqrtf(block_sum(ssd, red) / H + eps) : 1.f;
+  float sum[8];
   float ssc = 0.f;
+  {
+    float ga[8], gb[8];
 #pragma unroll
-  for (int u = 0; u < kCombMaxChunks; ++u) {
-    const int c = threadIdx.x + u * kCombThreads;
-    if (c < nch) {
-      float ga[8], gb[8];
-      if (g_pd) unpack8(__ldg(reinterpret_cast<const uint4*>(g_pd) + c), ga);
-      if (g_pm) unpack8(__ldg(reinterpret_cast<const uint4*>(g_pm) + c), gb);
+    for (int i = 0; i < 8; ++i) ga[i] = gb[i] = 1.f;
+    if (on && g_pd) unpack8(__ldg(reinterpret_cast<const uint4*>(g_pd) + c), ga);
+    if (on && g_pm) unpack8(__ldg(reinterpret_cast<const uint4*>(g_pm) + c), gb);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float a = g_pd ? d[u][i] * rd * ga[i] : d[u][i];
-        const float b = g_pm ? m[u][i] * rm * gb[i] : m[u][i];
-        m[u][i] = a + b;  // reuse m for the sum
-        ssc = fmaf(m[u][i], m[u][i], ssc);
-      }
+    for (int i = 0; i < 8; ++i) {
+      const float a = g_pd ? d[i] * rd * ga[i] : d[i];
+      const float b = g_pm ? m[i] * rm * gb[i] : m[i];
+      sum[i] = a + b;
+      ssc = fmaf(sum[i], sum[i], ssc);
     }
   }
   const float rc = 1.0f / sqrtf(block_sum(ssc, red) / H + eps);
+  if (on) {
+    float xf[8], g[8], o[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + c), xf);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(g_ff) + c), g);
 #pragma unroll
-  for (int u = 0; u < kCombMaxChunks; ++u) {
-    const int c = threadIdx.x + u * kCombThreads;
-    if (c < nch) {
-      float xf[8], g[8], o[8];
-      unpack8(__ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + c), xf);
-      unpack8(__ldg(reinterpret_cast<const uint4*>(g_ff) + c), g);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = xf[i] + m[u][i] * rc * g[i];
-      reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = pack8(o);
-    }
+    for (int i = 0; i < 8; ++i) o[i] = xf[i] + sum[i] * rc * g[i];
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = pack8(o);
   }
 }
 
 // moe_out[t] = sum_j Y[t*k + j] in fp32, slot order, rounded to bf16.
-__global__ void __launch_bounds__(kCombThreads) combine_moe_kernel(int H, int k,
-                                                                   const uint16_t* __restrict__ y,
-                                                                   uint16_t* __restrict__ moe_out) {
+__global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
+                                                          const uint16_t* __restrict__ y,
+                                                          uint16_t* __restrict__ moe_out) {
   const int t = blockIdx.x;
-  for (int c = threadIdx.x; c < (H >> 3); c += kCombThreads) {
+  for (int c = threadIdx.x; c < (H >> 3); c += 256) {
     float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < k; ++j) {
       float f[8];
@@ -114,14 +112,15 @@ cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t*
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s) {
-  combine_block_kernel<<<T, kCombThreads, 0, s>>>(H, k, eps, x, y, dense, g_post_moe,
-                                                  g_post_dense, g_post_ff, out, moe_out);
+  const int threads = ((H >> 3) + 31) / 32 * 32;
+  combine_block_kernel<<<T, threads, 0, s>>>(H, k, eps, x, y, dense, g_post_moe, g_post_dense,
+                                             g_post_ff, out, moe_out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, uint16_t* moe_out,
                                cudaStream_t s) {
-  combine_moe_kernel<<<T, kCombThreads, 0, s>>>(H, k, y, moe_out);
+  combine_moe_kernel<<<T, 256, 0, s>>>(H, k, y, moe_out);
   return cudaGetLastError();
 }
 

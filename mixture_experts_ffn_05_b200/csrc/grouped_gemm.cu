@@ -19,17 +19,18 @@
 // stores its fp32 partial tile; the last piece to arrive (an atomic counter) sums all
 // partials in piece order, so the result does not depend on arrival order.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads into a ring of shared-memory
-// stages, warp 1 issues tcgen05.mma into one of two TMEM accumulators, warps 2-5 read
-// the accumulator back (tcgen05.ld) and run the epilogue while the next tile is being
-// multiplied.  Every wait is bounded; a wait that runs out records a timeout in the
+// Warp roles (320 threads): warp 0 issues TMA loads into a ring of shared-memory
+// stages, warp 1 issues tcgen05.mma into one of 2-4 TMEM accumulators, and two groups of
+// four warps (2-5 and 6-9) take alternate pieces, read the accumulator back (tcgen05.ld)
+// and run the epilogue while later pieces are being multiplied.  Every wait is bounded; a wait that runs out records a timeout in the
 // status word and the CTA winds down.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;  // producer warp, MMA warp, 2 x 4 epilogue warps
+constexpr int kMaxSplit = 4;       // K pieces per tile at most
 constexpr int kMaxEntries = 258;  // groups of problem 0 (<= 256) + problem 1 (1) + 1
 
 template <int BN>
@@ -38,16 +39,19 @@ struct Cfg {
   static constexpr int kBBytes = BN * 64 * 2;   // BN token rows x 64 K
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kStages = BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4));
-  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+  // TMEM accumulators: 4 for narrow tiles (the epilogue of a weight-streaming piece is
+  // latency-bound and must not hold up the MMAs), 2 for wide ones (512 columns max).
+  static constexpr int kAcc = BN <= 64 ? 4 : 2;
+  static constexpr int kTmemCols = kAcc * BN < 32 ? 32 : kAcc * BN;
   // after the stages: barriers, bookkeeping, the gate/up exchange buffer
   static constexpr int kBarOff = kStages * kStage;
-  static constexpr int kNumBars = 2 * kStages + 5;  // full, empty, acc_full x2, acc_empty x2, drain
+  static constexpr int kNumBars = 2 * kStages + 2 * kAcc + 1;  // full, empty, acc_full, acc_empty, drain
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kMiscInts = 8;               // tmem slot, abort, bcast, ...
   static constexpr int kPreOff = kMiscOff + kMiscInts * 4;
   static constexpr int kTabInts = 4 * kMaxEntries;  // pre, cnt, b0, ng
   static constexpr int kXchgOff = ((kPreOff + kTabInts * 4) + 15) & ~15;
-  static constexpr int kXchgBytes = 16 * 64 * 4;
+  static constexpr int kXchgBytes = 2 * 16 * 64 * 4;  // one per epilogue group
   static constexpr int kSmem = kXchgOff + kXchgBytes + 1024;  // + alignment slack
   static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment");
 };
@@ -101,8 +105,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* empty = full + C::kStages;
   uint64_t* acc_full = empty + C::kStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + C::kAcc;
+  uint64_t* drain = acc_empty + C::kAcc;
   int* misc = reinterpret_cast<int*>(smem + C::kMiscOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 0);
   volatile int* abort_flag = misc + 1;
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::kAcc; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 128);
     }
@@ -270,8 +274,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         umma_commit(&acc_full[ab]);
-        ab ^= 1;
-        if (ab == 0) aph ^= 1u;
+        if (++ab == C::kAcc) {
+          ab = 0;
+          aph ^= 1u;
+        }
       }
       if (!ok) {
         record_status(P.status, kStatusTimeout);
@@ -283,18 +289,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // ================= epilogue (warps 2..5, TMEM lanes by warp % 4) =================
+    // ================= epilogue: two groups of 4 warps take alternate pieces ============
+    // Warp w reads TMEM lanes 32*(w%4)..+31; each group covers all 128 lanes.  Two groups
+    // keep the latency-bound part of an epilogue (partials, counters) off the MMA's path.
+    const int grp = (warp - 2) >> 2;
     const int q = warp & 3;
     const int row = q * 32 + lane;  // accumulator row = TMEM lane
-    const int et = threadIdx.x - 64;
-    int ab = 0;
-    uint32_t aph = 0;
-    for (int piece = blockIdx.x; piece < total; piece += gridDim.x) {
+    const int et = threadIdx.x - 64 - 128 * grp;
+    const uint32_t bar = 1 + grp;
+    volatile int* gb = bcast + grp;
+    float* xg = xchg + grp * 16 * 64;
+    int local = 0;
+    for (int piece = blockIdx.x; piece < total; piece += gridDim.x, ++local) {
+      if ((local & 1) != grp) continue;
+      const int ab = local % C::kAcc;
+      const uint32_t aph = static_cast<uint32_t>(local / C::kAcc) & 1u;
       const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
       const GemmProblem& pr = P.prob[pc.p];
-      if (et == 0) *bcast = mbar_wait(&acc_full[ab], aph, tmo, abort_flag) ? 1 : 0;
-      named_sync(1, 128);
-      if (!*bcast) {
+      if (et == 0) *gb = mbar_wait(&acc_full[ab], aph, tmo, abort_flag) ? 1 : 0;
+      named_sync(bar, 128);
+      if (!*gb) {
         if (et == 0) {
           record_status(P.status, kStatusTimeout);
           *abort_flag = 1;
@@ -314,17 +328,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) __stcg(part + (c0 + i) * 128 + row, v[i]);
         }
-        __threadfence();
-        named_sync(1, 128);
+        // Publish with one release: the barrier orders every thread's partial before the
+        // elected thread's atomic, whose acq_rel also acquires the other pieces' partials.
+        named_sync(bar, 128);
         if (et == 0) {
-          const unsigned old = atomicAdd(P.counters + pc.first_piece, 1u);
+          const unsigned old = atom_add_acq_rel_gpu(P.counters + pc.first_piece, 1u);
           const int l = (old == static_cast<unsigned>(pr.split - 1)) ? 1 : 0;
           if (l) P.counters[pc.first_piece] = 0u;  // ready for the next launch
-          *bcast = l;
+          *gb = l;
         }
-        named_sync(1, 128);
-        last = *bcast != 0;
-        if (last) __threadfence();
+        named_sync(bar, 128);
+        last = *gb != 0;
       }
       if (last) {
         const int out_col0 = pc.m * (pr.kind == 0 ? 64 : 128);
@@ -338,17 +352,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           float v[16];
           tmem_ld16(tbase + c0, v);
           if (pr.split > 1) {
+            // every other piece's partial is loaded first, then all are summed in piece
+            // order (the same order whichever piece arrives last)
+            float pv[kMaxSplit][16];
+#pragma unroll
+            for (int s2 = 0; s2 < kMaxSplit; ++s2) {
+              if (s2 < pr.split && s2 != pc.s) {
+                const float* qp = P.partials + static_cast<size_t>(pc.first_piece + s2) * BN * 128;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pv[s2][i] = __ldcg(qp + (c0 + i) * 128 + row);
+              }
+            }
             float acc[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-            for (int s2 = 0; s2 < pr.split; ++s2) {
-              if (s2 == pc.s) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] += v[i];
-              } else {
-                const float* qp = P.partials + static_cast<size_t>(pc.first_piece + s2) * BN * 128;
+            for (int s2 = 0; s2 < kMaxSplit; ++s2) {
+              if (s2 < pr.split) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] += __ldcg(qp + (c0 + i) * 128 + row);
+                for (int i = 0; i < 16; ++i) acc[i] += (s2 == pc.s) ? v[i] : pv[s2][i];
               }
             }
 #pragma unroll
@@ -357,21 +379,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (pr.kind == 0) {
             if (row >= 64) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) xchg[i * 64 + (row - 64)] = v[i] * sc;
+              for (int i = 0; i < 16; ++i) xg[i * 64 + (row - 64)] = v[i] * sc;
             }
-            named_sync(1, 128);
+            named_sync(bar, 128);
             if (row < 64) {
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const int col = c0 + i;
                 if (col < pc.n_valid) {
-                  const float h = gelu_tanh(v[i] * sc) * xchg[i * 64 + row];
+                  const float h = gelu_tanh(v[i] * sc) * xg[i * 64 + row];
                   const size_t orow = static_cast<size_t>(pc.b_row0 + pc.n * BN + col);
                   pr.out[orow * pr.out_ld + out_col0 + row] = bf16_bits(h);
                 }
               }
             }
-            named_sync(1, 128);
+            named_sync(bar, 128);
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -390,10 +412,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       tc_fence_before();
-      named_sync(1, 128);  // every flag of this piece is read before the next is written
+      named_sync(bar, 128);  // every flag of this piece is read before the next is written
       mbar_arrive(&acc_empty[ab]);
-      ab ^= 1;
-      if (ab == 0) aph ^= 1u;
     }
   }
 

@@ -48,15 +48,17 @@ struct GemmMaps {
 };
 
 // kernels/*.cu launchers.  All return cudaSuccess or the launch error.
-cudaError_t launch_router_logits(int T, int H, int E, float eps, float inv_sqrt_h,
-                                 const uint16_t* x, const uint16_t* router_scale,
-                                 const uint16_t* w_router, const float* bias,
-                                 const uint16_t* g_pre_moe, const uint16_t* g_pre_dense,
-                                 uint16_t* xn_moe, uint16_t* xn_dense, float* logits,
-                                 cudaStream_t s);
-cudaError_t launch_router_topk(int T, int E, int k, const float* logits,
-                               const uint16_t* per_expert_scale, int* topk_idx, float* topk_w,
-                               cudaStream_t s);
+// Router + pre norms + top-k in one launch; when offsets != NULL (and T*k fits the
+// single-block sort, see permute_blocks) also the token-to-expert counting sort.
+// counters: router_counters(T) words, zero on entry (left zero on exit).
+cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t* x,
+                          const uint16_t* router_scale, const uint16_t* w_router,
+                          const float* bias, const uint16_t* per_expert_scale,
+                          const uint16_t* g_pre_moe, const uint16_t* g_pre_dense,
+                          uint16_t* xn_moe, uint16_t* xn_dense, float* logits, int* topk_idx,
+                          float* topk_w, unsigned* counters, int* offsets, int* sorted_src,
+                          int* inv_pos, cudaStream_t s);
+int router_counters(int T);
 cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int* sorted_src,
                            int* inv_pos, int* block_hist, int* block_base, cudaStream_t s);
 int permute_blocks(int n);  // blocks of the multi-block path (0 = single-block path)

@@ -67,11 +67,11 @@ int choose_bn(const Dims& d) {
 // so that the tile list is fine enough to keep every SM streaming to the end.
 int choose_split(int k_steps, int bn) {
   if (bn != 16) return 1;
-  return std::max(1, std::min(k_steps, (k_steps + 10) / 11));
+  return std::max(1, std::min(std::min(k_steps, 4), (k_steps + 10) / 11));
 }
 
 struct Layout {
-  size_t status, counters, logits, bhist, bbase, topk_idx, topk_w, offsets, sorted, inv;
+  size_t status, rcounters, counters, logits, bhist, bbase, topk_idx, topk_w, offsets, sorted, inv;
   size_t xn_moe, xn_dense, aperm, h, y, hd, dense, partials, total;
   size_t counters_bytes;
   int bn, split_gu, split_dgu, split_d, split_dd;
@@ -102,9 +102,12 @@ Layout layout_of(const Dims& d) {
     off = align_up(off + std::max<size_t>(bytes, 1), kAlign);
     return at;
   };
-  L.status = take(256);
+  // status word, router counters and GEMM counters are contiguous: one memset clears them
+  L.status = 0;
+  L.rcounters = 256;
+  L.counters = align_up(L.rcounters + static_cast<size_t>(router_counters(d.T)) * 4, 256);
   L.counters_bytes = static_cast<size_t>(pieces) * 4;
-  L.counters = take(L.counters_bytes);
+  off = align_up(L.counters + L.counters_bytes, kAlign);
   L.logits = take(static_cast<size_t>(T) * d.E * 4);
   L.bhist = take(static_cast<size_t>(nb) * d.E * 4);
   L.bbase = take(static_cast<size_t>(nb) * d.E * 4);
@@ -214,14 +217,18 @@ bool mark(void* const* ev, int i, cudaStream_t s) {
   return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
 }
 
+// Clears the status word and every counter of the workspace.
+moe_status_t clear_counters(const Layout& L, void* ws, cudaStream_t s) {
+  return cudaMemsetAsync(ws, 0, L.counters + L.counters_bytes, s) == cudaSuccess ? MOE_OK
+                                                                                 : MOE_ERR_CUDA;
+}
+
 moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& j,
-                       cudaStream_t s, void* const* ev = nullptr) {
+                       cudaStream_t s, bool clear, void* const* ev = nullptr) {
   const int64_t Tk = static_cast<int64_t>(d.T) * d.k;
   const int grid = sm_count();
   if (grid <= 0) return MOE_ERR_CUDA;
-  if (cudaMemsetAsync(at<uint8_t>(ws, L.status), 0, L.counters - L.status + L.counters_bytes, s) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (clear && clear_counters(L, ws, s) != MOE_OK) return MOE_ERR_CUDA;
   if (!mark(ev, 4, s)) return MOE_ERR_CUDA;
   uint16_t* h = at<uint16_t>(ws, L.h);
   uint16_t* hd = at<uint16_t>(ws, L.hd);
@@ -328,6 +335,7 @@ moe_status_t moe_router(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
   Dims d;
   moe_status_t st = check_cfg(cfg, T, &d);
   if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
   for (const void* p : {(const void*)x, (const void*)router_scale, (const void*)w_router,
                         (const void*)per_expert_scale, (const void*)g_pre_moe,
                         (const void*)g_pre_dense, (const void*)topk_idx, (const void*)topk_w,
@@ -336,14 +344,12 @@ moe_status_t moe_router(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
   if (logit_bias != nullptr && !aligned16(logit_bias)) return MOE_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* logits = at<float>(ws, L.logits);
-  st = cuda_status(launch_router_logits(d.T, d.H, d.E, d.eps, 1.0f / sqrtf(static_cast<float>(d.H)),
-                                        x, router_scale, w_router, logit_bias, g_pre_moe,
-                                        g_pre_dense, xn_moe, xn_dense, logits, s));
-  if (st != MOE_OK) return st;
-  return cuda_status(launch_router_topk(d.T, d.E, d.k, logits, per_expert_scale, topk_idx, topk_w, s));
+  if ((st = clear_counters(L, ws, s)) != MOE_OK) return st;
+  return cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, x, router_scale, w_router,
+                                   logit_bias, per_expert_scale, g_pre_moe, g_pre_dense, xn_moe,
+                                   xn_dense, at<float>(ws, L.logits), topk_idx, topk_w,
+                                   at<unsigned>(ws, L.rcounters), nullptr, nullptr, nullptr, s));
 }
 
 moe_status_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx,
@@ -352,12 +358,12 @@ moe_status_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk
   Dims d;
   moe_status_t st = check_cfg(cfg, T, &d);
   if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
   for (const void* p : {(const void*)topk_idx, (const void*)expert_offsets,
                         (const void*)sorted_src, (const void*)inv_pos})
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
   return cuda_status(launch_permute(d.T * d.k, d.E, topk_idx, expert_offsets, sorted_src, inv_pos,
                                     at<int>(ws, L.bhist), at<int>(ws, L.bbase),
                                     static_cast<cudaStream_t>(stream)));
@@ -371,6 +377,7 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   Dims d;
   moe_status_t st = check_cfg(cfg, T, &d);
   if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
   for (const void* p : {(const void*)xn_moe, (const void*)topk_w, (const void*)expert_offsets,
                         (const void*)sorted_src, (const void*)inv_pos, (const void*)moe_out})
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
@@ -378,7 +385,6 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   if (d.int8) return MOE_ERR_UNSUPPORTED;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int Tk = d.T * d.k;
   uint16_t* aperm = at<uint16_t>(ws, L.aperm);
@@ -396,7 +402,7 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   j.sorted_src = sorted_src;
   j.topk_w = topk_w;
   j.y = y;
-  if ((st = run_gemms(d, L, ws, j, s)) != MOE_OK) return st;
+  if ((st = run_gemms(d, L, ws, j, s, true)) != MOE_OK) return st;
   return cuda_status(launch_combine_moe(d.T, d.H, d.k, y, moe_out, s));
 }
 
@@ -406,19 +412,19 @@ moe_status_t dense_mlp_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   Dims d;
   moe_status_t st = check_cfg(cfg, T, &d);
   if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
   for (const void* p : {(const void*)xn_dense, (const void*)w_gate_up, (const void*)w_down,
                         (const void*)dense_out})
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
   GemmJob j{};
   j.dense = true;
   j.xn_dense = xn_dense;
   j.w_dgu = w_gate_up;
   j.w_dd = w_down;
   j.dense_out = dense_out;
-  return run_gemms(d, L, ws, j, static_cast<cudaStream_t>(stream));
+  return run_gemms(d, L, ws, j, static_cast<cudaStream_t>(stream), true);
 }
 
 moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
@@ -428,6 +434,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   Dims d;
   moe_status_t st = check_cfg(cfg, T, &d);
   if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
   if (w == nullptr) return MOE_ERR_INVALID_ARG;
   for (const void* p : {(const void*)x, (const void*)out, (const void*)w->router_scale,
                         (const void*)w->w_router, (const void*)w->per_expert_scale,
@@ -442,7 +449,6 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   if (d.int8) return MOE_ERR_UNSUPPORTED;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int Tk = d.T * d.k;
   int* topk_idx = at<int>(ws, L.topk_idx);
@@ -461,16 +467,17 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
     for (int i = 0; i < MOE_BLOCK_EVENTS; ++i)
       if (ev[i] == nullptr) return MOE_ERR_INVALID_ARG;
   if (!mark(ev, 0, s)) return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_router_logits(
-           d.T, d.H, d.E, d.eps, 1.0f / sqrtf(static_cast<float>(d.H)), x, w->router_scale,
-           w->w_router, w->logit_bias, w->g_pre_moe, w->g_pre_dense, xn_moe, xn_dense, logits,
-           s))) != MOE_OK)
-    return st;
-  if ((st = cuda_status(launch_router_topk(d.T, d.E, d.k, logits, w->per_expert_scale, topk_idx,
-                                           topk_w, s))) != MOE_OK)
+  if ((st = clear_counters(L, ws, s)) != MOE_OK) return st;
+  const bool fused_sort = permute_blocks(Tk) == 0;
+  if ((st = cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, x, w->router_scale, w->w_router,
+                                      w->logit_bias, w->per_expert_scale, w->g_pre_moe,
+                                      w->g_pre_dense, xn_moe, xn_dense, logits, topk_idx, topk_w,
+                                      at<unsigned>(ws, L.rcounters), fused_sort ? offsets : nullptr,
+                                      sorted, inv, s))) != MOE_OK)
     return st;
   if (!mark(ev, 1, s)) return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_permute(Tk, d.E, topk_idx, offsets, sorted, inv, at<int>(ws, L.bhist),
+  if (!fused_sort &&
+      (st = cuda_status(launch_permute(Tk, d.E, topk_idx, offsets, sorted, inv, at<int>(ws, L.bhist),
                                        at<int>(ws, L.bbase), s))) != MOE_OK)
     return st;
   if (!mark(ev, 2, s)) return MOE_ERR_CUDA;
@@ -493,7 +500,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   j.w_dgu = w->w_dense_gate_up;
   j.w_dd = w->w_dense_down;
   j.dense_out = dense;
-  if ((st = run_gemms(d, L, ws, j, s, ev)) != MOE_OK) return st;
+  if ((st = run_gemms(d, L, ws, j, s, false, ev)) != MOE_OK) return st;
   if ((st = cuda_status(launch_combine_block(d.T, d.H, d.k, d.eps, x, y, dense, w->g_post_moe,
                                              w->g_post_dense, w->g_post_ff, out, moe_out, s))) !=
       MOE_OK)

@@ -135,18 +135,20 @@ def zipf_bias(seed: int, E: int, alpha: float, s: float = 1.1) -> np.ndarray:
 
 
 def make_router(seed: int, shape: Shape, layer: int = 0, std: float = 0.02,
-                gains=(0.5, 1.5)) -> dict:
-    """The router's tensors of one layer (the same draws make_layer returns)."""
+                gains=(0.5, 1.5), router_std=None) -> dict:
+    """The router's tensors of one layer (the same draws make_layer returns).
+    router_std (default: std) sets the spread of the router weights alone."""
     lo, hi = gains
     return {
-        "w_router": normal_bf16(seed, (W_ROUTER, layer), (shape.E, shape.H), std),
+        "w_router": normal_bf16(seed, (W_ROUTER, layer), (shape.E, shape.H),
+                                std if router_std is None else router_std),
         "router_scale": uniform_bf16(seed, (ROUTER_SCALE, layer), (shape.H,), lo, hi),
         "per_expert_scale": uniform_bf16(seed, (PER_EXPERT_SCALE, layer), (shape.E,), lo, hi),
     }
 
 
 def make_layer(seed: int, shape: Shape, layer: int = 0, std: float = 0.02,
-               gains=(0.5, 1.5)) -> dict:
+               gains=(0.5, 1.5), router_std=None) -> dict:
     """All weights of one layer as bf16 bit patterns (numpy uint16).
 
     Layout (row-major, K contiguous):
@@ -162,7 +164,7 @@ def make_layer(seed: int, shape: Shape, layer: int = 0, std: float = 0.02,
     lo, hi = gains
     L = layer
     return {
-        **make_router(seed, shape, layer, std, gains),
+        **make_router(seed, shape, layer, std, gains, router_std),
         "w_gate_up": normal_bf16(seed, (W_GATE_UP, L), (E, 2 * I, H), std),
         "w_down": normal_bf16(seed, (W_DOWN, L), (E, H, I), std),
         "w_dense_gate_up": normal_bf16(seed, (W_DENSE_GATE_UP, L), (2 * D, H), std),

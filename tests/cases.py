@@ -107,13 +107,13 @@ _CASE_CACHE = _Lru(16)
 
 
 def make_case(shape: synth.Shape, seed: int = 1234, zipf: bool = False, layer: int = 0,
-              gap: bool = True) -> Case:
-    ckey = (shape, seed, zipf, layer, gap)
+              gap: bool = True, router_std=None) -> Case:
+    ckey = (shape, seed, zipf, layer, gap, router_std)
     if ckey in _CASE_CACHE:
         return _CASE_CACHE[ckey]
-    key = (shape.H, shape.E, shape.I, shape.D, seed, layer)
+    key = (shape.H, shape.E, shape.I, shape.D, seed, layer, router_std)
     p = _LAYER_CACHE[key] if key in _LAYER_CACHE else _LAYER_CACHE.put(
-        key, synth.make_layer(seed, shape, layer))
+        key, synth.make_layer(seed, shape, layer, router_std=router_std))
     bias = synth.zipf_bias(seed, shape.E, zipf_alpha()) if zipf else None
     if gap:
         x = gap_filtered_x(seed + 1, shape, p, bias, layer=layer)
