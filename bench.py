@@ -58,6 +58,48 @@ def peaks():
                 "source": "fallback"}
 
 
+# ---------------------------------------------------------------------------- ncu traffic
+
+PROFILES = os.path.join(ROOT, "profiles")
+GEMM_SOURCES = [os.path.join(ROOT, "mixture_experts_ffn_05_b200", "csrc", f)
+                for f in ("grouped_gemm.cu", "common.cuh")]
+
+
+def kernel_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(summary: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the kernel's
+    source has changed since the counters were taken."""
+    try:
+        vals = {}
+        with open(os.path.join(PROFILES, summary)) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.strip().split(":", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("source_sha256") != kernel_sha():
+            return None
+        return int(vals["traffic_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def max_over_ranks(t_ms: float, world: int, device) -> float:
+    """The slowest rank's time (every rank takes part)."""
+    if world <= 1:
+        return t_ms
+    tt = torch.tensor([t_ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+    return float(tt.item())
+
+
 # ---------------------------------------------------------------------------- clocks
 
 class Clocks:
@@ -193,11 +235,7 @@ def run_ours(args, wl, rank, world, device):
     for ev in stage_ev:
         for j, n in enumerate(stages):
             stages[n].append(ev[j].elapsed_time(ev[j + 1]))
-    t_max = t_ms
-    if world > 1:
-        tt = torch.tensor([t_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        t_max = float(tt.item())
+    t_max = max_over_ranks(t_ms, world, device)
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     x_host = torch.empty(W + K, T, shape.H, dtype=torch.bfloat16, pin_memory=True)
@@ -223,11 +261,7 @@ def run_ours(args, wl, rank, world, device):
         e2e_step(W + i, i)
     f1.record(stream)
     torch.cuda.synchronize(device)
-    te = f0.elapsed_time(f1)
-    if world > 1:
-        tt = torch.tensor([te], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        te = float(tt.item())
+    te = max_over_ranks(f0.elapsed_time(f1), world, device)
     if mf.moe_check_device_status(ws) != mf.MOE_OK:
         raise RuntimeError("device status after the end-to-end region")
 
@@ -249,7 +283,8 @@ def run_ours(args, wl, rank, world, device):
                 "peak_source": f"bf16_tflops of {pk['source']} peaks"}
     else:
         roof = {"bound": "hbm", "achieved": round(gu_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(gu_gbs / pk["hbm_gbs"], 4), "traffic": None,
+                "frac": round(gu_gbs / pk["hbm_gbs"], 4),
+                "traffic": ncu_traffic("grouped_gemm_gate_up_decode_T8.md") if T == 8 else None,
                 "kernel": "grouped_gemm_kernel (gate_up launch)",
                 "peak_source": f"hbm_gbs of {pk['source']} peaks"}
     t_hbm = blk_bytes / (pk["hbm_gbs"] * 1e9)
