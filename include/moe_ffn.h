@@ -142,6 +142,29 @@ moe_status_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk
                          int32_t* expert_offsets, int32_t* sorted_src, int32_t* inv_pos,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* The token-to-expert permutation of moe_permute for callers that cannot hand the
+ * library any scratch memory: plugin hosts that pass only input and output buffers and
+ * offer no allocator, processes whose device memory is already reserved by another
+ * framework's caching allocator, and latency-critical loops that must not call
+ * cudaMalloc (which can synchronise the device).  The model pages have no counterpart;
+ * this is an interface convenience, computing exactly what moe_permute computes.
+ *   Arguments and results as in moe_permute, without `ws`.
+ *   Scratch: a fixed array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (512 KiB) in the
+ *   library's device memory, present on every GPU that loads the library until the
+ *   process exits.  Nothing is allocated or freed by this call.
+ *   Limits: T*k <= MOE_PERMUTE_NOALLOC_MAX_PAIRS (2^20); larger batches return
+ *   MOE_ERR_UNSUPPORTED before anything is launched (use moe_permute with a workspace).
+ *   The first call on a device looks up the scratch array's device address (once per
+ *   device, with that device current); make that first call before any stream capture.
+ *   Every call shares the one scratch array: calls whose kernels overlap on the GPU (on
+ *   different streams, or from several threads) race and must be serialised by the
+ *   caller.  Each call fully writes the scratch it reads, so nothing carries over. */
+#define MOE_PERMUTE_NOALLOC_MAX_PAIRS (1 << 20)
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (512 * 1024)
+moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx,
+                                 int32_t* expert_offsets, int32_t* sorted_src,
+                                 int32_t* inv_pos, void* stream);
+
 /* Routed experts (ONNX export card, "Mixture of Experts" row; Inferentia2 card,
  * "How it works": outputs weighted by the routing weights and summed).
  *   xn_moe [T][H] bf16; topk_w [T][k] fp32; expert_offsets, sorted_src, inv_pos as

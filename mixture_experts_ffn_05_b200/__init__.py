@@ -28,9 +28,11 @@ MOE_W_BF16 = 0
 MOE_W_INT8 = 1
 
 # Entry points of include/moe_ffn.h (the CPU tests check the header declares exactly these).
-ENTRY_POINTS = ("moe_workspace_size", "moe_router", "moe_permute", "moe_ffn_forward",
-                "dense_mlp_forward", "moe_block_forward", "moe_quantize_int8",
-                "moe_check_device_status", "moe_status_string", "moe_abi_version")
+ENTRY_POINTS = ("moe_workspace_size", "moe_router", "moe_permute", "moe_permute_noalloc",
+                "moe_ffn_forward", "dense_mlp_forward", "moe_block_forward",
+                "moe_quantize_int8", "moe_check_device_status", "moe_status_string",
+                "moe_abi_version")
+PERMUTE_NOALLOC_MAX_PAIRS = 1 << 20
 
 
 class MoeError(RuntimeError):
@@ -66,6 +68,7 @@ _SIG = {
     "moe_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(CConfig), _I32]),
     "moe_router": (_I32, [ctypes.POINTER(CConfig), _I32] + [_P] * 12 + [ctypes.c_size_t, _P]),
     "moe_permute": (_I32, [ctypes.POINTER(CConfig), _I32] + [_P] * 5 + [ctypes.c_size_t, _P]),
+    "moe_permute_noalloc": (_I32, [ctypes.POINTER(CConfig), _I32] + [_P] * 4 + [_P]),
     "moe_ffn_forward": (_I32, [ctypes.POINTER(CConfig), _I32, _P, _P, _P, _P, _P,
                                ctypes.POINTER(CExpertWeights), _P, _P, ctypes.c_size_t, _P]),
     "dense_mlp_forward": (_I32, [ctypes.POINTER(CConfig), _I32] + [_P] * 5 + [ctypes.c_size_t, _P]),
@@ -178,6 +181,18 @@ def moe_permute(cfg, topk_idx, expert_offsets, sorted_src, inv_pos, ws, stream=N
                            _ptr(inv_pos, torch.int32, "inv_pos"), _ptr(ws, torch.uint8, "ws"),
                            ws.numel(), _stream(stream))
     _check("moe_permute", st)
+
+
+def moe_permute_noalloc(cfg, topk_idx, expert_offsets, sorted_src, inv_pos, stream=None):
+    """moe_permute without a workspace, for callers that cannot provide scratch memory:
+    the library's own fixed device array (512 KiB, up to 2^20 pairs) is used instead.
+    Calls that overlap on the GPU share that array and must be serialised."""
+    T = topk_idx.shape[0]
+    st = lib().moe_permute_noalloc(ctypes.byref(cfg.c()), T, _ptr(topk_idx, torch.int32, "topk_idx"),
+                                   _ptr(expert_offsets, torch.int32, "expert_offsets"),
+                                   _ptr(sorted_src, torch.int32, "sorted_src"),
+                                   _ptr(inv_pos, torch.int32, "inv_pos"), _stream(stream))
+    _check("moe_permute_noalloc", st)
 
 
 def _experts(cfg, e: dict) -> CExpertWeights:

@@ -534,3 +534,59 @@ moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream) {
 }
 
 }  // extern "C"
+
+// ================================================================ no-workspace permutation
+//
+// For callers that can hand the library no scratch memory (see moe_permute_noalloc in
+// include/moe_ffn.h).  The multi-block counting sort needs per-block histograms and
+// per-block bases (2 x 256 blocks x 256 experts ints); they live in this fixed device
+// array instead of a caller workspace.  Its host-side name is only a handle: the
+// device address is looked up once per device with cudaGetSymbolAddress and cached.
+
+namespace {
+
+constexpr int kNoAllocMaxBlocks = MOE_PERMUTE_NOALLOC_MAX_PAIRS / 4096;  // blocks of 4096 pairs
+constexpr int kNoAllocInts = 2 * kNoAllocMaxBlocks * 256;
+static_assert(kNoAllocInts * 4 == MOE_PERMUTE_NOALLOC_SCRATCH_BYTES, "scratch size");
+
+static __device__ __align__(256) int g_permute_scratch[kNoAllocInts];
+
+std::mutex g_scratch_mu;
+int* g_scratch_ptr[64] = {};
+
+// Device address of the scratch array on the current device (NULL on failure).
+int* permute_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int32_t T,
+                                            const int32_t* topk_idx, int32_t* expert_offsets,
+                                            int32_t* sorted_src, int32_t* inv_pos,
+                                            void* stream) {
+  Dims d;
+  moe_status_t st = check_cfg(cfg, T, &d);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  for (const void* p : {(const void*)topk_idx, (const void*)expert_offsets,
+                        (const void*)sorted_src, (const void*)inv_pos})
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const int64_t n = static_cast<int64_t>(d.T) * d.k;
+  if (n > MOE_PERMUTE_NOALLOC_MAX_PAIRS) return MOE_ERR_UNSUPPORTED;
+  int* scratch = permute_scratch();
+  if (scratch == nullptr) return MOE_ERR_CUDA;
+  // block histograms in the first half, block bases in the second (nb * E <= 256 * 256)
+  return cuda_status(launch_permute(static_cast<int>(n), d.E, topk_idx, expert_offsets,
+                                    sorted_src, inv_pos, scratch,
+                                    scratch + kNoAllocMaxBlocks * 256,
+                                    static_cast<cudaStream_t>(stream)));
+}
