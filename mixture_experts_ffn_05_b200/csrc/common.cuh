@@ -132,6 +132,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy
+// (tcgen05.mma reads its operands through it).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 // 2-D tiled bulk copy global -> shared; completion counted on `bar` in bytes.
 // c0 is the innermost (contiguous) coordinate in elements, c1 the row.

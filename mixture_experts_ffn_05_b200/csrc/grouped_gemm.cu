@@ -22,39 +22,92 @@
 // Warp roles (320 threads): warp 0 issues TMA loads into a ring of shared-memory
 // stages, warp 1 issues tcgen05.mma into one of 2-4 TMEM accumulators, and two groups of
 // four warps (2-5 and 6-9) take alternate pieces, read the accumulator back (tcgen05.ld)
-// and run the epilogue while later pieces are being multiplied.  Every wait is bounded; a wait that runs out records a timeout in the
+// and run the epilogue while later pieces are being multiplied.  With int8 expert
+// weights (the int8 build of the Inferentia2 card: per-channel symmetric INT8 experts),
+// warps 10-13 convert each raw int8 tile to bf16 in shared memory inside the mainloop,
+// and the per-row scale multiplies the fp32 accumulator in the epilogue (it factors out
+// of the K sum, so this is exact).  Every wait is bounded; a wait that runs out records a timeout in the
 // status word and the CTA winds down.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
-constexpr int kGemmThreads = 320;  // producer warp, MMA warp, 2 x 4 epilogue warps
 constexpr int kMaxSplit = 4;       // K pieces per tile at most
-constexpr int kMaxEntries = 258;  // groups of problem 0 (<= 256) + problem 1 (1) + 1
+constexpr int kMaxEntries = 258;   // groups of problem 0 (<= 256) + problem 1 (1) + 1
+constexpr int kConvWarp0 = 10;     // first converter warp of the int8 variant
 
-template <int BN>
+// W8 = false: the A tile (weights, bf16) goes from HBM to shared memory by TMA, already
+//   in the 128-byte-swizzled K-major layout the MMA reads.
+// W8 = true: TMA lands the raw A tile (int8 codes, or bf16 rows of a bf16 problem in the
+//   same launch) unswizzled; four converter warps turn it into the bf16 swizzled layout
+//   in a second, shallower ring.  The int8 row scales are applied in the epilogue.
+template <int BN, bool W8>
 struct Cfg {
-  static constexpr int kABytes = 128 * 64 * 2;  // 128 weight rows x 64 K (bf16)
-  static constexpr int kBBytes = BN * 64 * 2;   // BN token rows x 64 K
-  static constexpr int kStage = kABytes + kBBytes;
-  static constexpr int kStages = BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4));
+  static constexpr int kThreads = W8 ? 448 : 320;  // producer, MMA, 2x4 epilogue (+4 converters)
+  static constexpr int kABytes = 128 * 64 * 2;     // bf16 A tile: 128 weight rows x 64 K
+  static constexpr int kBBytes = BN * 64 * 2;      // BN token rows x 64 K
+  static constexpr int kStage = kABytes + kBBytes; // (W8: the raw A region has the same size)
+  static constexpr int kStages = W8 ? (BN <= 16 ? 8 : (BN <= 32 ? 7 : (BN <= 64 ? 6 : (BN <= 128 ? 4 : 3))))
+                                    : (BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4)));
+  static constexpr int kConv = W8 ? 4 : 0;          // converted bf16 A stages
   // TMEM accumulators: 4 for narrow tiles (the epilogue of a weight-streaming piece is
   // latency-bound and must not hold up the MMAs), 2 for wide ones (512 columns max).
   static constexpr int kAcc = BN <= 64 ? 4 : 2;
   static constexpr int kTmemCols = kAcc * BN < 32 ? 32 : kAcc * BN;
-  // after the stages: barriers, bookkeeping, the gate/up exchange buffer
-  static constexpr int kBarOff = kStages * kStage;
-  static constexpr int kNumBars = 2 * kStages + 2 * kAcc + 1;  // full, empty, acc_full, acc_empty, drain
+  // after the stages: converted stages, barriers, bookkeeping, the gate/up exchange buffer
+  static constexpr int kConvOff = kStages * kStage;
+  static constexpr int kBarOff = kConvOff + kConv * kABytes;
+  static constexpr int kNumBars = 2 * kStages + 2 * kConv + 2 * kAcc + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kMiscInts = 8;               // tmem slot, abort, bcast, ...
+  static constexpr int kMiscInts = 8;               // tmem slot, abort, bcast x2, converter flag
   static constexpr int kPreOff = kMiscOff + kMiscInts * 4;
   static constexpr int kTabInts = 4 * kMaxEntries;  // pre, cnt, b0, ng
   static constexpr int kXchgOff = ((kPreOff + kTabInts * 4) + 15) & ~15;
   static constexpr int kXchgBytes = 2 * 16 * 64 * 4;  // one per epilogue group
   static constexpr int kSmem = kXchgOff + kXchgBytes + 1024;  // + alignment slack
   static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(kSmem <= 232448, "shared memory");
 };
+
+// ---- int8 -> bf16 in the converter warps.  Each code q in [-127, 127] becomes the fp32
+// number 2^23 + (q + 128) by placing the unsigned byte q + 128 in the mantissa of 2^23
+// (exponent-bias construction), minus 2^23 + 128; both steps are exact, and so is the
+// rounding to bf16 since |q| < 2^8.
+__device__ __forceinline__ float i8_to_f32(uint32_t biased_word, uint32_t byte) {
+  return __int_as_float(static_cast<int>(__byte_perm(biased_word, 0x4B000000u, 0x7440u + byte))) -
+         8388736.0f;
+}
+
+// Row `r` of the converted tile: 64 K values as 8 chunks of 16 bytes, chunk c stored at
+// chunk position c ^ (r % 8) (the 128-byte swizzle, for a 1024-byte-aligned tile).
+__device__ __forceinline__ void convert_row_i8(const uint8_t* src, uint8_t* dst, int r) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const uint4 q = s[h];
+    const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u,
+                           q.w ^ 0x80808080u};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[2 * i] = pack2(i8_to_f32(w[i], 0), i8_to_f32(w[i], 1));
+      o[2 * i + 1] = pack2(i8_to_f32(w[i], 2), i8_to_f32(w[i], 3));
+    }
+    const int c0 = 2 * h, c1 = 2 * h + 1;
+    *reinterpret_cast<uint4*>(dst + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + ((c1 ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+__device__ __forceinline__ void convert_row_bf16(const uint8_t* src, uint8_t* dst, int r) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+  uint4 v[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) v[c] = s[c];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + ((c ^ (r & 7)) << 4)) = v[c];
+}
 
 struct Piece {
   int p, g, m, n, s;
@@ -95,22 +148,25 @@ __device__ __forceinline__ Piece decode_piece(int piece, const GemmParams& P, co
   return pc;
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <int BN, bool W8>
+__global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams P) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, W8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* empty = full + C::kStages;
-  uint64_t* acc_full = empty + C::kStages;
+  uint64_t* conv_full = empty + C::kStages;
+  uint64_t* conv_empty = conv_full + C::kConv;
+  uint64_t* acc_full = conv_empty + C::kConv;
   uint64_t* acc_empty = acc_full + C::kAcc;
   uint64_t* drain = acc_empty + C::kAcc;
   int* misc = reinterpret_cast<int*>(smem + C::kMiscOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 0);
   volatile int* abort_flag = misc + 1;
-  volatile int* bcast = misc + 2;
+  volatile int* bcast = misc + 2;        // [2], one per epilogue group
+  volatile int* conv_flag = misc + 4;    // converter warps
   int* pre = reinterpret_cast<int*>(smem + C::kPreOff);
   int* cnt = pre + kMaxEntries;
   int* b0 = cnt + kMaxEntries;
@@ -124,7 +180,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], W8 ? 2 : 1);  // W8: the MMA (B) and the converters (raw A)
+    }
+    for (int i = 0; i < C::kConv; ++i) {
+      mbar_init(&conv_full[i], 1);
+      mbar_init(&conv_empty[i], 1);
     }
     for (int i = 0; i < C::kAcc; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -144,7 +204,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < nent; i += kGemmThreads) {
+  for (int i = threadIdx.x; i < nent; i += C::kThreads) {
     const int p = i < P.prob[0].groups ? 0 : 1;
     const int g = p == 0 ? i : i - P.prob[0].groups;
     const GemmProblem& pr = P.prob[p];
@@ -213,10 +273,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           uint8_t* sa = smem + stage * C::kStage;
-          mbar_arrive_expect_tx(&full[stage], C::kStage);
+          // A bytes: a bf16 tile, or (W8 with int8 weights) a tile of int8 codes
+          const int abytes = (W8 && pr.w8) ? C::kABytes / 2 : C::kABytes;
+          mbar_arrive_expect_tx(&full[stage], abytes + C::kBBytes);
           if (pr.kind == 0) {
             tma_load_2d(sa, ma, &full[stage], ks * 64, arow, pol_w);
-            tma_load_2d(sa + C::kABytes / 2, ma, &full[stage], ks * 64, arow + pr.nw, pol_w);
+            tma_load_2d(sa + abytes / 2, ma, &full[stage], ks * 64, arow + pr.nw, pol_w);
           } else {
             tma_load_2d(sa, ma, &full[stage], ks * 64, arow, pol_w);
           }
@@ -241,6 +303,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      int cs = 0;
+      uint32_t cph = 0;
       int ab = 0;
       uint32_t aph = 0;
       bool ok = true, issued = false;
@@ -254,17 +318,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(ab * BN);
         for (int ks = pc.k0; ks < pc.k1; ++ks) {
-          if (!mbar_wait(&full[stage], phase, tmo, abort_flag)) {
+          if (!mbar_wait(&full[stage], phase, tmo, abort_flag) ||
+              (W8 && !mbar_wait(&conv_full[cs], cph, tmo, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * C::kStage);
-          const uint64_t ad = sdesc_k_sw128(sa);
+          const uint32_t sA = W8 ? smem_u32(smem + C::kConvOff + cs * C::kABytes) : sa;
+          const uint64_t ad = sdesc_k_sw128(sA);
           const uint64_t bd = sdesc_k_sw128(sa + C::kABytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (ks > pc.k0 || kk > 0) ? 1u : 0u);
+          if (W8) {
+            umma_commit(&conv_empty[cs]);
+            if (++cs == C::kConv) {
+              cs = 0;
+              cph ^= 1u;
+            }
+          }
           umma_commit(&empty[stage]);
           issued = true;
           if (++stage == C::kStages) {
@@ -286,6 +359,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           umma_commit(drain);
           mbar_wait(drain, 0, tmo, nullptr);
         }
+      }
+    }
+  } else if (W8 && warp >= kConvWarp0) {
+    // ================= converters (W8): raw A stage -> swizzled bf16 stage ============
+    const int ct = threadIdx.x - kConvWarp0 * 32;  // the row of the tile this thread owns
+    int stage = 0;
+    uint32_t phase = 0;
+    int cs = 0;
+    uint32_t cph = 0;
+    for (int piece = blockIdx.x; piece < total; piece += gridDim.x) {
+      const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
+      const bool i8 = P.prob[pc.p].w8 != 0;
+      bool ok = true;
+      for (int ks = pc.k0; ks < pc.k1; ++ks) {
+        if (ct == 0)
+          *conv_flag = (mbar_wait(&full[stage], phase, tmo, abort_flag) &&
+                        mbar_wait(&conv_empty[cs], cph ^ 1u, tmo, abort_flag))
+                           ? 1
+                           : 0;
+        named_sync(3, 128);
+        if (!*conv_flag) {
+          ok = false;
+          break;
+        }
+        const uint8_t* raw = smem + stage * C::kStage;
+        uint8_t* dst = smem + C::kConvOff + cs * C::kABytes + ct * 128;
+        if (i8)
+          convert_row_i8(raw + ct * 64, dst, ct);
+        else
+          convert_row_bf16(raw + ct * 128, dst, ct);
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        named_sync(3, 128);
+        if (ct == 0) {
+          mbar_arrive(&conv_full[cs]);
+          mbar_arrive(&empty[stage]);
+        }
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (++cs == C::kConv) {
+          cs = 0;
+          cph ^= 1u;
+        }
+      }
+      if (!ok) {
+        if (ct == 0) {
+          record_status(P.status, kStatusTimeout);
+          *abort_flag = 1;
+        }
+        break;
       }
     }
   } else {
@@ -426,37 +550,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-template <int BN>
+template <int BN, bool W8>
 static cudaError_t launch_bn(const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s) {
-  const int smem = Cfg<BN>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  using C = Cfg<BN, W8>;
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, W8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<BN><<<grid, kGemmThreads, smem, s>>>(maps, p);
+  grouped_gemm_kernel<BN, W8><<<grid, C::kThreads, C::kSmem, s>>>(maps, p);
   return cudaGetLastError();
 }
 
-size_t grouped_gemm_smem_bytes(int bn) {
+template <bool W8>
+static cudaError_t launch_w(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
+                            cudaStream_t s) {
   switch (bn) {
-    case 16: return Cfg<16>::kSmem;
-    case 32: return Cfg<32>::kSmem;
-    case 64: return Cfg<64>::kSmem;
-    case 128: return Cfg<128>::kSmem;
-    case 256: return Cfg<256>::kSmem;
+    case 16: return launch_bn<16, W8>(maps, p, grid, s);
+    case 32: return launch_bn<32, W8>(maps, p, grid, s);
+    case 64: return launch_bn<64, W8>(maps, p, grid, s);
+    case 128: return launch_bn<128, W8>(maps, p, grid, s);
+    case 256: return launch_bn<256, W8>(maps, p, grid, s);
   }
-  return 0;
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                                 cudaStream_t s) {
-  switch (bn) {
-    case 16: return launch_bn<16>(maps, p, grid, s);
-    case 32: return launch_bn<32>(maps, p, grid, s);
-    case 64: return launch_bn<64>(maps, p, grid, s);
-    case 128: return launch_bn<128>(maps, p, grid, s);
-    case 256: return launch_bn<256>(maps, p, grid, s);
-  }
-  return cudaErrorInvalidValue;
+  return p.int8_weights ? launch_w<true>(bn, maps, p, grid, s) : launch_w<false>(bn, maps, p, grid, s);
 }
 
 }  // namespace moe

@@ -30,12 +30,13 @@ struct GemmProblem {
   const int* out_rows;   // down: output row of B row pos (sorted_src); NULL = pos
   const float* route_w;  // down: weight per output row (topk_w flattened); NULL = 1
   const float* wscale;   // int8 row scales [groups][w_rows_per_group]; NULL for bf16
+  int w8;                // A operand is int8 codes (needs a launch with int8_weights)
 };
 
 struct GemmParams {
   GemmProblem prob[2];
   int nprob;
-  int int8_weights;     // A operand stored as int8 (converted in shared memory)
+  int int8_weights;     // a problem has int8 A: use the variant with converter warps
   float* partials;      // split-K partial tiles, [piece][BN][128] fp32
   unsigned* counters;   // split-K arrival counters, zero between launches
   unsigned* status;     // device status word
@@ -66,7 +67,6 @@ cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src
                                const uint16_t* src, uint16_t* dst, cudaStream_t s);
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                                 cudaStream_t s);
-size_t grouped_gemm_smem_bytes(int bn);
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
                                  const uint16_t* y, const uint16_t* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,

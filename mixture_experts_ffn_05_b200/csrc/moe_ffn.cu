@@ -169,23 +169,34 @@ int sm_count() {
   return g_sm_count[dev];
 }
 
-// K-major 2-D map: rows x cols elements, box 64 (K) x box_rows, 128-byte swizzle.
+// K-major 2-D map: rows x cols elements, box of 64 K elements x box_rows rows.
 bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
-               CUtensorMapDataType dt, int elem_bytes) {
+               CUtensorMapDataType dt, int elem_bytes, CUtensorMapSwizzle swz) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t es[2] = {1, 1};
   const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
+// bf16 tile as the MMA reads it (128-byte swizzle).
 bool encode_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
-  return encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2);
+  return encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Raw weight tile for the converter warps: unswizzled rows of int8 codes or bf16 values.
+bool encode_raw(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
+                bool int8) {
+  return int8 ? encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)
+              : encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -235,13 +246,21 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
 
   GemmParams gu{}, dn{};
   GemmMaps mgu{}, mdn{};
+  // int8 experts: the launches take the converter-warp variant, whose A maps are raw
+  // (unswizzled) for every problem of the launch, the bf16 dense MLP included.
+  const bool w8 = j.experts && d.int8;
   for (GemmParams* P : {&gu, &dn}) {
     P->partials = at<float>(ws, L.partials);
     P->counters = at<unsigned>(ws, L.counters);
     P->status = at<unsigned>(ws, L.status);
     P->timeout_ns = kWaitTimeoutNs;
-    P->int8_weights = 0;
+    P->int8_weights = w8 ? 1 : 0;
   }
+  auto encode_a = [&](CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
+                      bool int8) {
+    return w8 ? encode_raw(m, base, rows, cols, box_rows, int8)
+              : encode_bf16(m, base, rows, cols, box_rows);
+  };
   int np = 0;
   if (j.experts) {
     GemmProblem& a = gu.prob[np];
@@ -249,15 +268,16 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     a.kind = 0; a.groups = d.E; a.offsets = j.offsets; a.n_tokens = static_cast<int>(Tk);
     a.k_steps = d.H / 64; a.m_tiles = d.I / 64; a.w_rows_per_group = 2 * d.I; a.nw = d.I;
     a.split = L.split_gu; a.map = np; a.out = h; a.out_ld = d.I; a.wscale = j.s_gate_up;
+    a.w8 = d.int8;
     GemmProblem& b = dn.prob[np];
     b = GemmProblem{};
     b.kind = 1; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = static_cast<int>(Tk);
     b.k_steps = d.I / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H; b.nw = 0;
     b.split = L.split_d; b.map = np; b.out = j.y; b.out_ld = d.H; b.out_rows = j.sorted_src;
-    b.route_w = j.topk_w; b.wscale = j.s_down;
-    if (!encode_bf16(&mgu.a[np], j.w_gate_up, static_cast<int64_t>(d.E) * 2 * d.I, d.H, 64) ||
+    b.route_w = j.topk_w; b.wscale = j.s_down; b.w8 = d.int8;
+    if (!encode_a(&mgu.a[np], j.w_gate_up, static_cast<int64_t>(d.E) * 2 * d.I, d.H, 64, d.int8) ||
         !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, L.bn) ||
-        !encode_bf16(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128) ||
+        !encode_a(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128, d.int8) ||
         !encode_bf16(&mdn.b[np], h, Tk, d.I, L.bn))
       return MOE_ERR_CUDA;
     ++np;
@@ -273,9 +293,9 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.kind = 1; b.groups = 1; b.offsets = nullptr; b.n_tokens = d.T;
     b.k_steps = d.D / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H;
     b.split = L.split_dd; b.map = np; b.out = j.dense_out; b.out_ld = d.H;
-    if (!encode_bf16(&mgu.a[np], j.w_dgu, 2 * static_cast<int64_t>(d.D), d.H, 64) ||
+    if (!encode_a(&mgu.a[np], j.w_dgu, 2 * static_cast<int64_t>(d.D), d.H, 64, false) ||
         !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, L.bn) ||
-        !encode_bf16(&mdn.a[np], j.w_dd, d.H, d.D, 128) ||
+        !encode_a(&mdn.a[np], j.w_dd, d.H, d.D, 128, false) ||
         !encode_bf16(&mdn.b[np], hd, d.T, d.D, L.bn))
       return MOE_ERR_CUDA;
     ++np;
@@ -382,7 +402,6 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
                         (const void*)sorted_src, (const void*)inv_pos, (const void*)moe_out})
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (!w_ok(experts, d.int8)) return MOE_ERR_INVALID_ARG;
-  if (d.int8) return MOE_ERR_UNSUPPORTED;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -446,7 +465,6 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
                         (const void*)w->g_post_moe, (const void*)w->g_post_dense})
     if (p != nullptr && !aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (!w_ok(&w->experts, d.int8)) return MOE_ERR_INVALID_ARG;
-  if (d.int8) return MOE_ERR_UNSUPPORTED;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -90,3 +90,34 @@ def run_block(cfg, case, layer, want_moe=True, ws=None, x=None):
     st = mf.moe_check_device_status(ws)
     assert st == mf.MOE_OK, mf.status_string(st)
     return out, moe
+
+
+_INT8_CACHE = cases._Lru(2)
+
+
+def int8_experts(case: cases.Case):
+    """Quantise the case's expert weights on the GPU (moe_quantize_int8) and with the
+    oracle; return (device tensors for the library, oracle.Experts built from the
+    oracle's own codes and scales, whether the two quantisations are identical)."""
+    key = id(case.p)
+    if key in _INT8_CACHE and _INT8_CACHE[key][0] is case.p:
+        return _INT8_CACHE[key][1]
+    dev = {}
+    host = {}
+    same = True
+    for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down")):
+        w = case.p[name]
+        rows, cols = int(np.prod(w.shape[:-1])), w.shape[-1]
+        q = torch.empty(w.shape, dtype=torch.int8, device="cuda")
+        s = torch.empty(w.shape[:-1], dtype=torch.float32, device="cuda")
+        mf.moe_quantize_int8(to_dev(w).view(rows, cols), q.view(rows, cols), s.view(rows))
+        qo, so = oracle.quantize_int8_per_channel(w)
+        same = same and np.array_equal(q.cpu().numpy(), qo) and \
+            np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+        dev[name], dev[sname] = q, s
+        host[name], host[sname] = qo, so
+    ex = oracle.Experts(q_gate_up=host["w_gate_up"], s_gate_up=host["s_gate_up"],
+                        q_down=host["w_down"], s_down=host["s_down"])
+    res = (dev, ex, same)
+    _INT8_CACHE.put(key, (case.p, res))
+    return res
