@@ -37,10 +37,25 @@ METRIC = ("MoE-FFN tokens/s (1 B200) at T=8..16K; % HBM roofline (decode) / "
 UNIT = "tokens/s"
 
 WORKLOADS = {
-    "decode": dict(shape=synth.DECODE, layers=8, zipf=False, steps=3000, warmup=100,
+    "decode": dict(shape=synth.DECODE, layers=8, steps=3000, warmup=100,
                    name="Gemma-4-26B-A4B-shaped MoE-FFN layer, decode T=8 (bf16 experts)"),
-    "prefill": dict(shape=synth.PREFILL, layers=4, zipf=True, steps=200, warmup=10,
+    "decode_T64": dict(shape=synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                       steps=2000, warmup=100,
+                       name="Gemma-4-26B-A4B-shaped MoE-FFN layer, T=64 (bf16 experts)"),
+    "prefill": dict(shape=synth.PREFILL, layers=4, zipf=True, steps=300, warmup=10,
                     name="Gemma-4-26B-A4B-shaped MoE-FFN layer, prefill T=2048, Zipf-skewed router"),
+    "int8_T1": dict(shape=synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                    int8=True, steps=3000, warmup=100,
+                    name="same layer with per-channel int8 experts, T=1"),
+    "int8_T64": dict(shape=synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                     int8=True, steps=2000, warmup=100,
+                     name="same layer with per-channel int8 experts, T=64"),
+    "int8_T1024": dict(shape=synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                       int8=True, steps=500, warmup=20,
+                       name="same layer with per-channel int8 experts, T=1024"),
+    "stack": dict(shape=synth.Shape(T=synth.STACK_T, H=2816, E=128, k=8, I=704, D=2112),
+                  layers=synth.STACK_LAYERS, chain=True, steps=3, warmup=1,
+                  name="stack of 30 distinct MoE-FFN layers, residual-chained, T=16384 (one 16K chunk)"),
 }
 ZIPF_ALPHA_FILE = os.path.join(ROOT, "tests", "golden", "zipf_alpha.json")
 
@@ -147,82 +162,129 @@ class Clocks:
 
 # ---------------------------------------------------------------------------- work model
 
-def algorithmic(shape, used_experts: int):
+def algorithmic(shape, used_experts: int, int8: bool = False):
     """Bytes that must move and FLOPs that must run for one block call.
 
-    Bytes: the weights of the experts that received a token, the dense MLP, the router
-    and the norm vectors, plus x in and out.  Intermediates are implementation traffic.
+    Bytes: the weights of the experts that received a token (int8 codes plus fp32 row
+    scales for int8 experts), the dense MLP, the router and the norm vectors, plus x in
+    and out.  Intermediates are implementation traffic.
     """
     H, E, k, I, D, T = shape.H, shape.E, shape.k, shape.I, shape.D, shape.T
-    b_experts = used_experts * 3 * I * H * 2
+    wb = 1 if int8 else 2
+    b_experts = used_experts * (3 * I * H * wb + ((2 * I + H) * 4 if int8 else 0))
     b_dense = 3 * D * H * 2
     b = b_experts + b_dense + E * H * 2 + 6 * H * 2 + E * 2 + 2 * T * H * 2
     flops = T * (2 * k * 3 * I * H + 2 * 3 * D * H + 2 * E * H)
     # the gate_up launch alone: its weights, its token rows in, h out
-    b_gate_up = used_experts * 2 * I * H * 2 + 2 * D * H * 2 + (T * k + T) * H * 2 + (T * k * I + T * D) * 2
+    b_gate_up = (used_experts * (2 * I * H * wb + (2 * I * 4 if int8 else 0)) + 2 * D * H * 2
+                 + (T * k + T) * H * 2 + (T * k * I + T * D) * 2)
     f_gate_up = T * (2 * k * 2 * I * H + 2 * 2 * D * H)
     return {"bytes": b, "flops": flops, "gate_up_bytes": b_gate_up, "gate_up_flops": f_gate_up}
 
 
 # ---------------------------------------------------------------------------- our arm
 
+def _make_layers(mf, cfg, shape, wl, n, seed, device):
+    layers, alpha = [], None
+    for l in range(n):
+        t = synth.torch_layer(shape, seed, l, device)
+        if wl.get("zipf"):
+            with open(ZIPF_ALPHA_FILE) as f:
+                alpha = float(json.load(f)["alpha"])
+            t["logit_bias"] = torch.from_numpy(synth.zipf_bias(seed, shape.E, alpha)).to(device)
+        if wl.get("int8"):
+            for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down")):
+                w = t.pop(name)
+                cols = w.shape[-1]
+                q = torch.empty(w.shape, dtype=torch.int8, device=device)
+                sc = torch.empty(w.shape[:-1], dtype=torch.float32, device=device)
+                mf.moe_quantize_int8(w.view(-1, cols), q.view(-1, cols), sc.view(-1))
+                t[name], t[sname] = q, sc
+                del w
+        layers.append(t)
+    torch.cuda.synchronize(device)
+    return layers, alpha
+
+
 def run_ours(args, wl, rank, world, device):
     import mixture_experts_ffn_05_b200 as mf
     mf.lib()  # fails loudly without the built CUDA library
     shape = wl["shape"]
     T = shape.T
-    cfg = mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps)
+    int8 = bool(wl.get("int8"))
+    chain = bool(wl.get("chain"))
+    cfg = mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps, int8)
     seed = 1234 + 7919 * rank
-    alpha = None
-    layers = []
-    for l in range(args.layers or wl["layers"]):
-        t = synth.torch_layer(shape, seed, l, device)
-        if wl["zipf"]:
-            with open(ZIPF_ALPHA_FILE) as f:
-                alpha = float(json.load(f)["alpha"])
-            t["logit_bias"] = torch.from_numpy(synth.zipf_bias(seed, shape.E, alpha)).to(device)
-        layers.append(t)
+    nl = args.layers or wl["layers"]
+    layers, alpha = _make_layers(mf, cfg, shape, wl, nl, seed, device)
     bws = [mf.BlockWeights(cfg, t) for t in layers]
     W, K = args.warmup, args.steps
     xs = [synth.torch_x(shape, seed, i, device) for i in range(W + K)]
     out = torch.empty(T, shape.H, dtype=torch.bfloat16, device=device)
+    bufs = [torch.empty_like(out), torch.empty_like(out)]
     ws = mf.workspace(cfg, T, device)
     stream = torch.cuda.current_stream(device)
 
-    # routing of each timed step (outside the timed region): experts that receive tokens
+    def calls(i, x=None, final=None):
+        """(layer, input, output) of step i: one layer, or every layer chained."""
+        x = xs[i] if x is None else x
+        if not chain:
+            return [(i % nl, x, out if final is None else final)]
+        res, cur = [], x
+        for l in range(nl):
+            dst = (out if final is None else final) if l == nl - 1 else bufs[l % 2]
+            res.append((l, cur, dst))
+            cur = dst
+        return res
+
+    def step(i, evs=None, x=None, final=None):
+        for c, (l, xin, dst) in enumerate(calls(i, x, final)):
+            mf.moe_block_forward(cfg, xin, bws[l], dst, ws, stream=stream,
+                                 stage_events=None if evs is None else evs[c])
+
+    # experts that receive tokens in each timed call (outside the timed region)
     used = []
     ti = torch.empty(T, shape.k, dtype=torch.int32, device=device)
     tw = torch.empty(T, shape.k, dtype=torch.float32, device=device)
     xa = torch.empty(T, shape.H, dtype=torch.bfloat16, device=device)
     xb = torch.empty_like(xa)
     for i in range(K):
-        L = layers[(W + i) % len(layers)]
-        mf.moe_router(cfg, xs[W + i], L["router_scale"], L["w_router"], L.get("logit_bias"),
-                      L["per_expert_scale"], L["g_pre_moe"], L["g_pre_dense"], ti, tw, xa, xb, ws)
-        used.append(int(torch.unique(ti).numel()))
-
-    def step(i, ev=None):
-        mf.moe_block_forward(cfg, xs[i], bws[i % len(bws)], out, ws, stream=stream, stage_events=ev)
+        for (l, xin, dst) in calls(W + i):
+            L = layers[l]
+            mf.moe_router(cfg, xin, L["router_scale"], L["w_router"], L.get("logit_bias"),
+                          L["per_expert_scale"], L["g_pre_moe"], L["g_pre_dense"], ti, tw, xa, xb, ws)
+            used.append(int(torch.unique(ti).numel()))
+            if chain:
+                mf.moe_block_forward(cfg, xin, bws[l], dst, ws, stream=stream)
 
     for i in range(W):
         step(i)
     torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(mf.MOE_BLOCK_EVENTS)]
-                for _ in range(K)]
+    ncalls = len(calls(0))
+    stage_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(mf.MOE_BLOCK_EVENTS)]
+                 for _ in range(ncalls)] for _ in range(K)]
     for evs in stage_ev:  # create the CUDA events before the timed region
-        for e in evs:
-            e.record(stream)
+        for ev in evs:
+            for e in ev:
+                e.record(stream)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     clocks = Clocks(device)
     time.sleep(0.15)
     torch.cuda.synchronize(device)
+    # timed region 1: the steps alone (events inside a step would order its kernels and
+    # hide the overlap of consecutive launches)
     e0.record(stream)
     for i in range(K):
-        step(W + i, stage_ev[i])
+        step(W + i)
     e1.record(stream)
+    torch.cuda.synchronize(device)
+    # timed region 2: the same steps with events at every stage boundary, for the
+    # duration of each kernel (the roofline of the dominant one)
+    for i in range(K):
+        step(W + i, stage_ev[i])
     torch.cuda.synchronize(device)
     clk = clocks.stop()
     if world > 1:
@@ -232,9 +294,10 @@ def run_ours(args, wl, rank, world, device):
         raise RuntimeError(f"device status after the timed region: {mf.status_string(st)}")
     t_ms = e0.elapsed_time(e1)
     stages = {n: [] for n in ("router", "permute", "gather", "clear", "gate_up", "down", "combine")}
-    for ev in stage_ev:
-        for j, n in enumerate(stages):
-            stages[n].append(ev[j].elapsed_time(ev[j + 1]))
+    for evs in stage_ev:
+        for ev in evs:
+            for j, n in enumerate(stages):
+                stages[n].append(ev[j].elapsed_time(ev[j + 1]))
     t_max = max_over_ranks(t_ms, world, device)
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
@@ -243,11 +306,12 @@ def run_ours(args, wl, rank, world, device):
         x_host[i].copy_(xs[i])
     out_host = torch.empty(K, T, shape.H, dtype=torch.bfloat16, pin_memory=True)
     x_dev = torch.empty(T, shape.H, dtype=torch.bfloat16, device=device)
+    y_dev = torch.empty_like(x_dev)
 
     def e2e_step(i, j):
         x_dev.copy_(x_host[i], non_blocking=True)
-        mf.moe_block_forward(cfg, x_dev, bws[i % len(bws)], out, ws, stream=stream)
-        out_host[j].copy_(out, non_blocking=True)
+        step(i, x=x_dev, final=y_dev)
+        out_host[j].copy_(y_dev, non_blocking=True)
 
     for i in range(min(W, 10)):
         e2e_step(i, 0)
@@ -267,57 +331,65 @@ def run_ours(args, wl, rank, world, device):
 
     # ---- roofline of the dominant kernel (the gate_up grouped GEMM) and of the block
     pk = peaks()
-    alg = [algorithmic(shape, u) for u in used]
-    gu_bytes = sum(a["gate_up_bytes"] for a in alg)
+    long_step = t_max / K > 10.0  # ms: a kernel inside a long step meets the sustained peak
+    tc_peak = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
+    alg = [algorithmic(shape, u, int8) for u in used]
     gu_ms = sum(stages["gate_up"])
+    gu_bytes = sum(a["gate_up_bytes"] for a in alg)
+    gu_flops = sum(a["gate_up_flops"] for a in alg)
     gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
+    gu_tf = gu_flops / (gu_ms * 1e-3) / 1e12
     blk_bytes = sum(a["bytes"] for a in alg) / K
     blk_flops = sum(a["flops"] for a in alg) / K
     ms_step = t_max / K
-    prefill = T >= 1024
-    if prefill:
-        gu_tf = sum(a["gate_up_flops"] for a in alg) / (gu_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(gu_tf, 2), "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": round(gu_tf / pk["bf16_tflops"], 4), "traffic": None,
-                "kernel": "grouped_gemm_kernel (gate_up launch)",
-                "peak_source": f"bf16_tflops of {pk['source']} peaks"}
+    gu_t_hbm = gu_bytes / (pk["hbm_gbs"] * 1e9)
+    gu_t_tc = gu_flops / (tc_peak * 1e12)
+    kern = "grouped_gemm_kernel (gate_up launch" + (", int8 converter variant)" if int8 else ")")
+    if gu_t_tc > gu_t_hbm:
+        roof = {"bound": "tensor", "achieved": round(gu_tf, 2), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(gu_tf / tc_peak, 4), "traffic": None,
+                "kernel": kern,
+                "peak_source": ("bf16_tflops_sustained" if long_step else "bf16_tflops")
+                               + f" of {pk['source']} peaks"}
     else:
+        summary = {(8, False): "grouped_gemm_gate_up_decode_T8.md"}.get((T, int8))
         roof = {"bound": "hbm", "achieved": round(gu_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gu_gbs / pk["hbm_gbs"], 4),
-                "traffic": ncu_traffic("grouped_gemm_gate_up_decode_T8.md") if T == 8 else None,
-                "kernel": "grouped_gemm_kernel (gate_up launch)",
-                "peak_source": f"hbm_gbs of {pk['source']} peaks"}
+                "traffic": ncu_traffic(summary) if summary else None,
+                "kernel": kern, "peak_source": f"hbm_gbs of {pk['source']} peaks"}
     t_hbm = blk_bytes / (pk["hbm_gbs"] * 1e9)
-    t_tc = blk_flops / (pk["bf16_tflops"] * 1e12)
+    t_tc = blk_flops / (tc_peak * 1e12)
     block_roof = {"bytes_per_step": int(blk_bytes), "flops_per_step": int(blk_flops),
                   "hbm_frac": round(t_hbm / (ms_step * 1e-3), 4),
                   "tc_frac": round(t_tc / (ms_step * 1e-3), 4),
                   "binding_frac": round(max(t_hbm, t_tc) / (ms_step * 1e-3), 4),
-                  "mean_used_experts": round(sum(used) / K, 2)}
-    launches_per_step = 2 + (1 if T * shape.k <= 8192 else 3) + 1 + 2 + 1
+                  "mean_used_experts": round(sum(used) / len(used), 2)}
+    # router (with the sort when T*k <= 8192, else 3 sort kernels), gather, 2 GEMMs, combine
+    launches_per_call = 5 + (0 if T * shape.k <= 8192 else 3)
     res = {
         "metric": METRIC, "value": round(world * T * K / (t_max * 1e-3), 1), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init weights of the layer's shape)",
         "config": {"workload": wl["name"], "T": T, "H": shape.H, "E": shape.E, "top_k": shape.k,
-                   "expert_inter": shape.I, "dense_inter": shape.D, "expert_weights": "bf16",
-                   "router_bias": ("zipf s=1.1, alpha=%.5f" % alpha) if wl["zipf"] else "none",
-                   "layers_rotated": len(layers),
-                   "l2": "steps rotate over %d distinct layers (%.1f GB of weights) and distinct "
-                         "inputs; no step's weights are L2-resident" %
-                         (len(layers), len(layers) * 3 * shape.E * shape.I * shape.H * 2 / 1e9),
+                   "expert_inter": shape.I, "dense_inter": shape.D,
+                   "expert_weights": "int8 per-channel" if int8 else "bf16",
+                   "router_bias": ("zipf s=1.1, alpha=%.5f" % alpha) if wl.get("zipf") else "none",
+                   "layers": nl, "chained": chain,
+                   "l2": ("steps rotate over %d distinct layers (%.1f GB of weights) and distinct "
+                          "inputs; no step's weights are L2-resident" %
+                          (nl, nl * 3 * shape.E * shape.I * shape.H * (1 if int8 else 2) / 1e9)),
                    "parallelism": f"dp{world} (replicas, no collective)"},
         "roofline": roof,
         "block_roofline": block_roof,
         "stages_ms": {n: round(statistics.mean(v), 5) for n, v in stages.items()},
         "e2e": {"value": round(world * T * K / (te * 1e-3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": launches_per_call * ncalls * K,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(shape, layers[0], xs[W], wl, alpha)
+        res["cpu_baseline"] = cpu_baseline(shape, layers[0], xs[W], wl, alpha, nl if chain else 1)
     return res
 
 
@@ -348,12 +420,21 @@ def _oracle_rows(shape):
     return shape.T if shape.T <= 64 else 64
 
 
-def cpu_baseline(shape, layer, x, wl, alpha, budget_s=15.0):
-    """The oracle, as it stands, on the host cores: tokens/s over a bounded sample."""
+def _oracle_experts(p):
+    import oracle
+    if "s_gate_up" in p:
+        return oracle.Experts(q_gate_up=p["w_gate_up"], s_gate_up=p["s_gate_up"],
+                              q_down=p["w_down"], s_down=p["s_down"])
+    return oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
+
+
+def cpu_baseline(shape, layer, x, wl, alpha, layers_per_step=1, budget_s=15.0):
+    """The oracle, as it stands, on the host cores: tokens/s over a bounded sample.
+    For the chained stack one layer is timed and the rate divided by the layer count."""
     import oracle
     p = _host_layer(layer)
     bias = p.pop("logit_bias", None)
-    ex = oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
+    ex = _oracle_experts(p)
     rows = _oracle_rows(shape)
     xh = x[:rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
     n, t0 = 0, time.perf_counter()
@@ -363,10 +444,12 @@ def cpu_baseline(shape, layer, x, wl, alpha, budget_s=15.0):
         el = time.perf_counter() - t0
         if el > budget_s or n >= 200:
             break
-    return {"value": round(n * rows / el, 3), "unit": UNIT, "cores": _blas_threads(),
-            "kind": "oracle",
+    extra = (f"; one layer timed, rate divided by {layers_per_step} layers"
+             if layers_per_step > 1 else "")
+    return {"value": round(n * rows / el / layers_per_step, 3), "unit": UNIT,
+            "cores": _blas_threads(), "kind": "oracle",
             "sample": f"{n} oracle block calls of {rows} tokens of the {wl['name']} workload "
-                      f"(layer 0), {el:.1f} s"}
+                      f"(layer 0), {el:.1f} s{extra}"}
 
 
 def run_reference(args, wl, rank, world):
@@ -376,12 +459,18 @@ def run_reference(args, wl, rank, world):
     shape = wl["shape"]
     layer = synth.torch_layer(shape, 1234, 0, "cpu")
     alpha = None
-    if wl["zipf"]:
+    if wl.get("zipf"):
         with open(ZIPF_ALPHA_FILE) as f:
             alpha = float(json.load(f)["alpha"])
     p = _host_layer(layer)
-    bias = synth.zipf_bias(1234, shape.E, alpha) if wl["zipf"] else None
-    ex = oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
+    bias = synth.zipf_bias(1234, shape.E, alpha) if wl.get("zipf") else None
+    if wl.get("int8"):
+        qg, sg = oracle.quantize_int8_per_channel(p["w_gate_up"])
+        qd, sd = oracle.quantize_int8_per_channel(p["w_down"])
+        ex = oracle.Experts(q_gate_up=qg, s_gate_up=sg, q_down=qd, s_down=sd)
+    else:
+        ex = oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
+    per_step = wl["layers"] if wl.get("chain") else 1
     rows = _oracle_rows(shape)
     xs = [synth.torch_x(shape, 1234, i, "cpu")[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
           for i in range(args.warmup + args.steps)]
@@ -391,8 +480,9 @@ def run_reference(args, wl, rank, world):
     for i in range(args.steps):
         oracle.block_forward(xs[args.warmup + i], p, ex, shape.k, shape.eps, bias)
     el = time.perf_counter() - t0
-    v = round(args.steps * rows / el, 3)
-    sample = f"{args.steps} timed oracle block calls of {rows} tokens each ({wl['name']})"
+    v = round(args.steps * rows / el / per_step, 3)
+    sample = f"{args.steps} timed oracle block calls of {rows} tokens each ({wl['name']})" + (
+        f"; one layer per call, rate divided by {per_step} layers" if per_step > 1 else "")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

@@ -34,6 +34,8 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
   __shared__ float red[kCombMaxThreads / 32];
   const int t = blockIdx.x;
   const int c = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const bool on = c < (H >> 3);
   float m[8], d[8];
 #pragma unroll
@@ -95,6 +97,8 @@ __global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
                                                           const uint16_t* __restrict__ y,
                                                           uint16_t* __restrict__ moe_out) {
   const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   for (int c = threadIdx.x; c < (H >> 3); c += 256) {
     float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < k; ++j) {
@@ -111,17 +115,15 @@ cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t*
                                  const uint16_t* y, const uint16_t* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, bool pdl) {
   const int threads = ((H >> 3) + 31) / 32 * 32;
-  combine_block_kernel<<<T, threads, 0, s>>>(H, k, eps, x, y, dense, g_post_moe, g_post_dense,
-                                             g_post_ff, out, moe_out);
-  return cudaGetLastError();
+  return launch_k(combine_block_kernel, dim3(T), dim3(threads), 0, s, pdl, H, k, eps, x, y, dense,
+                  g_post_moe, g_post_dense, g_post_ff, out, moe_out);
 }
 
 cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, uint16_t* moe_out,
-                               cudaStream_t s) {
-  combine_moe_kernel<<<T, 256, 0, s>>>(H, k, y, moe_out);
-  return cudaGetLastError();
+                               cudaStream_t s, bool pdl) {
+  return launch_k(combine_moe_kernel, dim3(T), dim3(256), 0, s, pdl, H, k, y, moe_out);
 }
 
 }  // namespace moe

@@ -36,6 +36,7 @@ namespace moe {
 constexpr int kMaxSplit = 4;       // K pieces per tile at most
 constexpr int kMaxEntries = 258;   // groups of problem 0 (<= 256) + problem 1 (1) + 1
 constexpr int kConvWarp0 = 10;     // first converter warp of the int8 variant
+constexpr int kConvWarps = 4;      // converter warps, 32 rows of the 128-row tile each
 
 // W8 = false: the A tile (weights, bf16) goes from HBM to shared memory by TMA, already
 //   in the 128-byte-swizzled K-major layout the MMA reads.
@@ -65,7 +66,10 @@ struct Cfg {
   static constexpr int kTabInts = 4 * kMaxEntries;  // pre, cnt, b0, ng
   static constexpr int kXchgOff = ((kPreOff + kTabInts * 4) + 15) & ~15;
   static constexpr int kXchgBytes = 2 * 16 * 64 * 4;  // one per epilogue group
-  static constexpr int kSmem = kXchgOff + kXchgBytes + 1024;  // + alignment slack
+  // per epilogue group: each column's output row and routing weight (down launches)
+  static constexpr int kRouteOff = kXchgOff + kXchgBytes;
+  static constexpr int kRouteBytes = 2 * BN * 8;
+  static constexpr int kSmem = kRouteOff + kRouteBytes + 1024;  // + alignment slack
   static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(kSmem <= 232448, "shared memory");
 };
@@ -79,13 +83,20 @@ __device__ __forceinline__ float i8_to_f32(uint32_t biased_word, uint32_t byte) 
          8388736.0f;
 }
 
-// Row `r` of the converted tile: 64 K values as 8 chunks of 16 bytes, chunk c stored at
-// chunk position c ^ (r % 8) (the 128-byte swizzle, for a 1024-byte-aligned tile).
-__device__ __forceinline__ void convert_row_i8(const uint8_t* src, uint8_t* dst, int r) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
+// A converter warp owns 32 rows of the tile.  Its lanes read the warp's slice of the raw
+// tile contiguously (16 bytes per lane per step, conflict-free), so a lane converts a
+// piece of a row; the converted row r keeps the 128-byte swizzle of the MMA operand:
+// 16-byte chunk c of row r at chunk position c ^ (r % 8) (1024-byte-aligned tile).
+//   int8 raw rows are 64 bytes: step j, lane l -> row 8j + l/4, codes 16*(l%4)..+15,
+//     i.e. output chunks 2*(l%4) and 2*(l%4)+1.
+//   bf16 raw rows are 128 bytes: step j, lane l -> row 4j + l/8, chunk l%8.
+__device__ __forceinline__ void convert_rows_i8(const uint8_t* raw, uint8_t* conv, int row0,
+                                                int lane) {
 #pragma unroll
-  for (int h = 0; h < 4; ++h) {
-    const uint4 q = s[h];
+  for (int j = 0; j < 4; ++j) {
+    const uint4 q = *reinterpret_cast<const uint4*>(raw + (row0 * 64) + 512 * j + 16 * lane);
+    const int r = row0 + 8 * j + (lane >> 2);
+    const int c0 = 2 * (lane & 3);
     const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u,
                            q.w ^ 0x80808080u};
     uint32_t o[8];
@@ -94,19 +105,24 @@ __device__ __forceinline__ void convert_row_i8(const uint8_t* src, uint8_t* dst,
       o[2 * i] = pack2(i8_to_f32(w[i], 0), i8_to_f32(w[i], 1));
       o[2 * i + 1] = pack2(i8_to_f32(w[i], 2), i8_to_f32(w[i], 3));
     }
-    const int c0 = 2 * h, c1 = 2 * h + 1;
-    *reinterpret_cast<uint4*>(dst + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(dst + ((c1 ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+    uint8_t* row = conv + r * 128;
+    *reinterpret_cast<uint4*>(row + (((c0) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 
-__device__ __forceinline__ void convert_row_bf16(const uint8_t* src, uint8_t* dst, int r) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
+__device__ __forceinline__ void convert_rows_bf16(const uint8_t* raw, uint8_t* conv, int row0,
+                                                  int lane) {
   uint4 v[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) v[c] = s[c];
+  for (int j = 0; j < 8; ++j)
+    v[j] = *reinterpret_cast<const uint4*>(raw + (row0 * 128) + 512 * j + 16 * lane);
 #pragma unroll
-  for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + ((c ^ (r & 7)) << 4)) = v[c];
+  for (int j = 0; j < 8; ++j) {
+    const int r = row0 + 4 * j + (lane >> 3);
+    const int c = lane & 7;
+    *reinterpret_cast<uint4*>(conv + r * 128 + ((c ^ (r & 7)) << 4)) = v[j];
+  }
 }
 
 struct Piece {
@@ -166,7 +182,6 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 0);
   volatile int* abort_flag = misc + 1;
   volatile int* bcast = misc + 2;        // [2], one per epilogue group
-  volatile int* conv_flag = misc + 4;    // converter warps
   int* pre = reinterpret_cast<int*>(smem + C::kPreOff);
   int* cnt = pre + kMaxEntries;
   int* b0 = cnt + kMaxEntries;
@@ -180,10 +195,11 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], W8 ? 2 : 1);  // W8: the MMA (B) and the converters (raw A)
+      // W8: the stage is free once the MMA (B) and every converter warp (raw A) are done
+      mbar_init(&empty[i], W8 ? 1 + kConvWarps : 1);
     }
     for (int i = 0; i < C::kConv; ++i) {
-      mbar_init(&conv_full[i], 1);
+      mbar_init(&conv_full[i], kConvWarps);
       mbar_init(&conv_empty[i], 1);
     }
     for (int i = 0; i < C::kAcc; ++i) {
@@ -204,6 +220,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
+  // everything above overlaps the previous kernel on the stream; its results (routing,
+  // gathered rows, h) are read only below
+  pdl_wait();
+  pdl_trigger();
   for (int i = threadIdx.x; i < nent; i += C::kThreads) {
     const int p = i < P.prob[0].groups ? 0 : 1;
     const int g = p == 0 ? i : i - P.prob[0].groups;
@@ -363,35 +383,39 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     }
   } else if (W8 && warp >= kConvWarp0) {
     // ================= converters (W8): raw A stage -> swizzled bf16 stage ============
-    const int ct = threadIdx.x - kConvWarp0 * 32;  // the row of the tile this thread owns
+    // Each warp owns 32 rows of the tile (one per lane) and runs on its own: an elected
+    // lane waits for the raw stage and a free converted stage, the warp converts, fences
+    // its writes to the async proxy, and lane 0 arrives for the warp.
     int stage = 0;
     uint32_t phase = 0;
     int cs = 0;
     uint32_t cph = 0;
-    for (int piece = blockIdx.x; piece < total; piece += gridDim.x) {
+    bool ok = true;
+    for (int piece = blockIdx.x; piece < total && ok; piece += gridDim.x) {
       const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
       const bool i8 = P.prob[pc.p].w8 != 0;
-      bool ok = true;
       for (int ks = pc.k0; ks < pc.k1; ++ks) {
-        if (ct == 0)
-          *conv_flag = (mbar_wait(&full[stage], phase, tmo, abort_flag) &&
-                        mbar_wait(&conv_empty[cs], cph ^ 1u, tmo, abort_flag))
-                           ? 1
-                           : 0;
-        named_sync(3, 128);
-        if (!*conv_flag) {
+        int good = 1;
+        if (lane == 0)
+          good = (mbar_wait(&full[stage], phase, tmo, abort_flag) &&
+                  mbar_wait(&conv_empty[cs], cph ^ 1u, tmo, abort_flag))
+                     ? 1
+                     : 0;
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) {
           ok = false;
           break;
         }
         const uint8_t* raw = smem + stage * C::kStage;
-        uint8_t* dst = smem + C::kConvOff + cs * C::kABytes + ct * 128;
+        uint8_t* conv = smem + C::kConvOff + cs * C::kABytes;
+        const int row0 = (warp - kConvWarp0) * 32;
         if (i8)
-          convert_row_i8(raw + ct * 64, dst, ct);
+          convert_rows_i8(raw, conv, row0, lane);
         else
-          convert_row_bf16(raw + ct * 128, dst, ct);
+          convert_rows_bf16(raw, conv, row0, lane);
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-        named_sync(3, 128);
-        if (ct == 0) {
+        __syncwarp();
+        if (lane == 0) {
           mbar_arrive(&conv_full[cs]);
           mbar_arrive(&empty[stage]);
         }
@@ -404,13 +428,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
           cph ^= 1u;
         }
       }
-      if (!ok) {
-        if (ct == 0) {
-          record_status(P.status, kStatusTimeout);
-          *abort_flag = 1;
-        }
-        break;
-      }
+    }
+    if (!ok && lane == 0) {
+      record_status(P.status, kStatusTimeout);
+      *abort_flag = 1;
     }
   } else {
     // ================= epilogue: two groups of 4 warps take alternate pieces ============
@@ -423,6 +444,8 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     const uint32_t bar = 1 + grp;
     volatile int* gb = bcast + grp;
     float* xg = xchg + grp * 16 * 64;
+    int* col_row = reinterpret_cast<int*>(smem + C::kRouteOff) + grp * 2 * BN;  // [BN]
+    float* col_w = reinterpret_cast<float*>(col_row + BN);                       // [BN]
     int local = 0;
     for (int piece = blockIdx.x; piece < total; piece += gridDim.x, ++local) {
       if ((local & 1) != grp) continue;
@@ -465,6 +488,18 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
         last = *gb != 0;
       }
       if (last) {
+        if (pr.kind == 1) {
+          // stage the tile's output rows and routing weights once (no global loads in
+          // the column loop below)
+          for (int c = et; c < pc.n_valid; c += 128) {
+            const int pos = pc.b_row0 + pc.n * BN + c;
+            int orow = pr.out_rows ? pr.out_rows[pos] : pos;
+            if (orow < 0 || orow >= pr.n_tokens) orow = -1;
+            col_row[c] = orow;
+            col_w[c] = (orow >= 0 && pr.route_w) ? pr.route_w[orow] : 1.f;
+          }
+          named_sync(bar, 128);
+        }
         const int out_col0 = pc.m * (pr.kind == 0 ? 64 : 128);
         float sc = 1.f;
         if (pr.wscale) {
@@ -523,13 +558,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
             for (int i = 0; i < 16; ++i) {
               const int col = c0 + i;
               if (col < pc.n_valid) {
-                const int pos = pc.b_row0 + pc.n * BN + col;
-                const int orow = pr.out_rows ? pr.out_rows[pos] : pos;
-                if (orow >= 0 && orow < pr.n_tokens) {
-                  const float w = pr.route_w ? pr.route_w[orow] : 1.f;
+                const int orow = col_row[col];
+                if (orow >= 0)
                   pr.out[static_cast<size_t>(orow) * pr.out_ld + out_col0 + row] =
-                      bf16_bits(v[i] * sc * w);
-                }
+                      bf16_bits(v[i] * sc * col_w[col]);
               }
             }
           }
@@ -551,31 +583,33 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
 }
 
 template <int BN, bool W8>
-static cudaError_t launch_bn(const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s) {
+static cudaError_t launch_bn(const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s,
+                             bool pdl) {
   using C = Cfg<BN, W8>;
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, W8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<BN, W8><<<grid, C::kThreads, C::kSmem, s>>>(maps, p);
-  return cudaGetLastError();
+  return launch_k(grouped_gemm_kernel<BN, W8>, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl,
+                  maps, p);
 }
 
 template <bool W8>
 static cudaError_t launch_w(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
-                            cudaStream_t s) {
+                            cudaStream_t s, bool pdl) {
   switch (bn) {
-    case 16: return launch_bn<16, W8>(maps, p, grid, s);
-    case 32: return launch_bn<32, W8>(maps, p, grid, s);
-    case 64: return launch_bn<64, W8>(maps, p, grid, s);
-    case 128: return launch_bn<128, W8>(maps, p, grid, s);
-    case 256: return launch_bn<256, W8>(maps, p, grid, s);
+    case 16: return launch_bn<16, W8>(maps, p, grid, s, pdl);
+    case 32: return launch_bn<32, W8>(maps, p, grid, s, pdl);
+    case 64: return launch_bn<64, W8>(maps, p, grid, s, pdl);
+    case 128: return launch_bn<128, W8>(maps, p, grid, s, pdl);
+    case 256: return launch_bn<256, W8>(maps, p, grid, s, pdl);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
-                                cudaStream_t s) {
-  return p.int8_weights ? launch_w<true>(bn, maps, p, grid, s) : launch_w<false>(bn, maps, p, grid, s);
+                                cudaStream_t s, bool pdl) {
+  return p.int8_weights ? launch_w<true>(bn, maps, p, grid, s, pdl)
+                        : launch_w<false>(bn, maps, p, grid, s, pdl);
 }
 
 }  // namespace moe

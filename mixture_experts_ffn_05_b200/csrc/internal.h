@@ -48,7 +48,28 @@ struct GemmMaps {
   CUtensorMap b[2];  // tokens of problem map 0 / 1
 };
 
-// kernels/*.cu launchers.  All return cudaSuccess or the launch error.
+// Launches kernel<<<grid, block, smem, s>>>(args...).  With pdl the launch is a
+// programmatic dependent of the previous kernel on s: it may start (and run its setup)
+// before that kernel ends, and waits in pdl_wait() before reading its results.  The
+// first kernel of every entry point is launched without it, so that nothing overlaps
+// work that an earlier call left on the stream.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Launchers.  All return cudaSuccess or the launch error.
 // Router + pre norms + top-k in one launch; when offsets != NULL (and T*k fits the
 // single-block sort, see permute_blocks) also the token-to-expert counting sort.
 // counters: router_counters(T) words, zero on entry (left zero on exit).
@@ -58,22 +79,24 @@ cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t*
                           const uint16_t* g_pre_moe, const uint16_t* g_pre_dense,
                           uint16_t* xn_moe, uint16_t* xn_dense, float* logits, int* topk_idx,
                           float* topk_w, unsigned* counters, int* offsets, int* sorted_src,
-                          int* inv_pos, cudaStream_t s);
+                          int* inv_pos, cudaStream_t s, bool pdl = false);
 int router_counters(int T);
 cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int* sorted_src,
-                           int* inv_pos, int* block_hist, int* block_base, cudaStream_t s);
+                           int* inv_pos, int* block_hist, int* block_base, cudaStream_t s,
+                           bool pdl = false);
 int permute_blocks(int n);  // blocks of the multi-block path (0 = single-block path)
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
-                               const uint16_t* src, uint16_t* dst, cudaStream_t s);
+                               const uint16_t* src, uint16_t* dst, cudaStream_t s,
+                               bool pdl = false);
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
-                                cudaStream_t s);
+                                cudaStream_t s, bool pdl = false);
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
                                  const uint16_t* y, const uint16_t* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
-                                 cudaStream_t s);
+                                 cudaStream_t s, bool pdl = false);
 cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, uint16_t* moe_out,
-                               cudaStream_t s);
+                               cudaStream_t s, bool pdl = false);
 cudaError_t launch_quantize_int8(const uint16_t* w, int64_t rows, int cols, int8_t* q,
                                  float* scales, cudaStream_t s);
 

@@ -305,10 +305,12 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     mgu.a[1] = mgu.a[0]; mgu.b[1] = mgu.b[0];
     mdn.a[1] = mdn.a[0]; mdn.b[1] = mdn.b[0];
   }
-  moe_status_t st = cuda_status(launch_grouped_gemm(L.bn, mgu, gu, grid, s));
+  // after a memset the gate_up launch is ordinary; after a kernel it overlaps that
+  // kernel's tail (programmatic dependent launch)
+  moe_status_t st = cuda_status(launch_grouped_gemm(L.bn, mgu, gu, grid, s, !clear));
   if (st != MOE_OK) return st;
   if (!mark(ev, 5, s)) return MOE_ERR_CUDA;
-  st = cuda_status(launch_grouped_gemm(L.bn, mdn, dn, grid, s));
+  st = cuda_status(launch_grouped_gemm(L.bn, mdn, dn, grid, s, true));
   if (st != MOE_OK) return st;
   return mark(ev, 6, s) ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -422,7 +424,7 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   j.topk_w = topk_w;
   j.y = y;
   if ((st = run_gemms(d, L, ws, j, s, true)) != MOE_OK) return st;
-  return cuda_status(launch_combine_moe(d.T, d.H, d.k, y, moe_out, s));
+  return cuda_status(launch_combine_moe(d.T, d.H, d.k, y, moe_out, s, true));
 }
 
 moe_status_t dense_mlp_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* xn_dense,
@@ -496,10 +498,11 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   if (!mark(ev, 1, s)) return MOE_ERR_CUDA;
   if (!fused_sort &&
       (st = cuda_status(launch_permute(Tk, d.E, topk_idx, offsets, sorted, inv, at<int>(ws, L.bhist),
-                                       at<int>(ws, L.bbase), s))) != MOE_OK)
+                                       at<int>(ws, L.bbase), s, true))) != MOE_OK)
     return st;
   if (!mark(ev, 2, s)) return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe, aperm, s))) != MOE_OK)
+  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe, aperm, s, true))) !=
+      MOE_OK)
     return st;
   if (!mark(ev, 3, s)) return MOE_ERR_CUDA;
   GemmJob j{};
@@ -520,8 +523,8 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   j.dense_out = dense;
   if ((st = run_gemms(d, L, ws, j, s, false, ev)) != MOE_OK) return st;
   if ((st = cuda_status(launch_combine_block(d.T, d.H, d.k, d.eps, x, y, dense, w->g_post_moe,
-                                             w->g_post_dense, w->g_post_ff, out, moe_out, s))) !=
-      MOE_OK)
+                                             w->g_post_dense, w->g_post_ff, out, moe_out, s,
+                                             true))) != MOE_OK)
     return st;
   return mark(ev, 7, s) ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_small_kernel(
     int n, int E, const int* __restrict__ idx, int* __restrict__ offsets,
     int* __restrict__ sorted_src, int* __restrict__ inv_pos) {
   __shared__ PermuteSmem<kPermThreads> s;
+  pdl_wait();
+  pdl_trigger();
   permute_block<kPermThreads>(n, E, idx, offsets, sorted_src, inv_pos, s);
 }
 
@@ -30,6 +32,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(int n, int E
                                                                     int* __restrict__ block_hist) {
   __shared__ int cnt[kPermMaxE];
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
   __syncthreads();
   const int p0 = blockIdx.x * kPermPerBlock;
@@ -50,6 +54,8 @@ __global__ void __launch_bounds__(kPermMaxE) permute_scan_kernel(int nb, int E,
   __shared__ int tot[kPermMaxE];
   __shared__ int off[kPermMaxE + 1];
   const int e = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (e < E) {
     int s = 0;
     for (int b = 0; b < nb; ++b) s += block_hist[b * E + e];
@@ -75,6 +81,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
     int* __restrict__ sorted_src, int* __restrict__ inv_pos) {
   __shared__ int base[kPermMaxE];
   __shared__ int wcnt[kPermThreads / 32][kPermMaxE];
+  pdl_wait();
+  pdl_trigger();
   for (int e = threadIdx.x; e < E; e += kPermThreads) base[e] = block_base[blockIdx.x * E + e];
   __syncthreads();
   const int p0 = blockIdx.x * kPermPerBlock;
@@ -87,17 +95,20 @@ int permute_blocks(int n) {
 }
 
 cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int* sorted_src,
-                           int* inv_pos, int* block_hist, int* block_base, cudaStream_t s) {
+                           int* inv_pos, int* block_hist, int* block_base, cudaStream_t s,
+                           bool pdl) {
   const int nb = permute_blocks(n);
-  if (nb == 0) {
-    permute_small_kernel<<<1, kPermThreads, 0, s>>>(n, E, topk_idx, offsets, sorted_src, inv_pos);
-    return cudaGetLastError();
-  }
-  permute_hist_kernel<<<nb, kPermThreads, 0, s>>>(n, E, topk_idx, block_hist);
-  permute_scan_kernel<<<1, kPermMaxE, 0, s>>>(nb, E, block_hist, block_base, offsets);
-  permute_scatter_kernel<<<nb, kPermThreads, 0, s>>>(n, E, topk_idx, block_base, sorted_src,
-                                                     inv_pos);
-  return cudaGetLastError();
+  if (nb == 0)
+    return launch_k(permute_small_kernel, dim3(1), dim3(kPermThreads), 0, s, pdl, n, E, topk_idx,
+                    offsets, sorted_src, inv_pos);
+  cudaError_t e = launch_k(permute_hist_kernel, dim3(nb), dim3(kPermThreads), 0, s, pdl, n, E,
+                           topk_idx, block_hist);
+  if (e != cudaSuccess) return e;
+  e = launch_k(permute_scan_kernel, dim3(1), dim3(kPermMaxE), 0, s, true, nb, E,
+               (const int*)block_hist, block_base, offsets);
+  if (e != cudaSuccess) return e;
+  return launch_k(permute_scatter_kernel, dim3(nb), dim3(kPermThreads), 0, s, true, n, E, topk_idx,
+                  (const int*)block_base, sorted_src, inv_pos);
 }
 
 // dst[q] = src[sorted_src[q] / k] for the n sorted pairs; one thread per 16 bytes.
@@ -107,6 +118,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(int n, int k, int H, i
                                                           const uint16_t* __restrict__ src,
                                                           uint16_t* __restrict__ dst) {
   const int nch = H >> 3;
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   if (i >= static_cast<int64_t>(n) * nch) return;
   const int q = static_cast<int>(i / nch), c = static_cast<int>(i % nch);
@@ -118,11 +131,10 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(int n, int k, int H, i
 }
 
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
-                               const uint16_t* src, uint16_t* dst, cudaStream_t s) {
+                               const uint16_t* src, uint16_t* dst, cudaStream_t s, bool pdl) {
   const int64_t total = static_cast<int64_t>(n) * (H >> 3);
-  gather_rows_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(n, k, H, T, sorted_src,
-                                                                               src, dst);
-  return cudaGetLastError();
+  return launch_k(gather_rows_kernel, dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256),
+                  0, s, pdl, n, k, H, T, sorted_src, src, dst);
 }
 
 }  // namespace moe

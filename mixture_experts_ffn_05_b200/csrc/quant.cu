@@ -14,6 +14,7 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(int64_t rows, int co
                                                             int8_t* __restrict__ q,
                                                             float* __restrict__ scales) {
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  pdl_wait();
   if (r >= rows) return;
   const int lane = threadIdx.x & 31;
   const uint4* wr = reinterpret_cast<const uint4*>(w + r * cols);

@@ -107,6 +107,8 @@ __global__ void __launch_bounds__(kRThreads) router_kernel(const RouterArgs a) {
   const int H = a.H, E = a.E;
   const int t0 = blockIdx.x * kRT;
   const int nch = H >> 3;  // chunks of 8 values
+  pdl_wait();
+  pdl_trigger();
 
   // ---- normalise the CTA's tokens into z; the first expert slice writes the pre norms
   {
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(kRThreads) router_kernel(const RouterArgs a) {
 }
 
 template <int EB>
-static cudaError_t launch_eb(const RouterArgs& a, cudaStream_t s) {
+static cudaError_t launch_eb(const RouterArgs& a, cudaStream_t s, bool pdl) {
   const size_t smem = static_cast<size_t>(kRT) * a.H * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(router_kernel<EB>,
@@ -272,8 +274,7 @@ static cudaError_t launch_eb(const RouterArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   dim3 grid((a.T + kRT - 1) / kRT, (a.E + EB - 1) / EB);
-  router_kernel<EB><<<grid, kRThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(router_kernel<EB>, grid, dim3(kRThreads), smem, s, pdl, a);
 }
 
 int router_counters(int T) { return (T + kRT - 1) / kRT + 1; }
@@ -284,14 +285,14 @@ cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t*
                           const uint16_t* g_pre_moe, const uint16_t* g_pre_dense,
                           uint16_t* xn_moe, uint16_t* xn_dense, float* logits, int* topk_idx,
                           float* topk_w, unsigned* counters, int* offsets, int* sorted_src,
-                          int* inv_pos, cudaStream_t s) {
+                          int* inv_pos, cudaStream_t s, bool pdl) {
   RouterArgs a{T, H, E, k, eps, 1.0f / sqrtf(static_cast<float>(H)), x, router_scale, w_router,
                bias, per_expert_scale, g_pre_moe, g_pre_dense, xn_moe, xn_dense, logits,
                topk_idx, topk_w, counters, offsets, sorted_src, inv_pos};
   // Narrow expert slices for small batches (more CTAs streaming W_r), wide ones for
   // large batches (fewer redundant normalisations).
-  if (T <= 64) return launch_eb<4>(a, s);
-  return launch_eb<32>(a, s);
+  if (T <= 64) return launch_eb<4>(a, s, pdl);
+  return launch_eb<32>(a, s, pdl);
 }
 
 }  // namespace moe
