@@ -13,49 +13,68 @@ namespace moe {
 
 constexpr int kCombMaxThreads = 768;  // H <= 6144: one 8-column chunk per thread
 
-// Block reduction in a fixed order (deterministic).  nthreads is a multiple of 32.
-__device__ __forceinline__ float block_sum(float v, float* red) {
-  v = warp_sum(v);
+// Sums of two values over the block in a fixed order (deterministic).
+__device__ __forceinline__ float2 block_sum2(float a, float b, float2* red) {
+  a = warp_sum(a);
+  b = warp_sum(b);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __syncthreads();  // red may still be read by a previous call
-  if (lane == 0) red[warp] = v;
+  if (lane == 0) red[warp] = make_float2(a, b);
   __syncthreads();
-  float s = 0.f;
-  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) s += red[w];
+  float2 s = make_float2(0.f, 0.f);
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+    s.x += red[w].x;
+    s.y += red[w].y;
+  }
   return s;
 }
 
-// One CTA per token, one 8-column chunk per thread.
+// One CTA per token, one 8-column chunk per thread; every input is requested before
+// the first reduction.
 __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
     int H, int k, float eps, const uint16_t* __restrict__ x, const uint16_t* __restrict__ y,
     const uint16_t* __restrict__ dense, const uint16_t* __restrict__ g_pm,
     const uint16_t* __restrict__ g_pd, const uint16_t* __restrict__ g_ff,
     uint16_t* __restrict__ out, uint16_t* __restrict__ moe_out) {
-  __shared__ float red[kCombMaxThreads / 32];
+  __shared__ float2 red[kCombMaxThreads / 32];
   const int t = blockIdx.x;
   const int c = threadIdx.x;
+  const bool on = c < (H >> 3);
+  const int cc = on ? c : 0;
+  // inputs that do not depend on the previous kernel: gains and the residual
+  uint4 vgd = make_uint4(0u, 0u, 0u, 0u), vgm = vgd, vgf, vx;
+  if (g_pd) vgd = __ldg(reinterpret_cast<const uint4*>(g_pd) + cc);
+  if (g_pm) vgm = __ldg(reinterpret_cast<const uint4*>(g_pm) + cc);
+  vgf = __ldg(reinterpret_cast<const uint4*>(g_ff) + cc);
+  vx = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + cc);
   pdl_wait();
   pdl_trigger();
-  const bool on = c < (H >> 3);
   float m[8], d[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = d[i] = 0.f;
-  if (on) {
-    const uint4* yr = reinterpret_cast<const uint4*>(y + static_cast<size_t>(t) * k * H) + c;
-    uint4 buf[16];
+  {
+    const uint4* yr = reinterpret_cast<const uint4*>(y + static_cast<size_t>(t) * k * H) + cc;
+    const uint4 vd = __ldg(reinterpret_cast<const uint4*>(dense + static_cast<size_t>(t) * H) + cc);
+    for (int j0 = 0; j0 < k; j0 += 8) {  // 8 slots in flight at a time, summed in slot order
+      uint4 buf[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k) buf[j] = __ldg(yr + static_cast<size_t>(j) * (H >> 3));
+      for (int j = 0; j < 8; ++j)
+        if (j0 + j < k) buf[j] = __ldg(yr + static_cast<size_t>(j0 + j) * (H >> 3));
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k) {  // slot order j = 0..k-1
-        float f[8];
-        unpack8(buf[j], f);
+      for (int j = 0; j < 8; ++j)
+        if (j0 + j < k) {
+          float f[8];
+          unpack8(buf[j], f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m[i] += f[i];
-      }
-    unpack8(__ldg(reinterpret_cast<const uint4*>(dense + static_cast<size_t>(t) * H) + c), d);
-    if (moe_out) reinterpret_cast<uint4*>(moe_out + static_cast<size_t>(t) * H)[c] = pack8(m);
+          for (int i = 0; i < 8; ++i) m[i] += f[i];
+        }
+    }
+    unpack8(vd, d);
+    if (!on) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = d[i] = 0.f;
+    }
+    if (on && moe_out) reinterpret_cast<uint4*>(moe_out + static_cast<size_t>(t) * H)[c] = pack8(m);
   }
   float ssm = 0.f, ssd = 0.f;
 #pragma unroll
@@ -63,29 +82,25 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
     ssm = fmaf(m[i], m[i], ssm);
     ssd = fmaf(d[i], d[i], ssd);
   }
-  const float rm = g_pm ? 1.0f / sqrtf(block_sum(ssm, red) / H + eps) : 1.f;
-  const float rd = g_pd ? 1.0f / sqrtf(block_sum(ssd, red) / H + eps) : 1.f;
-  float sum[8];
+  const float2 ss = block_sum2(ssm, ssd, red);
+  const float rm = g_pm ? 1.0f / sqrtf(ss.x / H + eps) : 1.f;
+  const float rd = g_pd ? 1.0f / sqrtf(ss.y / H + eps) : 1.f;
+  float sum[8], ga[8], gb[8];
+  unpack8(vgd, ga);
+  unpack8(vgm, gb);
   float ssc = 0.f;
-  {
-    float ga[8], gb[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) ga[i] = gb[i] = 1.f;
-    if (on && g_pd) unpack8(__ldg(reinterpret_cast<const uint4*>(g_pd) + c), ga);
-    if (on && g_pm) unpack8(__ldg(reinterpret_cast<const uint4*>(g_pm) + c), gb);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float a = g_pd ? d[i] * rd * ga[i] : d[i];
-      const float b = g_pm ? m[i] * rm * gb[i] : m[i];
-      sum[i] = a + b;
-      ssc = fmaf(sum[i], sum[i], ssc);
-    }
+  for (int i = 0; i < 8; ++i) {
+    const float av = g_pd ? d[i] * rd * ga[i] : d[i];
+    const float bv = g_pm ? m[i] * rm * gb[i] : m[i];
+    sum[i] = av + bv;
+    ssc = fmaf(sum[i], sum[i], ssc);
   }
-  const float rc = 1.0f / sqrtf(block_sum(ssc, red) / H + eps);
+  const float rc = 1.0f / sqrtf(block_sum2(ssc, 0.f, red).x / H + eps);
   if (on) {
     float xf[8], g[8], o[8];
-    unpack8(__ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + c), xf);
-    unpack8(__ldg(reinterpret_cast<const uint4*>(g_ff) + c), g);
+    unpack8(vx, xf);
+    unpack8(vgf, g);
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i] = xf[i] + sum[i] * rc * g[i];
     reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = pack8(o);

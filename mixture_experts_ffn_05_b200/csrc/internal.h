@@ -78,8 +78,8 @@ cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t*
                           const float* bias, const uint16_t* per_expert_scale,
                           const uint16_t* g_pre_moe, const uint16_t* g_pre_dense,
                           uint16_t* xn_moe, uint16_t* xn_dense, float* logits, int* topk_idx,
-                          float* topk_w, unsigned* counters, int* offsets, int* sorted_src,
-                          int* inv_pos, cudaStream_t s, bool pdl = false);
+                          float* topk_w, unsigned* counters, unsigned* status, int* offsets,
+                          int* sorted_src, int* inv_pos, cudaStream_t s, bool pdl = false);
 int router_counters(int T);
 cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int* sorted_src,
                            int* inv_pos, int* block_hist, int* block_base, cudaStream_t s,

@@ -371,7 +371,8 @@ moe_status_t moe_router(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
   return cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, x, router_scale, w_router,
                                    logit_bias, per_expert_scale, g_pre_moe, g_pre_dense, xn_moe,
                                    xn_dense, at<float>(ws, L.logits), topk_idx, topk_w,
-                                   at<unsigned>(ws, L.rcounters), nullptr, nullptr, nullptr, s));
+                                   at<unsigned>(ws, L.rcounters), at<unsigned>(ws, L.status),
+                                   nullptr, nullptr, nullptr, s));
 }
 
 moe_status_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx,
@@ -492,8 +493,8 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   if ((st = cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, x, w->router_scale, w->w_router,
                                       w->logit_bias, w->per_expert_scale, w->g_pre_moe,
                                       w->g_pre_dense, xn_moe, xn_dense, logits, topk_idx, topk_w,
-                                      at<unsigned>(ws, L.rcounters), fused_sort ? offsets : nullptr,
-                                      sorted, inv, s))) != MOE_OK)
+                                      at<unsigned>(ws, L.rcounters), at<unsigned>(ws, L.status),
+                                      fused_sort ? offsets : nullptr, sorted, inv, s))) != MOE_OK)
     return st;
   if (!mark(ev, 1, s)) return MOE_ERR_CUDA;
   if (!fused_sort &&
