@@ -293,7 +293,7 @@ def run_ours(args, wl, rank, world, device):
     if st != mf.MOE_OK:
         raise RuntimeError(f"device status after the timed region: {mf.status_string(st)}")
     t_ms = e0.elapsed_time(e1)
-    stages = {n: [] for n in ("router", "permute", "gather", "clear", "gate_up", "down", "combine")}
+    stages = {n: [] for n in ("router", "permute", "gather", "gate_up", "down", "combine")}
     for evs in stage_ev:
         for ev in evs:
             for j, n in enumerate(stages):

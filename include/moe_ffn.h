@@ -28,7 +28,11 @@
  *   - Every pointer is device memory owned by the caller, 16-byte aligned, unless
  *     marked "host".  The library never allocates or frees memory in these calls;
  *     scratch comes from the caller's workspace `ws` of `ws_bytes` bytes, which must
- *     be at least moe_workspace_size(cfg, T) and 256-byte aligned.
+ *     be at least moe_workspace_size(cfg, T) and 256-byte aligned.  A new workspace
+ *     must be zeroed once before its first use (e.g. cudaMemsetAsync); every call that
+ *     completes leaves its counters at zero again, so later calls need no clearing.
+ *     After MOE_ERR_DEVICE_TIMEOUT, zero the workspace again.  A workspace that was
+ *     not zeroed gives wrong results, never an out-of-bounds access or a hang.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
  *     only enqueues work on that stream and returns; results are ready when the
  *     stream reaches that point.  Calls on different streams must not share `ws`.
@@ -192,9 +196,9 @@ moe_status_t dense_mlp_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
  *   stage_events: NULL, or a host array of MOE_BLOCK_EVENTS cudaEvent_t that the call
  *   records on `stream` at its stage boundaries, for timing each stage:
  *     [0] start  [1] router done (with the permutation for small batches)
- *     [2] permutation done  [3] row gather done  [4] GEMMs start
- *     [5] gate_up GEMMs done  [6] down GEMMs done  [7] combine done */
-#define MOE_BLOCK_EVENTS 8
+ *     [2] permutation done  [3] row gather done  [4] gate_up GEMMs done
+ *     [5] down GEMMs done  [6] combine done */
+#define MOE_BLOCK_EVENTS 7
 moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
                                const moe_block_weights_t* w, moe_bf16_t* out,
                                moe_bf16_t* moe_out, void* ws, size_t ws_bytes, void* stream,
@@ -215,7 +219,8 @@ moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream);
 /* A short constant English description of a status code. */
 const char* moe_status_string(moe_status_t status);
 
-/* Version of this interface (increases when a signature changes). */
+/* Version of this interface (increases when a signature or a calling contract changes;
+ * 2: the workspace is zeroed once by the caller, MOE_BLOCK_EVENTS is 7). */
 int32_t moe_abi_version(void);
 
 #ifdef __cplusplus

@@ -149,11 +149,12 @@ def workspace_size(cfg: Config, T: int) -> int:
 
 
 def workspace(cfg: Config, T: int, device=None) -> torch.Tensor:
-    """A device buffer of moe_workspace_size bytes (torch allocations are 512-byte aligned)."""
+    """A zeroed device buffer of moe_workspace_size bytes, ready for its first use
+    (torch allocations are 512-byte aligned)."""
     n = workspace_size(cfg, T)
     if n == 0:
         raise MoeError("moe_workspace_size", MOE_ERR_INVALID_ARG)
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
 BF16 = torch.bfloat16
@@ -247,7 +248,7 @@ class BlockWeights:
             vals["w_dense_down"])
 
 
-MOE_BLOCK_EVENTS = 8
+MOE_BLOCK_EVENTS = 7
 
 
 def moe_block_forward(cfg, x, weights: BlockWeights, out, ws, moe_out=None, stream=None,

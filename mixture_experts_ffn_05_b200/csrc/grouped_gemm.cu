@@ -48,17 +48,21 @@ struct Cfg {
   static constexpr int kThreads = W8 ? 448 : 320;  // producer, MMA, 2x4 epilogue (+4 converters)
   static constexpr int kABytes = 128 * 64 * 2;     // bf16 A tile: 128 weight rows x 64 K
   static constexpr int kBBytes = BN * 64 * 2;      // BN token rows x 64 K
-  static constexpr int kStage = kABytes + kBBytes; // (W8: the raw A region has the same size)
-  static constexpr int kStages = W8 ? (BN <= 16 ? 8 : (BN <= 32 ? 7 : (BN <= 64 ? 6 : (BN <= 128 ? 4 : 3))))
+  // W8 stages hold a raw A tile of 16 KB (int8 codes for 128 K, or bf16 for 64 K) and
+  // up to two B tiles (an int8 step covers two 64-wide MMA sub-steps).
+  static constexpr int kBSlots = W8 ? 2 : 1;
+  static constexpr int kStage = kABytes + kBSlots * kBBytes;
+  static constexpr int kStages = W8 ? (BN <= 16 ? 7 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 3 : 2))))
                                     : (BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4)));
-  static constexpr int kConv = W8 ? 4 : 0;          // converted bf16 A stages
+  static constexpr int kConvBytes = 2 * kABytes;   // converted stage: two 64-wide sub-tiles
+  static constexpr int kConv = W8 ? (BN >= 256 ? 1 : 2) : 0;
   // TMEM accumulators: 4 for narrow tiles (the epilogue of a weight-streaming piece is
   // latency-bound and must not hold up the MMAs), 2 for wide ones (512 columns max).
   static constexpr int kAcc = BN <= 64 ? 4 : 2;
   static constexpr int kTmemCols = kAcc * BN < 32 ? 32 : kAcc * BN;
   // after the stages: converted stages, barriers, bookkeeping, the gate/up exchange buffer
   static constexpr int kConvOff = kStages * kStage;
-  static constexpr int kBarOff = kConvOff + kConv * kABytes;
+  static constexpr int kBarOff = kConvOff + kConv * kConvBytes;
   static constexpr int kNumBars = 2 * kStages + 2 * kConv + 2 * kAcc + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kMiscInts = 8;               // tmem slot, abort, bcast x2, converter flag
@@ -85,17 +89,18 @@ __device__ __forceinline__ float i8_to_f32(uint32_t biased_word, uint32_t byte) 
 
 // A converter warp owns 32 rows of the tile.  Its lanes read the warp's slice of the raw
 // tile contiguously (16 bytes per lane per step, conflict-free), so a lane converts a
-// piece of a row; the converted row r keeps the 128-byte swizzle of the MMA operand:
-// 16-byte chunk c of row r at chunk position c ^ (r % 8) (1024-byte-aligned tile).
-//   int8 raw rows are 64 bytes: step j, lane l -> row 8j + l/4, codes 16*(l%4)..+15,
-//     i.e. output chunks 2*(l%4) and 2*(l%4)+1.
-//   bf16 raw rows are 128 bytes: step j, lane l -> row 4j + l/8, chunk l%8.
+// piece of a row; the converted rows keep the 128-byte swizzle of the MMA operand:
+// 16-byte chunk c of row r at chunk position c ^ (r % 8) (1024-byte-aligned sub-tile).
+//   int8 raw rows are 128 codes (two 64-wide sub-tiles): step j, lane l -> row
+//     4j + l/8, codes 16*(l%8)..+15 -> sub-tile (l%8)/4, chunks 2*(l%4) and 2*(l%4)+1.
+//   bf16 raw rows are 64 values (one sub-tile): step j, lane l -> row 4j + l/8, chunk l%8.
 __device__ __forceinline__ void convert_rows_i8(const uint8_t* raw, uint8_t* conv, int row0,
                                                 int lane) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 q = *reinterpret_cast<const uint4*>(raw + (row0 * 64) + 512 * j + 16 * lane);
-    const int r = row0 + 8 * j + (lane >> 2);
+  for (int j = 0; j < 8; ++j) {
+    const uint4 q = *reinterpret_cast<const uint4*>(raw + (row0 * 128) + 512 * j + 16 * lane);
+    const int r = row0 + 4 * j + (lane >> 3);
+    const int sub = (lane & 7) >> 2;
     const int c0 = 2 * (lane & 3);
     const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u,
                            q.w ^ 0x80808080u};
@@ -105,8 +110,8 @@ __device__ __forceinline__ void convert_rows_i8(const uint8_t* raw, uint8_t* con
       o[2 * i] = pack2(i8_to_f32(w[i], 0), i8_to_f32(w[i], 1));
       o[2 * i + 1] = pack2(i8_to_f32(w[i], 2), i8_to_f32(w[i], 3));
     }
-    uint8_t* row = conv + r * 128;
-    *reinterpret_cast<uint4*>(row + (((c0) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    uint8_t* row = conv + sub * (128 * 128) + r * 128;
+    *reinterpret_cast<uint4*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
@@ -293,16 +298,20 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
             break;
           }
           uint8_t* sa = smem + stage * C::kStage;
-          // A bytes: a bf16 tile, or (W8 with int8 weights) a tile of int8 codes
-          const int abytes = (W8 && pr.w8) ? C::kABytes / 2 : C::kABytes;
-          mbar_arrive_expect_tx(&full[stage], abytes + C::kBBytes);
+          // a step covers 64 K (bf16 weights) or 128 K (int8 codes, two B sub-tiles);
+          // the A tile is 16 KB either way
+          const int kw = (W8 && pr.w8) ? 128 : 64;
+          const int nb = kw / 64;
+          mbar_arrive_expect_tx(&full[stage], C::kABytes + nb * C::kBBytes);
           if (pr.kind == 0) {
-            tma_load_2d(sa, ma, &full[stage], ks * 64, arow, pol_w);
-            tma_load_2d(sa + abytes / 2, ma, &full[stage], ks * 64, arow + pr.nw, pol_w);
+            tma_load_2d(sa, ma, &full[stage], ks * kw, arow, pol_w);
+            tma_load_2d(sa + C::kABytes / 2, ma, &full[stage], ks * kw, arow + pr.nw, pol_w);
           } else {
-            tma_load_2d(sa, ma, &full[stage], ks * 64, arow, pol_w);
+            tma_load_2d(sa, ma, &full[stage], ks * kw, arow, pol_w);
           }
-          tma_load_2d(sa + C::kABytes, mb, &full[stage], ks * 64, brow, pol_b);
+          for (int b = 0; b < nb; ++b)
+            tma_load_2d(sa + C::kABytes + b * C::kBBytes, mb, &full[stage], ks * kw + 64 * b, brow,
+                        pol_b);
           armed[stage] = static_cast<int>(phase);
           if (++stage == C::kStages) {
             stage = 0;
@@ -345,12 +354,16 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * C::kStage);
-          const uint32_t sA = W8 ? smem_u32(smem + C::kConvOff + cs * C::kABytes) : sa;
-          const uint64_t ad = sdesc_k_sw128(sA);
-          const uint64_t bd = sdesc_k_sw128(sa + C::kABytes);
+          const uint32_t sA = W8 ? smem_u32(smem + C::kConvOff + cs * C::kConvBytes) : sa;
+          const int nsub = (W8 && P.prob[pc.p].w8) ? 2 : 1;  // 64-wide sub-steps
+          for (int sub = 0; sub < nsub; ++sub) {
+            const uint64_t ad = sdesc_k_sw128(sA + sub * C::kABytes);
+            const uint64_t bd = sdesc_k_sw128(sa + C::kABytes + sub * C::kBBytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (ks > pc.k0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc,
+                        (ks > pc.k0 || sub > 0 || kk > 0) ? 1u : 0u);
+          }
           if (W8) {
             umma_commit(&conv_empty[cs]);
             if (++cs == C::kConv) {
@@ -407,7 +420,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
           break;
         }
         const uint8_t* raw = smem + stage * C::kStage;
-        uint8_t* conv = smem + C::kConvOff + cs * C::kABytes;
+        uint8_t* conv = smem + C::kConvOff + cs * C::kConvBytes;
         const int row0 = (warp - kConvWarp0) * 32;
         if (i8)
           convert_rows_i8(raw, conv, row0, lane);

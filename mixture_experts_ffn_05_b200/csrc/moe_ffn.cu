@@ -83,9 +83,10 @@ Layout layout_of(const Dims& d) {
   Layout L{};
   const int64_t T = d.T, Tk = static_cast<int64_t>(d.T) * d.k;
   L.bn = choose_bn(d);
-  L.split_gu = choose_split(d.H / 64, L.bn);
+  const int kw = d.int8 ? 128 : 64;  // K per pipeline step of the expert GEMMs
+  L.split_gu = choose_split((d.H + kw - 1) / kw, L.bn);
   L.split_dgu = choose_split(d.H / 64, L.bn);
-  L.split_d = choose_split(d.I / 64, L.bn);
+  L.split_d = choose_split((d.I + kw - 1) / kw, L.bn);
   L.split_dd = choose_split(d.D / 64, L.bn);
   // Upper bound of the N tiles: every non-empty expert has a partial tile.
   const int64_t ntl_e = std::min<int64_t>(d.E, Tk) + ceil_div(Tk, L.bn);
@@ -169,14 +170,14 @@ int sm_count() {
   return g_sm_count[dev];
 }
 
-// K-major 2-D map: rows x cols elements, box of 64 K elements x box_rows rows.
+// K-major 2-D map: rows x cols elements, box of 128 bytes of K x box_rows rows.
 bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
                CUtensorMapDataType dt, int elem_bytes, CUtensorMapSwizzle swz) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t es[2] = {1, 1};
   const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -190,7 +191,8 @@ bool encode_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, i
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Raw weight tile for the converter warps: unswizzled rows of int8 codes or bf16 values.
+// Raw weight tile for the converter warps: unswizzled 128-byte rows of int8 codes
+// (128 K) or bf16 values (64 K).
 bool encode_raw(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
                 bool int8) {
   return int8 ? encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
@@ -228,19 +230,15 @@ bool mark(void* const* ev, int i, cudaStream_t s) {
   return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
 }
 
-// Clears the status word and every counter of the workspace.
-moe_status_t clear_counters(const Layout& L, void* ws, cudaStream_t s) {
-  return cudaMemsetAsync(ws, 0, L.counters + L.counters_bytes, s) == cudaSuccess ? MOE_OK
-                                                                                 : MOE_ERR_CUDA;
-}
-
+// The counters in the workspace start at zero (the caller zeroes a new workspace once)
+// and every kernel that uses one returns it to zero, so no call clears them.
+// first_kernel: the gate_up launch is the entry point's first kernel (no dependent
+// launch on whatever the stream ran before).
 moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& j,
-                       cudaStream_t s, bool clear, void* const* ev = nullptr) {
+                       cudaStream_t s, bool first_kernel, void* const* ev = nullptr) {
   const int64_t Tk = static_cast<int64_t>(d.T) * d.k;
   const int grid = sm_count();
   if (grid <= 0) return MOE_ERR_CUDA;
-  if (clear && clear_counters(L, ws, s) != MOE_OK) return MOE_ERR_CUDA;
-  if (!mark(ev, 4, s)) return MOE_ERR_CUDA;
   uint16_t* h = at<uint16_t>(ws, L.h);
   uint16_t* hd = at<uint16_t>(ws, L.hd);
 
@@ -265,15 +263,19 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
   if (j.experts) {
     GemmProblem& a = gu.prob[np];
     a = GemmProblem{};
+    // int8 steps cover 128 K (a ragged last step reads zeros past K through the maps)
+    const int kw = d.int8 ? 128 : 64;
     a.kind = 0; a.groups = d.E; a.offsets = j.offsets; a.n_tokens = static_cast<int>(Tk);
-    a.k_steps = d.H / 64; a.m_tiles = d.I / 64; a.w_rows_per_group = 2 * d.I; a.nw = d.I;
-    a.split = L.split_gu; a.map = np; a.out = h; a.out_ld = d.I; a.wscale = j.s_gate_up;
+    a.k_steps = (d.H + kw - 1) / kw; a.m_tiles = d.I / 64; a.w_rows_per_group = 2 * d.I; a.nw = d.I;
+    a.split = std::min(L.split_gu, a.k_steps); a.map = np; a.out = h; a.out_ld = d.I;
+    a.wscale = j.s_gate_up;
     a.w8 = d.int8;
     GemmProblem& b = dn.prob[np];
     b = GemmProblem{};
     b.kind = 1; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = static_cast<int>(Tk);
-    b.k_steps = d.I / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H; b.nw = 0;
-    b.split = L.split_d; b.map = np; b.out = j.y; b.out_ld = d.H; b.out_rows = j.sorted_src;
+    b.k_steps = (d.I + kw - 1) / kw; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H; b.nw = 0;
+    b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_ld = d.H;
+    b.out_rows = j.sorted_src;
     b.route_w = j.topk_w; b.wscale = j.s_down; b.w8 = d.int8;
     if (!encode_a(&mgu.a[np], j.w_gate_up, static_cast<int64_t>(d.E) * 2 * d.I, d.H, 64, d.int8) ||
         !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, L.bn) ||
@@ -305,14 +307,14 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     mgu.a[1] = mgu.a[0]; mgu.b[1] = mgu.b[0];
     mdn.a[1] = mdn.a[0]; mdn.b[1] = mdn.b[0];
   }
-  // after a memset the gate_up launch is ordinary; after a kernel it overlaps that
-  // kernel's tail (programmatic dependent launch)
-  moe_status_t st = cuda_status(launch_grouped_gemm(L.bn, mgu, gu, grid, s, !clear));
+  // after a kernel of the same entry point the gate_up launch overlaps that kernel's tail
+  // (programmatic dependent launch)
+  moe_status_t st = cuda_status(launch_grouped_gemm(L.bn, mgu, gu, grid, s, !first_kernel));
   if (st != MOE_OK) return st;
-  if (!mark(ev, 5, s)) return MOE_ERR_CUDA;
+  if (!mark(ev, 4, s)) return MOE_ERR_CUDA;
   st = cuda_status(launch_grouped_gemm(L.bn, mdn, dn, grid, s, true));
   if (st != MOE_OK) return st;
-  return mark(ev, 6, s) ? MOE_OK : MOE_ERR_CUDA;
+  return mark(ev, 5, s) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 bool w_ok(const moe_expert_weights_t* w, bool int8) {
@@ -328,7 +330,7 @@ bool w_ok(const moe_expert_weights_t* w, bool int8) {
 
 extern "C" {
 
-int32_t moe_abi_version(void) { return 1; }
+int32_t moe_abi_version(void) { return 2; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -367,7 +369,6 @@ moe_status_t moe_router(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = clear_counters(L, ws, s)) != MOE_OK) return st;
   return cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, x, router_scale, w_router,
                                    logit_bias, per_expert_scale, g_pre_moe, g_pre_dense, xn_moe,
                                    xn_dense, at<float>(ws, L.logits), topk_idx, topk_w,
@@ -424,7 +425,7 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   j.sorted_src = sorted_src;
   j.topk_w = topk_w;
   j.y = y;
-  if ((st = run_gemms(d, L, ws, j, s, true)) != MOE_OK) return st;
+  if ((st = run_gemms(d, L, ws, j, s, false)) != MOE_OK) return st;
   return cuda_status(launch_combine_moe(d.T, d.H, d.k, y, moe_out, s, true));
 }
 
@@ -488,7 +489,6 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
     for (int i = 0; i < MOE_BLOCK_EVENTS; ++i)
       if (ev[i] == nullptr) return MOE_ERR_INVALID_ARG;
   if (!mark(ev, 0, s)) return MOE_ERR_CUDA;
-  if ((st = clear_counters(L, ws, s)) != MOE_OK) return st;
   const bool fused_sort = permute_blocks(Tk) == 0;
   if ((st = cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, x, w->router_scale, w->w_router,
                                       w->logit_bias, w->per_expert_scale, w->g_pre_moe,
@@ -527,7 +527,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
                                              w->g_post_dense, w->g_post_ff, out, moe_out, s,
                                              true))) != MOE_OK)
     return st;
-  return mark(ev, 7, s) ? MOE_OK : MOE_ERR_CUDA;
+  return mark(ev, 6, s) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, int8_t* q,

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
     for s in range(6):
         assert mf.status_string(s)
     assert mf.status_string(99) == "unknown status"
@@ -114,7 +114,8 @@ def test_every_entry_point_validates(lib):
                                  None, None) == mf.MOE_ERR_WORKSPACE
     assert lib.moe_block_forward(c, 0, FAKE, ctypes.byref(bw), FAKE, None, FAKE, n,
                                  None, None) == mf.MOE_OK
-    ev = (ctypes.c_void_p * 8)(*([FAKE] * 7 + [None]))  # an event missing
+    ev = (ctypes.c_void_p * mf.MOE_BLOCK_EVENTS)(*([FAKE] * (mf.MOE_BLOCK_EVENTS - 1) + [None]))
+    # an event missing
     assert lib.moe_block_forward(c, 8, FAKE, ctypes.byref(bw), FAKE, None, FAKE, n,
                                  None, ev) == mf.MOE_ERR_INVALID_ARG
     bw.g_post_moe = FAKE + 4
