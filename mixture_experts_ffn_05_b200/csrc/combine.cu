@@ -5,7 +5,7 @@
 // layernorms" add a post norm on each branch:
 //   m   = sum_{j=0..k-1} Y[t*k + j]          (weights already applied, fixed slot order)
 //   out = x + N_post_ff( N_post_dense(d) + N_post_moe(m) ),  N_g(v) = v / rms(v) * g
-// All sums in fp32; the output is rounded to bf16 once.
+// Y and d arrive in fp32; all sums are fp32 and the output is rounded to bf16 once.
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,11 +29,19 @@ __device__ __forceinline__ float2 block_sum2(float a, float b, float2* red) {
   return s;
 }
 
+// 8 fp32 values from two 16-byte loads.
+__device__ __forceinline__ void load8f(const float* p, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
 // One CTA per token, one 8-column chunk per thread; every input is requested before
 // the first reduction.
 __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
-    int H, int k, float eps, const uint16_t* __restrict__ x, const uint16_t* __restrict__ y,
-    const uint16_t* __restrict__ dense, const uint16_t* __restrict__ g_pm,
+    int H, int k, float eps, const uint16_t* __restrict__ x, const float* __restrict__ y,
+    const float* __restrict__ dense, const uint16_t* __restrict__ g_pm,
     const uint16_t* __restrict__ g_pd, const uint16_t* __restrict__ g_ff,
     uint16_t* __restrict__ out, uint16_t* __restrict__ moe_out) {
   __shared__ float2 red[kCombMaxThreads / 32];
@@ -53,23 +61,20 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = d[i] = 0.f;
   {
-    const uint4* yr = reinterpret_cast<const uint4*>(y + static_cast<size_t>(t) * k * H) + cc;
-    const uint4 vd = __ldg(reinterpret_cast<const uint4*>(dense + static_cast<size_t>(t) * H) + cc);
-    for (int j0 = 0; j0 < k; j0 += 8) {  // 8 slots in flight at a time, summed in slot order
-      uint4 buf[8];
+    const float* yr = y + static_cast<size_t>(t) * k * H + cc * 8;
+    load8f(dense + static_cast<size_t>(t) * H + cc * 8, d);
+    for (int j0 = 0; j0 < k; j0 += 4) {  // 4 slots in flight at a time, summed in slot order
+      float buf[4][8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j0 + j < k) buf[j] = __ldg(yr + static_cast<size_t>(j0 + j) * (H >> 3));
+      for (int j = 0; j < 4; ++j)
+        if (j0 + j < k) load8f(yr + static_cast<size_t>(j0 + j) * H, buf[j]);
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
+      for (int j = 0; j < 4; ++j)
         if (j0 + j < k) {
-          float f[8];
-          unpack8(buf[j], f);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] += f[i];
+          for (int i = 0; i < 8; ++i) m[i] += buf[j][i];
         }
     }
-    unpack8(vd, d);
     if (!on) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) m[i] = d[i] = 0.f;
@@ -109,7 +114,7 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
 
 // moe_out[t] = sum_j Y[t*k + j] in fp32, slot order, rounded to bf16.
 __global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
-                                                          const uint16_t* __restrict__ y,
+                                                          const float* __restrict__ y,
                                                           uint16_t* __restrict__ moe_out) {
   const int t = blockIdx.x;
   pdl_wait();
@@ -118,7 +123,7 @@ __global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
     float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < k; ++j) {
       float f[8];
-      unpack8(__ldg(reinterpret_cast<const uint4*>(y + (static_cast<size_t>(t) * k + j) * H) + c), f);
+      load8f(y + (static_cast<size_t>(t) * k + j) * H + c * 8, f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) m[i] += f[i];
     }
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
 }
 
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
-                                 const uint16_t* y, const uint16_t* dense,
+                                 const float* y, const float* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s, bool pdl) {
@@ -136,7 +141,7 @@ cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t*
                   g_post_moe, g_post_dense, g_post_ff, out, moe_out);
 }
 
-cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, uint16_t* moe_out,
+cudaError_t launch_combine_moe(int T, int H, int k, const float* y, uint16_t* moe_out,
                                cudaStream_t s, bool pdl) {
   return launch_k(combine_moe_kernel, dim3(T), dim3(256), 0, s, pdl, H, k, y, moe_out);
 }

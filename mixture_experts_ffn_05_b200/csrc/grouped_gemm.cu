@@ -2,7 +2,7 @@
 //
 // Used for both halves of every expert MLP and of the shared dense MLP:
 //   gate_up (kind 0): h[pos][i] = gelu_tanh(g) * u, g/u = xn[pos] . W_gate_up[e][i or I+i]
-//   down    (kind 1): Y[row][o] = w(row) * (h[pos] . W_down[e][o])
+//   down    (kind 1): Y[row][o] = w(row) * (h[pos] . W_down[e][o])   (bf16 or fp32)
 // (ONNX export card, "Truthful graph contracts", "Mixture of Experts" and "MoE topology"
 // rows; Inferentia2 card, "How it works": expert outputs weighted by the routing weight).
 //
@@ -561,7 +561,8 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
                 if (col < pc.n_valid) {
                   const float h = gelu_tanh(v[i] * sc) * xg[i * 64 + row];
                   const size_t orow = static_cast<size_t>(pc.b_row0 + pc.n * BN + col);
-                  pr.out[orow * pr.out_ld + out_col0 + row] = bf16_bits(h);
+                  static_cast<uint16_t*>(pr.out)[orow * pr.out_ld + out_col0 + row] =
+                      bf16_bits(h);
                 }
               }
             }
@@ -572,9 +573,14 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
               const int col = c0 + i;
               if (col < pc.n_valid) {
                 const int orow = col_row[col];
-                if (orow >= 0)
-                  pr.out[static_cast<size_t>(orow) * pr.out_ld + out_col0 + row] =
-                      bf16_bits(v[i] * sc * col_w[col]);
+                if (orow >= 0) {
+                  const size_t o = static_cast<size_t>(orow) * pr.out_ld + out_col0 + row;
+                  const float val = v[i] * sc * col_w[col];
+                  if (pr.out_f32)
+                    static_cast<float*>(pr.out)[o] = val;
+                  else
+                    static_cast<uint16_t*>(pr.out)[o] = bf16_bits(val);
+                }
               }
             }
           }

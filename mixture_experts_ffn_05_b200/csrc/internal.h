@@ -12,7 +12,7 @@ namespace moe {
 //   kind 0 (gate_up): each M tile is 64 gate rows + the 64 matching up rows of one
 //     group; the epilogue writes h = gelu_tanh(gate) * up as bf16.
 //   kind 1 (down): each M tile is 128 rows of the output; the epilogue scales by the
-//     int8 row scale (if any) and the routing weight (if any) and writes bf16.
+//     int8 row scale (if any) and the routing weight (if any) and writes bf16 or fp32.
 struct GemmProblem {
   int kind;              // 0 gate_up, 1 down
   int groups;            // experts, or 1 for the dense MLP
@@ -25,7 +25,9 @@ struct GemmProblem {
   int nw;                // gate_up: Nw (first up row); down: unused
   int split;             // pieces per tile along K (>= 1)
   int map;               // tensor-map pair: 0 or 1
-  uint16_t* out;         // bf16 output
+  void* out;             // output: bf16 (gate_up always), or fp32 when out_f32
+  int out_f32;           // down: fp32 output (the block's branch outputs before the
+                         // combine keep fp32, so no rounding is added before the norms)
   int out_ld;            // elements per output row
   const int* out_rows;   // down: output row of B row pos (sorted_src); NULL = pos
   const float* route_w;  // down: weight per output row (topk_w flattened); NULL = 1
@@ -81,21 +83,38 @@ cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t*
                           float* topk_w, unsigned* counters, unsigned* status, int* offsets,
                           int* sorted_src, int* inv_pos, cudaStream_t s, bool pdl = false);
 int router_counters(int T);
+
+// The tensor-core router (router_tc.cu) serves batches of more than kRouterTcMinT
+// tokens.  It needs two E x H bf16 buffers for the split W' = s * W_r / sqrt(H) and
+// the tensor maps below: x [T][H] with 64 x 128 boxes, W'hi and W'lo [E][H] with
+// 64 x ne boxes (ne = E rounded up to 16), all with 128-byte swizzling.
+constexpr int kRouterTcMinT = 128;
+bool router_uses_tc(int T);
+struct RouterTcMaps {
+  CUtensorMap x, whi, wlo;
+};
+cudaError_t launch_router_tc(const RouterTcMaps& maps, int T, int H, int E, int k, float eps,
+                             const uint16_t* w_router, const uint16_t* router_scale,
+                             uint16_t* whi, uint16_t* wlo, const float* bias,
+                             const uint16_t* per_expert_scale, const uint16_t* g_pre_moe,
+                             const uint16_t* g_pre_dense, uint16_t* xn_moe, uint16_t* xn_dense,
+                             int* topk_idx, float* topk_w, unsigned* status,
+                             uint64_t timeout_ns, cudaStream_t s, bool pdl = false);
 cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int* sorted_src,
                            int* inv_pos, int* block_hist, int* block_base, cudaStream_t s,
                            bool pdl = false);
-int permute_blocks(int n);  // blocks of the multi-block path (0 = single-block path)
+int permute_blocks(int n);  // blocks of the multi-block path, <= 256 (0 = single-block path)
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
                                const uint16_t* src, uint16_t* dst, cudaStream_t s,
                                bool pdl = false);
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                                 cudaStream_t s, bool pdl = false);
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
-                                 const uint16_t* y, const uint16_t* dense,
+                                 const float* y, const float* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s, bool pdl = false);
-cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, uint16_t* moe_out,
+cudaError_t launch_combine_moe(int T, int H, int k, const float* y, uint16_t* moe_out,
                                cudaStream_t s, bool pdl = false);
 cudaError_t launch_quantize_int8(const uint16_t* w, int64_t rows, int cols, int8_t* q,
                                  float* scales, cudaStream_t s);

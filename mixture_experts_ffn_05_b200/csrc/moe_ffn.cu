@@ -72,7 +72,7 @@ int choose_split(int k_steps, int bn) {
 
 struct Layout {
   size_t status, rcounters, counters, logits, bhist, bbase, topk_idx, topk_w, offsets, sorted, inv;
-  size_t xn_moe, xn_dense, aperm, h, y, hd, dense, partials, total;
+  size_t xn_moe, xn_dense, aperm, h, y, hd, dense, partials, wr_hi, wr_lo, total;
   size_t counters_bytes;
   int bn, split_gu, split_dgu, split_d, split_dd;
 };
@@ -121,10 +121,14 @@ Layout layout_of(const Dims& d) {
   L.xn_dense = take(T * d.H * 2);
   L.aperm = take(Tk * d.H * 2);
   L.h = take(Tk * d.I * 2);
-  L.y = take(Tk * d.H * 2);
+  L.y = take(Tk * d.H * 4);
   L.hd = take(T * d.D * 2);
-  L.dense = take(T * d.H * 2);
+  L.dense = take(T * d.H * 4);
   L.partials = take(any_split ? static_cast<size_t>(pieces) * L.bn * 128 * 4 : 0);
+  // the tensor-core router's two-term split of the scaled router weights
+  const size_t wr_bytes = router_uses_tc(d.T) ? static_cast<size_t>(d.E) * d.H * 2 : 0;
+  L.wr_hi = take(wr_bytes);
+  L.wr_lo = take(wr_bytes);
   L.total = off;
   return L;
 }
@@ -216,13 +220,14 @@ struct GemmJob {
   const int* offsets;
   const int* sorted_src;
   const float* topk_w;
-  uint16_t* y;               // [Tk][H] weighted expert outputs
+  float* y;                  // [Tk][H] weighted expert outputs
   // dense MLP (problem 1 when experts are present, else problem 0), may be absent
   bool dense;
   const uint16_t* xn_dense;  // [T][H]
   const uint16_t* w_dgu;     // [2D][H]
   const uint16_t* w_dd;      // [H][D]
-  uint16_t* dense_out;       // [T][H]
+  void* dense_out;           // [T][H], bf16 or (dense_f32) fp32
+  int dense_f32;
 };
 
 // Records ev[i] on s when a stage-event array was given.
@@ -274,7 +279,8 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b = GemmProblem{};
     b.kind = 1; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = static_cast<int>(Tk);
     b.k_steps = (d.I + kw - 1) / kw; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H; b.nw = 0;
-    b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_ld = d.H;
+    b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_f32 = 1;
+    b.out_ld = d.H;
     b.out_rows = j.sorted_src;
     b.route_w = j.topk_w; b.wscale = j.s_down; b.w8 = d.int8;
     if (!encode_a(&mgu.a[np], j.w_gate_up, static_cast<int64_t>(d.E) * 2 * d.I, d.H, 64, d.int8) ||
@@ -294,7 +300,8 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b = GemmProblem{};
     b.kind = 1; b.groups = 1; b.offsets = nullptr; b.n_tokens = d.T;
     b.k_steps = d.D / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H;
-    b.split = L.split_dd; b.map = np; b.out = j.dense_out; b.out_ld = d.H;
+    b.split = L.split_dd; b.map = np; b.out = j.dense_out; b.out_f32 = j.dense_f32;
+    b.out_ld = d.H;
     if (!encode_a(&mgu.a[np], j.w_dgu, 2 * static_cast<int64_t>(d.D), d.H, 64, false) ||
         !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, L.bn) ||
         !encode_a(&mdn.a[np], j.w_dd, d.H, d.D, 128, false) ||
@@ -315,6 +322,52 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
   st = cuda_status(launch_grouped_gemm(L.bn, mdn, dn, grid, s, true));
   if (st != MOE_OK) return st;
   return mark(ev, 5, s) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Inputs and outputs of the router step.
+struct RouteJob {
+  const uint16_t* x;
+  const uint16_t* router_scale;
+  const uint16_t* w_router;
+  const float* logit_bias;
+  const uint16_t* per_expert_scale;
+  const uint16_t* g_pre_moe;
+  const uint16_t* g_pre_dense;
+  int* topk_idx;
+  float* topk_w;
+  uint16_t* xn_moe;
+  uint16_t* xn_dense;
+  int* offsets;  // with sorted_src and inv_pos: sort the pairs in the same launch; or NULL
+  int* sorted_src;
+  int* inv_pos;
+};
+
+// The router step, launched as the first kernel of the entry point: the tensor-core
+// router for large batches, the CUDA-core one (router.cu) for small ones.  Only the
+// CUDA-core router sorts the pairs in the same launch (r.offsets); the caller asks for
+// it for batches of the CUDA-core router.
+moe_status_t run_router(const Dims& d, const Layout& L, void* ws, const RouteJob& r,
+                        cudaStream_t s) {
+  unsigned* counters = at<unsigned>(ws, L.rcounters);
+  unsigned* status = at<unsigned>(ws, L.status);
+  if (!router_uses_tc(d.T))
+    return cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, r.x, r.router_scale, r.w_router,
+                                     r.logit_bias, r.per_expert_scale, r.g_pre_moe,
+                                     r.g_pre_dense, r.xn_moe, r.xn_dense,
+                                     at<float>(ws, L.logits), r.topk_idx, r.topk_w, counters,
+                                     status, r.offsets, r.sorted_src, r.inv_pos, s));
+  uint16_t* whi = at<uint16_t>(ws, L.wr_hi);
+  uint16_t* wlo = at<uint16_t>(ws, L.wr_lo);
+  const int ne = (d.E + 15) / 16 * 16;
+  if (r.offsets != nullptr) return MOE_ERR_INVALID_ARG;  // no fused sort on this path
+  RouterTcMaps m;
+  if (!encode_bf16(&m.x, r.x, d.T, d.H, 128) || !encode_bf16(&m.whi, whi, d.E, d.H, ne) ||
+      !encode_bf16(&m.wlo, wlo, d.E, d.H, ne))
+    return MOE_ERR_CUDA;
+  return cuda_status(launch_router_tc(m, d.T, d.H, d.E, d.k, d.eps, r.w_router, r.router_scale,
+                                      whi, wlo, r.logit_bias, r.per_expert_scale, r.g_pre_moe,
+                                      r.g_pre_dense, r.xn_moe, r.xn_dense, r.topk_idx, r.topk_w,
+                                      status, kWaitTimeoutNs, s));
 }
 
 bool w_ok(const moe_expert_weights_t* w, bool int8) {
@@ -368,12 +421,9 @@ moe_status_t moe_router(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
   if (logit_bias != nullptr && !aligned16(logit_bias)) return MOE_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, x, router_scale, w_router,
-                                   logit_bias, per_expert_scale, g_pre_moe, g_pre_dense, xn_moe,
-                                   xn_dense, at<float>(ws, L.logits), topk_idx, topk_w,
-                                   at<unsigned>(ws, L.rcounters), at<unsigned>(ws, L.status),
-                                   nullptr, nullptr, nullptr, s));
+  const RouteJob r{x, router_scale, w_router, logit_bias, per_expert_scale, g_pre_moe,
+                   g_pre_dense, topk_idx, topk_w, xn_moe, xn_dense, nullptr, nullptr, nullptr};
+  return run_router(d, L, ws, r, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx,
@@ -411,7 +461,7 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int Tk = d.T * d.k;
   uint16_t* aperm = at<uint16_t>(ws, L.aperm);
-  uint16_t* y = at<uint16_t>(ws, L.y);
+  float* y = at<float>(ws, L.y);
   if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted_src, xn_moe, aperm, s))) != MOE_OK)
     return st;
   GemmJob j{};
@@ -481,21 +531,18 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   uint16_t* xn_moe = at<uint16_t>(ws, L.xn_moe);
   uint16_t* xn_dense = at<uint16_t>(ws, L.xn_dense);
   uint16_t* aperm = at<uint16_t>(ws, L.aperm);
-  uint16_t* y = at<uint16_t>(ws, L.y);
-  uint16_t* dense = at<uint16_t>(ws, L.dense);
-  float* logits = at<float>(ws, L.logits);
+  float* y = at<float>(ws, L.y);
+  float* dense = at<float>(ws, L.dense);
 
   if (ev != nullptr)
     for (int i = 0; i < MOE_BLOCK_EVENTS; ++i)
       if (ev[i] == nullptr) return MOE_ERR_INVALID_ARG;
   if (!mark(ev, 0, s)) return MOE_ERR_CUDA;
-  const bool fused_sort = permute_blocks(Tk) == 0;
-  if ((st = cuda_status(launch_router(d.T, d.H, d.E, d.k, d.eps, x, w->router_scale, w->w_router,
-                                      w->logit_bias, w->per_expert_scale, w->g_pre_moe,
-                                      w->g_pre_dense, xn_moe, xn_dense, logits, topk_idx, topk_w,
-                                      at<unsigned>(ws, L.rcounters), at<unsigned>(ws, L.status),
-                                      fused_sort ? offsets : nullptr, sorted, inv, s))) != MOE_OK)
-    return st;
+  const bool fused_sort = !router_uses_tc(d.T) && permute_blocks(Tk) == 0;
+  const RouteJob r{x, w->router_scale, w->w_router, w->logit_bias, w->per_expert_scale,
+                   w->g_pre_moe, w->g_pre_dense, topk_idx, topk_w, xn_moe, xn_dense,
+                   fused_sort ? offsets : nullptr, sorted, inv};
+  if ((st = run_router(d, L, ws, r, s)) != MOE_OK) return st;
   if (!mark(ev, 1, s)) return MOE_ERR_CUDA;
   if (!fused_sort &&
       (st = cuda_status(launch_permute(Tk, d.E, topk_idx, offsets, sorted, inv, at<int>(ws, L.bhist),
@@ -522,6 +569,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   j.w_dgu = w->w_dense_gate_up;
   j.w_dd = w->w_dense_down;
   j.dense_out = dense;
+  j.dense_f32 = 1;
   if ((st = run_gemms(d, L, ws, j, s, false, ev)) != MOE_OK) return st;
   if ((st = cuda_status(launch_combine_block(d.T, d.H, d.k, d.eps, x, y, dense, w->g_post_moe,
                                              w->g_post_dense, w->g_post_ff, out, moe_out, s,
@@ -567,7 +615,7 @@ moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream) {
 
 namespace {
 
-constexpr int kNoAllocMaxBlocks = MOE_PERMUTE_NOALLOC_MAX_PAIRS / 4096;  // blocks of 4096 pairs
+constexpr int kNoAllocMaxBlocks = 256;  // the multi-block sort uses at most 256 blocks
 constexpr int kNoAllocInts = 2 * kNoAllocMaxBlocks * 256;
 static_assert(kNoAllocInts * 4 == MOE_PERMUTE_NOALLOC_SCRATCH_BYTES, "scratch size");
 

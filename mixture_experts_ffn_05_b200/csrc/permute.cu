@@ -6,7 +6,10 @@
 // token), computed exactly:
 //   histogram -> exclusive scan (expert_offsets) -> stable scatter (sorted_src, inv_pos).
 // Up to kPermSmallMax pairs one block does everything; beyond that, per-block
-// histograms, one scan block, and a per-block stable scatter.
+// histograms, one scan block, and a per-block stable scatter over at most
+// kPermMaxBlocks blocks of a multiple of kPermThreads pairs each.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "permute_impl.cuh"
@@ -14,8 +17,16 @@
 namespace moe {
 
 constexpr int kPermThreads = 1024;
-constexpr int kPermPerBlock = 4096;  // pairs per block of the multi-block path
-constexpr int kPermSmallMax = 8192;  // pairs handled by the single-block path
+constexpr int kPermSmallMax = 2048;  // pairs handled by the single-block path
+constexpr int kPermMaxBlocks = 256;  // blocks of the multi-block path at most
+
+// Pairs per block of the multi-block path: one pass of the block's threads when that
+// keeps the grid within kPermMaxBlocks, else the smallest multiple that does.
+int pairs_per_block(int n) {
+  const int64_t per = (static_cast<int64_t>(n) + kPermMaxBlocks - 1) / kPermMaxBlocks;
+  return static_cast<int>(std::max<int64_t>(1, (per + kPermThreads - 1) / kPermThreads) *
+                          kPermThreads);
+}
 
 __global__ void __launch_bounds__(kPermThreads) permute_small_kernel(
     int n, int E, const int* __restrict__ idx, int* __restrict__ offsets,
@@ -27,7 +38,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_small_kernel(
 }
 
 // Multi-block pass 1: per-block histograms block_hist[b][e].
-__global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(int n, int E,
+__global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(int n, int E, int ppb,
                                                                     const int* __restrict__ idx,
                                                                     int* __restrict__ block_hist) {
   __shared__ int cnt[kPermMaxE];
@@ -36,8 +47,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(int n, int E
   pdl_trigger();
   for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
   __syncthreads();
-  const int p0 = blockIdx.x * kPermPerBlock;
-  const int p1 = min(n, p0 + kPermPerBlock);
+  const int p0 = blockIdx.x * ppb;
+  const int p1 = min(n, p0 + ppb);
   for (int p = p0 + tid; p < p1; p += kPermThreads) {
     const int e = idx[p];
     if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
@@ -77,7 +88,7 @@ __global__ void __launch_bounds__(kPermMaxE) permute_scan_kernel(int nb, int E,
 
 // Multi-block pass 3: stable scatter of each block's pairs.
 __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
-    int n, int E, const int* __restrict__ idx, const int* __restrict__ block_base,
+    int n, int E, int ppb, const int* __restrict__ idx, const int* __restrict__ block_base,
     int* __restrict__ sorted_src, int* __restrict__ inv_pos) {
   __shared__ int base[kPermMaxE];
   __shared__ int wcnt[kPermThreads / 32][kPermMaxE];
@@ -85,13 +96,14 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
   pdl_trigger();
   for (int e = threadIdx.x; e < E; e += kPermThreads) base[e] = block_base[blockIdx.x * E + e];
   __syncthreads();
-  const int p0 = blockIdx.x * kPermPerBlock;
-  scatter_range<kPermThreads>(p0, min(n, p0 + kPermPerBlock), E, idx, base, wcnt, sorted_src,
-                              inv_pos);
+  const int p0 = blockIdx.x * ppb;
+  scatter_range<kPermThreads>(p0, min(n, p0 + ppb), E, idx, base, wcnt, sorted_src, inv_pos);
 }
 
 int permute_blocks(int n) {
-  return n <= kPermSmallMax ? 0 : (n + kPermPerBlock - 1) / kPermPerBlock;
+  if (n <= kPermSmallMax) return 0;
+  const int ppb = pairs_per_block(n);
+  return (n + ppb - 1) / ppb;
 }
 
 cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int* sorted_src,
@@ -101,14 +113,15 @@ cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int*
   if (nb == 0)
     return launch_k(permute_small_kernel, dim3(1), dim3(kPermThreads), 0, s, pdl, n, E, topk_idx,
                     offsets, sorted_src, inv_pos);
+  const int ppb = pairs_per_block(n);
   cudaError_t e = launch_k(permute_hist_kernel, dim3(nb), dim3(kPermThreads), 0, s, pdl, n, E,
-                           topk_idx, block_hist);
+                           ppb, topk_idx, block_hist);
   if (e != cudaSuccess) return e;
   e = launch_k(permute_scan_kernel, dim3(1), dim3(kPermMaxE), 0, s, true, nb, E,
                (const int*)block_hist, block_base, offsets);
   if (e != cudaSuccess) return e;
-  return launch_k(permute_scatter_kernel, dim3(nb), dim3(kPermThreads), 0, s, true, n, E, topk_idx,
-                  (const int*)block_base, sorted_src, inv_pos);
+  return launch_k(permute_scatter_kernel, dim3(nb), dim3(kPermThreads), 0, s, true, n, E, ppb,
+                  topk_idx, (const int*)block_base, sorted_src, inv_pos);
 }
 
 // dst[q] = src[sorted_src[q] / k] for the n sorted pairs; one thread per 16 bytes.
