@@ -3,9 +3,13 @@
 // ONNX export card, "Truthful graph contracts", "MoE topology" row: the block returns
 // post_ff_norm(dense + moe) + residual; the Inferentia2 card's "four feed-forward
 // layernorms" add a post norm on each branch:
-//   m   = sum_{j=0..k-1} Y[t*k + j]          (weights already applied, fixed slot order)
+//   m   = sum_{j=0..k-1} w[t,j] * Y[inv_pos[t*k + j]]        (fixed slot order)
 //   out = x + N_post_ff( N_post_dense(d) + N_post_moe(m) ),  N_g(v) = v / rms(v) * g
-// Y and d arrive in fp32; all sums are fp32 and the output is rounded to bf16 once.
+// Y (the expert outputs in sorted order, unweighted) and d arrive in fp32; all sums are
+// fp32 and the output is rounded to bf16 once.  A slot whose inv_pos does not point back
+// at it through sorted_src (a pair the permutation dropped) contributes nothing.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -37,14 +41,33 @@ __device__ __forceinline__ void load8f(const float* p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+// Row of Y and routing weight of each slot of token t, in shared memory (row -1: none).
+__device__ __forceinline__ void load_slots(int t, int k, int n, const int* __restrict__ inv_pos,
+                                           const int* __restrict__ sorted_src,
+                                           const float* __restrict__ topk_w, int* s_q,
+                                           float* s_w) {
+  if (threadIdx.x < k) {
+    const int p = t * k + threadIdx.x;
+    const int q = inv_pos[p];
+    const bool ok = q >= 0 && q < n && sorted_src[q] == p;
+    s_q[threadIdx.x] = ok ? q : -1;
+    s_w[threadIdx.x] = topk_w[p];
+  }
+  __syncthreads();
+}
+
 // One CTA per token, one 8-column chunk per thread; every input is requested before
 // the first reduction.
 __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
     int H, int k, float eps, const uint16_t* __restrict__ x, const float* __restrict__ y,
-    const float* __restrict__ dense, const uint16_t* __restrict__ g_pm,
+    const int* __restrict__ inv_pos, const int* __restrict__ sorted_src,
+    const float* __restrict__ topk_w, const float* __restrict__ dense,
+    const uint16_t* __restrict__ g_pm,
     const uint16_t* __restrict__ g_pd, const uint16_t* __restrict__ g_ff,
     uint16_t* __restrict__ out, uint16_t* __restrict__ moe_out) {
   __shared__ float2 red[kCombMaxThreads / 32];
+  __shared__ int s_q[16];
+  __shared__ float s_w[16];
   const int t = blockIdx.x;
   const int c = threadIdx.x;
   const bool on = c < (H >> 3);
@@ -57,22 +80,24 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
   vx = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + cc);
   pdl_wait();
   pdl_trigger();
+  load_slots(t, k, gridDim.x * k, inv_pos, sorted_src, topk_w, s_q, s_w);
   float m[8], d[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = d[i] = 0.f;
   {
-    const float* yr = y + static_cast<size_t>(t) * k * H + cc * 8;
     load8f(dense + static_cast<size_t>(t) * H + cc * 8, d);
     for (int j0 = 0; j0 < k; j0 += 4) {  // 4 slots in flight at a time, summed in slot order
       float buf[4][8];
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if (j0 + j < k) load8f(yr + static_cast<size_t>(j0 + j) * H, buf[j]);
+        if (j0 + j < k && s_q[j0 + j] >= 0)
+          load8f(y + static_cast<size_t>(s_q[j0 + j]) * H + cc * 8, buf[j]);
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if (j0 + j < k) {
+        if (j0 + j < k && s_q[j0 + j] >= 0) {
+          const float w = s_w[j0 + j];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] += buf[j][i];
+          for (int i = 0; i < 8; ++i) m[i] = fmaf(w, buf[j][i], m[i]);
         }
     }
     if (!on) {
@@ -112,38 +137,50 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
   }
 }
 
-// moe_out[t] = sum_j Y[t*k + j] in fp32, slot order, rounded to bf16.
+// moe_out[t] = sum_j w[t,j] * Y[inv_pos[t*k + j]] in fp32, slot order, rounded to bf16.
 __global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
                                                           const float* __restrict__ y,
+                                                          const int* __restrict__ inv_pos,
+                                                          const int* __restrict__ sorted_src,
+                                                          const float* __restrict__ topk_w,
                                                           uint16_t* __restrict__ moe_out) {
+  __shared__ int s_q[16];
+  __shared__ float s_w[16];
   const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
+  load_slots(t, k, gridDim.x * k, inv_pos, sorted_src, topk_w, s_q, s_w);
   for (int c = threadIdx.x; c < (H >> 3); c += 256) {
     float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < k; ++j) {
+      if (s_q[j] < 0) continue;
       float f[8];
-      load8f(y + (static_cast<size_t>(t) * k + j) * H + c * 8, f);
+      load8f(y + static_cast<size_t>(s_q[j]) * H + c * 8, f);
+      const float w = s_w[j];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] += f[i];
+      for (int i = 0; i < 8; ++i) m[i] = fmaf(w, f[i], m[i]);
     }
     reinterpret_cast<uint4*>(moe_out + static_cast<size_t>(t) * H)[c] = pack8(m);
   }
 }
 
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
-                                 const float* y, const float* dense,
+                                 const float* y, const int* inv_pos, const int* sorted_src,
+                                 const float* topk_w, const float* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s, bool pdl) {
-  const int threads = ((H >> 3) + 31) / 32 * 32;
-  return launch_k(combine_block_kernel, dim3(T), dim3(threads), 0, s, pdl, H, k, eps, x, y, dense,
-                  g_post_moe, g_post_dense, g_post_ff, out, moe_out);
+  const int threads = std::max(32, ((H >> 3) + 31) / 32 * 32);
+  return launch_k(combine_block_kernel, dim3(T), dim3(threads), 0, s, pdl, H, k, eps, x, y,
+                  inv_pos, sorted_src, topk_w, dense, g_post_moe, g_post_dense, g_post_ff, out,
+                  moe_out);
 }
 
-cudaError_t launch_combine_moe(int T, int H, int k, const float* y, uint16_t* moe_out,
+cudaError_t launch_combine_moe(int T, int H, int k, const float* y, const int* inv_pos,
+                               const int* sorted_src, const float* topk_w, uint16_t* moe_out,
                                cudaStream_t s, bool pdl) {
-  return launch_k(combine_moe_kernel, dim3(T), dim3(256), 0, s, pdl, H, k, y, moe_out);
+  return launch_k(combine_moe_kernel, dim3(T), dim3(256), 0, s, pdl, H, k, y, inv_pos,
+                  sorted_src, topk_w, moe_out);
 }
 
 }  // namespace moe

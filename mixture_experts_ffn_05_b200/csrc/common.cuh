@@ -160,6 +160,43 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 5-D tiled bulk copy global -> shared (coordinates innermost first).
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3,
+                                            int32_t c4, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+      "r"(c3), "r"(c4), "l"(policy)
+      : "memory");
+}
+
+// 2-D tiled bulk copy shared -> global, tracked in this thread's bulk group.  The
+// shared-memory writes it reads must be fenced to the async proxy first
+// (fence_proxy_async_smem) by the threads that made them.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0,
+                                             int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most one of this thread's committed bulk groups still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// Wait until every bulk group committed by this thread has completed (writes done).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // 1-D bulk copy global -> shared of `bytes` (both addresses 16-byte aligned, bytes a
 // multiple of 16); completion counted on `bar`.
 __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
@@ -272,11 +309,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 }
 
 // ------------------------------------------------------------------ math
-// gelu_pytorch_tanh: 0.5 a (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3))).
+// gelu_pytorch_tanh: 0.5 a (1 + tanh(u)), u = sqrt(2/pi) (a + 0.044715 a^3).
+// Since 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)), it is evaluated as a / (1 + exp(-2u)):
+// one exponential and one division (relative error a few units of 2^-23 for the
+// arguments that reach it; h is stored in bf16).  For very negative a, exp(-2u)
+// overflows to +inf and the quotient is the correct limit, -0.
 __device__ __forceinline__ float gelu_tanh(float a) {
   const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
   const float k1 = 0.044715f;
-  return 0.5f * a * (1.0f + tanhf(k0 * (a + k1 * a * a * a)));
+  const float u = k0 * fmaf(k1 * a, a * a, a);
+  return __fdividef(a, 1.0f + __expf(-2.0f * u));
 }
 
 }  // namespace moe

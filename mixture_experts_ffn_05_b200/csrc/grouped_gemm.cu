@@ -68,12 +68,12 @@ struct Cfg {
   static constexpr int kMiscInts = 8;               // tmem slot, abort, bcast x2, converter flag
   static constexpr int kPreOff = kMiscOff + kMiscInts * 4;
   static constexpr int kTabInts = 4 * kMaxEntries;  // pre, cnt, b0, ng
-  static constexpr int kXchgOff = ((kPreOff + kTabInts * 4) + 15) & ~15;
-  static constexpr int kXchgBytes = 2 * 16 * 64 * 4;  // one per epilogue group
-  // per epilogue group: each column's output row and routing weight (down launches)
-  static constexpr int kRouteOff = kXchgOff + kXchgBytes;
-  static constexpr int kRouteBytes = 2 * BN * 8;
-  static constexpr int kSmem = kRouteOff + kRouteBytes + 1024;  // + alignment slack
+  // output staging for the TMA stores: two 1 KB buffers per epilogue warp (one where
+  // two do not fit next to the pipeline)
+  static constexpr int kStgBytes = 1024;
+  static constexpr int kStgOff = ((kPreOff + kTabInts * 4) + 127) & ~127;
+  static constexpr int kStgBufs = (kStgOff + 8 * 2 * kStgBytes + 1024 <= 232448) ? 2 : 1;
+  static constexpr int kSmem = kStgOff + 8 * kStgBufs * kStgBytes + 1024;  // + alignment slack
   static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(kSmem <= 232448, "shared memory");
 };
@@ -128,6 +128,16 @@ __device__ __forceinline__ void convert_rows_bf16(const uint8_t* raw, uint8_t* c
     const int c = lane & 7;
     *reinterpret_cast<uint4*>(conv + r * 128 + ((c ^ (r & 7)) << 4)) = v[j];
   }
+}
+
+// Before a staging buffer is rewritten: the TMA store that last read it has done so
+// (with two buffers, the store of the other buffer may still be reading).
+template <int NBUF>
+__device__ __forceinline__ void stg_wait() {
+  if (NBUF >= 2)
+    bulk_wait_read1();
+  else
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 struct Piece {
@@ -191,7 +201,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
   int* cnt = pre + kMaxEntries;
   int* b0 = cnt + kMaxEntries;
   int* ng = b0 + kMaxEntries;
-  float* xchg = reinterpret_cast<float*>(smem + C::kXchgOff);
+  uint8_t* stg_all = smem + C::kStgOff;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nent = P.prob[0].groups + (P.nprob > 1 ? P.prob[1].groups : 0);
@@ -290,7 +300,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
         const GemmProblem& pr = P.prob[pc.p];
         const CUtensorMap* ma = &maps.a[pr.map];
         const CUtensorMap* mb = &maps.b[pr.map];
-        const int arow = pc.g * pr.w_rows_per_group + pc.m * (pr.kind == 0 ? 64 : 128);
+        const int arow = pc.g * pr.w_rows_per_group + pc.m * 128;  // down only
         const int brow = pc.b_row0 + pc.n * BN;
         for (int ks = pc.k0; ks < pc.k1; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
@@ -303,12 +313,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
           const int kw = (W8 && pr.w8) ? 128 : 64;
           const int nb = kw / 64;
           mbar_arrive_expect_tx(&full[stage], C::kABytes + nb * C::kBBytes);
-          if (pr.kind == 0) {
+          if (pr.kind == 0)  // 8 gate rows, the 8 matching up rows, ... (one 5-D box)
+            tma_load_5d(sa, ma, &full[stage], ks * kw, 0, 0, pc.m * 8, pc.g, pol_w);
+          else
             tma_load_2d(sa, ma, &full[stage], ks * kw, arow, pol_w);
-            tma_load_2d(sa + C::kABytes / 2, ma, &full[stage], ks * kw, arow + pr.nw, pol_w);
-          } else {
-            tma_load_2d(sa, ma, &full[stage], ks * kw, arow, pol_w);
-          }
           for (int b = 0; b < nb; ++b)
             tma_load_2d(sa + C::kABytes + b * C::kBBytes, mb, &full[stage], ks * kw + 64 * b, brow,
                         pol_b);
@@ -450,15 +458,23 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     // ================= epilogue: two groups of 4 warps take alternate pieces ============
     // Warp w reads TMEM lanes 32*(w%4)..+31; each group covers all 128 lanes.  Two groups
     // keep the latency-bound part of an epilogue (partials, counters) off the MMA's path.
+    // Each warp then writes its own slice of the output tile: it stages the values in its
+    // shared-memory buffers and one lane stores them with a TMA copy, so the epilogue
+    // issues a few bulk stores per tile instead of one global store per value.
+    //   gate_up: lanes l and l^8 hold the gate and up row of one feature (the A tile is
+    //     8 gate rows, the matching 8 up rows, ...); a shuffle pairs them, the gate lane
+    //     finishes columns 0-7 of each 16 and the up lane columns 8-15.  Warp q covers
+    //     features 16q..16q+15 of the tile's 64.
+    //   down: lane l holds output row 32q + l of the tile's 128.
+    // Output rows are the tile's B rows (sorted order).  A 16-column chunk (gate_up) or
+    // 8-column half chunk (down) that is not all valid is written with plain stores.
     const int grp = (warp - 2) >> 2;
     const int q = warp & 3;
-    const int row = q * 32 + lane;  // accumulator row = TMEM lane
     const int et = threadIdx.x - 64 - 128 * grp;
     const uint32_t bar = 1 + grp;
     volatile int* gb = bcast + grp;
-    float* xg = xchg + grp * 16 * 64;
-    int* col_row = reinterpret_cast<int*>(smem + C::kRouteOff) + grp * 2 * BN;  // [BN]
-    float* col_w = reinterpret_cast<float*>(col_row + BN);                       // [BN]
+    uint8_t* stg = stg_all + (warp - 2) * C::kStgBufs * C::kStgBytes;
+    int nstg = 0;  // staging buffers used by this warp so far
     int local = 0;
     for (int piece = blockIdx.x; piece < total; piece += gridDim.x, ++local) {
       if ((local & 1) != grp) continue;
@@ -478,6 +494,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(ab * BN);
+      const int row = q * 32 + lane;  // accumulator row = TMEM lane
       const int ncols = (pc.n_valid + 15) & ~15;
       bool last = true;
       if (pr.split > 1) {
@@ -501,23 +518,13 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
         last = *gb != 0;
       }
       if (last) {
-        if (pr.kind == 1) {
-          // stage the tile's output rows and routing weights once (no global loads in
-          // the column loop below)
-          for (int c = et; c < pc.n_valid; c += 128) {
-            const int pos = pc.b_row0 + pc.n * BN + c;
-            int orow = pr.out_rows ? pr.out_rows[pos] : pos;
-            if (orow < 0 || orow >= pr.n_tokens) orow = -1;
-            col_row[c] = orow;
-            col_w[c] = (orow >= 0 && pr.route_w) ? pr.route_w[orow] : 1.f;
-          }
-          named_sync(bar, 128);
-        }
-        const int out_col0 = pc.m * (pr.kind == 0 ? 64 : 128);
+        const int pos0 = pc.b_row0 + pc.n * BN;  // output row of column 0
         float sc = 1.f;
         if (pr.wscale) {
-          const int wr = pr.kind == 0 ? (row < 64 ? out_col0 + row : pr.nw + out_col0 + row - 64)
-                                      : out_col0 + row;
+          // gate_up row r of the tile: feature 8*(r/16) + r%8 of its 64, gate or up by bit 3
+          const int wr = pr.kind == 0
+                             ? pc.m * 64 + 8 * (row >> 4) + (row & 7) + ((row & 8) ? pr.nw : 0)
+                             : pc.m * 128 + row;
           sc = pr.wscale[static_cast<size_t>(pc.g) * pr.w_rows_per_group + wr];
         }
         for (int c0 = 0; c0 < ncols; c0 += 16) {
@@ -548,38 +555,82 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = acc[i];
           }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] *= sc;
           if (pr.kind == 0) {
-            if (row >= 64) {
+            // pair gate and up, 8 columns per lane
+            const bool up = (lane & 8) != 0;
+            float h[8];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) xg[i * 64 + (row - 64)] = v[i] * sc;
+            for (int i = 0; i < 8; ++i) {
+              const float mine = up ? v[8 + i] : v[i];          // gate: cols 0-7, up: 8-15
+              const float give = up ? v[i] : v[8 + i];          // what the partner needs
+              const float other = __shfl_xor_sync(0xffffffffu, give, 8);
+              h[i] = up ? gelu_tanh(other) * mine : gelu_tanh(mine) * other;
             }
-            named_sync(bar, 128);
-            if (row < 64) {
+            uint8_t* buf = stg + (nstg % C::kStgBufs) * C::kStgBytes;
+            ++nstg;
+            if (lane == 0) stg_wait<C::kStgBufs>();
+            __syncwarp();
+            // [16 columns][16 features] bf16
+            uint16_t* b16 = reinterpret_cast<uint16_t*>(buf);
+            const int f = 8 * (lane >> 4) + (lane & 7);
+            const int cb = up ? 8 : 0;
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int col = c0 + i;
-                if (col < pc.n_valid) {
-                  const float h = gelu_tanh(v[i] * sc) * xg[i * 64 + row];
-                  const size_t orow = static_cast<size_t>(pc.b_row0 + pc.n * BN + col);
-                  static_cast<uint16_t*>(pr.out)[orow * pr.out_ld + out_col0 + row] =
-                      bf16_bits(h);
-                }
+            for (int i = 0; i < 8; ++i) b16[(cb + i) * 16 + f] = bf16_bits(h[i]);
+            const int fx = pc.m * 64 + 16 * q;  // first output feature of this warp
+            if (c0 + 16 <= pc.n_valid) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&maps.o[pr.map], buf, fx, pos0 + c0);
+                bulk_commit();
               }
+            } else {
+              __syncwarp();
+              if (lane == 0) bulk_commit();  // an empty group keeps the buffer accounting
+              // ragged chunk: lane l writes feature l%16 of columns l/16, l/16+2, ...
+              uint16_t* out = static_cast<uint16_t*>(pr.out);
+              for (int c = lane >> 4; c0 + c < pc.n_valid; c += 2)
+                out[static_cast<size_t>(pos0 + c0 + c) * pr.out_ld + fx + (lane & 15)] =
+                    b16[c * 16 + (lane & 15)];
             }
-            named_sync(bar, 128);
           } else {
+            // two halves of 8 columns: [8 columns][32 rows] fp32 or bf16
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int col = c0 + i;
-              if (col < pc.n_valid) {
-                const int orow = col_row[col];
-                if (orow >= 0) {
-                  const size_t o = static_cast<size_t>(orow) * pr.out_ld + out_col0 + row;
-                  const float val = v[i] * sc * col_w[col];
+            for (int hh = 0; hh < 2; ++hh) {
+              uint8_t* buf = stg + (nstg % C::kStgBufs) * C::kStgBytes;
+              ++nstg;
+              if (lane == 0) stg_wait<C::kStgBufs>();
+              __syncwarp();
+              if (pr.out_f32) {
+                float* bf = reinterpret_cast<float*>(buf);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bf[i * 32 + lane] = v[8 * hh + i];
+              } else {
+                uint16_t* bh = reinterpret_cast<uint16_t*>(buf);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bh[i * 32 + lane] = bf16_bits(v[8 * hh + i]);
+              }
+              const int cc = c0 + 8 * hh;
+              const int fx = pc.m * 128 + 32 * q;
+              if (cc + 8 <= pc.n_valid) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_2d(&maps.o[pr.map], buf, fx, pos0 + cc);
+                  bulk_commit();
+                }
+              } else {
+                __syncwarp();
+                if (lane == 0) bulk_commit();  // an empty group keeps the buffer accounting
+                for (int c = 0; cc + c < pc.n_valid; ++c) {
+                  const size_t o = static_cast<size_t>(pos0 + cc + c) * pr.out_ld + fx + lane;
                   if (pr.out_f32)
-                    static_cast<float*>(pr.out)[o] = val;
+                    static_cast<float*>(pr.out)[o] = reinterpret_cast<const float*>(buf)[c * 32 + lane];
                   else
-                    static_cast<uint16_t*>(pr.out)[o] = bf16_bits(val);
+                    static_cast<uint16_t*>(pr.out)[o] =
+                        reinterpret_cast<const uint16_t*>(buf)[c * 32 + lane];
                 }
               }
             }
@@ -590,6 +641,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
       named_sync(bar, 128);  // every flag of this piece is read before the next is written
       mbar_arrive(&acc_empty[ab]);
     }
+    if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
   }
 
   // ---- teardown

@@ -8,11 +8,13 @@
 namespace moe {
 
 // One GEMM problem of a grouped launch.  The weights are the M operand (rows of a
-// K-major matrix streamed by TMA), the tokens the N operand.
-//   kind 0 (gate_up): each M tile is 64 gate rows + the 64 matching up rows of one
-//     group; the epilogue writes h = gelu_tanh(gate) * up as bf16.
+// K-major matrix streamed by TMA), the tokens the N operand.  Output row = B row.
+//   kind 0 (gate_up): each M tile holds 64 features of one group as 8 gate rows, the
+//     8 matching up rows, the next 8 gate rows, ... (a 5-D tensor map over
+//     [group][gate|up][feature/8][8][K]); the epilogue writes h = gelu_tanh(gate) * up
+//     as bf16.
 //   kind 1 (down): each M tile is 128 rows of the output; the epilogue scales by the
-//     int8 row scale (if any) and the routing weight (if any) and writes bf16 or fp32.
+//     int8 row scale (if any) and writes bf16 or fp32.
 struct GemmProblem {
   int kind;              // 0 gate_up, 1 down
   int groups;            // experts, or 1 for the dense MLP
@@ -29,8 +31,6 @@ struct GemmProblem {
   int out_f32;           // down: fp32 output (the block's branch outputs before the
                          // combine keep fp32, so no rounding is added before the norms)
   int out_ld;            // elements per output row
-  const int* out_rows;   // down: output row of B row pos (sorted_src); NULL = pos
-  const float* route_w;  // down: weight per output row (topk_w flattened); NULL = 1
   const float* wscale;   // int8 row scales [groups][w_rows_per_group]; NULL for bf16
   int w8;                // A operand is int8 codes (needs a launch with int8_weights)
 };
@@ -48,6 +48,8 @@ struct GemmParams {
 struct GemmMaps {
   CUtensorMap a[2];  // weights of problem map 0 / 1
   CUtensorMap b[2];  // tokens of problem map 0 / 1
+  CUtensorMap o[2];  // outputs (TMA stores), unswizzled: gate_up boxes of 16 features x
+                     // 16 rows (bf16), down boxes of 32 features x 8 rows
 };
 
 // Launches kernel<<<grid, block, smem, s>>>(args...).  With pdl the launch is a
@@ -109,12 +111,16 @@ cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src
                                bool pdl = false);
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                                 cudaStream_t s, bool pdl = false);
+// y holds the expert outputs in sorted order (row inv_pos[t*k+j] for slot j of token
+// t), unweighted; the combine applies topk_w.
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
-                                 const float* y, const float* dense,
+                                 const float* y, const int* inv_pos, const int* sorted_src,
+                                 const float* topk_w, const float* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s, bool pdl = false);
-cudaError_t launch_combine_moe(int T, int H, int k, const float* y, uint16_t* moe_out,
+cudaError_t launch_combine_moe(int T, int H, int k, const float* y, const int* inv_pos,
+                               const int* sorted_src, const float* topk_w, uint16_t* moe_out,
                                cudaStream_t s, bool pdl = false);
 cudaError_t launch_quantize_int8(const uint16_t* w, int64_t rows, int cols, int8_t* q,
                                  float* scales, cudaStream_t s);

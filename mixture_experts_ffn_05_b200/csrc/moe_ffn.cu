@@ -205,6 +205,56 @@ bool encode_raw(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, in
                           CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// gate_up weights [groups][2F][K] (gate rows 0..F-1, up rows F..2F-1) as a 5-D map over
+// (K, row in 8, gate|up, feature group of 8, group): one box of 128 bytes of K x 8 rows x
+// gate|up x 8 groups lands as 8 gate rows, the matching 8 up rows, the next 8 gate
+// rows, ...  The strides are not increasing (gate|up is outside the feature groups in
+// memory but inside them in the box).
+bool encode_gate_up(CUtensorMap* m, const void* base, int64_t groups, int64_t F, int64_t K,
+                    bool raw, bool int8) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
+  if (fn == nullptr) return false;
+  const int es = int8 ? 1 : 2;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(K), 8, 2, static_cast<cuuint64_t>(F / 8),
+                        static_cast<cuuint64_t>(groups)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(K * es), static_cast<cuuint64_t>(F * K * es),
+                           static_cast<cuuint64_t>(8 * K * es),
+                           static_cast<cuuint64_t>(2 * F * K * es)};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / es), 8, 2, 8, 1};
+  cuuint32_t el[5] = {1, 1, 1, 1, 1};
+  const CUresult r =
+      fn(m, int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+         const_cast<void*>(base), dims, strides, box, el, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         raw ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Output map for the epilogue's TMA stores: rows x cols, unswizzled boxes.
+bool encode_out(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int box_cols,
+                int box_rows, bool f32) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
+  if (fn == nullptr) return false;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * es};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t el[2] = {1, 1};
+  const CUresult r =
+      fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
+         dims, strides, box, el, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Output boxes of the two GEMM kinds (see GemmMaps).
+bool encode_h_out(CUtensorMap* m, void* base, int64_t rows, int64_t cols) {
+  return encode_out(m, base, rows, cols, 16, 16, false);
+}
+bool encode_y_out(CUtensorMap* m, void* base, int64_t rows, int64_t cols, bool f32) {
+  return encode_out(m, base, rows, cols, 32, 8, f32);
+}
+
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // ---------------------------------------------------------------- the expert / dense GEMMs
@@ -220,7 +270,7 @@ struct GemmJob {
   const int* offsets;
   const int* sorted_src;
   const float* topk_w;
-  float* y;                  // [Tk][H] weighted expert outputs
+  float* y;                  // [Tk][H] expert outputs in sorted order, unweighted
   // dense MLP (problem 1 when experts are present, else problem 0), may be absent
   bool dense;
   const uint16_t* xn_dense;  // [T][H]
@@ -281,12 +331,13 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.k_steps = (d.I + kw - 1) / kw; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H; b.nw = 0;
     b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_f32 = 1;
     b.out_ld = d.H;
-    b.out_rows = j.sorted_src;
-    b.route_w = j.topk_w; b.wscale = j.s_down; b.w8 = d.int8;
-    if (!encode_a(&mgu.a[np], j.w_gate_up, static_cast<int64_t>(d.E) * 2 * d.I, d.H, 64, d.int8) ||
+    b.wscale = j.s_down; b.w8 = d.int8;
+    if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, w8, d.int8) ||
         !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, L.bn) ||
+        !encode_h_out(&mgu.o[np], h, Tk, d.I) ||
         !encode_a(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128, d.int8) ||
-        !encode_bf16(&mdn.b[np], h, Tk, d.I, L.bn))
+        !encode_bf16(&mdn.b[np], h, Tk, d.I, L.bn) ||
+        !encode_y_out(&mdn.o[np], j.y, Tk, d.H, true))
       return MOE_ERR_CUDA;
     ++np;
   }
@@ -302,17 +353,19 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.k_steps = d.D / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H;
     b.split = L.split_dd; b.map = np; b.out = j.dense_out; b.out_f32 = j.dense_f32;
     b.out_ld = d.H;
-    if (!encode_a(&mgu.a[np], j.w_dgu, 2 * static_cast<int64_t>(d.D), d.H, 64, false) ||
+    if (!encode_gate_up(&mgu.a[np], j.w_dgu, 1, d.D, d.H, w8, false) ||
         !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, L.bn) ||
+        !encode_h_out(&mgu.o[np], hd, d.T, d.D) ||
         !encode_a(&mdn.a[np], j.w_dd, d.H, d.D, 128, false) ||
-        !encode_bf16(&mdn.b[np], hd, d.T, d.D, L.bn))
+        !encode_bf16(&mdn.b[np], hd, d.T, d.D, L.bn) ||
+        !encode_y_out(&mdn.o[np], j.dense_out, d.T, d.H, j.dense_f32 != 0))
       return MOE_ERR_CUDA;
     ++np;
   }
   gu.nprob = dn.nprob = np;
-  if (np == 1) {  // unused second pair: a valid copy of the first
-    mgu.a[1] = mgu.a[0]; mgu.b[1] = mgu.b[0];
-    mdn.a[1] = mdn.a[0]; mdn.b[1] = mdn.b[0];
+  if (np == 1) {  // unused second set: a valid copy of the first
+    mgu.a[1] = mgu.a[0]; mgu.b[1] = mgu.b[0]; mgu.o[1] = mgu.o[0];
+    mdn.a[1] = mdn.a[0]; mdn.b[1] = mdn.b[0]; mdn.o[1] = mdn.o[0];
   }
   // after a kernel of the same entry point the gate_up launch overlaps that kernel's tail
   // (programmatic dependent launch)
@@ -476,7 +529,8 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   j.topk_w = topk_w;
   j.y = y;
   if ((st = run_gemms(d, L, ws, j, s, false)) != MOE_OK) return st;
-  return cuda_status(launch_combine_moe(d.T, d.H, d.k, y, moe_out, s, true));
+  return cuda_status(launch_combine_moe(d.T, d.H, d.k, y, inv_pos, sorted_src, topk_w, moe_out,
+                                        s, true));
 }
 
 moe_status_t dense_mlp_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* xn_dense,
@@ -571,7 +625,8 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   j.dense_out = dense;
   j.dense_f32 = 1;
   if ((st = run_gemms(d, L, ws, j, s, false, ev)) != MOE_OK) return st;
-  if ((st = cuda_status(launch_combine_block(d.T, d.H, d.k, d.eps, x, y, dense, w->g_post_moe,
+  if ((st = cuda_status(launch_combine_block(d.T, d.H, d.k, d.eps, x, y, inv, sorted, topk_w,
+                                             dense, w->g_post_moe,
                                              w->g_post_dense, w->g_post_ff, out, moe_out, s,
                                              true))) != MOE_OK)
     return st;
