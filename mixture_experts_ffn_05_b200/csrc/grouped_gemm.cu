@@ -40,20 +40,29 @@ constexpr int kConvWarps = 4;      // converter warps, 32 rows of the 128-row ti
 
 // W8 = false: the A tile (weights, bf16) goes from HBM to shared memory by TMA, already
 //   in the 128-byte-swizzled K-major layout the MMA reads.
+// PAIR = true (bf16 only, wide token tiles): clusters of two CTAs run M = 256 MMAs
+//   (cta_group::2).  A work item covers two neighbouring M tiles, one per CTA, and
+//   both CTAs load half of the item's token rows, so each CTA streams 16 KB of
+//   weights and 16 KB of tokens per 64-wide K step for a 128 x 256 share of the
+//   product (instead of 16 + 32 KB alone): a third less shared-memory fill traffic per
+//   FLOP, which is what bounds the wide tiles.
 // W8 = true: TMA lands the raw A tile (int8 codes, or bf16 rows of a bf16 problem in the
 //   same launch) unswizzled; four converter warps turn it into the bf16 swizzled layout
 //   in a second, shallower ring.  The int8 row scales are applied in the epilogue.
-template <int BN, bool W8>
+template <int BN, bool W8, bool PAIR>
 struct Cfg {
+  static_assert(!(W8 && PAIR), "CTA pairs take bf16 weights only");
   static constexpr int kThreads = W8 ? 448 : 320;  // producer, MMA, 2x4 epilogue (+4 converters)
   static constexpr int kABytes = 128 * 64 * 2;     // bf16 A tile: 128 weight rows x 64 K
-  static constexpr int kBBytes = BN * 64 * 2;      // BN token rows x 64 K
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;  // token rows in this CTA's B tile
+  static constexpr int kBBytes = kBRows * 64 * 2;
   // W8 stages hold a raw A tile of 16 KB (int8 codes for 128 K, or bf16 for 64 K) and
   // up to two B tiles (an int8 step covers two 64-wide MMA sub-steps).
   static constexpr int kBSlots = W8 ? 2 : 1;
   static constexpr int kStage = kABytes + kBSlots * kBBytes;
-  static constexpr int kStages = W8 ? (BN <= 16 ? 7 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 3 : 2))))
-                                    : (BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4)));
+  static constexpr int kStages = PAIR ? (BN <= 128 ? 8 : 6)
+                                : W8 ? (BN <= 16 ? 7 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 3 : 2))))
+                                     : (BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4)));
   static constexpr int kConvBytes = 2 * kABytes;   // converted stage: two 64-wide sub-tiles
   static constexpr int kConv = W8 ? (BN >= 256 ? 1 : 2) : 0;
   // TMEM accumulators: 4 for narrow tiles (the epilogue of a weight-streaming piece is
@@ -156,6 +165,7 @@ __device__ __forceinline__ int find_entry(const int* pre, int nent, int piece) {
   return lo;
 }
 
+// With PAIR, pc.m numbers pairs of M tiles.
 template <int BN>
 __device__ __forceinline__ Piece decode_piece(int piece, const GemmParams& P, const int* pre,
                                               const int* b0, const int* ng, int nent) {
@@ -179,10 +189,10 @@ __device__ __forceinline__ Piece decode_piece(int piece, const GemmParams& P, co
   return pc;
 }
 
-template <int BN, bool W8>
-__global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
+template <int BN, bool W8, bool PAIR>
+__global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
     grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams P) {
-  using C = Cfg<BN, W8>;
+  using C = Cfg<BN, W8, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -205,6 +215,11 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nent = P.prob[0].groups + (P.nprob > 1 ? P.prob[1].groups : 0);
+  // work items: one per CTA, or (PAIR) one per cluster of two, dealt round-robin
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int first_item = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int item_stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   // ---- setup: barriers, TMEM, the piece table
   if (threadIdx.x == 0) {
@@ -219,7 +234,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     }
     for (int i = 0; i < C::kAcc; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 128);
+      mbar_init(&acc_empty[i], PAIR ? 256 : 128);  // PAIR: both CTAs' epilogues (leader's)
     }
     mbar_init(drain, 1);
     mbar_fence_init();
@@ -232,9 +247,16 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
+  // the peer's barriers are initialised before either CTA signals the other
+  if (PAIR) cluster_sync();
   // everything above overlaps the previous kernel on the stream; its results (routing,
   // gathered rows, h) are read only below
   pdl_wait();
@@ -259,7 +281,8 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     }
     b0[i] = s0;
     ng[i] = n;
-    cnt[i] = pr.m_tiles * ((n + BN - 1) / BN) * pr.split;
+    const int m_items = PAIR ? (pr.m_tiles + 1) / 2 : pr.m_tiles;
+    cnt[i] = m_items * ((n + BN - 1) / BN) * pr.split;
   }
   __syncthreads();
   if (warp == 0) {
@@ -295,13 +318,19 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
       int armed[C::kStages];
       for (int i = 0; i < C::kStages; ++i) armed[i] = -1;
       bool ok = true;
-      for (int piece = blockIdx.x; piece < total && ok; piece += gridDim.x) {
+      for (int piece = first_item; piece < total && ok; piece += item_stride) {
         const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
         const GemmProblem& pr = P.prob[pc.p];
         const CUtensorMap* ma = &maps.a[pr.map];
         const CUtensorMap* mb = &maps.b[pr.map];
-        const int arow = pc.g * pr.w_rows_per_group + pc.m * 128;  // down only
-        const int brow = pc.b_row0 + pc.n * BN;
+        // this CTA's M tile; PAIR: the second tile of an odd count lies past the group's
+        // rows (zero-filled for gate_up, another group's rows for down: never stored)
+        const int mt = PAIR ? 2 * pc.m + static_cast<int>(rank) : pc.m;
+        const int arow = pc.g * pr.w_rows_per_group + mt * 128;  // down only
+        // PAIR: the leader loads the first half of the item's (16-rounded) token columns,
+        // the other CTA the second half
+        const int half = ((pc.n_valid + 15) & ~15) >> 1;
+        const int brow = pc.b_row0 + pc.n * BN + (PAIR ? static_cast<int>(rank) * half : 0);
         for (int ks = pc.k0; ks < pc.k1; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
             ok = false;
@@ -312,14 +341,25 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
           // the A tile is 16 KB either way
           const int kw = (W8 && pr.w8) ? 128 : 64;
           const int nb = kw / 64;
-          mbar_arrive_expect_tx(&full[stage], C::kABytes + nb * C::kBBytes);
-          if (pr.kind == 0)  // 8 gate rows, the 8 matching up rows, ... (one 5-D box)
-            tma_load_5d(sa, ma, &full[stage], ks * kw, 0, 0, pc.m * 8, pc.g, pol_w);
-          else
-            tma_load_2d(sa, ma, &full[stage], ks * kw, arow, pol_w);
-          for (int b = 0; b < nb; ++b)
-            tma_load_2d(sa + C::kABytes + b * C::kBBytes, mb, &full[stage], ks * kw + 64 * b, brow,
-                        pol_b);
+          if (PAIR) {
+            // both CTAs' bytes land on the leader's barrier; the leader expects them all
+            const uint32_t fb = cluster_addr(&full[stage], 0);
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::kABytes + C::kBBytes));
+            if (pr.kind == 0)
+              tma_load_5d_pair(sa, ma, fb, ks * 64, 0, 0, mt * 8, pc.g, pol_w);
+            else
+              tma_load_2d_pair(sa, ma, fb, ks * 64, arow, pol_w);
+            tma_load_2d_pair(sa + C::kABytes, mb, fb, ks * 64, brow, pol_b);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::kABytes + nb * C::kBBytes);
+            if (pr.kind == 0)  // 8 gate rows, the 8 matching up rows, ... (one 5-D box)
+              tma_load_5d(sa, ma, &full[stage], ks * kw, 0, 0, pc.m * 8, pc.g, pol_w);
+            else
+              tma_load_2d(sa, ma, &full[stage], ks * kw, arow, pol_w);
+            for (int b = 0; b < nb; ++b)
+              tma_load_2d(sa + C::kABytes + b * C::kBBytes, mb, &full[stage], ks * kw + 64 * b,
+                          brow, pol_b);
+          }
           armed[stage] = static_cast<int>(phase);
           if (++stage == C::kStages) {
             stage = 0;
@@ -330,14 +370,16 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
       if (!ok) {
         record_status(P.status, kStatusTimeout);
         *abort_flag = 1;
-        // Let every copy already issued land before the CTA winds down.
-        for (int i = 0; i < C::kStages; ++i)
-          if (armed[i] >= 0) mbar_wait(&full[i], static_cast<uint32_t>(armed[i]), tmo, nullptr);
+        // Let every copy already issued land before the CTA winds down (PAIR: the
+        // leader's barriers count both CTAs' copies).
+        if (!PAIR || leader)
+          for (int i = 0; i < C::kStages; ++i)
+            if (armed[i] >= 0) mbar_wait(&full[i], static_cast<uint32_t>(armed[i]), tmo, nullptr);
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0) {
+    // ================= MMA issuer (PAIR: the leader's, for both CTAs) =================
+    if (lane == 0 && (!PAIR || leader)) {
       int stage = 0;
       uint32_t phase = 0;
       int cs = 0;
@@ -345,9 +387,12 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
       int ab = 0;
       uint32_t aph = 0;
       bool ok = true, issued = false;
-      for (int piece = blockIdx.x; piece < total && ok; piece += gridDim.x) {
+      // PAIR: stage and accumulator releases go to the barriers of both CTAs
+      const uint32_t peer_empty0 = PAIR ? cluster_addr(&empty[0], 1) : 0u;
+      const uint32_t peer_acc0 = PAIR ? cluster_addr(&acc_full[0], 1) : 0u;
+      for (int piece = first_item; piece < total && ok; piece += item_stride) {
         const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
-        const uint32_t idesc = idesc_bf16_f32(128, (pc.n_valid + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32(PAIR ? 256 : 128, (pc.n_valid + 15) & ~15);
         if (!mbar_wait(&acc_empty[ab], aph ^ 1u, tmo, abort_flag)) {
           ok = false;
           break;
@@ -368,9 +413,13 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
             const uint64_t ad = sdesc_k_sw128(sA + sub * C::kABytes);
             const uint64_t bd = sdesc_k_sw128(sa + C::kABytes + sub * C::kBBytes);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc,
-                        (ks > pc.k0 || sub > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (ks > pc.k0 || sub > 0 || kk > 0) ? 1u : 0u;
+              if (PAIR)
+                umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+              else
+                umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+            }
           }
           if (W8) {
             umma_commit(&conv_empty[cs]);
@@ -379,7 +428,12 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
               cph ^= 1u;
             }
           }
-          umma_commit(&empty[stage]);
+          if (PAIR) {
+            umma_commit_pair(smem_u32(&empty[stage]));
+            umma_commit_pair(peer_empty0 + stage * 8);
+          } else {
+            umma_commit(&empty[stage]);
+          }
           issued = true;
           if (++stage == C::kStages) {
             stage = 0;
@@ -387,7 +441,12 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
           }
         }
         if (!ok) break;
-        umma_commit(&acc_full[ab]);
+        if (PAIR) {
+          umma_commit_pair(smem_u32(&acc_full[ab]));
+          umma_commit_pair(peer_acc0 + ab * 8);
+        } else {
+          umma_commit(&acc_full[ab]);
+        }
         if (++ab == C::kAcc) {
           ab = 0;
           aph ^= 1u;
@@ -397,7 +456,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
         record_status(P.status, kStatusTimeout);
         *abort_flag = 1;
         if (issued) {  // wait for the MMAs in flight before TMEM is released
-          umma_commit(drain);
+          if (PAIR)
+            umma_commit_pair(smem_u32(drain));
+          else
+            umma_commit(drain);
           mbar_wait(drain, 0, tmo, nullptr);
         }
       }
@@ -412,7 +474,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     int cs = 0;
     uint32_t cph = 0;
     bool ok = true;
-    for (int piece = blockIdx.x; piece < total && ok; piece += gridDim.x) {
+    for (int piece = first_item; piece < total && ok; piece += item_stride) {
       const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
       const bool i8 = P.prob[pc.p].w8 != 0;
       for (int ks = pc.k0; ks < pc.k1; ++ks) {
@@ -476,7 +538,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
     uint8_t* stg = stg_all + (warp - 2) * C::kStgBufs * C::kStgBytes;
     int nstg = 0;  // staging buffers used by this warp so far
     int local = 0;
-    for (int piece = blockIdx.x; piece < total; piece += gridDim.x, ++local) {
+    for (int piece = first_item; piece < total; piece += item_stride, ++local) {
       if ((local & 1) != grp) continue;
       const int ab = local % C::kAcc;
       const uint32_t aph = static_cast<uint32_t>(local / C::kAcc) & 1u;
@@ -496,8 +558,9 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
                              static_cast<uint32_t>(ab * BN);
       const int row = q * 32 + lane;  // accumulator row = TMEM lane
       const int ncols = (pc.n_valid + 15) & ~15;
-      bool last = true;
-      if (pr.split > 1) {
+      const int mt = PAIR ? 2 * pc.m + static_cast<int>(rank) : pc.m;  // this CTA's M tile
+      bool last = mt < pr.m_tiles;  // PAIR: the second tile of an odd count is not stored
+      if (pr.split > 1) {  // (never with PAIR)
         float* part = P.partials + static_cast<size_t>(piece) * BN * 128;
         for (int c0 = 0; c0 < ncols; c0 += 16) {
           float v[16];
@@ -523,8 +586,8 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
         if (pr.wscale) {
           // gate_up row r of the tile: feature 8*(r/16) + r%8 of its 64, gate or up by bit 3
           const int wr = pr.kind == 0
-                             ? pc.m * 64 + 8 * (row >> 4) + (row & 7) + ((row & 8) ? pr.nw : 0)
-                             : pc.m * 128 + row;
+                             ? mt * 64 + 8 * (row >> 4) + (row & 7) + ((row & 8) ? pr.nw : 0)
+                             : mt * 128 + row;
           sc = pr.wscale[static_cast<size_t>(pc.g) * pr.w_rows_per_group + wr];
         }
         for (int c0 = 0; c0 < ncols; c0 += 16) {
@@ -578,7 +641,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
             const int cb = up ? 8 : 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) b16[(cb + i) * 16 + f] = bf16_bits(h[i]);
-            const int fx = pc.m * 64 + 16 * q;  // first output feature of this warp
+            const int fx = mt * 64 + 16 * q;  // first output feature of this warp
             if (c0 + 16 <= pc.n_valid) {
               fence_proxy_async_smem();
               __syncwarp();
@@ -613,7 +676,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
                 for (int i = 0; i < 8; ++i) bh[i * 32 + lane] = bf16_bits(v[8 * hh + i]);
               }
               const int cc = c0 + 8 * hh;
-              const int fx = pc.m * 128 + 32 * q;
+              const int fx = mt * 128 + 32 * q;
               if (cc + 8 <= pc.n_valid) {
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -639,7 +702,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
       }
       tc_fence_before();
       named_sync(bar, 128);  // every flag of this piece is read before the next is written
-      mbar_arrive(&acc_empty[ab]);
+      if (PAIR)
+        mbar_arrive_cluster(cluster_addr(&acc_empty[ab], 0));  // the leader's MMA waits
+      else
+        mbar_arrive(&acc_empty[ab]);
     }
     if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
   }
@@ -647,38 +713,69 @@ __global__ void __launch_bounds__((Cfg<BN, W8>::kThreads), 1)
   // ---- teardown
   tc_fence_before();
   __syncthreads();
+  // PAIR: neither CTA releases TMEM or exits while its peer may still signal it or read
+  // its shared memory
+  if (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if (PAIR)
+      tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else
+      tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
-template <int BN, bool W8>
+template <int BN, bool W8, bool PAIR>
 static cudaError_t launch_bn(const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s,
                              bool pdl) {
-  using C = Cfg<BN, W8>;
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, W8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  using C = Cfg<BN, W8, PAIR>;
+  auto kernel = grouped_gemm_kernel<BN, W8, PAIR>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  return launch_k(grouped_gemm_kernel<BN, W8>, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl,
-                  maps, p);
+  if (!PAIR) return launch_k(kernel, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl, maps, p);
+  // clusters of two CTAs (an even grid), optionally a programmatic dependent launch
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid & ~1);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, maps, p);
 }
 
 template <bool W8>
 static cudaError_t launch_w(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                             cudaStream_t s, bool pdl) {
   switch (bn) {
-    case 16: return launch_bn<16, W8>(maps, p, grid, s, pdl);
-    case 32: return launch_bn<32, W8>(maps, p, grid, s, pdl);
-    case 64: return launch_bn<64, W8>(maps, p, grid, s, pdl);
-    case 128: return launch_bn<128, W8>(maps, p, grid, s, pdl);
-    case 256: return launch_bn<256, W8>(maps, p, grid, s, pdl);
+    case 16: return launch_bn<16, W8, false>(maps, p, grid, s, pdl);
+    case 32: return launch_bn<32, W8, false>(maps, p, grid, s, pdl);
+    case 64: return launch_bn<64, W8, false>(maps, p, grid, s, pdl);
+    case 128: return launch_bn<128, W8, false>(maps, p, grid, s, pdl);
+    case 256: return launch_bn<256, W8, false>(maps, p, grid, s, pdl);
   }
   return cudaErrorInvalidValue;
 }
 
+bool gemm_pairs_allowed(int bn, bool int8_weights) { return !int8_weights && bn >= 128; }
+
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                                 cudaStream_t s, bool pdl) {
+  if (p.pairs) {
+    if (!gemm_pairs_allowed(bn, p.int8_weights != 0)) return cudaErrorInvalidValue;
+
+    if (bn == 128) return launch_bn<128, false, true>(maps, p, grid, s, pdl);
+    if (bn == 256) return launch_bn<256, false, true>(maps, p, grid, s, pdl);
+    return cudaErrorInvalidValue;
+  }
   return p.int8_weights ? launch_w<true>(bn, maps, p, grid, s, pdl)
                         : launch_w<false>(bn, maps, p, grid, s, pdl);
 }

@@ -39,6 +39,7 @@ struct GemmParams {
   GemmProblem prob[2];
   int nprob;
   int int8_weights;     // a problem has int8 A: use the variant with converter warps
+  int pairs;            // run on CTA pairs (see gemm_pairs_allowed)
   float* partials;      // split-K partial tiles, [piece][BN][128] fp32
   unsigned* counters;   // split-K arrival counters, zero between launches
   unsigned* status;     // device status word
@@ -87,11 +88,14 @@ cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t*
 int router_counters(int T);
 
 // The tensor-core router (router_tc.cu) serves batches of more than kRouterTcMinT
-// tokens.  It needs two E x H bf16 buffers for the split W' = s * W_r / sqrt(H) and
-// the tensor maps below: x [T][H] with 64 x 128 boxes, W'hi and W'lo [E][H] with
-// 64 x ne boxes (ne = E rounded up to 16), all with 128-byte swizzling.
+// tokens.  It needs two E x H bf16 buffers for the split W' = s * W_r / sqrt(H), the
+// logits buffer [T][E] fp32 and one counter per 128 tokens when it splits the experts
+// into router_tc_slices(T, E) > 1 slices, and the tensor maps below: x [T][H] with
+// 64 x 128 boxes, W'hi and W'lo [E][H] with 64 x (E rounded up to 16) / slices boxes,
+// all with 128-byte swizzling.
 constexpr int kRouterTcMinT = 128;
 bool router_uses_tc(int T);
+int router_tc_slices(int T, int E);
 struct RouterTcMaps {
   CUtensorMap x, whi, wlo;
 };
@@ -100,8 +104,9 @@ cudaError_t launch_router_tc(const RouterTcMaps& maps, int T, int H, int E, int 
                              uint16_t* whi, uint16_t* wlo, const float* bias,
                              const uint16_t* per_expert_scale, const uint16_t* g_pre_moe,
                              const uint16_t* g_pre_dense, uint16_t* xn_moe, uint16_t* xn_dense,
-                             int* topk_idx, float* topk_w, unsigned* status,
-                             uint64_t timeout_ns, cudaStream_t s, bool pdl = false);
+                             int* topk_idx, float* topk_w, float* logits, unsigned* counters,
+                             unsigned* status, uint64_t timeout_ns, cudaStream_t s,
+                             bool pdl = false);
 cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int* sorted_src,
                            int* inv_pos, int* block_hist, int* block_base, cudaStream_t s,
                            bool pdl = false);
@@ -109,6 +114,12 @@ int permute_blocks(int n);  // blocks of the multi-block path, <= 256 (0 = singl
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
                                const uint16_t* src, uint16_t* dst, cudaStream_t s,
                                bool pdl = false);
+// A launch may run on CTA pairs (GemmParams::pairs) when its weights are bf16 and its
+// token tiles are 128 or 256 wide; its B maps then take boxes of bn / 2 rows (each CTA
+// loads half of a tile's token rows), and the grid is even.  A pair takes two M tiles:
+// with an odd count the second CTA of the last pair computes on zero or foreign weight
+// rows and stores nothing.
+bool gemm_pairs_allowed(int bn, bool int8_weights);
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                                 cudaStream_t s, bool pdl = false);
 // y holds the expert outputs in sorted order (row inv_pos[t*k+j] for slot j of token

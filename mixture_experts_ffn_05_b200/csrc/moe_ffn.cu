@@ -314,6 +314,19 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     return w8 ? encode_raw(m, base, rows, cols, box_rows, int8)
               : encode_bf16(m, base, rows, cols, box_rows);
   };
+  // CTA pairs load half of each token tile.  A pair takes two M tiles; with an odd count
+  // the last pair's second tile is idle, which costs more than pairs save when the tiles
+  // are full (tensor-bound), and less when most tiles are partly filled (weight-stream
+  // bound: mean tokens per expert below the tile width).
+  const bool pairs_ok = gemm_pairs_allowed(L.bn, w8);
+  const bool streaming = static_cast<double>(d.T) * d.k / d.E < L.bn;
+  const bool gu_pairs = pairs_ok && (streaming || ((!j.experts || (d.I / 64) % 2 == 0) &&
+                                                   (!j.dense || (d.D / 64) % 2 == 0)));
+  const bool dn_pairs = pairs_ok && (streaming || (d.H / 128) % 2 == 0);
+  gu.pairs = gu_pairs ? 1 : 0;
+  dn.pairs = dn_pairs ? 1 : 0;
+  const int bbox_gu = gu_pairs ? L.bn / 2 : L.bn;
+  const int bbox_dn = dn_pairs ? L.bn / 2 : L.bn;
   int np = 0;
   if (j.experts) {
     GemmProblem& a = gu.prob[np];
@@ -333,10 +346,10 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.out_ld = d.H;
     b.wscale = j.s_down; b.w8 = d.int8;
     if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, w8, d.int8) ||
-        !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, L.bn) ||
+        !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, bbox_gu) ||
         !encode_h_out(&mgu.o[np], h, Tk, d.I) ||
         !encode_a(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128, d.int8) ||
-        !encode_bf16(&mdn.b[np], h, Tk, d.I, L.bn) ||
+        !encode_bf16(&mdn.b[np], h, Tk, d.I, bbox_dn) ||
         !encode_y_out(&mdn.o[np], j.y, Tk, d.H, true))
       return MOE_ERR_CUDA;
     ++np;
@@ -354,10 +367,10 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.split = L.split_dd; b.map = np; b.out = j.dense_out; b.out_f32 = j.dense_f32;
     b.out_ld = d.H;
     if (!encode_gate_up(&mgu.a[np], j.w_dgu, 1, d.D, d.H, w8, false) ||
-        !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, L.bn) ||
+        !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, bbox_gu) ||
         !encode_h_out(&mgu.o[np], hd, d.T, d.D) ||
         !encode_a(&mdn.a[np], j.w_dd, d.H, d.D, 128, false) ||
-        !encode_bf16(&mdn.b[np], hd, d.T, d.D, L.bn) ||
+        !encode_bf16(&mdn.b[np], hd, d.T, d.D, bbox_dn) ||
         !encode_y_out(&mdn.o[np], j.dense_out, d.T, d.H, j.dense_f32 != 0))
       return MOE_ERR_CUDA;
     ++np;
@@ -411,7 +424,7 @@ moe_status_t run_router(const Dims& d, const Layout& L, void* ws, const RouteJob
                                      status, r.offsets, r.sorted_src, r.inv_pos, s));
   uint16_t* whi = at<uint16_t>(ws, L.wr_hi);
   uint16_t* wlo = at<uint16_t>(ws, L.wr_lo);
-  const int ne = (d.E + 15) / 16 * 16;
+  const int ne = (d.E + 15) / 16 * 16 / router_tc_slices(d.T, d.E);  // experts per CTA
   if (r.offsets != nullptr) return MOE_ERR_INVALID_ARG;  // no fused sort on this path
   RouterTcMaps m;
   if (!encode_bf16(&m.x, r.x, d.T, d.H, 128) || !encode_bf16(&m.whi, whi, d.E, d.H, ne) ||
@@ -420,7 +433,8 @@ moe_status_t run_router(const Dims& d, const Layout& L, void* ws, const RouteJob
   return cuda_status(launch_router_tc(m, d.T, d.H, d.E, d.k, d.eps, r.w_router, r.router_scale,
                                       whi, wlo, r.logit_bias, r.per_expert_scale, r.g_pre_moe,
                                       r.g_pre_dense, r.xn_moe, r.xn_dense, r.topk_idx, r.topk_w,
-                                      status, kWaitTimeoutNs, s));
+                                      at<float>(ws, L.logits), counters, status, kWaitTimeoutNs,
+                                      s));
 }
 
 bool w_ok(const moe_expert_weights_t* w, bool int8) {

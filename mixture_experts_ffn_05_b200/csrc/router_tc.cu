@@ -13,14 +13,19 @@
 // x.W'lo into the same fp32 accumulator, so the logits carry the accuracy of an fp32 dot
 // product (every bf16 x bf16 product is exact in fp32).
 //
-// One CTA per 128 tokens (the 128 TMEM lanes), all E experts as the N dimension.
+// One CTA per 128 tokens (the 128 TMEM lanes) and slice of the experts (the N dimension:
+// all E experts when the batch has enough token tiles to fill the GPU, else E/2, E/4 or
+// E/8 of them, so that small batches still spread over most SMs).
 // Warp roles:
 //   0      TMA producer: per 64-wide K step the x tile and the W'hi, W'lo tiles
 //          (phase 1), then the x tiles again, several per ring stage (phase 2);
 //   1      MMA issuer (two MMAs per 16 K) and TMEM owner;
 //   2..5   sums of x^2 of one token row per thread, read from the x tiles of phase 1;
-//          afterwards the top-k of the same row from its TMEM lane;
-//   6..13  phase 2: xn_moe = x * rinv * g_pre_moe and xn_dense = x * rinv * g_pre_dense.
+//          afterwards the top-k of the same row from its TMEM lane (one expert slice),
+//          or the row's logits of the slice to global memory (several slices: the last
+//          CTA of a token tile to finish then takes the top-k of its 128 tokens);
+//   6..13  phase 2: xn_moe = x * rinv * g_pre_moe and xn_dense = x * rinv * g_pre_dense,
+//          for the CTA's share of the columns (its slice of the 64-wide K steps).
 // Every wait is bounded.
 #include <algorithm>
 
@@ -39,7 +44,8 @@ constexpr int kTcMaxE = 256;
 
 struct RouterTcArgs {
   int T, H, E, k;
-  int ne;               // E rounded up to a multiple of 16 (the MMA N)
+  int ne;               // experts per CTA (a multiple of 16: the MMA N)
+  int slices;           // expert slices (gridDim.y); ne * slices >= E
   int stages;           // ring stages
   int stage_bytes;      // x tile + W'hi tile + W'lo tile
   int tiles_per_stage;  // x tiles per stage in phase 2
@@ -52,6 +58,8 @@ struct RouterTcArgs {
   uint16_t* xn_dense;
   int* topk_idx;
   float* topk_w;
+  float* logits;       // [T][E], several slices only
+  unsigned* counters;  // one per token tile, zero on entry and on exit (several slices)
   unsigned* status;
   uint64_t timeout_ns;
 };
@@ -67,6 +75,66 @@ __device__ __forceinline__ uint32_t order_key(float l) {
 __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
+
+// Top-k of one token's logits, fed in ascending expert order: a strictly larger key
+// enters the sorted list, so among equal logits the lower expert id comes first.
+template <int KMAX>
+struct TopK {
+  uint32_t key[KMAX];
+  int id[KMAX];
+
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      key[j] = 0u;
+      id[j] = 0;
+    }
+  }
+
+  __device__ __forceinline__ void push(float l, int e) {
+    uint32_t ck = order_key(l);
+    if (ck > key[KMAX - 1]) {
+      int ci = e;
+      bool shift = false;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        const bool g = shift || ck > key[j];
+        const uint32_t tk = g ? key[j] : ck;
+        const int ti = g ? id[j] : ci;
+        key[j] = g ? ck : key[j];
+        id[j] = g ? ci : id[j];
+        ck = tk;
+        ci = ti;
+        shift = g;
+      }
+    }
+  }
+
+  // softmax restricted to the selected experts (the full denominator cancels in the
+  // renormalisation), summed in slot order; then per_expert_scale
+  __device__ __forceinline__ void write(int t, int k, const uint16_t* pes, int* topk_idx,
+                                        float* topk_w) const {
+    const float top = key_value(key[0]);
+    float ex[KMAX];
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ex[j] = 0.f;
+      if (j < k) {
+        ex[j] = expf(key_value(key[j]) - top);
+        sum += ex[j];
+      }
+    }
+    int* oi = topk_idx + static_cast<size_t>(t) * k;
+    float* ow = topk_w + static_cast<size_t>(t) * k;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j < k) {
+        oi[j] = id[j];
+        ow[j] = ex[j] / sum * __uint_as_float(static_cast<uint32_t>(pes[id[j]]) << 16);
+      }
+  }
+};
 
 // All lanes wait; the warp continues only if every lane saw the phase complete.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
@@ -89,14 +157,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   __shared__ float s_rinv[kTcTokens];
+  __shared__ int s_last;
   __shared__ float s_bias[kTcMaxE];
   __shared__ uint16_t s_pes[kTcMaxE];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kTcTokens;
+  const int e0 = blockIdx.y * a.ne;  // first expert of this CTA's slice
   const int KS = a.H / 64;
   const int S = a.stages;
-  const int J2 = (KS + a.tiles_per_stage - 1) / a.tiles_per_stage;
+  // phase 2 covers this slice's share of the K steps
+  const int ks0 = static_cast<int>(blockIdx.y) * KS / a.slices;
+  const int ks1 = static_cast<int>(blockIdx.y + 1) * KS / a.slices;
+  const int J2 = (ks1 - ks0 + a.tiles_per_stage - 1) / a.tiles_per_stage;
   const uint32_t b_bytes = static_cast<uint32_t>(a.ne) * 128u;
   const uint32_t tmem_cols = a.ne <= 32 ? 32u : a.ne <= 64 ? 64u : a.ne <= 128 ? 128u : 256u;
 
@@ -154,11 +227,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (j < KS) {
           mbar_arrive_expect_tx(&full[s], kTcTile + 2 * b_bytes);
           tma_load_2d(st, &maps.x, &full[s], j * 64, t0, keep);
-          tma_load_2d(st + kTcTile, &maps.whi, &full[s], j * 64, 0, keep);
-          tma_load_2d(st + kTcTile + b_bytes, &maps.wlo, &full[s], j * 64, 0, keep);
+          tma_load_2d(st + kTcTile, &maps.whi, &full[s], j * 64, e0, keep);
+          tma_load_2d(st + kTcTile + b_bytes, &maps.wlo, &full[s], j * 64, e0, keep);
         } else {
-          const int q0 = (j - KS) * a.tiles_per_stage;
-          const int nt = min(a.tiles_per_stage, KS - q0);
+          const int q0 = ks0 + (j - KS) * a.tiles_per_stage;
+          const int nt = min(a.tiles_per_stage, ks1 - q0);
           mbar_arrive_expect_tx(&full[s], nt * kTcTile);
           for (int i = 0; i < nt; ++i)
             tma_load_2d(st + i * kTcTile, &maps.x, &full[s], (q0 + i) * 64, t0, keep);
@@ -247,65 +320,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     } else {
       tc_fence_after();
-      // top-k of this row's logits, experts in ascending order; a strictly larger key
-      // enters the sorted list, so among equal logits the lower expert id comes first
-      uint32_t key[KMAX];
-      int id[KMAX];
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        key[j] = 0u;
-        id[j] = 0;
-      }
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c = 0; c < a.ne; c += 16) {
-        float v[16];
-        tmem_ld16(lane_base + c, v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int e = c + i;
-          if (e < a.E) {
-            uint32_t ck = order_key(v[i] * rinv + s_bias[e]);
-            if (ck > key[KMAX - 1]) {
-              int ci = e;
-              bool shift = false;
-#pragma unroll
-              for (int j = 0; j < KMAX; ++j) {
-                const bool g = shift || ck > key[j];
-                const uint32_t tk = g ? key[j] : ck;
-                const int ti = g ? id[j] : ci;
-                key[j] = g ? ck : key[j];
-                id[j] = g ? ci : id[j];
-                ck = tk;
-                ci = ti;
-                shift = g;
-              }
-            }
-          }
-        }
-      }
       const int t = t0 + r;
-      if (t < a.T) {
-        // softmax restricted to the selected experts (the full denominator cancels in
-        // the renormalisation), summed in slot order; then per_expert_scale
-        const float top = key_value(key[0]);
-        float ex[KMAX];
-        float sum = 0.f;
+      if (a.slices == 1) {
+        TopK<KMAX> tk;
+        tk.init();
+        for (int c = 0; c < a.ne; c += 16) {
+          float v[16];
+          tmem_ld16(lane_base + c, v);
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-          ex[j] = 0.f;
-          if (j < a.k) {
-            ex[j] = expf(key_value(key[j]) - top);
-            sum += ex[j];
+          for (int i = 0; i < 16; ++i)
+            if (c + i < a.E) tk.push(v[i] * rinv + s_bias[c + i], c + i);
+        }
+        if (t < a.T) tk.write(t, a.k, s_pes, a.topk_idx, a.topk_w);
+      } else {
+        // the slice's logits to global memory; the last CTA of the tile selects
+        for (int c = 0; c < a.ne; c += 16) {
+          float v[16];
+          tmem_ld16(lane_base + c, v);
+          if (t < a.T) {
+            float* lr = a.logits + static_cast<size_t>(t) * a.E + e0 + c;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (e0 + c + i < a.E) lr[i] = v[i] * rinv + s_bias[e0 + c + i];
           }
         }
-        int* oi = a.topk_idx + static_cast<size_t>(t) * a.k;
-        float* ow = a.topk_w + static_cast<size_t>(t) * a.k;
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-          if (j < a.k) {
-            oi[j] = id[j];
-            ow[j] = ex[j] / sum * __uint_as_float(static_cast<uint32_t>(s_pes[id[j]]) << 16);
-          }
       }
     }
   } else {
@@ -324,8 +363,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       const uint8_t* st = ring + static_cast<size_t>(s) * a.stage_bytes;
-      const int q0 = (j - KS) * a.tiles_per_stage;
-      const int nt = min(a.tiles_per_stage, KS - q0);
+      const int q0 = ks0 + (j - KS) * a.tiles_per_stage;
+      const int nt = min(a.tiles_per_stage, ks1 - q0);
       for (int i = 0; i < nt; ++i) {
         const uint8_t* tile = st + i * kTcTile;
         const int cb = (q0 + i) * 8;  // first 8-wide chunk of this tile's columns
@@ -363,6 +402,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }
+  if (a.slices == 1) return;
+
+  // ---- several slices: the last CTA of this token tile to finish takes the top-k
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned old = atomicAdd(a.counters + blockIdx.x, 1u);
+    s_last = old == gridDim.y - 1;
+    if (s_last) {
+      a.counters[blockIdx.x] = 0u;
+      __threadfence();
+    }
+  }
+  __syncthreads();
+  if (!s_last || threadIdx.x < 64 || threadIdx.x >= 64 + kTcTokens) return;
+  const int t = t0 + static_cast<int>(threadIdx.x) - 64;
+  if (t >= a.T) return;
+  TopK<KMAX> tk;
+  tk.init();
+  const float* lr = a.logits + static_cast<size_t>(t) * a.E;
+  for (int e = 0; e < a.E; ++e) tk.push(__ldcg(lr + e), e);
+  tk.write(t, a.k, s_pes, a.topk_idx, a.topk_w);
 }
 
 // W'hi, W'lo = the two-term bf16 split of s[h] * W_r[e,h] / sqrt(H); one thread per 8.
@@ -392,6 +452,14 @@ __global__ void __launch_bounds__(256) router_prep_kernel(int E, int H, float in
 
 bool router_uses_tc(int T) { return T > kRouterTcMinT; }
 
+int router_tc_slices(int T, int E) {
+  const int tiles = (T + kTcTokens - 1) / kTcTokens;
+  const int groups16 = (E + 15) / 16;  // every slice is a multiple of 16 experts
+  int sl = 1;
+  while (sl < 8 && tiles * sl * 2 <= 148 && groups16 % (sl * 2) == 0) sl *= 2;
+  return sl;
+}
+
 template <int KMAX>
 static cudaError_t launch_tc(const RouterTcMaps& maps, const RouterTcArgs& a, size_t smem,
                              cudaStream_t s) {
@@ -399,8 +467,9 @@ static cudaError_t launch_tc(const RouterTcMaps& maps, const RouterTcArgs& a, si
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_k(router_tc_kernel<KMAX>, dim3((a.T + kTcTokens - 1) / kTcTokens),
-                  dim3(kTcThreads), smem, s, true, maps, a);
+  return launch_k(router_tc_kernel<KMAX>,
+                  dim3((a.T + kTcTokens - 1) / kTcTokens, a.slices), dim3(kTcThreads), smem, s,
+                  true, maps, a);
 }
 
 cudaError_t launch_router_tc(const RouterTcMaps& maps, int T, int H, int E, int k, float eps,
@@ -408,8 +477,8 @@ cudaError_t launch_router_tc(const RouterTcMaps& maps, int T, int H, int E, int 
                              uint16_t* whi, uint16_t* wlo, const float* bias,
                              const uint16_t* per_expert_scale, const uint16_t* g_pre_moe,
                              const uint16_t* g_pre_dense, uint16_t* xn_moe, uint16_t* xn_dense,
-                             int* topk_idx, float* topk_w, unsigned* status,
-                             uint64_t timeout_ns, cudaStream_t s, bool pdl) {
+                             int* topk_idx, float* topk_w, float* logits, unsigned* counters,
+                             unsigned* status, uint64_t timeout_ns, cudaStream_t s, bool pdl) {
   const int64_t nch = static_cast<int64_t>(E) * (H / 8);
   cudaError_t e = launch_k(router_prep_kernel, dim3(static_cast<unsigned>((nch + 255) / 256)),
                            dim3(256), 0, s, pdl, E, H, 1.0f / sqrtf(static_cast<float>(H)),
@@ -417,14 +486,15 @@ cudaError_t launch_router_tc(const RouterTcMaps& maps, int T, int H, int E, int 
   if (e != cudaSuccess) return e;
   RouterTcArgs a{};
   a.T = T; a.H = H; a.E = E; a.k = k;
-  a.ne = (E + 15) / 16 * 16;
+  a.slices = router_tc_slices(T, E);
+  a.ne = (E + 15) / 16 * 16 / a.slices;
   a.stage_bytes = static_cast<int>(kTcTile) + 2 * a.ne * 128;
   a.stages = std::min(kTcMaxStages, kTcSmemBudget / a.stage_bytes);
   a.tiles_per_stage = a.stage_bytes / static_cast<int>(kTcTile);
   a.eps = eps;
   a.bias = bias; a.pes = per_expert_scale; a.gm = g_pre_moe; a.gd = g_pre_dense;
   a.xn_moe = xn_moe; a.xn_dense = xn_dense; a.topk_idx = topk_idx; a.topk_w = topk_w;
-  a.status = status; a.timeout_ns = timeout_ns;
+  a.logits = logits; a.counters = counters; a.status = status; a.timeout_ns = timeout_ns;
   const size_t smem = static_cast<size_t>(a.stages) * a.stage_bytes + 1024;
   return k <= 8 ? launch_tc<8>(maps, a, smem, s) : launch_tc<16>(maps, a, smem, s);
 }
