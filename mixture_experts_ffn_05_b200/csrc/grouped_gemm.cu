@@ -257,9 +257,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
   }
   // the peer's barriers are initialised before either CTA signals the other
   if (PAIR) cluster_sync();
-  // everything above overlaps the previous kernel on the stream; its results (routing,
-  // gathered rows, h) are read only below
-  pdl_wait();
+  // Everything up to the producer's first token-tile load overlaps the previous kernel
+  // on the stream.  The routing tables read here (offsets) come from kernels that
+  // completed before that kernel started; only the token tiles (gathered rows, h) are
+  // its own results, and the producer loads them after the dependency wait.
   pdl_trigger();
   for (int i = threadIdx.x; i < nent; i += C::kThreads) {
     const int p = i < P.prob[0].groups ? 0 : 1;
@@ -318,6 +319,32 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       int armed[C::kStages];
       for (int i = 0; i < C::kStages; ++i) armed[i] = -1;
       bool ok = true;
+      // Weight tiles are never written by an earlier kernel, so the first ring fill of
+      // them is issued before the dependency wait; the token-tile loads of those stages
+      // are held here and issued after it.
+      bool waited = false;
+      int nd = 0, steps = 0;
+      uint8_t* d_dst[2 * C::kStages];
+      const CUtensorMap* d_map[2 * C::kStages];
+      int d_c0[2 * C::kStages], d_c1[2 * C::kStages];
+      uint64_t* d_bar[2 * C::kStages];
+      auto load_b = [&](uint8_t* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+        if (waited) {
+          if (PAIR)
+            tma_load_2d_pair(dst, map, cluster_addr(bar, 0), c0, c1, pol_b);
+          else
+            tma_load_2d(dst, map, bar, c0, c1, pol_b);
+        } else {
+          d_dst[nd] = dst; d_map[nd] = map; d_c0[nd] = c0; d_c1[nd] = c1; d_bar[nd] = bar;
+          ++nd;
+        }
+      };
+      auto release_b = [&]() {
+        pdl_wait();
+        waited = true;
+        for (int i = 0; i < nd; ++i) load_b(d_dst[i], d_map[i], d_c0[i], d_c1[i], d_bar[i]);
+        nd = 0;
+      };
       for (int piece = first_item; piece < total && ok; piece += item_stride) {
         const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
         const GemmProblem& pr = P.prob[pc.p];
@@ -332,10 +359,12 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         const int half = ((pc.n_valid + 15) & ~15) >> 1;
         const int brow = pc.b_row0 + pc.n * BN + (PAIR ? static_cast<int>(rank) * half : 0);
         for (int ks = pc.k0; ks < pc.k1; ++ks) {
+          if (!waited && steps == C::kStages) release_b();  // the ring is full
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
             ok = false;
             break;
           }
+          ++steps;
           uint8_t* sa = smem + stage * C::kStage;
           // a step covers 64 K (bf16 weights) or 128 K (int8 codes, two B sub-tiles);
           // the A tile is 16 KB either way
@@ -349,7 +378,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
               tma_load_5d_pair(sa, ma, fb, ks * 64, 0, 0, mt * 8, pc.g, pol_w);
             else
               tma_load_2d_pair(sa, ma, fb, ks * 64, arow, pol_w);
-            tma_load_2d_pair(sa + C::kABytes, mb, fb, ks * 64, brow, pol_b);
+            load_b(sa + C::kABytes, mb, ks * 64, brow, &full[stage]);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kABytes + nb * C::kBBytes);
             if (pr.kind == 0)  // 8 gate rows, the 8 matching up rows, ... (one 5-D box)
@@ -357,8 +386,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
             else
               tma_load_2d(sa, ma, &full[stage], ks * kw, arow, pol_w);
             for (int b = 0; b < nb; ++b)
-              tma_load_2d(sa + C::kABytes + b * C::kBBytes, mb, &full[stage], ks * kw + 64 * b,
-                          brow, pol_b);
+              load_b(sa + C::kABytes + b * C::kBBytes, mb, ks * kw + 64 * b, brow, &full[stage]);
           }
           armed[stage] = static_cast<int>(phase);
           if (++stage == C::kStages) {
@@ -367,6 +395,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
           }
         }
       }
+      if (!waited) release_b();  // fewer steps than stages, or a wait that gave up
       if (!ok) {
         record_status(P.status, kStatusTimeout);
         *abort_flag = 1;
