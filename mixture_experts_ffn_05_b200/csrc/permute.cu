@@ -124,30 +124,46 @@ cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int*
                   topk_idx, (const int*)block_base, sorted_src, inv_pos);
 }
 
-// dst[q] = src[sorted_src[q] / k] for the n sorted pairs; one thread per 16 bytes.
-// A pair index outside [0, T*k) yields a zero row (never an out-of-bounds read).
-__global__ void __launch_bounds__(256) gather_rows_kernel(int n, int k, int H, int T,
-                                                          const int* __restrict__ sorted_src,
-                                                          const uint16_t* __restrict__ src,
-                                                          uint16_t* __restrict__ dst) {
+// dst[q] = src[sorted_src[q] / k] for the n sorted pairs.  One warp per row: each lane
+// requests up to 8 of the row's 16-byte chunks before storing any, so a warp keeps
+// 4 KB of loads in flight.  A pair index outside [0, T*k) yields a zero row (never an
+// out-of-bounds read).
+constexpr int kGatherWarps = 8;
+
+__global__ void __launch_bounds__(32 * kGatherWarps) gather_rows_kernel(
+    int n, int k, int H, int T, const int* __restrict__ sorted_src,
+    const uint16_t* __restrict__ src, uint16_t* __restrict__ dst) {
   const int nch = H >> 3;
   pdl_wait();
   pdl_trigger();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
-  if (i >= static_cast<int64_t>(n) * nch) return;
-  const int q = static_cast<int>(i / nch), c = static_cast<int>(i % nch);
+  const int q = static_cast<int>(blockIdx.x) * kGatherWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (q >= n) return;
   const int p = sorted_src[q];
   const int t = (p >= 0 && p < n) ? p / k : -1;
-  uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (t >= 0 && t < T) v = __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * H) + c);
-  reinterpret_cast<uint4*>(dst + static_cast<size_t>(q) * H)[c] = v;
+  const uint4* s = (t >= 0 && t < T) ? reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * H)
+                                     : nullptr;
+  uint4* d = reinterpret_cast<uint4*>(dst + static_cast<size_t>(q) * H);
+  for (int c0 = lane; c0 < nch; c0 += 32 * 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + 32 * u;
+      v[u] = (s != nullptr && c < nch) ? __ldg(s + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nch) d[c] = v[u];
+    }
+  }
 }
 
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
                                const uint16_t* src, uint16_t* dst, cudaStream_t s, bool pdl) {
-  const int64_t total = static_cast<int64_t>(n) * (H >> 3);
-  return launch_k(gather_rows_kernel, dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256),
-                  0, s, pdl, n, k, H, T, sorted_src, src, dst);
+  const int blocks = (n + kGatherWarps - 1) / kGatherWarps;
+  return launch_k(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)),
+                  dim3(32 * kGatherWarps), 0, s, pdl, n, k, H, T, sorted_src, src, dst);
 }
 
 }  // namespace moe
