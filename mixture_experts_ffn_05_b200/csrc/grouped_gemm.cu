@@ -72,9 +72,17 @@ struct Cfg {
   // after the stages: converted stages, barriers, bookkeeping, the gate/up exchange buffer
   static constexpr int kConvOff = kStages * kStage;
   static constexpr int kBarOff = kConvOff + kConv * kConvBytes;
-  static constexpr int kNumBars = 2 * kStages + 2 * kConv + 2 * kAcc + 1;
+  // Single CTAs with wide tiles take their pieces from a global counter (the fastest SMs
+  // take more, which shortens the tail of long pieces); the producer passes them to the
+  // other roles through a queue of kQ slots.  Narrow (weight-streaming) tiles keep the
+  // round-robin deal, which measured faster for their short pieces.
+  static constexpr bool kDyn = !PAIR && BN >= 64;
+  static constexpr int kQ = 8;
+  static constexpr int kQConsumers = 1 + 2 + (W8 ? kConvWarps : 0);  // MMA, 2 groups, converters
+  static constexpr int kNumBars = 2 * kStages + 2 * kConv + 2 * kAcc + 1 + 2 * kQ;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kMiscInts = 8;               // tmem slot, abort, bcast x2, converter flag
+  // tmem slot, abort, bcast x2, group piece broadcast 2 x 2, queue slots
+  static constexpr int kMiscInts = 8 + kQ;
   static constexpr int kPreOff = kMiscOff + kMiscInts * 4;
   static constexpr int kTabInts = 4 * kMaxEntries;  // pre, cnt, b0, ng
   // output staging for the TMA stores: two 1 KB buffers per epilogue warp (one where
@@ -203,10 +211,14 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
   uint64_t* acc_full = conv_empty + C::kConv;
   uint64_t* acc_empty = acc_full + C::kAcc;
   uint64_t* drain = acc_empty + C::kAcc;
+  uint64_t* q_full = drain + 1;
+  uint64_t* q_empty = q_full + C::kQ;
   int* misc = reinterpret_cast<int*>(smem + C::kMiscOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 0);
   volatile int* abort_flag = misc + 1;
   volatile int* bcast = misc + 2;        // [2], one per epilogue group
+  volatile int* gpiece = misc + 4;       // [2][2]: each group's piece ids, by parity
+  volatile int* q_piece = misc + 8;      // [kQ]
   int* pre = reinterpret_cast<int*>(smem + C::kPreOff);
   int* cnt = pre + kMaxEntries;
   int* b0 = cnt + kMaxEntries;
@@ -237,6 +249,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       mbar_init(&acc_empty[i], PAIR ? 256 : 128);  // PAIR: both CTAs' epilogues (leader's)
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < C::kQ; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], C::kQConsumers);
+    }
     mbar_fence_init();
     *abort_flag = 0;
     tma_prefetch_map(&maps.a[0]);
@@ -309,6 +325,27 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
   const int total = pre[nent];
   const uint64_t tmo = P.timeout_ns;
 
+  // The piece queue (kDyn): the producer pushes each piece it takes, then -1; every
+  // consumer role pops the same sequence (one elected thread per role).
+  auto q_push = [&](int n_pushed, int v) -> bool {
+    const int slot = n_pushed % C::kQ;
+    if (n_pushed >= C::kQ &&
+        !mbar_wait(&q_empty[slot], static_cast<uint32_t>((n_pushed / C::kQ) - 1) & 1u, tmo,
+                   abort_flag))
+      return false;
+    q_piece[slot] = v;
+    mbar_arrive(&q_full[slot]);
+    return true;
+  };
+  auto q_pop = [&](int n_popped, int* v) -> bool {
+    const int slot = n_popped % C::kQ;
+    if (!mbar_wait(&q_full[slot], static_cast<uint32_t>(n_popped / C::kQ) & 1u, tmo, abort_flag))
+      return false;
+    *v = q_piece[slot];
+    mbar_arrive(&q_empty[slot]);
+    return true;
+  };
+
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
@@ -345,7 +382,15 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         for (int i = 0; i < nd; ++i) load_b(d_dst[i], d_map[i], d_c0[i], d_c1[i], d_bar[i]);
         nd = 0;
       };
-      for (int piece = first_item; piece < total && ok; piece += item_stride) {
+      int n_pushed = 0;
+      int piece = C::kDyn ? static_cast<int>(atomicAdd(P.sched, 1u)) : first_item;
+      for (; piece < total && ok;) {
+        // the next piece is taken one ahead, so the atomic's latency hides behind loads
+        const int next = C::kDyn ? static_cast<int>(atomicAdd(P.sched, 1u)) : piece + item_stride;
+        if (C::kDyn && !q_push(n_pushed++, piece)) {
+          ok = false;
+          break;
+        }
         const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
         const GemmProblem& pr = P.prob[pc.p];
         const CUtensorMap* ma = &maps.a[pr.map];
@@ -394,7 +439,9 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
             phase ^= 1u;
           }
         }
+        piece = next;
       }
+      if (C::kDyn && ok && !q_push(n_pushed++, -1)) ok = false;  // end of the sequence
       if (!waited) release_b();  // fewer steps than stages, or a wait that gave up
       if (!ok) {
         record_status(P.status, kStatusTimeout);
@@ -419,7 +466,13 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       // PAIR: stage and accumulator releases go to the barriers of both CTAs
       const uint32_t peer_empty0 = PAIR ? cluster_addr(&empty[0], 1) : 0u;
       const uint32_t peer_acc0 = PAIR ? cluster_addr(&acc_full[0], 1) : 0u;
-      for (int piece = first_item; piece < total && ok; piece += item_stride) {
+      int n_popped = 0;
+      for (int piece = first_item; ok; piece += item_stride) {
+        if (C::kDyn && !q_pop(n_popped++, &piece)) {
+          ok = false;
+          break;
+        }
+        if (piece < 0 || piece >= total) break;
         const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
         const uint32_t idesc = idesc_bf16_f32(PAIR ? 256 : 128, (pc.n_valid + 15) & ~15);
         if (!mbar_wait(&acc_empty[ab], aph ^ 1u, tmo, abort_flag)) {
@@ -503,7 +556,19 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
     int cs = 0;
     uint32_t cph = 0;
     bool ok = true;
-    for (int piece = first_item; piece < total && ok; piece += item_stride) {
+    int n_popped = 0;
+    for (int piece = first_item; ok; piece += item_stride) {
+      if (C::kDyn) {
+        int v = -2;
+        if (lane == 0 && !q_pop(n_popped, &v)) v = -2;
+        ++n_popped;
+        piece = __shfl_sync(0xffffffffu, v, 0);
+        if (piece == -2) {
+          ok = false;
+          break;
+        }
+      }
+      if (piece < 0 || piece >= total) break;
       const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
       const bool i8 = P.prob[pc.p].w8 != 0;
       for (int ks = pc.k0; ks < pc.k1; ++ks) {
@@ -567,7 +632,26 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
     uint8_t* stg = stg_all + (warp - 2) * C::kStgBufs * C::kStgBytes;
     int nstg = 0;  // staging buffers used by this warp so far
     int local = 0;
-    for (int piece = first_item; piece < total; piece += item_stride, ++local) {
+    for (int piece = first_item;; piece += item_stride, ++local) {
+      if (C::kDyn) {
+        // the group's elected thread pops; the slot alternates by parity, so it is not
+        // rewritten before every thread of the group has read it
+        volatile int* slot = gpiece + 2 * grp + (local & 1);
+        if (et == 0) {
+          int v = -2;
+          *slot = q_pop(local, &v) ? v : -2;
+        }
+        named_sync(bar, 128);
+        piece = *slot;
+        if (piece == -2) {
+          if (et == 0) {
+            record_status(P.status, kStatusTimeout);
+            *abort_flag = 1;
+          }
+          break;
+        }
+      }
+      if (piece < 0 || piece >= total) break;
       if ((local & 1) != grp) continue;
       const int ab = local % C::kAcc;
       const uint32_t aph = static_cast<uint32_t>(local / C::kAcc) & 1u;
@@ -742,6 +826,15 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
   // ---- teardown
   tc_fence_before();
   __syncthreads();
+  if (C::kDyn && threadIdx.x == 0) {
+    // the last CTA to finish returns the piece counter to zero for the next launch
+    __threadfence();
+    if (atomicAdd(P.sched + 1, 1u) == gridDim.x - 1) {
+      P.sched[0] = 0u;
+      P.sched[1] = 0u;
+      __threadfence();
+    }
+  }
   // PAIR: neither CTA releases TMEM or exits while its peer may still signal it or read
   // its shared memory
   if (PAIR) cluster_sync();

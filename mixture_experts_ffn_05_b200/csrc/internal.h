@@ -42,6 +42,8 @@ struct GemmParams {
   int pairs;            // run on CTA pairs (see gemm_pairs_allowed)
   float* partials;      // split-K partial tiles, [piece][BN][128] fp32
   unsigned* counters;   // split-K arrival counters, zero between launches
+  unsigned* sched;      // [2] piece counter and finished CTAs (single-CTA launches), zero
+                        // between launches; launches that may overlap need their own
   unsigned* status;     // device status word
   uint64_t timeout_ns;  // bound of every wait
 };

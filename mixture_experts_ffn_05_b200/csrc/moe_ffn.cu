@@ -72,7 +72,7 @@ int choose_split(int k_steps, int bn) {
 
 struct Layout {
   size_t status, rcounters, counters, logits, bhist, bbase, topk_idx, topk_w, offsets, sorted, inv;
-  size_t xn_moe, xn_dense, aperm, h, y, hd, dense, partials, wr_hi, wr_lo, total;
+  size_t xn_moe, xn_dense, aperm, h, y, hd, dense, partials, wr_hi, wr_lo, sched, total;
   size_t counters_bytes;
   int bn, split_gu, split_dgu, split_d, split_dd;
 };
@@ -129,6 +129,7 @@ Layout layout_of(const Dims& d) {
   const size_t wr_bytes = router_uses_tc(d.T) ? static_cast<size_t>(d.E) * d.H * 2 : 0;
   L.wr_hi = take(wr_bytes);
   L.wr_lo = take(wr_bytes);
+  L.sched = take(16);  // the GEMM launches' piece counters: [0..1] gate_up, [2..3] down
   L.total = off;
   return L;
 }
@@ -302,6 +303,8 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
   // int8 experts: the launches take the converter-warp variant, whose A maps are raw
   // (unswizzled) for every problem of the launch, the bf16 dense MLP included.
   const bool w8 = j.experts && d.int8;
+  gu.sched = at<unsigned>(ws, L.sched);
+  dn.sched = at<unsigned>(ws, L.sched) + 2;  // the down launch may start before gate_up ends
   for (GemmParams* P : {&gu, &dn}) {
     P->partials = at<float>(ws, L.partials);
     P->counters = at<unsigned>(ws, L.counters);
