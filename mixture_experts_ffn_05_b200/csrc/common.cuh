@@ -172,31 +172,6 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// 2-D tiled bulk copy shared -> global, tracked in this thread's bulk group.  The
-// shared-memory writes it reads must be fenced to the async proxy first
-// (fence_proxy_async_smem) by the threads that made them.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0,
-                                             int32_t c1) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(smem_u32(src)), "r"(c0), "r"(c1)
-               : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until at most one of this thread's committed bulk groups still reads shared memory.
-__device__ __forceinline__ void bulk_wait_read1() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-
-// Wait until every bulk group committed by this thread has completed (writes done).
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // 1-D bulk copy global -> shared of `bytes` (both addresses 16-byte aligned, bytes a
 // multiple of 16); completion counted on `bar`.
 __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,

@@ -2,22 +2,25 @@
 //
 // Used for both halves of every expert MLP and of the shared dense MLP:
 //   gate_up (kind 0): h[pos][i] = gelu_tanh(g) * u, g/u = xn[pos] . W_gate_up[e][i or I+i]
-//   down    (kind 1): Y[row][o] = w(row) * (h[pos] . W_down[e][o])   (bf16 or fp32)
-// (ONNX export card, "Truthful graph contracts", "Mixture of Experts" and "MoE topology"
-// rows; Inferentia2 card, "How it works": expert outputs weighted by the routing weight).
+//   down    (kind 1): Y[pos][o] = h[pos] . W_down[e][o]   (bf16 or fp32)
+// pos is the token row in sorted (expert-major) order; the routing weights are applied
+// where the slots of a token are summed (combine.cu).  (ONNX export card, "Truthful graph
+// contracts", "Mixture of Experts" and "MoE topology" rows; Inferentia2 card, "How it
+// works": expert outputs weighted by the routing weight.)
 //
 // Orientation: the weights are the M operand (128 rows per tile, streamed once from
 // HBM by TMA), the tokens of one expert are the N operand (BN columns).  A decode
 // batch puts a handful of tokens on each expert, so N is small and the kernel is a
-// weight stream; a prefill batch fills N up to 256.  For gate_up, each 128-row tile is
-// 64 gate rows followed by the 64 matching up rows, so one accumulator holds both
-// halves and the epilogue pairs them.
+// weight stream; a prefill batch fills N up to 256.  A gate_up tile holds 64 features as
+// 8 gate rows, the 8 matching up rows, the next 8 gate rows, ... (one 5-D TMA box), so
+// the gate and up accumulators of a feature land in TMEM lanes l and l^8 of one warp.
 //
 // Work list: for each problem (experts, then the optional dense MLP), for each group,
-// for each M tile, for each N tile of BN tokens, `split` pieces along K.  Pieces are
-// dealt round-robin to a persistent grid (one CTA per SM).  When split > 1 each piece
+// for each M tile (PAIR: pair of M tiles), for each N tile of BN tokens, `split` pieces
+// along K.  Narrow tiles deal pieces round-robin to the persistent grid (one CTA per
+// SM); wide single-CTA tiles take them from a global counter.  When split > 1 each piece
 // stores its fp32 partial tile; the last piece to arrive (an atomic counter) sums all
-// partials in piece order, so the result does not depend on arrival order.
+// partials in piece order, so the result does not depend on arrival order or schedule.
 //
 // Warp roles (320 threads): warp 0 issues TMA loads into a ring of shared-memory
 // stages, warp 1 issues tcgen05.mma into one of 2-4 TMEM accumulators, and two groups of
@@ -26,8 +29,8 @@
 // weights (the int8 build of the Inferentia2 card: per-channel symmetric INT8 experts),
 // warps 10-13 convert each raw int8 tile to bf16 in shared memory inside the mainloop,
 // and the per-row scale multiplies the fp32 accumulator in the epilogue (it factors out
-// of the K sum, so this is exact).  Every wait is bounded; a wait that runs out records a timeout in the
-// status word and the CTA winds down.
+// of the K sum, so this is exact).  Every wait is bounded; a wait that runs out records
+// a timeout in the status word and the CTA winds down.
 #include "common.cuh"
 #include "internal.h"
 
@@ -85,8 +88,9 @@ struct Cfg {
   static constexpr int kMiscInts = 8 + kQ;
   static constexpr int kPreOff = kMiscOff + kMiscInts * 4;
   static constexpr int kTabInts = 4 * kMaxEntries;  // pre, cnt, b0, ng
-  // output staging for the TMA stores: two 1 KB buffers per epilogue warp (one where
-  // two do not fit next to the pipeline)
+  // output staging (transposes a warp's slice of the tile so that each lane stores 16 or
+  // 32 contiguous bytes): two 1 KB buffers per epilogue warp (one where two do not fit
+  // next to the pipeline)
   static constexpr int kStgBytes = 1024;
   static constexpr int kStgOff = ((kPreOff + kTabInts * 4) + 127) & ~127;
   static constexpr int kStgBufs = (kStgOff + 8 * 2 * kStgBytes + 1024 <= 232448) ? 2 : 1;
@@ -145,16 +149,6 @@ __device__ __forceinline__ void convert_rows_bf16(const uint8_t* raw, uint8_t* c
     const int c = lane & 7;
     *reinterpret_cast<uint4*>(conv + r * 128 + ((c ^ (r & 7)) << 4)) = v[j];
   }
-}
-
-// Before a staging buffer is rewritten: the TMA store that last read it has done so
-// (with two buffers, the store of the other buffer may still be reading).
-template <int NBUF>
-__device__ __forceinline__ void stg_wait() {
-  if (NBUF >= 2)
-    bulk_wait_read1();
-  else
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 struct Piece {
@@ -615,15 +609,15 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
     // Warp w reads TMEM lanes 32*(w%4)..+31; each group covers all 128 lanes.  Two groups
     // keep the latency-bound part of an epilogue (partials, counters) off the MMA's path.
     // Each warp then writes its own slice of the output tile: it stages the values in its
-    // shared-memory buffers and one lane stores them with a TMA copy, so the epilogue
-    // issues a few bulk stores per tile instead of one global store per value.
+    // shared-memory buffers, transposed, so that every lane stores 16 or 32 contiguous
+    // bytes of an output row (a warp store covers 512 bytes).
     //   gate_up: lanes l and l^8 hold the gate and up row of one feature (the A tile is
     //     8 gate rows, the matching 8 up rows, ...); a shuffle pairs them, the gate lane
     //     finishes columns 0-7 of each 16 and the up lane columns 8-15.  Warp q covers
     //     features 16q..16q+15 of the tile's 64.
     //   down: lane l holds output row 32q + l of the tile's 128.
-    // Output rows are the tile's B rows (sorted order).  A 16-column chunk (gate_up) or
-    // 8-column half chunk (down) that is not all valid is written with plain stores.
+    // Output rows are the tile's B rows (sorted order); columns past the tile's valid
+    // count are not stored.
     const int grp = (warp - 2) >> 2;
     const int q = warp & 3;
     const int et = threadIdx.x - 64 - 128 * grp;
@@ -746,38 +740,30 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
             }
             uint8_t* buf = stg + (nstg % C::kStgBufs) * C::kStgBytes;
             ++nstg;
-            if (lane == 0) stg_wait<C::kStgBufs>();
-            __syncwarp();
-            // [16 columns][16 features] bf16
+            __syncwarp();  // the buffer's last reads (two chunks ago) are done
+            // [16 columns][16 features] bf16, then one 16-byte store per lane: lane l
+            // writes features 8*(l&1)..+7 of column l/2
             uint16_t* b16 = reinterpret_cast<uint16_t*>(buf);
             const int f = 8 * (lane >> 4) + (lane & 7);
             const int cb = up ? 8 : 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) b16[(cb + i) * 16 + f] = bf16_bits(h[i]);
+            __syncwarp();
             const int fx = mt * 64 + 16 * q;  // first output feature of this warp
-            if (c0 + 16 <= pc.n_valid) {
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&maps.o[pr.map], buf, fx, pos0 + c0);
-                bulk_commit();
-              }
-            } else {
-              __syncwarp();
-              if (lane == 0) bulk_commit();  // an empty group keeps the buffer accounting
-              // ragged chunk: lane l writes feature l%16 of columns l/16, l/16+2, ...
-              uint16_t* out = static_cast<uint16_t*>(pr.out);
-              for (int c = lane >> 4; c0 + c < pc.n_valid; c += 2)
-                out[static_cast<size_t>(pos0 + c0 + c) * pr.out_ld + fx + (lane & 15)] =
-                    b16[c * 16 + (lane & 15)];
+            const int c = lane >> 1;
+            if (c0 + c < pc.n_valid) {
+              const uint4 val = *reinterpret_cast<const uint4*>(b16 + c * 16 + 8 * (lane & 1));
+              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(pr.out) +
+                                        static_cast<size_t>(pos0 + c0 + c) * pr.out_ld + fx +
+                                        8 * (lane & 1)) = val;
             }
           } else {
-            // two halves of 8 columns: [8 columns][32 rows] fp32 or bf16
+            // two halves of 8 columns: [8 columns][32 rows] fp32 or bf16, then lane l
+            // writes rows 8*(l&3)..+7 of column l/4
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               uint8_t* buf = stg + (nstg % C::kStgBufs) * C::kStgBytes;
               ++nstg;
-              if (lane == 0) stg_wait<C::kStgBufs>();
               __syncwarp();
               if (pr.out_f32) {
                 float* bf = reinterpret_cast<float*>(buf);
@@ -788,25 +774,20 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) bh[i * 32 + lane] = bf16_bits(v[8 * hh + i]);
               }
+              __syncwarp();
               const int cc = c0 + 8 * hh;
               const int fx = mt * 128 + 32 * q;
-              if (cc + 8 <= pc.n_valid) {
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                  tma_store_2d(&maps.o[pr.map], buf, fx, pos0 + cc);
-                  bulk_commit();
-                }
-              } else {
-                __syncwarp();
-                if (lane == 0) bulk_commit();  // an empty group keeps the buffer accounting
-                for (int c = 0; cc + c < pc.n_valid; ++c) {
-                  const size_t o = static_cast<size_t>(pos0 + cc + c) * pr.out_ld + fx + lane;
-                  if (pr.out_f32)
-                    static_cast<float*>(pr.out)[o] = reinterpret_cast<const float*>(buf)[c * 32 + lane];
-                  else
-                    static_cast<uint16_t*>(pr.out)[o] =
-                        reinterpret_cast<const uint16_t*>(buf)[c * 32 + lane];
+              const int c = lane >> 2, g = lane & 3;
+              if (cc + c < pc.n_valid) {
+                const size_t o = static_cast<size_t>(pos0 + cc + c) * pr.out_ld + fx + 8 * g;
+                if (pr.out_f32) {
+                  const float4* src = reinterpret_cast<const float4*>(buf) + c * 8 + 2 * g;
+                  float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + o);
+                  dst[0] = src[0];
+                  dst[1] = src[1];
+                } else {
+                  *reinterpret_cast<uint4*>(static_cast<uint16_t*>(pr.out) + o) =
+                      *(reinterpret_cast<const uint4*>(buf) + c * 4 + g);
                 }
               }
             }
@@ -820,7 +801,6 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       else
         mbar_arrive(&acc_empty[ab]);
     }
-    if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
   }
 
   // ---- teardown

@@ -51,8 +51,6 @@ struct GemmParams {
 struct GemmMaps {
   CUtensorMap a[2];  // weights of problem map 0 / 1
   CUtensorMap b[2];  // tokens of problem map 0 / 1
-  CUtensorMap o[2];  // outputs (TMA stores), unswizzled: gate_up boxes of 16 features x
-                     // 16 rows (bf16), down boxes of 32 features x 8 rows
 };
 
 // Launches kernel<<<grid, block, smem, s>>>(args...).  With pdl the launch is a

@@ -231,31 +231,6 @@ bool encode_gate_up(CUtensorMap* m, const void* base, int64_t groups, int64_t F,
   return r == CUDA_SUCCESS;
 }
 
-// Output map for the epilogue's TMA stores: rows x cols, unswizzled boxes.
-bool encode_out(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int box_cols,
-                int box_rows, bool f32) {
-  PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
-  if (fn == nullptr) return false;
-  const int es = f32 ? 4 : 2;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * es};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t el[2] = {1, 1};
-  const CUresult r =
-      fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
-         dims, strides, box, el, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// Output boxes of the two GEMM kinds (see GemmMaps).
-bool encode_h_out(CUtensorMap* m, void* base, int64_t rows, int64_t cols) {
-  return encode_out(m, base, rows, cols, 16, 16, false);
-}
-bool encode_y_out(CUtensorMap* m, void* base, int64_t rows, int64_t cols, bool f32) {
-  return encode_out(m, base, rows, cols, 32, 8, f32);
-}
-
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // ---------------------------------------------------------------- the expert / dense GEMMs
@@ -350,10 +325,8 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.wscale = j.s_down; b.w8 = d.int8;
     if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, w8, d.int8) ||
         !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, bbox_gu) ||
-        !encode_h_out(&mgu.o[np], h, Tk, d.I) ||
         !encode_a(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128, d.int8) ||
-        !encode_bf16(&mdn.b[np], h, Tk, d.I, bbox_dn) ||
-        !encode_y_out(&mdn.o[np], j.y, Tk, d.H, true))
+        !encode_bf16(&mdn.b[np], h, Tk, d.I, bbox_dn))
       return MOE_ERR_CUDA;
     ++np;
   }
@@ -371,17 +344,15 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.out_ld = d.H;
     if (!encode_gate_up(&mgu.a[np], j.w_dgu, 1, d.D, d.H, w8, false) ||
         !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, bbox_gu) ||
-        !encode_h_out(&mgu.o[np], hd, d.T, d.D) ||
         !encode_a(&mdn.a[np], j.w_dd, d.H, d.D, 128, false) ||
-        !encode_bf16(&mdn.b[np], hd, d.T, d.D, bbox_dn) ||
-        !encode_y_out(&mdn.o[np], j.dense_out, d.T, d.H, j.dense_f32 != 0))
+        !encode_bf16(&mdn.b[np], hd, d.T, d.D, bbox_dn))
       return MOE_ERR_CUDA;
     ++np;
   }
   gu.nprob = dn.nprob = np;
   if (np == 1) {  // unused second set: a valid copy of the first
-    mgu.a[1] = mgu.a[0]; mgu.b[1] = mgu.b[0]; mgu.o[1] = mgu.o[0];
-    mdn.a[1] = mdn.a[0]; mdn.b[1] = mdn.b[0]; mdn.o[1] = mdn.o[0];
+    mgu.a[1] = mgu.a[0]; mgu.b[1] = mgu.b[0];
+    mdn.a[1] = mdn.a[0]; mdn.b[1] = mdn.b[0];
   }
   // after a kernel of the same entry point the gate_up launch overlaps that kernel's tail
   // (programmatic dependent launch)
