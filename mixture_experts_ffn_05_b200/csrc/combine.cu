@@ -49,7 +49,8 @@ __device__ __forceinline__ void load_slots(int t, int k, int n, const int* __res
   if (threadIdx.x < k) {
     const int p = t * k + threadIdx.x;
     const int q = inv_pos[p];
-    const bool ok = q >= 0 && q < n && sorted_src[q] == p;
+    // sorted_src == NULL: the permutation comes from this library's own sort (no check)
+    const bool ok = q >= 0 && q < n && (sorted_src == nullptr || sorted_src[q] == p);
     s_q[threadIdx.x] = ok ? q : -1;
     s_w[threadIdx.x] = topk_w[p];
   }
@@ -57,15 +58,18 @@ __device__ __forceinline__ void load_slots(int t, int k, int n, const int* __res
 }
 
 // One CTA per token, one 8-column chunk per thread; every input is requested before
-// the first reduction.
-__global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
+// the first reduction.  NSLOT slots of Y are in flight at a time: 8 when there are
+// fewer tokens than SMs (one CTA per SM: the shortest chain of loads), else 4 (two CTAs
+// fit on an SM, which measured faster for large batches).
+template <int MAXT, int NSLOT>
+__global__ void __launch_bounds__(MAXT) combine_block_kernel(
     int H, int k, float eps, const uint16_t* __restrict__ x, const float* __restrict__ y,
     const int* __restrict__ inv_pos, const int* __restrict__ sorted_src,
     const float* __restrict__ topk_w, const float* __restrict__ dense,
     const uint16_t* __restrict__ g_pm,
     const uint16_t* __restrict__ g_pd, const uint16_t* __restrict__ g_ff,
     uint16_t* __restrict__ out, uint16_t* __restrict__ moe_out) {
-  __shared__ float2 red[kCombMaxThreads / 32];
+  __shared__ float2 red[MAXT / 32];
   __shared__ int s_q[16];
   __shared__ float s_w[16];
   const int t = blockIdx.x;
@@ -86,14 +90,14 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_block_kernel(
   for (int i = 0; i < 8; ++i) m[i] = d[i] = 0.f;
   {
     load8f(dense + static_cast<size_t>(t) * H + cc * 8, d);
-    for (int j0 = 0; j0 < k; j0 += 4) {  // 4 slots in flight at a time, summed in slot order
-      float buf[4][8];
+    for (int j0 = 0; j0 < k; j0 += NSLOT) {  // NSLOT slots in flight, summed in slot order
+      float buf[NSLOT][8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < NSLOT; ++j)
         if (j0 + j < k && s_q[j0 + j] >= 0)
           load8f(y + static_cast<size_t>(s_q[j0 + j]) * H + cc * 8, buf[j]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < NSLOT; ++j)
         if (j0 + j < k && s_q[j0 + j] >= 0) {
           const float w = s_w[j0 + j];
 #pragma unroll
@@ -171,9 +175,17 @@ cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t*
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s, bool pdl) {
   const int threads = std::max(32, ((H >> 3) + 31) / 32 * 32);
-  return launch_k(combine_block_kernel, dim3(T), dim3(threads), 0, s, pdl, H, k, eps, x, y,
-                  inv_pos, sorted_src, topk_w, dense, g_post_moe, g_post_dense, g_post_ff, out,
-                  moe_out);
+  if (threads <= 384 && T <= 148)
+    return launch_k(combine_block_kernel<384, 8>, dim3(T), dim3(threads), 0, s, pdl, H, k, eps,
+                    x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe, g_post_dense,
+                    g_post_ff, out, moe_out);
+  if (threads <= 384)
+    return launch_k(combine_block_kernel<384, 4>, dim3(T), dim3(threads), 0, s, pdl, H, k, eps,
+                    x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe, g_post_dense,
+                    g_post_ff, out, moe_out);
+  return launch_k(combine_block_kernel<kCombMaxThreads, 4>, dim3(T), dim3(threads), 0, s, pdl,
+                  H, k, eps, x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe,
+                  g_post_dense, g_post_ff, out, moe_out);
 }
 
 cudaError_t launch_combine_moe(int T, int H, int k, const float* y, const int* inv_pos,

@@ -123,7 +123,9 @@ bool gemm_pairs_allowed(int bn, bool int8_weights);
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                                 cudaStream_t s, bool pdl = false);
 // y holds the expert outputs in sorted order (row inv_pos[t*k+j] for slot j of token
-// t), unweighted; the combine applies topk_w.
+// t), unweighted; the combine applies topk_w.  With sorted_src != NULL a slot counts
+// only if sorted_src[inv_pos[p]] == p (a caller-supplied permutation may have dropped
+// pairs); NULL skips that check (the permutation is this library's own).
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
                                  const float* y, const int* inv_pos, const int* sorted_src,
                                  const float* topk_w, const float* dense,

@@ -613,7 +613,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   j.dense_out = dense;
   j.dense_f32 = 1;
   if ((st = run_gemms(d, L, ws, j, s, false, ev)) != MOE_OK) return st;
-  if ((st = cuda_status(launch_combine_block(d.T, d.H, d.k, d.eps, x, y, inv, sorted, topk_w,
+  if ((st = cuda_status(launch_combine_block(d.T, d.H, d.k, d.eps, x, y, inv, nullptr, topk_w,
                                              dense, w->g_post_moe,
                                              w->g_post_dense, w->g_post_ff, out, moe_out, s,
                                              true))) != MOE_OK)
