@@ -99,13 +99,17 @@ struct Cfg {
   static_assert(kSmem <= 232448, "shared memory");
 };
 
-// ---- int8 -> bf16 in the converter warps.  Each code q in [-127, 127] becomes the fp32
-// number 2^23 + (q + 128) by placing the unsigned byte q + 128 in the mantissa of 2^23
-// (exponent-bias construction), minus 2^23 + 128; both steps are exact, and so is the
-// rounding to bf16 since |q| < 2^8.
-__device__ __forceinline__ float i8_to_f32(uint32_t biased_word, uint32_t byte) {
-  return __int_as_float(static_cast<int>(__byte_perm(biased_word, 0x4B000000u, 0x7440u + byte))) -
-         8388736.0f;
+// ---- int8 -> fp16 in the converter warps (int8 expert problems take fp16 operands).
+// For a code q in [-127, 127], the fp16 number whose exponent is that of 1024 and whose
+// low mantissa bits hold the byte q + 128 is 1024 + q + 128 (fp16 has 10 mantissa bits),
+// and subtracting 1152 in fp16 leaves q exactly (exponent-bias construction).  One byte
+// permute builds two such halves from a word of biased codes; one fp16x2 subtraction
+// finishes both.  sel 0x5140 takes codes 0 and 1 of the word, 0x5342 codes 2 and 3.
+__device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t biased_word, uint32_t sel) {
+  const uint32_t h = __byte_perm(biased_word, 0x64646464u, sel);
+  uint32_t r;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64806480u));
+  return r;
 }
 
 // A converter warp owns 32 rows of the tile.  Its lanes read the warp's slice of the raw
@@ -128,8 +132,8 @@ __device__ __forceinline__ void convert_rows_i8(const uint8_t* raw, uint8_t* con
     uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      o[2 * i] = pack2(i8_to_f32(w[i], 0), i8_to_f32(w[i], 1));
-      o[2 * i + 1] = pack2(i8_to_f32(w[i], 2), i8_to_f32(w[i], 3));
+      o[2 * i] = i8x2_to_f16x2(w[i], 0x5140u);
+      o[2 * i + 1] = i8x2_to_f16x2(w[i], 0x5342u);
     }
     uint8_t* row = conv + sub * (128 * 128) + r * 128;
     *reinterpret_cast<uint4*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -468,7 +472,9 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         }
         if (piece < 0 || piece >= total) break;
         const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
-        const uint32_t idesc = idesc_bf16_f32(PAIR ? 256 : 128, (pc.n_valid + 15) & ~15);
+        const int ncol = (pc.n_valid + 15) & ~15;
+        const uint32_t idesc = P.prob[pc.p].f16 ? idesc_f16_f32(PAIR ? 256 : 128, ncol)
+                                                : idesc_bf16_f32(PAIR ? 256 : 128, ncol);
         if (!mbar_wait(&acc_empty[ab], aph ^ 1u, tmo, abort_flag)) {
           ok = false;
           break;
@@ -747,7 +753,8 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
             const int f = 8 * (lane >> 4) + (lane & 7);
             const int cb = up ? 8 : 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) b16[(cb + i) * 16 + f] = bf16_bits(h[i]);
+            for (int i = 0; i < 8; ++i)
+              b16[(cb + i) * 16 + f] = pr.f16 ? f16_bits(h[i]) : bf16_bits(h[i]);
             __syncwarp();
             const int fx = mt * 64 + 16 * q;  // first output feature of this warp
             const int c = lane >> 1;

@@ -33,6 +33,8 @@ struct GemmProblem {
   int out_ld;            // elements per output row
   const float* wscale;   // int8 row scales [groups][w_rows_per_group]; NULL for bf16
   int w8;                // A operand is int8 codes (needs a launch with int8_weights)
+  int f16;               // A and B are fp16 (int8 codes are converted to fp16, exact);
+                         // gate_up writes h in fp16
 };
 
 struct GemmParams {
@@ -111,8 +113,9 @@ cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int*
                            int* inv_pos, int* block_hist, int* block_base, cudaStream_t s,
                            bool pdl = false);
 int permute_blocks(int n);  // blocks of the multi-block path, <= 256 (0 = single-block path)
+// to_f16: write the rows as fp16 (the operand type of int8 experts) instead of bf16.
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
-                               const uint16_t* src, uint16_t* dst, cudaStream_t s,
+                               const uint16_t* src, uint16_t* dst, bool to_f16, cudaStream_t s,
                                bool pdl = false);
 // A launch may run on CTA pairs (GemmParams::pairs) when its weights are bf16 and its
 // token tiles are 128 or 256 wide; its B maps then take boxes of bn / 2 rows (each CTA

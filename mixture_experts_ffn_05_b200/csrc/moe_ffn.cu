@@ -316,13 +316,14 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     a.split = std::min(L.split_gu, a.k_steps); a.map = np; a.out = h; a.out_ld = d.I;
     a.wscale = j.s_gate_up;
     a.w8 = d.int8;
+    a.f16 = d.int8;  // int8 codes become fp16 (exact); the gathered rows and h are fp16
     GemmProblem& b = dn.prob[np];
     b = GemmProblem{};
     b.kind = 1; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = static_cast<int>(Tk);
     b.k_steps = (d.I + kw - 1) / kw; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H; b.nw = 0;
     b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_f32 = 1;
     b.out_ld = d.H;
-    b.wscale = j.s_down; b.w8 = d.int8;
+    b.wscale = j.s_down; b.w8 = d.int8; b.f16 = d.int8;
     if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, w8, d.int8) ||
         !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, bbox_gu) ||
         !encode_a(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128, d.int8) ||
@@ -503,7 +504,8 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   const int Tk = d.T * d.k;
   uint16_t* aperm = at<uint16_t>(ws, L.aperm);
   float* y = at<float>(ws, L.y);
-  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted_src, xn_moe, aperm, s))) != MOE_OK)
+  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted_src, xn_moe, aperm,
+                                           d.int8 != 0, s))) != MOE_OK)
     return st;
   GemmJob j{};
   j.experts = true;
@@ -591,7 +593,8 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
                                        at<int>(ws, L.bbase), s, true))) != MOE_OK)
     return st;
   if (!mark(ev, 2, s)) return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe, aperm, s, true))) !=
+  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe, aperm, d.int8 != 0,
+                                           s, true))) !=
       MOE_OK)
     return st;
   if (!mark(ev, 3, s)) return MOE_ERR_CUDA;

@@ -130,6 +130,21 @@ cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int*
 // out-of-bounds read).
 constexpr int kGatherWarps = 8;
 
+// bf16 -> fp16 of 8 values (exact for |v| in the fp16 normal range; smaller values keep
+// fp16 subnormal precision, 2^-24 absolute).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& u) {
+  float f[8];
+  unpack8(u, f);
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+    o[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <bool F16>
 __global__ void __launch_bounds__(32 * kGatherWarps) gather_rows_kernel(
     int n, int k, int H, int T, const int* __restrict__ sorted_src,
     const uint16_t* __restrict__ src, uint16_t* __restrict__ dst) {
@@ -154,16 +169,19 @@ __global__ void __launch_bounds__(32 * kGatherWarps) gather_rows_kernel(
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int c = c0 + 32 * u;
-      if (c < nch) d[c] = v[u];
+      if (c < nch) d[c] = F16 ? bf16x8_to_f16x8(v[u]) : v[u];
     }
   }
 }
 
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
-                               const uint16_t* src, uint16_t* dst, cudaStream_t s, bool pdl) {
+                               const uint16_t* src, uint16_t* dst, bool to_f16, cudaStream_t s,
+                               bool pdl) {
   const int blocks = (n + kGatherWarps - 1) / kGatherWarps;
-  return launch_k(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)),
-                  dim3(32 * kGatherWarps), 0, s, pdl, n, k, H, T, sorted_src, src, dst);
+  return to_f16 ? launch_k(gather_rows_kernel<true>, dim3(static_cast<unsigned>(blocks)),
+                           dim3(32 * kGatherWarps), 0, s, pdl, n, k, H, T, sorted_src, src, dst)
+                : launch_k(gather_rows_kernel<false>, dim3(static_cast<unsigned>(blocks)),
+                           dim3(32 * kGatherWarps), 0, s, pdl, n, k, H, T, sorted_src, src, dst);
 }
 
 }  // namespace moe
