@@ -49,9 +49,12 @@ constexpr int kConvWarps = 4;      // converter warps, 32 rows of the 128-row ti
 //   weights and 16 KB of tokens per 64-wide K step for a 128 x 256 share of the
 //   product (instead of 16 + 32 KB alone): a third less shared-memory fill traffic per
 //   FLOP, which is what bounds the wide tiles.
-// W8 = true: TMA lands the raw A tile (int8 codes, or bf16 rows of a bf16 problem in the
-//   same launch) unswizzled; four converter warps turn it into the bf16 swizzled layout
-//   in a second, shallower ring.  The int8 row scales are applied in the epilogue.
+// W8 = true: TMA lands the A tile of an int8 problem as 128 rows of 128 codes (128-byte
+//   swizzled); four converter warps turn each row into fp16 in registers and store it in
+//   tensor memory, from which the MMA reads its A operand (tcgen05.mma with A in TMEM),
+//   so the converted tile never passes through shared memory.  A bf16 problem in the same
+//   launch (the dense MLP) is read by the MMA from shared memory as usual.  The int8 row
+//   scales are applied in the epilogue.
 template <int BN, bool W8, bool PAIR>
 struct Cfg {
   static_assert(!(W8 && PAIR), "CTA pairs take bf16 weights only");
@@ -64,17 +67,20 @@ struct Cfg {
   static constexpr int kBSlots = W8 ? 2 : 1;
   static constexpr int kStage = kABytes + kBSlots * kBBytes;
   static constexpr int kStages = PAIR ? (BN <= 128 ? 8 : 6)
-                                : W8 ? (BN <= 16 ? 7 : (BN <= 32 ? 6 : (BN <= 64 ? 4 : (BN <= 128 ? 3 : 2))))
+                                : W8 ? (BN <= 32 ? 8 : (BN <= 64 ? 6 : (BN <= 128 ? 4 : 2)))
                                      : (BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4)));
-  static constexpr int kConvBytes = 2 * kABytes;   // converted stage: two 64-wide sub-tiles
-  static constexpr int kConv = W8 ? (BN >= 256 ? 1 : 2) : 0;
+  // W8: TMEM buffers for converted A tiles, 64 columns (128 K of fp16 pairs) each
+  static constexpr int kConv = W8 ? 4 : 0;
   // TMEM accumulators: 4 for narrow tiles (the epilogue of a weight-streaming piece is
-  // latency-bound and must not hold up the MMAs), 2 for wide ones (512 columns max).
-  static constexpr int kAcc = BN <= 64 ? 4 : 2;
-  static constexpr int kTmemCols = kAcc * BN < 32 ? 32 : kAcc * BN;
-  // after the stages: converted stages, barriers, bookkeeping, the gate/up exchange buffer
-  static constexpr int kConvOff = kStages * kStage;
-  static constexpr int kBarOff = kConvOff + kConv * kConvBytes;
+  // latency-bound and must not hold up the MMAs), 2 for wide ones (512 columns max, less
+  // the converted A buffers of the W8 variant).
+  static constexpr int kAcc = BN <= 64 ? 4 : (W8 && BN >= 256 ? 1 : 2);
+  static constexpr int kTaCol = kAcc * BN;  // first TMEM column of the A buffers
+  static constexpr int kTmemCols =
+      W8 ? 512 : (kAcc * BN < 32 ? 32 : kAcc * BN);
+  static_assert(kTaCol + kConv * 64 <= kTmemCols, "tensor memory");
+  // after the stages: barriers, bookkeeping, the output staging buffers
+  static constexpr int kBarOff = kStages * kStage;
   // Single CTAs with wide tiles take their pieces from a global counter (the fastest SMs
   // take more, which shortens the tail of long pieces); the producer passes them to the
   // other roles through a queue of kQ slots.  Narrow (weight-streaming) tiles keep the
@@ -119,39 +125,29 @@ __device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t biased_word, uint32_t
 //   int8 raw rows are 128 codes (two 64-wide sub-tiles): step j, lane l -> row
 //     4j + l/8, codes 16*(l%8)..+15 -> sub-tile (l%8)/4, chunks 2*(l%4) and 2*(l%4)+1.
 //   bf16 raw rows are 64 values (one sub-tile): step j, lane l -> row 4j + l/8, chunk l%8.
-__device__ __forceinline__ void convert_rows_i8(const uint8_t* raw, uint8_t* conv, int row0,
-                                                int lane) {
+// A converter warp owns 32 rows of the tile, one per lane (its TMEM lane quarter).  A
+// lane reads its row's 128 codes from the swizzled tile (chunk c of row r at chunk
+// position c ^ (r % 8): the 32 lanes of a load hit 8 distinct positions), converts them
+// to 64 fp16 pairs and stores them in 64 consecutive TMEM columns of its lane: column j
+// holds codes 2j (low half) and 2j+1, the layout of an M x K fp16 A operand in TMEM.
+__device__ __forceinline__ void convert_row_i8_to_tmem(const uint8_t* raw, int r,
+                                                       uint32_t taddr) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint4 q = *reinterpret_cast<const uint4*>(raw + (row0 * 128) + 512 * j + 16 * lane);
-    const int r = row0 + 4 * j + (lane >> 3);
-    const int sub = (lane & 7) >> 2;
-    const int c0 = 2 * (lane & 3);
-    const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u,
-                           q.w ^ 0x80808080u};
-    uint32_t o[8];
+  for (int h = 0; h < 4; ++h) {  // 32 codes -> 16 columns at a time
+    uint32_t o[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      o[2 * i] = i8x2_to_f16x2(w[i], 0x5140u);
-      o[2 * i + 1] = i8x2_to_f16x2(w[i], 0x5342u);
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 2 * h + cc;
+      const uint4 q = *reinterpret_cast<const uint4*>(raw + r * 128 + ((c ^ (r & 7)) << 4));
+      const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u,
+                             q.w ^ 0x80808080u};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[8 * cc + 2 * i] = i8x2_to_f16x2(w[i], 0x5140u);
+        o[8 * cc + 2 * i + 1] = i8x2_to_f16x2(w[i], 0x5342u);
+      }
     }
-    uint8_t* row = conv + sub * (128 * 128) + r * 128;
-    *reinterpret_cast<uint4*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-  }
-}
-
-__device__ __forceinline__ void convert_rows_bf16(const uint8_t* raw, uint8_t* conv, int row0,
-                                                  int lane) {
-  uint4 v[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    v[j] = *reinterpret_cast<const uint4*>(raw + (row0 * 128) + 512 * j + 16 * lane);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int r = row0 + 4 * j + (lane >> 3);
-    const int c = lane & 7;
-    *reinterpret_cast<uint4*>(conv + r * 128 + ((c ^ (r & 7)) << 4)) = v[j];
+    tmem_st16(taddr + 16 * h, o);
   }
 }
 
@@ -204,7 +200,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* empty = full + C::kStages;
-  uint64_t* conv_full = empty + C::kStages;
+  uint64_t* conv_full = empty + C::kStages;  // converted A tile in TMEM buffer i is ready
   uint64_t* conv_empty = conv_full + C::kConv;
   uint64_t* acc_full = conv_empty + C::kConv;
   uint64_t* acc_empty = acc_full + C::kAcc;
@@ -481,33 +477,42 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(ab * BN);
+        // int8 problems (W8): A comes from the TMEM buffer the converters filled
+        const bool a_tmem = W8 && P.prob[pc.p].w8;
         for (int ks = pc.k0; ks < pc.k1; ++ks) {
           if (!mbar_wait(&full[stage], phase, tmo, abort_flag) ||
-              (W8 && !mbar_wait(&conv_full[cs], cph, tmo, abort_flag))) {
+              (a_tmem && !mbar_wait(&conv_full[cs], cph, tmo, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * C::kStage);
-          const uint32_t sA = W8 ? smem_u32(smem + C::kConvOff + cs * C::kConvBytes) : sa;
-          const int nsub = (W8 && P.prob[pc.p].w8) ? 2 : 1;  // 64-wide sub-steps
-          for (int sub = 0; sub < nsub; ++sub) {
-            const uint64_t ad = sdesc_k_sw128(sA + sub * C::kABytes);
-            const uint64_t bd = sdesc_k_sw128(sa + C::kABytes + sub * C::kBBytes);
+          if (a_tmem) {
+            // a 128-K step: two 64-wide sub-steps; A sub-step `sub`, K slice kk sits in
+            // TMEM columns [32 sub + 8 kk, +8) of the buffer
+            const uint32_t ta = tmem_base + static_cast<uint32_t>(C::kTaCol + cs * 64);
+            for (int sub = 0; sub < 2; ++sub) {
+              const uint64_t bd = sdesc_k_sw128(sa + C::kABytes + sub * C::kBBytes);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (ks > pc.k0 || sub > 0 || kk > 0) ? 1u : 0u;
-              if (PAIR)
-                umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
-              else
-                umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+              for (int kk = 0; kk < 4; ++kk)
+                umma_ta(d, ta + 32 * sub + 8 * kk, bd + 2 * kk, idesc,
+                        (ks > pc.k0 || sub > 0 || kk > 0) ? 1u : 0u);
             }
-          }
-          if (W8) {
             umma_commit(&conv_empty[cs]);
             if (++cs == C::kConv) {
               cs = 0;
               cph ^= 1u;
+            }
+          } else {
+            const uint64_t ad = sdesc_k_sw128(sa);
+            const uint64_t bd = sdesc_k_sw128(sa + C::kABytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (ks > pc.k0 || kk > 0) ? 1u : 0u;
+              if (PAIR)
+                umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+              else
+                umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
             }
           }
           if (PAIR) {
@@ -547,10 +552,11 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       }
     }
   } else if (W8 && warp >= kConvWarp0) {
-    // ================= converters (W8): raw A stage -> swizzled bf16 stage ============
-    // Each warp owns 32 rows of the tile (one per lane) and runs on its own: an elected
-    // lane waits for the raw stage and a free converted stage, the warp converts, fences
-    // its writes to the async proxy, and lane 0 arrives for the warp.
+    // ================= converters (W8): int8 A tile -> fp16 in TMEM ==================
+    // Each warp owns 32 rows of the tile (one per lane, its TMEM lane quarter) and runs on
+    // its own: an elected lane waits for the stage (and, for an int8 problem, a free TMEM
+    // buffer), the warp converts and stores, and lane 0 arrives for the warp.  Stages of
+    // a bf16 problem need no conversion: the warp only takes part in releasing them.
     int stage = 0;
     uint32_t phase = 0;
     int cs = 0;
@@ -571,11 +577,12 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       if (piece < 0 || piece >= total) break;
       const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
       const bool i8 = P.prob[pc.p].w8 != 0;
+      const int q = warp & 3;  // TMEM lane quarter
       for (int ks = pc.k0; ks < pc.k1; ++ks) {
         int good = 1;
         if (lane == 0)
           good = (mbar_wait(&full[stage], phase, tmo, abort_flag) &&
-                  mbar_wait(&conv_empty[cs], cph ^ 1u, tmo, abort_flag))
+                  (!i8 || mbar_wait(&conv_empty[cs], cph ^ 1u, tmo, abort_flag)))
                      ? 1
                      : 0;
         good = __shfl_sync(0xffffffffu, good, 0);
@@ -583,24 +590,25 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
           ok = false;
           break;
         }
-        const uint8_t* raw = smem + stage * C::kStage;
-        uint8_t* conv = smem + C::kConvOff + cs * C::kConvBytes;
-        const int row0 = (warp - kConvWarp0) * 32;
-        if (i8)
-          convert_rows_i8(raw, conv, row0, lane);
-        else
-          convert_rows_bf16(raw, conv, row0, lane);
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        if (i8) {
+          tc_fence_after();
+          const uint8_t* raw = smem + stage * C::kStage;
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                 static_cast<uint32_t>(C::kTaCol + cs * 64);
+          convert_row_i8_to_tmem(raw, q * 32 + lane, taddr);
+          tmem_st_wait();
+          tc_fence_before();
+        }
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&conv_full[cs]);
+          if (i8) mbar_arrive(&conv_full[cs]);
           mbar_arrive(&empty[stage]);
         }
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
-        if (++cs == C::kConv) {
+        if (i8 && ++cs == C::kConv) {
           cs = 0;
           cph ^= 1u;
         }

@@ -196,14 +196,10 @@ bool encode_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, i
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Raw weight tile for the converter warps: unswizzled 128-byte rows of int8 codes
-// (128 K) or bf16 values (64 K).
-bool encode_raw(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
-                bool int8) {
-  return int8 ? encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
-                          CU_TENSOR_MAP_SWIZZLE_NONE)
-              : encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                          CU_TENSOR_MAP_SWIZZLE_NONE);
+// int8 weight tile for the converter warps: 128-byte rows of 128 codes, 128-byte swizzle.
+bool encode_i8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  return encode_2d(m, base, rows, cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // gate_up weights [groups][2F][K] (gate rows 0..F-1, up rows F..2F-1) as a 5-D map over
@@ -212,7 +208,7 @@ bool encode_raw(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, in
 // rows, ...  The strides are not increasing (gate|up is outside the feature groups in
 // memory but inside them in the box).
 bool encode_gate_up(CUtensorMap* m, const void* base, int64_t groups, int64_t F, int64_t K,
-                    bool raw, bool int8) {
+                    bool int8) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
   if (fn == nullptr) return false;
   const int es = int8 ? 1 : 2;
@@ -226,7 +222,7 @@ bool encode_gate_up(CUtensorMap* m, const void* base, int64_t groups, int64_t F,
   const CUresult r =
       fn(m, int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
          const_cast<void*>(base), dims, strides, box, el, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         raw ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -275,8 +271,9 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
 
   GemmParams gu{}, dn{};
   GemmMaps mgu{}, mdn{};
-  // int8 experts: the launches take the converter-warp variant, whose A maps are raw
-  // (unswizzled) for every problem of the launch, the bf16 dense MLP included.
+  // int8 experts: the launches take the converter-warp variant (int8 A tiles are turned
+  // into fp16 in tensor memory; the bf16 dense MLP in the same launch reads its A tiles
+  // from shared memory as usual).
   const bool w8 = j.experts && d.int8;
   gu.sched = at<unsigned>(ws, L.sched);
   dn.sched = at<unsigned>(ws, L.sched) + 2;  // the down launch may start before gate_up ends
@@ -289,8 +286,8 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
   }
   auto encode_a = [&](CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
                       bool int8) {
-    return w8 ? encode_raw(m, base, rows, cols, box_rows, int8)
-              : encode_bf16(m, base, rows, cols, box_rows);
+    return int8 ? encode_i8(m, base, rows, cols, box_rows)
+                : encode_bf16(m, base, rows, cols, box_rows);
   };
   // CTA pairs load half of each token tile.  A pair takes two M tiles; with an odd count
   // the last pair's second tile is idle, which costs more than pairs save when the tiles
@@ -324,7 +321,7 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_f32 = 1;
     b.out_ld = d.H;
     b.wscale = j.s_down; b.w8 = d.int8; b.f16 = d.int8;
-    if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, w8, d.int8) ||
+    if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, d.int8) ||
         !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, bbox_gu) ||
         !encode_a(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128, d.int8) ||
         !encode_bf16(&mdn.b[np], h, Tk, d.I, bbox_dn))
@@ -343,7 +340,7 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.k_steps = d.D / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H;
     b.split = L.split_dd; b.map = np; b.out = j.dense_out; b.out_f32 = j.dense_f32;
     b.out_ld = d.H;
-    if (!encode_gate_up(&mgu.a[np], j.w_dgu, 1, d.D, d.H, w8, false) ||
+    if (!encode_gate_up(&mgu.a[np], j.w_dgu, 1, d.D, d.H, false) ||
         !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, bbox_gu) ||
         !encode_a(&mdn.a[np], j.w_dd, d.H, d.D, 128, false) ||
         !encode_bf16(&mdn.b[np], hd, d.T, d.D, bbox_dn))
