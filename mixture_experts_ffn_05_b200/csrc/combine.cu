@@ -5,8 +5,8 @@
 // layernorms" add a post norm on each branch:
 //   m   = sum_{j=0..k-1} w[t,j] * Y[inv_pos[t*k + j]]        (fixed slot order)
 //   out = x + N_post_ff( N_post_dense(d) + N_post_moe(m) ),  N_g(v) = v / rms(v) * g
-// Y (the expert outputs in sorted order, unweighted) and d arrive in fp32; all sums are
-// fp32 and the output is rounded to bf16 once.  A slot whose inv_pos does not point back
+// Y (the expert outputs in sorted order, unweighted) arrives in fp16 and d in fp32; all
+// sums are fp32 and the output is rounded to bf16 once.  A slot whose inv_pos does not point back
 // at it through sorted_src (a pair the permutation dropped) contributes nothing.
 #include <algorithm>
 
@@ -58,12 +58,11 @@ __device__ __forceinline__ void load_slots(int t, int k, int n, const int* __res
 }
 
 // One CTA per token, one 8-column chunk per thread; every input is requested before
-// the first reduction.  NSLOT slots of Y are in flight at a time: 8 when there are
-// fewer tokens than SMs (one CTA per SM: the shortest chain of loads), else 4 (two CTAs
-// fit on an SM, which measured faster for large batches).
+// the first reduction.  NSLOT slots of Y (16 bytes of fp16 each per thread) are in
+// flight at a time.
 template <int MAXT, int NSLOT>
 __global__ void __launch_bounds__(MAXT) combine_block_kernel(
-    int H, int k, float eps, const uint16_t* __restrict__ x, const float* __restrict__ y,
+    int H, int k, float eps, const uint16_t* __restrict__ x, const uint16_t* __restrict__ y,
     const int* __restrict__ inv_pos, const int* __restrict__ sorted_src,
     const float* __restrict__ topk_w, const float* __restrict__ dense,
     const uint16_t* __restrict__ g_pm,
@@ -91,17 +90,20 @@ __global__ void __launch_bounds__(MAXT) combine_block_kernel(
   {
     load8f(dense + static_cast<size_t>(t) * H + cc * 8, d);
     for (int j0 = 0; j0 < k; j0 += NSLOT) {  // NSLOT slots in flight, summed in slot order
-      float buf[NSLOT][8];
+      uint4 raw[NSLOT];
 #pragma unroll
       for (int j = 0; j < NSLOT; ++j)
-        if (j0 + j < k && s_q[j0 + j] >= 0)
-          load8f(y + static_cast<size_t>(s_q[j0 + j]) * H + cc * 8, buf[j]);
+        raw[j] = (j0 + j < k && s_q[j0 + j] >= 0)
+                     ? __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_q[j0 + j]) * H) + cc)
+                     : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int j = 0; j < NSLOT; ++j)
         if (j0 + j < k && s_q[j0 + j] >= 0) {
           const float w = s_w[j0 + j];
+          float f[8];
+          unpack8_f16(raw[j], f);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] = fmaf(w, buf[j][i], m[i]);
+          for (int i = 0; i < 8; ++i) m[i] = fmaf(w, f[i], m[i]);
         }
     }
     if (!on) {
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(MAXT) combine_block_kernel(
 
 // moe_out[t] = sum_j w[t,j] * Y[inv_pos[t*k + j]] in fp32, slot order, rounded to bf16.
 __global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
-                                                          const float* __restrict__ y,
+                                                          const uint16_t* __restrict__ y,
                                                           const int* __restrict__ inv_pos,
                                                           const int* __restrict__ sorted_src,
                                                           const float* __restrict__ topk_w,
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
     for (int j = 0; j < k; ++j) {
       if (s_q[j] < 0) continue;
       float f[8];
-      load8f(y + static_cast<size_t>(s_q[j]) * H + c * 8, f);
+      unpack8_f16(__ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_q[j]) * H) + c), f);
       const float w = s_w[j];
 #pragma unroll
       for (int i = 0; i < 8; ++i) m[i] = fmaf(w, f[i], m[i]);
@@ -169,26 +171,22 @@ __global__ void __launch_bounds__(256) combine_moe_kernel(int H, int k,
 }
 
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
-                                 const float* y, const int* inv_pos, const int* sorted_src,
+                                 const uint16_t* y, const int* inv_pos, const int* sorted_src,
                                  const float* topk_w, const float* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s, bool pdl) {
   const int threads = std::max(32, ((H >> 3) + 31) / 32 * 32);
-  if (threads <= 384 && T <= 148)
+  if (threads <= 384)
     return launch_k(combine_block_kernel<384, 8>, dim3(T), dim3(threads), 0, s, pdl, H, k, eps,
                     x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe, g_post_dense,
                     g_post_ff, out, moe_out);
-  if (threads <= 384)
-    return launch_k(combine_block_kernel<384, 4>, dim3(T), dim3(threads), 0, s, pdl, H, k, eps,
-                    x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe, g_post_dense,
-                    g_post_ff, out, moe_out);
-  return launch_k(combine_block_kernel<kCombMaxThreads, 4>, dim3(T), dim3(threads), 0, s, pdl,
+  return launch_k(combine_block_kernel<kCombMaxThreads, 8>, dim3(T), dim3(threads), 0, s, pdl,
                   H, k, eps, x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe,
                   g_post_dense, g_post_ff, out, moe_out);
 }
 
-cudaError_t launch_combine_moe(int T, int H, int k, const float* y, const int* inv_pos,
+cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, const int* inv_pos,
                                const int* sorted_src, const float* topk_w, uint16_t* moe_out,
                                cudaStream_t s, bool pdl) {
   return launch_k(combine_moe_kernel, dim3(T), dim3(256), 0, s, pdl, H, k, y, inv_pos,

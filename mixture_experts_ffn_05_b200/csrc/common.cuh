@@ -41,6 +41,23 @@ __device__ __forceinline__ uint16_t f16_bits(float a) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
+// fp16 rounding that saturates to +-65504 instead of overflowing to infinity.
+__device__ __forceinline__ uint16_t f16_bits_sat(float a) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(r) : "f"(a));
+  return r;
+}
+
+__device__ __forceinline__ void unpack8_f16(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[2 * i] = p.x;
+    f[2 * i + 1] = p.y;
+  }
+}
+
 __device__ __forceinline__ uint16_t bf16_bits(float a) {
   __nv_bfloat16 h = __float2bfloat16_rn(a);
   return *reinterpret_cast<uint16_t*>(&h);

@@ -780,14 +780,19 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
               uint8_t* buf = stg + (nstg % C::kStgBufs) * C::kStgBytes;
               ++nstg;
               __syncwarp();
-              if (pr.out_f32) {
+              if (pr.out_type == kOutF32) {
                 float* bf = reinterpret_cast<float*>(buf);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) bf[i * 32 + lane] = v[8 * hh + i];
               } else {
                 uint16_t* bh = reinterpret_cast<uint16_t*>(buf);
+                if (pr.out_type == kOutF16) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) bh[i * 32 + lane] = bf16_bits(v[8 * hh + i]);
+                  for (int i = 0; i < 8; ++i) bh[i * 32 + lane] = f16_bits_sat(v[8 * hh + i]);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) bh[i * 32 + lane] = bf16_bits(v[8 * hh + i]);
+                }
               }
               __syncwarp();
               const int cc = c0 + 8 * hh;
@@ -795,7 +800,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
               const int c = lane >> 2, g = lane & 3;
               if (cc + c < pc.n_valid) {
                 const size_t o = static_cast<size_t>(pos0 + cc + c) * pr.out_ld + fx + 8 * g;
-                if (pr.out_f32) {
+                if (pr.out_type == kOutF32) {
                   const float4* src = reinterpret_cast<const float4*>(buf) + c * 8 + 2 * g;
                   float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + o);
                   dst[0] = src[0];

@@ -27,15 +27,18 @@ struct GemmProblem {
   int nw;                // gate_up: Nw (first up row); down: unused
   int split;             // pieces per tile along K (>= 1)
   int map;               // tensor-map pair: 0 or 1
-  void* out;             // output: bf16 (gate_up always), or fp32 when out_f32
-  int out_f32;           // down: fp32 output (the block's branch outputs before the
-                         // combine keep fp32, so no rounding is added before the norms)
+  void* out;             // output: bf16 or fp16 (gate_up, see f16), or out_type (down)
+  int out_type;          // down: kOutBf16, kOutF32 or kOutF16 (the block's branch outputs
+                         // before the combine keep more precision than bf16: the dense
+                         // output fp32, the expert outputs fp16)
   int out_ld;            // elements per output row
   const float* wscale;   // int8 row scales [groups][w_rows_per_group]; NULL for bf16
   int w8;                // A operand is int8 codes (needs a launch with int8_weights)
   int f16;               // A and B are fp16 (int8 codes are converted to fp16, exact);
                          // gate_up writes h in fp16
 };
+
+constexpr int kOutBf16 = 0, kOutF32 = 1, kOutF16 = 2;
 
 struct GemmParams {
   GemmProblem prob[2];
@@ -130,12 +133,12 @@ cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& 
 // only if sorted_src[inv_pos[p]] == p (a caller-supplied permutation may have dropped
 // pairs); NULL skips that check (the permutation is this library's own).
 cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t* x,
-                                 const float* y, const int* inv_pos, const int* sorted_src,
+                                 const uint16_t* y, const int* inv_pos, const int* sorted_src,
                                  const float* topk_w, const float* dense,
                                  const uint16_t* g_post_moe, const uint16_t* g_post_dense,
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s, bool pdl = false);
-cudaError_t launch_combine_moe(int T, int H, int k, const float* y, const int* inv_pos,
+cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, const int* inv_pos,
                                const int* sorted_src, const float* topk_w, uint16_t* moe_out,
                                cudaStream_t s, bool pdl = false);
 cudaError_t launch_quantize_int8(const uint16_t* w, int64_t rows, int cols, int8_t* q,

@@ -121,7 +121,7 @@ Layout layout_of(const Dims& d) {
   L.xn_dense = take(T * d.H * 2);
   L.aperm = take(Tk * d.H * 2);
   L.h = take(Tk * d.I * 2);
-  L.y = take(Tk * d.H * 4);
+  L.y = take(Tk * d.H * 2);
   L.hd = take(T * d.D * 2);
   L.dense = take(T * d.H * 4);
   L.partials = take(any_split ? static_cast<size_t>(pieces) * L.bn * 128 * 4 : 0);
@@ -242,7 +242,7 @@ struct GemmJob {
   const int* offsets;
   const int* sorted_src;
   const float* topk_w;
-  float* y;                  // [Tk][H] expert outputs in sorted order, unweighted
+  uint16_t* y;               // [Tk][H] fp16 expert outputs in sorted order, unweighted
   // dense MLP (problem 1 when experts are present, else problem 0), may be absent
   bool dense;
   const uint16_t* xn_dense;  // [T][H]
@@ -318,7 +318,7 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b = GemmProblem{};
     b.kind = 1; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = static_cast<int>(Tk);
     b.k_steps = (d.I + kw - 1) / kw; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H; b.nw = 0;
-    b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_f32 = 1;
+    b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_type = kOutF16;
     b.out_ld = d.H;
     b.wscale = j.s_down; b.w8 = d.int8; b.f16 = d.int8;
     if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, d.int8) ||
@@ -338,7 +338,8 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b = GemmProblem{};
     b.kind = 1; b.groups = 1; b.offsets = nullptr; b.n_tokens = d.T;
     b.k_steps = d.D / 64; b.m_tiles = d.H / 128; b.w_rows_per_group = d.H;
-    b.split = L.split_dd; b.map = np; b.out = j.dense_out; b.out_f32 = j.dense_f32;
+    b.split = L.split_dd; b.map = np; b.out = j.dense_out;
+    b.out_type = j.dense_f32 ? kOutF32 : kOutBf16;
     b.out_ld = d.H;
     if (!encode_gate_up(&mgu.a[np], j.w_dgu, 1, d.D, d.H, false) ||
         !encode_bf16(&mgu.b[np], j.xn_dense, d.T, d.H, bbox_gu) ||
@@ -500,7 +501,7 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int Tk = d.T * d.k;
   uint16_t* aperm = at<uint16_t>(ws, L.aperm);
-  float* y = at<float>(ws, L.y);
+  uint16_t* y = at<uint16_t>(ws, L.y);
   if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted_src, xn_moe, aperm,
                                            d.int8 != 0, s))) != MOE_OK)
     return st;
@@ -572,7 +573,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   uint16_t* xn_moe = at<uint16_t>(ws, L.xn_moe);
   uint16_t* xn_dense = at<uint16_t>(ws, L.xn_dense);
   uint16_t* aperm = at<uint16_t>(ws, L.aperm);
-  float* y = at<float>(ws, L.y);
+  uint16_t* y = at<uint16_t>(ws, L.y);
   float* dense = at<float>(ws, L.dense);
 
   if (ev != nullptr)
