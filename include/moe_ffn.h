@@ -216,11 +216,22 @@ moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, 
  * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, or MOE_ERR_CUDA if the stream failed. */
 moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream);
 
+/* Self-test of the failure path of the bounded device waits (this library's own health
+ * check; the pages define no such call).  Enqueues one kernel that waits on a barrier
+ * that nothing completes, for `timeout_ns` nanoseconds (1e3 .. 1e10), then records
+ * MOE_ERR_DEVICE_TIMEOUT in the status word of `ws` exactly as a kernel of the block
+ * does when one of its waits runs out, and returns.  The GPU context stays usable; a
+ * following moe_check_device_status() returns MOE_ERR_DEVICE_TIMEOUT and clears the
+ * word.  Only the status word is written.  ws: 256-byte aligned, ws_bytes >= 256;
+ * otherwise MOE_ERR_WORKSPACE; a timeout out of range gives MOE_ERR_INVALID_ARG. */
+moe_status_t moe_wait_selftest(void* ws, size_t ws_bytes, uint64_t timeout_ns, void* stream);
+
 /* A short constant English description of a status code. */
 const char* moe_status_string(moe_status_t status);
 
 /* Version of this interface (increases when a signature or a calling contract changes;
- * 2: the workspace is zeroed once by the caller, MOE_BLOCK_EVENTS is 7). */
+ * 2: the workspace is zeroed once by the caller, MOE_BLOCK_EVENTS is 7;
+ * 3: moe_wait_selftest). */
 int32_t moe_abi_version(void);
 
 #ifdef __cplusplus

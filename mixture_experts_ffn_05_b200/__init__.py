@@ -30,8 +30,8 @@ MOE_W_INT8 = 1
 # Entry points of include/moe_ffn.h (the CPU tests check the header declares exactly these).
 ENTRY_POINTS = ("moe_workspace_size", "moe_router", "moe_permute", "moe_permute_noalloc",
                 "moe_ffn_forward", "dense_mlp_forward", "moe_block_forward",
-                "moe_quantize_int8", "moe_check_device_status", "moe_status_string",
-                "moe_abi_version")
+                "moe_quantize_int8", "moe_check_device_status", "moe_wait_selftest",
+                "moe_status_string", "moe_abi_version")
 PERMUTE_NOALLOC_MAX_PAIRS = 1 << 20
 
 
@@ -76,6 +76,7 @@ _SIG = {
                                  _P, _P, _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "moe_quantize_int8": (_I32, [_P, ctypes.c_int64, _I32, _P, _P, _P]),
     "moe_check_device_status": (_I32, [_P, ctypes.c_size_t, _P]),
+    "moe_wait_selftest": (_I32, [_P, ctypes.c_size_t, ctypes.c_uint64, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
     "moe_abi_version": (_I32, []),
 }
@@ -277,6 +278,13 @@ def moe_quantize_int8(w, q, scales, stream=None):
     st = lib().moe_quantize_int8(_ptr(w, BF16, "w"), rows, cols, _ptr(q, torch.int8, "q"),
                                  _ptr(scales, torch.float32, "scales"), _stream(stream))
     _check("moe_quantize_int8", st)
+
+
+def moe_wait_selftest(ws, timeout_ns: int, stream=None) -> None:
+    """Run one bounded device wait that is bound to run out (the failure path of every
+    kernel's waits); afterwards moe_check_device_status reports MOE_ERR_DEVICE_TIMEOUT."""
+    _check("moe_wait_selftest", lib().moe_wait_selftest(_ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                                         int(timeout_ns), _stream(stream)))
 
 
 def moe_check_device_status(ws, stream=None) -> int:

@@ -141,6 +141,7 @@ cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t*
 cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, const int* inv_pos,
                                const int* sorted_src, const float* topk_w, uint16_t* moe_out,
                                cudaStream_t s, bool pdl = false);
+cudaError_t launch_wait_selftest(unsigned* status, uint64_t timeout_ns, cudaStream_t s);
 cudaError_t launch_quantize_int8(const uint16_t* w, int64_t rows, int cols, int8_t* q,
                                  float* scales, cudaStream_t s);
 

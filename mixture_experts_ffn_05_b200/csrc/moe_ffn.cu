@@ -423,7 +423,7 @@ bool w_ok(const moe_expert_weights_t* w, bool int8) {
 
 extern "C" {
 
-int32_t moe_abi_version(void) { return 2; }
+int32_t moe_abi_version(void) { return 3; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -631,6 +631,14 @@ moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, 
     return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(scales) & 3u) != 0) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_quantize_int8(w, rows, cols, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_wait_selftest(void* ws, size_t ws_bytes, uint64_t timeout_ns, void* stream) {
+  if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return MOE_ERR_WORKSPACE;
+  if (timeout_ns < 1000ull || timeout_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_wait_selftest(static_cast<unsigned*>(ws), timeout_ns, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream) {

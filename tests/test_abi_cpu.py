@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 2
+    assert lib.moe_abi_version() == 3
     for s in range(6):
         assert mf.status_string(s)
     assert mf.status_string(99) == "unknown status"
@@ -121,6 +121,10 @@ def test_every_entry_point_validates(lib):
     bw.g_post_moe = FAKE + 4
     assert lib.moe_block_forward(c, 8, FAKE, ctypes.byref(bw), FAKE, None, FAKE, n,
                                  None, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_wait_selftest(None, 4096, 10**6, None) == mf.MOE_ERR_WORKSPACE
+    assert lib.moe_wait_selftest(FAKE + 16, 4096, 10**6, None) == mf.MOE_ERR_WORKSPACE
+    assert lib.moe_wait_selftest(FAKE, 4096, 10, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_wait_selftest(FAKE, 4096, 10**11, None) == mf.MOE_ERR_INVALID_ARG
     assert lib.moe_quantize_int8(FAKE, 4, 12, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG
     assert lib.moe_quantize_int8(None, 4, 16, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG
     assert lib.moe_quantize_int8(FAKE, 0, 16, FAKE, FAKE, None) == mf.MOE_OK
