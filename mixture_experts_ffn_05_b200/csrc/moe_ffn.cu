@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "internal.h"
@@ -63,11 +64,22 @@ int choose_bn(const Dims& d) {
   return bn;
 }
 
-// K pieces per tile: only for the narrowest token tiles (weight-streaming batches),
-// so that the tile list is fine enough to keep every SM streaming to the end.
-int choose_split(int k_steps, int bn) {
-  if (bn != 16) return 1;
+// K pieces per tile: only for the narrowest token tiles (weight-streaming batches), and
+// only when a launch has too few tiles to keep every SM streaming to the end (fewer than
+// kSplitTilesPerSm per SM); the partial sums cost more than the balance gains beyond.
+constexpr int kSplitTilesPerSm = 8;
+constexpr int kAssumedSms = 148;  // a B200; only shifts the threshold if the GPU differs
+
+int choose_split(int k_steps, int bn, double tiles) {
+  if (bn != 16 || tiles >= kSplitTilesPerSm * kAssumedSms) return 1;
   return std::max(1, std::min(std::min(k_steps, 4), (k_steps + 10) / 11));
+}
+
+// Expected number of experts that receive at least one of T*k uniformly routed pairs
+// (fewer when the routing is skewed, which only makes splitting more useful).
+double expected_used_experts(const Dims& d) {
+  const double pairs = static_cast<double>(d.T) * d.k;
+  return d.E * (1.0 - std::pow(1.0 - 1.0 / d.E, pairs));
 }
 
 struct Layout {
@@ -84,10 +96,15 @@ Layout layout_of(const Dims& d) {
   const int64_t T = d.T, Tk = static_cast<int64_t>(d.T) * d.k;
   L.bn = choose_bn(d);
   const int kw = d.int8 ? 128 : 64;  // K per pipeline step of the expert GEMMs
-  L.split_gu = choose_split((d.H + kw - 1) / kw, L.bn);
-  L.split_dgu = choose_split(d.H / 64, L.bn);
-  L.split_d = choose_split((d.I + kw - 1) / kw, L.bn);
-  L.split_dd = choose_split(d.D / 64, L.bn);
+  // expected tiles of the two launches (experts and the dense MLP share each launch)
+  const double u = expected_used_experts(d);
+  const double dense_nt = static_cast<double>(ceil_div(T, L.bn));
+  const double tiles_gu = u * (d.I / 64) + dense_nt * (d.D / 64);
+  const double tiles_dn = u * (d.H / 128) + dense_nt * (d.H / 128);
+  L.split_gu = choose_split((d.H + kw - 1) / kw, L.bn, tiles_gu);
+  L.split_dgu = choose_split(d.H / 64, L.bn, tiles_gu);
+  L.split_d = choose_split((d.I + kw - 1) / kw, L.bn, tiles_dn);
+  L.split_dd = choose_split(d.D / 64, L.bn, tiles_dn);
   // Upper bound of the N tiles: every non-empty expert has a partial tile.
   const int64_t ntl_e = std::min<int64_t>(d.E, Tk) + ceil_div(Tk, L.bn);
   const int64_t ntl_d = ceil_div(T, L.bn);
