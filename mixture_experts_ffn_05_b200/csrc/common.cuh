@@ -311,6 +311,38 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// tcgen05.ld 16x256b.x2: 16 TMEM lanes x 16 32-bit columns per warp.  Thread t receives,
+// with m = t % 4, for each half of 8 columns (r[0..3]: columns 0-7, r[4..7]: 8-15):
+//   (lane t/4, col 2m), (lane t/4, col 2m+1), (lane t/4+8, col 2m), (lane t/4+8, col 2m+1)
+// which is the 8x8 fragment layout of stmatrix.  Call tmem_ld_wait_16 before use.
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_wait_16(uint32_t (&r)[8], uint32_t (&s)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(s[0]), "+r"(s[1]), "+r"(s[2]), "+r"(s[3]),
+                 "+r"(s[4]), "+r"(s[5]), "+r"(s[6]), "+r"(s[7])
+               :
+               : "memory");
+}
+
+// Four 8x8 b16 matrices stored transposed: thread t gives the address of row t%8 of
+// matrix t/8 and holds row t/4, columns 2(t%4)..+1 of each matrix in a[i].
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t a0, uint32_t a1,
+                                                  uint32_t a2, uint32_t a3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(
+                   saddr),
+               "r"(a0), "r"(a1), "r"(a2), "r"(a3)
+               : "memory");
+}
+
 // ------------------------------------------------------------------ CTA pairs
 // A cluster of two CTAs on neighbouring SMs can run one MMA of M = 256 (cta_group::2):
 // each CTA holds half of A (its 128 rows) and half of B (half of the N rows) in its own

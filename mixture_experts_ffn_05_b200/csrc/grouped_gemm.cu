@@ -75,6 +75,10 @@ struct Cfg {
   // latency-bound and must not hold up the MMAs), 2 for wide ones (512 columns max, less
   // the converted A buffers of the W8 variant).
   static constexpr int kAcc = BN <= 64 ? 4 : (W8 && BN >= 256 ? 1 : 2);
+  // BN >= 32: both epilogue groups drain every tile, each taking alternate 16-column
+  // chunks, so an accumulator is released in half the time (such launches never split
+  // K); BN = 16: the groups take alternate pieces
+  static constexpr bool kColSplit = BN >= 32;
   static constexpr int kTaCol = kAcc * BN;  // first TMEM column of the A buffers
   static constexpr int kTmemCols =
       W8 ? 512 : (kAcc * BN < 32 ? 32 : kAcc * BN);
@@ -191,6 +195,24 @@ __device__ __forceinline__ Piece decode_piece(int piece, const GemmParams& P, co
   return pc;
 }
 
+// Transposed staging tiles of one epilogue warp (16-bit values, 16 token columns).
+// gate_up: [16 tokens][16 features], 32 bytes a token; down: [16 tokens][32 features],
+// 64 bytes a token.  The 16-byte chunks of a token are rotated by its index so that the
+// eight rows that one stmatrix matrix writes, and eight lanes' 16-byte reads, fall on
+// distinct banks.
+__device__ __forceinline__ uint32_t stg_glu_off(int tok, int chunk) {
+  return static_cast<uint32_t>(tok * 32 + ((chunk ^ ((tok >> 2) & 1)) << 4));
+}
+__device__ __forceinline__ uint32_t stg_dn_off(int tok, int chunk) {
+  return static_cast<uint32_t>(tok * 64 + ((chunk ^ ((tok >> 1) & 3)) << 4));
+}
+__device__ __forceinline__ uint32_t pack16(float lo, float hi, int mode) {
+  // mode 0: bf16, 1: fp16, 2: fp16 saturating at +-65504
+  const uint16_t a = mode == 0 ? bf16_bits(lo) : (mode == 1 ? f16_bits(lo) : f16_bits_sat(lo));
+  const uint16_t b = mode == 0 ? bf16_bits(hi) : (mode == 1 ? f16_bits(hi) : f16_bits_sat(hi));
+  return static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
+}
+
 template <int BN, bool W8, bool PAIR>
 __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
     grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams P) {
@@ -240,7 +262,8 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
     }
     for (int i = 0; i < C::kAcc; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], PAIR ? 256 : 128);  // PAIR: both CTAs' epilogues (leader's)
+      // every epilogue thread that drains the buffer arrives; PAIR: both CTAs' (leader's)
+      mbar_init(&acc_empty[i], (PAIR ? 2 : 1) * (C::kColSplit ? 256 : 128));
     }
     mbar_init(drain, 1);
     for (int i = 0; i < C::kQ; ++i) {
@@ -619,9 +642,11 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       *abort_flag = 1;
     }
   } else {
-    // ================= epilogue: two groups of 4 warps take alternate pieces ============
-    // Warp w reads TMEM lanes 32*(w%4)..+31; each group covers all 128 lanes.  Two groups
-    // keep the latency-bound part of an epilogue (partials, counters) off the MMA's path.
+    // ================= epilogue: two groups of 4 warps ==================================
+    // Warp w reads TMEM lanes 32*(w%4)..+31; each group covers all 128 lanes.  The groups
+    // take alternate 16-column chunks of every tile (kColSplit) or, at BN = 16, alternate
+    // pieces, which keeps the latency-bound part of a split-K epilogue (partials,
+    // counters) off the MMA's path.
     // Each warp then writes its own slice of the output tile: it stages the values in its
     // shared-memory buffers, transposed, so that every lane stores 16 or 32 contiguous
     // bytes of an output row (a warp store covers 512 bytes).
@@ -660,7 +685,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         }
       }
       if (piece < 0 || piece >= total) break;
-      if ((local & 1) != grp) continue;
+      if (!C::kColSplit && (local & 1) != grp) continue;
       const int ab = local % C::kAcc;
       const uint32_t aph = static_cast<uint32_t>(local / C::kAcc) & 1u;
       const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
@@ -701,7 +726,87 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         named_sync(bar, 128);
         last = *gb != 0;
       }
-      if (last) {
+      if (last && pr.split == 1 && (pr.kind == 0 || pr.out_type != kOutF32)) {
+        // 16-bit outputs of a whole-K tile: the accumulator is read 16 rows x 16 columns at
+        // a time (tcgen05.ld 16x256b: thread t holds rows t/4 and t/4+8 of each 16, columns
+        // 2(t%4)..+1 of each 8), which is stmatrix's fragment layout; stmatrix.trans writes
+        // it to shared memory as [token][features] and each lane stores 16 contiguous bytes
+        const int pos0 = pc.b_row0 + pc.n * BN;  // output row of column 0
+        const int fq = lane >> 2;
+        float sc[4] = {1.f, 1.f, 1.f, 1.f};  // [16-row half][row t/4, row t/4 + 8]
+        if (pr.wscale) {
+          const float* wsr = pr.wscale + static_cast<size_t>(pc.g) * pr.w_rows_per_group;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              // gate_up: rows 16h+fq (gate) and 16h+fq+8 (up) of warp q are feature
+              // 8(2q+h)+fq of the tile's 64; down: rows are output features
+              const int wr = pr.kind == 0 ? mt * 64 + 8 * (2 * q + h) + fq + (u ? pr.nw : 0)
+                                          : mt * 128 + 32 * q + 16 * h + 8 * u + fq;
+              sc[2 * h + u] = wsr[wr];
+            }
+        }
+        const int mode = pr.kind == 0 ? (pr.f16 ? 1 : 0) : (pr.out_type == kOutF16 ? 2 : 0);
+        const int mi = lane >> 3;  // the stmatrix matrix this lane addresses, row lane % 8
+        for (int c0 = C::kColSplit ? 16 * grp : 0; c0 < ncols; c0 += C::kColSplit ? 32 : 16) {
+          uint32_t r[8], s[8];
+          tmem_ld_16x256b_x2(tbase + c0, r);
+          tmem_ld_16x256b_x2(tbase + (16u << 16) + c0, s);
+          tmem_ld_wait_16(r, s);
+          float a[2][8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            a[0][i] = __uint_as_float(r[i]) * sc[(i >> 1) & 1];
+            a[1][i] = __uint_as_float(s[i]) * sc[2 + ((i >> 1) & 1)];
+          }
+          uint8_t* buf = stg + (nstg % C::kStgBufs) * C::kStgBytes;
+          ++nstg;
+          __syncwarp();  // this buffer's reads of an earlier chunk are done
+          const uint32_t sb = smem_u32(buf);
+          if (pr.kind == 0) {
+            // a[h][4j], a[h][4j+1]: gate of feature 8h+fq at columns 8j+2(t%4), +1;
+            // a[h][4j+2], a[h][4j+3]: up of the same feature and columns.  Matrix 2h+j:
+            // features 8h.. x columns 8j..
+            uint32_t m4[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                m4[2 * h + j] = pack16(gelu_tanh(a[h][4 * j]) * a[h][4 * j + 2],
+                                       gelu_tanh(a[h][4 * j + 1]) * a[h][4 * j + 3], mode);
+            stmatrix_x4_trans(sb + stg_glu_off((lane & 7) + 8 * (mi & 1), mi >> 1), m4[0], m4[1],
+                              m4[2], m4[3]);
+            __syncwarp();
+            const int tok = lane >> 1, ch = lane & 1;
+            if (c0 + tok < pc.n_valid) {
+              const uint4 val = *reinterpret_cast<const uint4*>(buf + stg_glu_off(tok, ch));
+              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(pr.out) +
+                                        static_cast<size_t>(pos0 + c0 + tok) * pr.out_ld +
+                                        mt * 64 + 16 * q + 8 * ch) = val;
+            }
+          } else {
+            // half h, matrix i: rows 16h + 8(i&1).. x columns 8(i>>1)..
+            const int tok_w = (lane & 7) + 8 * (mi >> 1);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              stmatrix_x4_trans(sb + stg_dn_off(tok_w, 2 * h + (mi & 1)),
+                                pack16(a[h][0], a[h][1], mode), pack16(a[h][2], a[h][3], mode),
+                                pack16(a[h][4], a[h][5], mode), pack16(a[h][6], a[h][7], mode));
+            __syncwarp();
+#pragma unroll
+            for (int rnd = 0; rnd < 2; ++rnd) {
+              const int tok = 8 * rnd + (lane >> 2), g = lane & 3;
+              if (c0 + tok < pc.n_valid) {
+                const uint4 val = *reinterpret_cast<const uint4*>(buf + stg_dn_off(tok, g));
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(pr.out) +
+                                          static_cast<size_t>(pos0 + c0 + tok) * pr.out_ld +
+                                          mt * 128 + 32 * q + 8 * g) = val;
+              }
+            }
+          }
+        }
+      } else if (last) {
         const int pos0 = pc.b_row0 + pc.n * BN;  // output row of column 0
         float sc = 1.f;
         if (pr.wscale) {
@@ -711,7 +816,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
                              : mt * 128 + row;
           sc = pr.wscale[static_cast<size_t>(pc.g) * pr.w_rows_per_group + wr];
         }
-        for (int c0 = 0; c0 < ncols; c0 += 16) {
+        for (int c0 = C::kColSplit ? 16 * grp : 0; c0 < ncols; c0 += C::kColSplit ? 32 : 16) {
           float v[16];
           tmem_ld16(tbase + c0, v);
           if (pr.split > 1) {
@@ -891,6 +996,9 @@ bool gemm_pairs_allowed(int bn, bool int8_weights) { return !int8_weights && bn 
 
 cudaError_t launch_grouped_gemm(int bn, const GemmMaps& maps, const GemmParams& p, int grid,
                                 cudaStream_t s, bool pdl) {
+  // split K only with BN = 16 (wider tiles split their epilogue by columns instead)
+  for (int i = 0; i < p.nprob; ++i)
+    if (bn != 16 && p.prob[i].split > 1) return cudaErrorInvalidValue;
   if (p.pairs) {
     if (!gemm_pairs_allowed(bn, p.int8_weights != 0)) return cudaErrorInvalidValue;
 
