@@ -364,8 +364,7 @@ def run_ours(args, wl, rank, world, device):
                   "tc_frac": round(t_tc / (ms_step * 1e-3), 4),
                   "binding_frac": round(max(t_hbm, t_tc) / (ms_step * 1e-3), 4),
                   "mean_used_experts": round(sum(used) / len(used), 2)}
-    # router (with the sort when T*k <= 8192, else 3 sort kernels), gather, 2 GEMMs, combine
-    launches_per_call = 5 + (0 if T * shape.k <= 8192 else 3)
+    launches_per_call = mf.moe_block_launch_count(cfg, T)  # the library's own count
     res = {
         "metric": METRIC, "value": round(world * T * K / (t_max * 1e-3), 1), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 5),

@@ -226,12 +226,19 @@ moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream);
  * otherwise MOE_ERR_WORKSPACE; a timeout out of range gives MOE_ERR_INVALID_ARG. */
 moe_status_t moe_wait_selftest(void* ws, size_t ws_bytes, uint64_t timeout_ns, void* stream);
 
+/* Number of kernels that one moe_block_forward(cfg, T, ...) launches (host-only, no
+ * GPU needed): the router (1, or 2 for the tensor-core router of T > 128: weight prep and
+ * router), the permutation (0 when the router sorts in the same launch, else 1 or 3),
+ * the row gather, the gate_up and down GEMMs and the combine (1 each).  0 for T = 0;
+ * -1 when cfg or T is invalid (the arguments moe_block_forward would reject). */
+int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T);
+
 /* A short constant English description of a status code. */
 const char* moe_status_string(moe_status_t status);
 
 /* Version of this interface (increases when a signature or a calling contract changes;
  * 2: the workspace is zeroed once by the caller, MOE_BLOCK_EVENTS is 7;
- * 3: moe_wait_selftest). */
+ * 3: moe_wait_selftest; 4: moe_block_launch_count). */
 int32_t moe_abi_version(void);
 
 #ifdef __cplusplus

@@ -31,7 +31,7 @@ MOE_W_INT8 = 1
 ENTRY_POINTS = ("moe_workspace_size", "moe_router", "moe_permute", "moe_permute_noalloc",
                 "moe_ffn_forward", "dense_mlp_forward", "moe_block_forward",
                 "moe_quantize_int8", "moe_check_device_status", "moe_wait_selftest",
-                "moe_status_string", "moe_abi_version")
+                "moe_block_launch_count", "moe_status_string", "moe_abi_version")
 PERMUTE_NOALLOC_MAX_PAIRS = 1 << 20
 
 
@@ -77,6 +77,7 @@ _SIG = {
     "moe_quantize_int8": (_I32, [_P, ctypes.c_int64, _I32, _P, _P, _P]),
     "moe_check_device_status": (_I32, [_P, ctypes.c_size_t, _P]),
     "moe_wait_selftest": (_I32, [_P, ctypes.c_size_t, ctypes.c_uint64, _P]),
+    "moe_block_launch_count": (_I32, [ctypes.POINTER(CConfig), _I32]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
     "moe_abi_version": (_I32, []),
 }
@@ -285,6 +286,11 @@ def moe_wait_selftest(ws, timeout_ns: int, stream=None) -> None:
     kernel's waits); afterwards moe_check_device_status reports MOE_ERR_DEVICE_TIMEOUT."""
     _check("moe_wait_selftest", lib().moe_wait_selftest(_ptr(ws, torch.uint8, "ws"), ws.numel(),
                                                          int(timeout_ns), _stream(stream)))
+
+
+def moe_block_launch_count(cfg, T: int) -> int:
+    """Kernels one moe_block_forward launches for this config and T (-1: invalid)."""
+    return int(lib().moe_block_launch_count(ctypes.byref(cfg.c()), int(T)))
 
 
 def moe_check_device_status(ws, stream=None) -> int:

@@ -440,7 +440,20 @@ bool w_ok(const moe_expert_weights_t* w, bool int8) {
 
 extern "C" {
 
-int32_t moe_abi_version(void) { return 3; }
+int32_t moe_abi_version(void) { return 4; }
+
+int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T) {
+  Dims d;
+  if (check_cfg(cfg, T, &d) != MOE_OK) return -1;
+  if (T == 0) return 0;
+  const int Tk = d.T * d.k;
+  // the same decisions as moe_block_forward
+  const bool tc = router_uses_tc(d.T);
+  const bool fused_sort = !tc && permute_blocks(Tk) == 0;
+  int n = tc ? 2 : 1;                                     // router (prep + router)
+  if (!fused_sort) n += permute_blocks(Tk) == 0 ? 1 : 3;  // permutation
+  return n + 4;                                           // gather, gate_up, down, combine
+}
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 3
+    assert lib.moe_abi_version() == 4
     for s in range(6):
         assert mf.status_string(s)
     assert mf.status_string(99) == "unknown status"
@@ -63,6 +63,21 @@ def test_workspace_size(lib):
         assert mf.workspace_size(c, 8) == 0, b
     assert lib.moe_workspace_size(None, 8) == 0
     assert mf.workspace_size(CFG, -1) == 0
+
+
+def test_block_launch_count(lib):
+    # router 1 (2 above T = 128: weight prep + tensor-core router); permutation 0 when the
+    # CUDA-core router sorts (T*k <= 2048), 1 (T*k <= 2048), else 3; gather, gate_up,
+    # down, combine 1 each
+    for T, n in ((1, 5), (8, 5), (64, 5), (128, 5), (129, 7), (256, 7), (257, 9), (2048, 9),
+                 (16384, 9)):
+        assert mf.moe_block_launch_count(CFG, T) == n, T
+    for T, n in ((8, 5), (512, 7), (513, 9)):  # top-4: T*k = 2048 at T = 512
+        assert mf.moe_block_launch_count(TINY, T) == n, T
+    assert mf.moe_block_launch_count(CFG, 0) == 0
+    assert mf.moe_block_launch_count(CFG, -1) == -1
+    assert mf.moe_block_launch_count(mf.Config(**{**CFG.__dict__, "top_k": 17}), 8) == -1
+    assert lib.moe_block_launch_count(None, 8) == -1
 
 
 FAKE = 1 << 20  # an aligned address that is never dereferenced
