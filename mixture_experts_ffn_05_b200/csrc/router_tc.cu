@@ -41,6 +41,11 @@ constexpr int kTcSmemBudget = 192 * 1024;
 constexpr uint32_t kTcTile = 128 * 128;  // one x tile: 128 rows of 64 bf16
 constexpr int kTcWriterThreads = 256;    // warps 6..13
 constexpr int kTcMaxE = 256;
+// the selection of a several-slice tile stages 128 x (E + 1) logits in the ring, whose
+// size is at least the budget less one stage of the widest slice (128 experts)
+static_assert(kTcSmemBudget - (static_cast<int>(kTcTile) + 2 * 128 * 128) >=
+                  kTcTokens * (kTcMaxE + 1) * 4,
+              "ring too small for the logits of a tile");
 
 struct RouterTcArgs {
   int T, H, E, k;
@@ -91,23 +96,22 @@ struct TopK {
     }
   }
 
+  // The new key's place is the number of kept keys >= it (they are sorted, so those are
+  // a prefix); every slot then updates independently of the others, so a push is a few
+  // dependent steps and no branch (a shifting insertion is a chain of KMAX steps, and in
+  // a warp of 32 rows nearly every push inserts somewhere).
   __device__ __forceinline__ void push(float l, int e) {
-    uint32_t ck = order_key(l);
-    if (ck > key[KMAX - 1]) {
-      int ci = e;
-      bool shift = false;
+    const uint32_t ck = order_key(l);
+    int pos = 0;
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        const bool g = shift || ck > key[j];
-        const uint32_t tk = g ? key[j] : ck;
-        const int ti = g ? id[j] : ci;
-        key[j] = g ? ck : key[j];
-        id[j] = g ? ci : id[j];
-        ck = tk;
-        ci = ti;
-        shift = g;
-      }
+    for (int j = 0; j < KMAX; ++j) pos += key[j] >= ck ? 1 : 0;
+#pragma unroll
+    for (int j = KMAX - 1; j > 0; --j) {
+      key[j] = j < pos ? key[j] : (j == pos ? ck : key[j - 1]);
+      id[j] = j < pos ? id[j] : (j == pos ? e : id[j - 1]);
     }
+    key[0] = pos > 0 ? key[0] : ck;
+    id[0] = pos > 0 ? id[0] : e;
   }
 
   // softmax restricted to the selected experts (the full denominator cancels in the
@@ -415,14 +419,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   __syncthreads();
-  if (!s_last || threadIdx.x < 64 || threadIdx.x >= 64 + kTcTokens) return;
-  const int t = t0 + static_cast<int>(threadIdx.x) - 64;
-  if (t >= a.T) return;
+  if (!s_last) return;
+  // The tile's logits go through shared memory (the ring is free now): coalesced loads by
+  // the whole CTA, rows padded to E + 1 floats so that the row-per-thread reads of the
+  // selection hit distinct banks.  (Read straight from global memory, each thread's
+  // row-wise loads made every warp request touch 32 rows; the selection took ~30 us.)
+  // With several slices a stage holds at least 144 KB of the 192 KB ring, more than
+  // the 128 x 257 floats of E = 256.
+  const int rows = min(kTcTokens, a.T - t0);
+  const int ld = a.E + 1;
+  float* sl = reinterpret_cast<float*>(ring);
+  const float* src = a.logits + static_cast<size_t>(t0) * a.E;
+  const int n = rows * a.E;
+  if ((a.E & 3) == 0) {  // 16-byte loads (a row starts on a 16-byte boundary)
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll 8
+    for (int i = threadIdx.x; i < n / 4; i += kTcThreads) {
+      const float4 v = __ldcg(s4 + i);
+      float* d = sl + (4 * i / a.E) * ld + (4 * i) % a.E;
+      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+    }
+  } else {
+#pragma unroll 8
+    for (int i = threadIdx.x; i < n; i += kTcThreads) sl[(i / a.E) * ld + i % a.E] = __ldcg(src + i);
+  }
+  __syncthreads();
+  if (threadIdx.x < 64 || threadIdx.x >= 64 + kTcTokens) return;
+  const int r = static_cast<int>(threadIdx.x) - 64;
+  if (r >= rows) return;
   TopK<KMAX> tk;
   tk.init();
-  const float* lr = a.logits + static_cast<size_t>(t) * a.E;
-  for (int e = 0; e < a.E; ++e) tk.push(__ldcg(lr + e), e);
-  tk.write(t, a.k, s_pes, a.topk_idx, a.topk_w);
+  const float* lr = sl + r * ld;
+  for (int e = 0; e < a.E; ++e) tk.push(lr[e], e);
+  tk.write(t0 + r, a.k, s_pes, a.topk_idx, a.topk_w);
 }
 
 // W'hi, W'lo = the two-term bf16 split of s[h] * W_r[e,h] / sqrt(H); one thread per 8.
