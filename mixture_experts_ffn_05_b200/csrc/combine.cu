@@ -16,6 +16,7 @@
 namespace moe {
 
 constexpr int kCombMaxThreads = 768;  // H <= 6144: one 8-column chunk per thread
+constexpr int kCombManyTokens = 256;  // from here on, occupancy over slots in flight
 
 // Sums of two values over the block in a fixed order (deterministic).
 __device__ __forceinline__ float2 block_sum2(float a, float b, float2* red) {
@@ -78,12 +79,14 @@ __global__ void __launch_bounds__(MAXT, MINB) combine_block_kernel(
   const int c = threadIdx.x;
   const bool on = c < (H >> 3);
   const int cc = on ? c : 0;
-  // the residual does not depend on the previous kernel (the gains, read late, are
-  // cache-resident)
+  // Read before the dependency wait: the residual, and the slot table.  inv_pos and
+  // topk_w come from the routing kernels, which completed before the kernel this one
+  // follows could start (the gather and GEMM launches wait for them); only Y and the dense
+  // output are the previous kernel's results.  (The gains, read late, are cache-resident.)
   const uint4 vx = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + cc);
+  load_slots(t, k, gridDim.x * k, inv_pos, sorted_src, topk_w, s_q, s_w);
   pdl_wait();
   pdl_trigger();
-  load_slots(t, k, gridDim.x * k, inv_pos, sorted_src, topk_w, s_q, s_w);
   float m[8], d[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = d[i] = 0.f;
@@ -177,9 +180,16 @@ cudaError_t launch_combine_block(int T, int H, int k, float eps, const uint16_t*
                                  const uint16_t* g_post_ff, uint16_t* out, uint16_t* moe_out,
                                  cudaStream_t s, bool pdl) {
   const int threads = std::max(32, ((H >> 3) + 31) / 32 * 32);
-  if (threads <= 384)
+  // Many tokens: resident CTAs hide the latency (4 slots in flight, 4 CTAs per SM).  Few
+  // tokens (up to about two CTAs per SM): every slot in flight at once (k <= 16), so that
+  // a token's Y rows cost one round trip.
+  if (threads <= 384 && T >= kCombManyTokens)
     return launch_k(combine_block_kernel<384, 4, 4>, dim3(T), dim3(threads), 0, s, pdl, H, k, eps,
                     x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe, g_post_dense,
+                    g_post_ff, out, moe_out);
+  if (threads <= 384)
+    return launch_k(combine_block_kernel<384, 16, 1>, dim3(T), dim3(threads), 0, s, pdl, H, k,
+                    eps, x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe, g_post_dense,
                     g_post_ff, out, moe_out);
   return launch_k(combine_block_kernel<kCombMaxThreads, 8, 1>, dim3(T), dim3(threads), 0, s, pdl,
                   H, k, eps, x, y, inv_pos, sorted_src, topk_w, dense, g_post_moe,
