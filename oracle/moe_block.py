@@ -15,6 +15,8 @@ Sources (page title, section):
        and "How it works".
   [P5] "Gemma-4 26B-A4B-it - ONNX MoE text decoder", table "Truthful graph
        contracts" (rows "Mixture of Experts", "MoE topology", "Router").
+  [P6] "Gemma 4 26B-A4B IT" (inference recipe), section "Quantized Variants" and its
+       variant list: FP8 (E4M3) weights with dynamic per-token activation quantization.
 
 Readings taken where the pages leave a step open (each also listed in the design notes):
   R1  RMSNorm multiplies by the stored gain as-is, eps inside the square root.
@@ -29,6 +31,14 @@ Readings taken where the pages leave a step open (each also listed in the design
   R8  gate_up rows 0..I-1 are the gate projection and rows I..2I-1 the up projection.
   R9  int8 experts: per output row s = max|w| / 127 (fp32), q = round-half-even(w / s)
       clamped to [-127, 127]; an all-zero row takes s = 1.
+  R10 fp8 experts ([P6]): E4M3 as the OCP 8-bit format defines it (1 sign, 4 exponent
+      bits of bias 7, 3 mantissa bits, subnormals, no infinities, largest finite 448).
+      Weights per output row and activations per token row (the rows entering each
+      expert matmul: the routed token's xn_moe, and h) take s = max|v| / 448 (fp32, an
+      all-zero row s = 1) and codes e4m3(v / s): the fp32 quotient rounded to nearest
+      even on the E4M3 grid, saturating at +-448.  The activations are quantised from
+      the bf16 values the expert matmuls receive (xn_moe and h are bf16 tensors), so both
+      sides take each rounding decision from the same number.
 """
 from __future__ import annotations
 
@@ -142,21 +152,34 @@ class Experts:
     """
 
     def __init__(self, w_gate_up=None, w_down=None, q_gate_up=None, s_gate_up=None,
-                 q_down=None, s_down=None):
-        self.int8 = q_gate_up is not None
+                 q_down=None, s_down=None, fp8: bool = False):
+        self.fp8 = fp8                     # q_* are E4M3 codes (uint8) and the activations
+        self.int8 = q_gate_up is not None and not fp8   # of both matmuls are quantised
         self.w_gate_up, self.w_down = w_gate_up, w_down
         self.q_gate_up, self.s_gate_up = q_gate_up, s_gate_up
         self.q_down, self.s_down = q_down, s_down
 
     def gate_up(self, e: int) -> np.ndarray:
+        if self.fp8:
+            return dequantize_fp8(self.q_gate_up[e], self.s_gate_up[e])
         if self.int8:
             return dequantize(self.q_gate_up[e], self.s_gate_up[e])
         return bf16(self.w_gate_up[e])
 
     def down(self, e: int) -> np.ndarray:
+        if self.fp8:
+            return dequantize_fp8(self.q_down[e], self.s_down[e])
         if self.int8:
             return dequantize(self.q_down[e], self.s_down[e])
         return bf16(self.w_down[e])
+
+
+
+def expert_mlp(experts, u: np.ndarray, e: int) -> np.ndarray:
+    """Expert e's gated MLP on rows u; fp8 experts run it on quantised activations (R10).
+    `experts` is anything with gate_up(e) and down(e) (and optionally fp8)."""
+    f = gated_mlp_fp8 if getattr(experts, "fp8", False) else gated_mlp
+    return f(u, experts.gate_up(e), experts.down(e))
 
 
 def moe_sparse(xn_moe: np.ndarray, topk_idx: np.ndarray, topk_w: np.ndarray,
@@ -171,7 +194,7 @@ def moe_sparse(xn_moe: np.ndarray, topk_idx: np.ndarray, topk_w: np.ndarray,
     y = np.zeros((T, k, xn.shape[1]), dtype=np.float64)
     for e in np.unique(topk_idx):
         tt, jj = np.nonzero(topk_idx == e)
-        y[tt, jj] = gated_mlp(xn[tt], experts.gate_up(int(e)), experts.down(int(e)))
+        y[tt, jj] = expert_mlp(experts, xn[tt], int(e))
     moe = np.zeros((T, xn.shape[1]), dtype=np.float64)
     for j in range(k):
         moe += topk_w[:, j:j + 1] * y[:, j]
@@ -184,7 +207,7 @@ def moe_all_experts_dense(xn_moe: np.ndarray, route: np.ndarray, experts: Expert
     xn = np.asarray(xn_moe, dtype=np.float64)
     moe = np.zeros_like(xn)
     for e in range(route.shape[1]):
-        moe += route[:, e:e + 1] * gated_mlp(xn, experts.gate_up(e), experts.down(e))
+        moe += route[:, e:e + 1] * expert_mlp(experts, xn, e)
     return moe
 
 
@@ -250,6 +273,96 @@ def quantize_int8_per_channel(w_bits: np.ndarray):
 def dequantize(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     """q * s per row, in float64."""
     return np.asarray(q, dtype=np.float64) * np.asarray(s, dtype=np.float64)[..., None]
+
+
+# ----------------------------------------------------------------------------- fp8 (E4M3)
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode_table() -> np.ndarray:
+    """Value of every E4M3 code 0..255, from the format's definition (R10): sign bit 7,
+    exponent bits 6..3 (bias 7), mantissa bits 2..0; exponent 0 is subnormal
+    (m/8 * 2^-6); code S.1111.111 is NaN."""
+    c = np.arange(256)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+    mag = np.where((e == 15) & ((c & 7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Round to the nearest E4M3 value, ties to even, saturating at +-448 (R10).
+
+    Normal binade [2^e, 2^(e+1)) has spacing 2^(e-3); below 2^-6 the spacing is 2^-9
+    (subnormals).  np.rint rounds half to even on the integer multiple of the spacing,
+    which is the even-mantissa rule of the format."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))       # a = f * 2^ex, f in [0.5, 1)
+    spacing = np.where(a < 2.0 ** -6, 2.0 ** -9, 2.0 ** (ex - 1 - 3.0))
+    q = np.rint(a / spacing) * spacing
+    return np.sign(v) * np.minimum(q, E4M3_MAX)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """Code (uint8) of E4M3 grid values (already rounded); -0 encodes as +0."""
+    tab = e4m3_decode_table()
+    pos = tab[:127]                                   # codes 0..126: 0 .. 448, increasing
+    v = np.asarray(v, dtype=np.float64)
+    idx = np.searchsorted(pos, np.abs(v))
+    assert np.all(pos[np.minimum(idx, 126)] == np.abs(v)), "not an E4M3 value"
+    return (idx + np.where(v < 0, 128, 0)).astype(np.uint8)
+
+
+def quantize_fp8_rows(v32: np.ndarray):
+    """Per-row E4M3 quantisation (R10) of fp32 values (rows = all axes but the last):
+    s = max|v| / 448 in fp32 (1 for an all-zero row), codes of e4m3(fp32(v / s)).
+    Returns (codes uint8, s fp32)."""
+    v = np.asarray(v32, dtype=np.float32)
+    amax = np.max(np.abs(v), axis=-1)
+    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    quot = (v / s[..., None]).astype(np.float32)      # the fp32 quotient the kernels round
+    return e4m3_encode(e4m3_round(quot)), s
+
+
+def quantize_fp8_per_channel(w_bits: np.ndarray):
+    """Per-output-row E4M3 quantisation of bf16 weights ([P6]; R10)."""
+    u = np.asarray(w_bits, dtype=np.uint16)
+    return quantize_fp8_rows((u.astype(np.uint32) << np.uint32(16)).view(np.float32))
+
+
+def dequantize_fp8(codes: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """E4M3 value times the row scale, in float64."""
+    return e4m3_decode_table()[np.asarray(codes, dtype=np.uint8)] * \
+        np.asarray(s, dtype=np.float64)[..., None]
+
+
+def bf16_round(v) -> np.ndarray:
+    """float64 -> fp32 (nearest) -> bf16 (nearest, ties to even), back as float64: the
+    value of an activation stored as bf16."""
+    f = np.asarray(v, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << np.uint32(16)
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def fp8_activation(v) -> np.ndarray:
+    """An expert matmul's activation rows as the fp8 path uses them (R10): stored as
+    bf16, quantised per row to E4M3, dequantised (float64)."""
+    q, s = quantize_fp8_rows(bf16_round(v).astype(np.float32))
+    return dequantize_fp8(q, s)
+
+
+def gated_mlp_fp8(u: np.ndarray, w_gate_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
+    """gated_mlp with both expert matmuls on fp8 activations (R10): the input rows and h
+    are quantised per row; the weights arrive already dequantised."""
+    I = w_gate_up.shape[0] // 2
+    uq = fp8_activation(u)
+    h = gelu_tanh(uq @ w_gate_up[:I].T) * (uq @ w_gate_up[I:].T)
+    return fp8_activation(h) @ w_down.T
 
 
 # ----------------------------------------------------------------------------- gaps

@@ -325,6 +325,79 @@ def test_int8_quantiser_pins():
     assert qq[0].tolist() == [127, 2, 4, -2, 0]
 
 
+# ------------------------------------------------------------------ fp8 (E4M3)
+
+def test_e4m3_decode_table_matches_torch():
+    """R10: the format written out (sign, 4 exponent bits of bias 7, 3 mantissa bits,
+    subnormals, NaN at S.1111.111) equals the library's float8_e4m3fn decoding."""
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    tab = oracle.e4m3_decode_table()
+    assert np.array_equal(np.isnan(tab), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(tab[ok], ref[ok])
+    assert tab[0x7E] == 448.0 and tab[0x01] == 2.0 ** -9 and tab[0x08] == 2.0 ** -6
+
+
+def test_e4m3_rounding_matches_torch_and_closed_forms():
+    """Round-to-nearest-even onto the E4M3 grid equals the library's fp32 -> float8_e4m3fn
+    conversion inside the finite range; ties, the subnormal floor and the saturation at
+    448 (the kernels' satfinite rounding, which the library conversion does not do) by
+    closed forms."""
+    tab = oracle.e4m3_decode_table()
+    fin = tab[np.isfinite(tab)]
+    assert np.array_equal(oracle.e4m3_round(fin), fin)           # grid values stay put
+    pos = np.unique(np.abs(fin))
+    mids = (pos[:-1] + pos[1:]) / 2                                # every exact tie
+    v = np.concatenate([RNG.uniform(-440, 440, 4000), RNG.uniform(-0.05, 0.05, 4000),
+                        mids, -mids, [0.0]]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.e4m3_round(v.astype(np.float64)), ref)
+    got = oracle.e4m3_round([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 449.0, 1e6, -1e6])
+    assert got.tolist() == [1.0, 1.25, 0.0, 2.0 ** -8, 448.0, 448.0, -448.0]
+    assert oracle.e4m3_encode(got[:4]).tolist() == [0x38, 0x3A, 0x00, 0x02]
+
+
+def test_fp8_quantiser_pins():
+    """R10: s = max|w| / 448; each value lands within half an E4M3 step (relative 2^-4,
+    or 2^-10 s absolute below the normal range) of w; the largest |w| of a row becomes
+    +-448 exactly; an all-zero row takes s = 1 and code 0."""
+    w = synth.normal_bf16(5, (98,), (6, 40), 0.02)
+    w[3] = 0
+    q, s = oracle.quantize_fp8_per_channel(w)
+    wf = synth.bf16_bits_to_f32(w).astype(np.float64)
+    assert q.dtype == np.uint8 and s.dtype == np.float32
+    deq = oracle.dequantize_fp8(q, s)
+    err = np.abs(deq - wf)
+    bound = np.maximum(np.abs(wf) * 2.0 ** -4, s[:, None] * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(err <= bound)
+    tab = oracle.e4m3_decode_table()
+    nz = [i for i in range(6) if i != 3]
+    assert np.all(np.abs(tab[q[nz]]).max(1) == 448.0)
+    assert s[3] == 1.0 and np.all(q[3] == 0)
+
+
+def test_fp8_activation_scale_is_per_token():
+    """R10 and [P6] (dynamic per-token activation scales): the all-experts-dense form runs
+    every token through every expert, the sparse form only the routed rows; the two agree
+    only if a token's quantisation does not depend on which other rows share the matmul."""
+    E, k, H, I, T = 6, 2, 32, 16, 9
+    wgu = synth.normal_bf16(21, (1,), (E, 2 * I, H), 0.2)
+    wd = synth.normal_bf16(21, (2,), (E, H, I), 0.2)
+    qg, sg = oracle.quantize_fp8_per_channel(wgu)
+    qd, sd = oracle.quantize_fp8_per_channel(wd)
+    ex = oracle.Experts(q_gate_up=qg, s_gate_up=sg, q_down=qd, s_down=sd, fp8=True)
+    xn = RNG.standard_normal((T, H))
+    idx = np.stack([RNG.permutation(E)[:k] for _ in range(T)])
+    tw = RNG.uniform(0.1, 1.0, (T, k))
+    sparse = oracle.moe_sparse(xn, idx, tw, ex)
+    dense = oracle.moe_all_experts_dense(xn, oracle.dense_route(idx, tw, E), ex)
+    np.testing.assert_allclose(sparse, dense, rtol=1e-12, atol=1e-12)
+    # and the quantisation is really there: the bf16-weight reading differs by ~ 2^-4
+    bfx = oracle.Experts(w_gate_up=wgu, w_down=wd)
+    rel = np.abs(sparse - oracle.moe_sparse(xn, idx, tw, bfx)).max() / np.abs(sparse).max()
+    assert 1e-3 < rel < 0.2
+
+
 # ------------------------------------------------------------------ the bar discriminates
 
 def test_fp16_accumulation_fails_the_bar():
