@@ -70,8 +70,10 @@ typedef enum {
 } moe_status_t;
 
 typedef enum {
-  MOE_W_BF16 = 0, /* expert weights in bf16 */
-  MOE_W_INT8 = 1  /* expert weights int8, one fp32 scale per output row */
+  MOE_W_BF16 = 0,    /* expert weights in bf16 */
+  MOE_W_INT8 = 1,    /* expert weights int8, one fp32 scale per output row */
+  MOE_W_FP8_E4M3 = 2 /* expert weights E4M3, one fp32 scale per output row; the expert
+                        matmuls' activations are quantised to E4M3 per token row */
 } moe_wdtype_t;
 
 /* Sizes of one layer. */
@@ -91,7 +93,14 @@ typedef struct {
  *   w_down    [E][H][I];
  *   bf16 (MOE_W_BF16): s_gate_up and s_down must be NULL.
  *   int8 (MOE_W_INT8): the weight is q * s, with s_gate_up [E][2I] and s_down [E][H]
- *                      fp32 per-output-row scales (see moe_quantize_int8). */
+ *                      fp32 per-output-row scales (see moe_quantize_int8).
+ *   fp8 (MOE_W_FP8_E4M3): the same layout of E4M3 codes (uint8) with the same scales
+ *                      (see moe_quantize_fp8).  This is the "FP8-dynamic" variant ("Gemma 4
+ *                      26B-A4B IT" recipe page, "Quantized Variants": E4M3 weights with
+ *                      dynamic per-token activation quantisation): each expert matmul's
+ *                      input rows (a routed token's xn_moe, its h) are quantised with
+ *                      their own scale max|row| / 448, codes rounded to nearest even and
+ *                      saturating; the products accumulate in fp32. */
 typedef struct {
   const void* w_gate_up;
   const void* w_down;
@@ -212,6 +221,14 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
 moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, int8_t* q,
                                float* scales, void* stream);
 
+/* Per-output-row E4M3 quantisation for MOE_W_FP8_E4M3, in fp32: s = max|w| / 448 (s = 1
+ * for an all-zero row), q = E4M3 code of w / s, rounded to nearest even, saturating at
+ * +-448 ("Gemma 4 26B-A4B IT", "Quantized Variants").  w [rows][cols] bf16 -> q
+ * [rows][cols] uint8 codes, scales [rows] fp32; cols a multiple of 8 (8..65536),
+ * rows >= 0; w and q 16-byte aligned. */
+moe_status_t moe_quantize_fp8(const moe_bf16_t* w, int64_t rows, int32_t cols, uint8_t* q,
+                              float* scales, void* stream);
+
 /* Waits for `stream`, then reads and clears the device status word in `ws`.
  * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, or MOE_ERR_CUDA if the stream failed. */
 moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream);
@@ -229,7 +246,8 @@ moe_status_t moe_wait_selftest(void* ws, size_t ws_bytes, uint64_t timeout_ns, v
 /* Number of kernels that one moe_block_forward(cfg, T, ...) launches (host-only, no
  * GPU needed): the router (1, or 2 for the tensor-core router of T > 128: weight prep and
  * router), the permutation (0 when the router sorts in the same launch, else 1 or 3),
- * the row gather, the gate_up and down GEMMs and the combine (1 each).  0 for T = 0;
+ * the row gather, the gate_up and down GEMMs and the combine (1 each), and for
+ * MOE_W_FP8_E4M3 the quantisation of h between the GEMMs.  0 for T = 0;
  * -1 when cfg or T is invalid (the arguments moe_block_forward would reject). */
 int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T);
 
@@ -238,7 +256,7 @@ const char* moe_status_string(moe_status_t status);
 
 /* Version of this interface (increases when a signature or a calling contract changes;
  * 2: the workspace is zeroed once by the caller, MOE_BLOCK_EVENTS is 7;
- * 3: moe_wait_selftest; 4: moe_block_launch_count). */
+ * 3: moe_wait_selftest; 4: moe_block_launch_count; 5: MOE_W_FP8_E4M3, moe_quantize_fp8). */
 int32_t moe_abi_version(void);
 
 #ifdef __cplusplus

@@ -26,11 +26,13 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 
 MOE_W_BF16 = 0
 MOE_W_INT8 = 1
+MOE_W_FP8 = 2
 
 # Entry points of include/moe_ffn.h (the CPU tests check the header declares exactly these).
 ENTRY_POINTS = ("moe_workspace_size", "moe_router", "moe_permute", "moe_permute_noalloc",
                 "moe_ffn_forward", "dense_mlp_forward", "moe_block_forward",
-                "moe_quantize_int8", "moe_check_device_status", "moe_wait_selftest",
+                "moe_quantize_int8", "moe_quantize_fp8", "moe_check_device_status",
+                "moe_wait_selftest",
                 "moe_block_launch_count", "moe_status_string", "moe_abi_version")
 PERMUTE_NOALLOC_MAX_PAIRS = 1 << 20
 
@@ -75,6 +77,7 @@ _SIG = {
     "moe_block_forward": (_I32, [ctypes.POINTER(CConfig), _I32, _P, ctypes.POINTER(CBlockWeights),
                                  _P, _P, _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "moe_quantize_int8": (_I32, [_P, ctypes.c_int64, _I32, _P, _P, _P]),
+    "moe_quantize_fp8": (_I32, [_P, ctypes.c_int64, _I32, _P, _P, _P]),
     "moe_check_device_status": (_I32, [_P, ctypes.c_size_t, _P]),
     "moe_wait_selftest": (_I32, [_P, ctypes.c_size_t, ctypes.c_uint64, _P]),
     "moe_block_launch_count": (_I32, [ctypes.POINTER(CConfig), _I32]),
@@ -119,10 +122,12 @@ class Config:
     dense_inter: int
     eps: float = 1e-6
     int8: bool = False
+    fp8: bool = False   # E4M3 expert weights, per-token E4M3 activations
 
     def c(self) -> CConfig:
+        wd = MOE_W_FP8 if self.fp8 else (MOE_W_INT8 if self.int8 else MOE_W_BF16)
         return CConfig(self.hidden, self.num_experts, self.top_k, self.expert_inter,
-                       self.dense_inter, self.eps, MOE_W_INT8 if self.int8 else MOE_W_BF16)
+                       self.dense_inter, self.eps, wd)
 
 
 def _ptr(t, dtype=None, name="tensor", nullable=False):
@@ -199,7 +204,7 @@ def moe_permute_noalloc(cfg, topk_idx, expert_offsets, sorted_src, inv_pos, stre
 
 
 def _experts(cfg, e: dict) -> CExpertWeights:
-    wt = torch.int8 if cfg.int8 else BF16
+    wt = torch.uint8 if cfg.fp8 else (torch.int8 if cfg.int8 else BF16)
     return CExpertWeights(_ptr(e["w_gate_up"], wt, "w_gate_up"), _ptr(e["w_down"], wt, "w_down"),
                           _ptr(e.get("s_gate_up"), torch.float32, "s_gate_up", True),
                           _ptr(e.get("s_down"), torch.float32, "s_down", True))
@@ -279,6 +284,15 @@ def moe_quantize_int8(w, q, scales, stream=None):
     st = lib().moe_quantize_int8(_ptr(w, BF16, "w"), rows, cols, _ptr(q, torch.int8, "q"),
                                  _ptr(scales, torch.float32, "scales"), _stream(stream))
     _check("moe_quantize_int8", st)
+
+
+def moe_quantize_fp8(w, q, scales, stream=None):
+    """Per-output-row E4M3 codes (uint8) and fp32 scales of bf16 weights."""
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    st = lib().moe_quantize_fp8(_ptr(w, BF16, "w"), rows, cols, _ptr(q, torch.uint8, "q"),
+                                _ptr(scales, torch.float32, "scales"), _stream(stream))
+    _check("moe_quantize_fp8", st)
 
 
 def moe_wait_selftest(ws, timeout_ns: int, stream=None) -> None:

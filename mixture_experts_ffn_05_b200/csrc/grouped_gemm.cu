@@ -428,19 +428,20 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
           }
           ++steps;
           uint8_t* sa = smem + stage * C::kStage;
-          // a step covers 64 K (bf16 weights) or 128 K (int8 codes, two B sub-tiles);
-          // the A tile is 16 KB either way
-          const int kw = (W8 && pr.w8) ? 128 : 64;
-          const int nb = kw / 64;
+          // a step covers 64 K (bf16), 128 K of int8 codes (two fp16 B sub-tiles) or 128 K
+          // of E4M3 codes (one B tile of 128-byte rows); the A tile is 16 KB in every case
+          const bool i8p = W8 && pr.w8;
+          const int kw = (i8p || pr.fp8) ? 128 : 64;
+          const int nb = i8p ? 2 : 1;
           if (PAIR) {
             // both CTAs' bytes land on the leader's barrier; the leader expects them all
             const uint32_t fb = cluster_addr(&full[stage], 0);
             if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::kABytes + C::kBBytes));
             if (pr.kind == 0)
-              tma_load_5d_pair(sa, ma, fb, ks * 64, 0, 0, mt * 8, pc.g, pol_w);
+              tma_load_5d_pair(sa, ma, fb, ks * kw, 0, 0, mt * 8, pc.g, pol_w);
             else
-              tma_load_2d_pair(sa, ma, fb, ks * 64, arow, pol_w);
-            load_b(sa + C::kABytes, mb, ks * 64, brow, &full[stage]);
+              tma_load_2d_pair(sa, ma, fb, ks * kw, arow, pol_w);
+            load_b(sa + C::kABytes, mb, ks * kw, brow, &full[stage]);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kABytes + nb * C::kBBytes);
             if (pr.kind == 0)  // 8 gate rows, the 8 matching up rows, ... (one 5-D box)
@@ -492,8 +493,10 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         if (piece < 0 || piece >= total) break;
         const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
         const int ncol = (pc.n_valid + 15) & ~15;
-        const uint32_t idesc = P.prob[pc.p].f16 ? idesc_f16_f32(PAIR ? 256 : 128, ncol)
-                                                : idesc_bf16_f32(PAIR ? 256 : 128, ncol);
+        // E4M3 operands take the A/B format code 0, as fp16 does under kind::f16
+        const bool f8 = P.prob[pc.p].fp8 != 0;
+        const uint32_t idesc = (P.prob[pc.p].f16 || f8) ? idesc_f16_f32(PAIR ? 256 : 128, ncol)
+                                                        : idesc_bf16_f32(PAIR ? 256 : 128, ncol);
         if (!mbar_wait(&acc_empty[ab], aph ^ 1u, tmo, abort_flag)) {
           ok = false;
           break;
@@ -529,13 +532,20 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
           } else {
             const uint64_t ad = sdesc_k_sw128(sa);
             const uint64_t bd = sdesc_k_sw128(sa + C::kABytes);
+            // four MMAs per 128-byte row: K = 16 bf16 or K = 32 E4M3 each
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t acc = (ks > pc.k0 || kk > 0) ? 1u : 0u;
-              if (PAIR)
+              if (f8) {
+                if (PAIR)
+                  umma_f8_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+                else
+                  umma_f8(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+              } else if (PAIR) {
                 umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
-              else
+              } else {
                 umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+              }
             }
           }
           if (PAIR) {
@@ -749,6 +759,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         }
         const int mode = pr.kind == 0 ? (pr.f16 ? 1 : 0) : (pr.out_type == kOutF16 ? 2 : 0);
         const int mi = lane >> 3;  // the stmatrix matrix this lane addresses, row lane % 8
+        const float* xsc = pr.xscale ? pr.xscale + pos0 : nullptr;  // fp8: per column
         for (int c0 = C::kColSplit ? 16 * grp : 0; c0 < ncols; c0 += C::kColSplit ? 32 : 16) {
           uint32_t r[8], s[8];
           tmem_ld_16x256b_x2(tbase + c0, r);
@@ -759,6 +770,20 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
           for (int i = 0; i < 8; ++i) {
             a[0][i] = __uint_as_float(r[i]) * sc[(i >> 1) & 1];
             a[1][i] = __uint_as_float(s[i]) * sc[2 + ((i >> 1) & 1)];
+          }
+          if (xsc != nullptr) {
+            // this thread's columns: 2m, 2m+1, 8+2m, 9+2m of the chunk (m = lane % 4)
+            float xs[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int col = c0 + 8 * (j >> 1) + 2 * (lane & 3) + (j & 1);
+              xs[j] = col < pc.n_valid ? __ldg(xsc + col) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              a[0][i] *= xs[((i >> 2) << 1) | (i & 1)];
+              a[1][i] *= xs[((i >> 2) << 1) | (i & 1)];
+            }
           }
           uint8_t* buf = stg + (nstg % C::kStgBufs) * C::kStgBytes;
           ++nstg;
@@ -846,6 +871,11 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] *= sc;
+          if (pr.xscale != nullptr) {  // fp8: the B rows' (tokens') scales, per column
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              v[i] *= c0 + i < pc.n_valid ? __ldg(pr.xscale + pos0 + c0 + i) : 0.f;
+          }
           if (pr.kind == 0) {
             // pair gate and up, 8 columns per lane
             const bool up = (lane & 8) != 0;

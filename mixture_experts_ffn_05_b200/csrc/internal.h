@@ -36,6 +36,9 @@ struct GemmProblem {
   int w8;                // A operand is int8 codes (needs a launch with int8_weights)
   int f16;               // A and B are fp16 (int8 codes are converted to fp16, exact);
                          // gate_up writes h in fp16
+  int fp8;               // A and B are E4M3 codes (kind::f8f6f4 MMAs, 128 K per step)
+  const float* xscale;   // fp8: scale of each B row (sorted order), applied per column
+                         // in the epilogue with wscale; NULL otherwise
 };
 
 constexpr int kOutBf16 = 0, kOutF32 = 1, kOutF16 = 2;
@@ -142,6 +145,14 @@ cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, const int
                                const int* sorted_src, const float* topk_w, uint16_t* moe_out,
                                cudaStream_t s, bool pdl = false);
 cudaError_t launch_wait_selftest(unsigned* status, uint64_t timeout_ns, cudaStream_t s);
+// dst[q] = E4M3 codes of row r(q) of src divided by scales[q] = max|row| / 448 (1 for an
+// all-zero row), r(q) = sorted_src[q] / k, or q when sorted_src is NULL; a source row
+// outside [0, T) gives a zero row.  cols a multiple of 8.
+cudaError_t launch_gather_quant_fp8(int n, int k, int cols, int T, const int* sorted_src,
+                                    const uint16_t* src, uint8_t* dst, float* scales,
+                                    cudaStream_t s, bool pdl);
+cudaError_t launch_quantize_fp8(const uint16_t* w, int64_t rows, int cols, uint8_t* q,
+                                float* scales, cudaStream_t s);
 cudaError_t launch_quantize_int8(const uint16_t* w, int64_t rows, int cols, int8_t* q,
                                  float* scales, cudaStream_t s);
 

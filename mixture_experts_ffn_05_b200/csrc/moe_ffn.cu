@@ -27,14 +27,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct Dims {
   int T, H, E, k, I, D;
   float eps;
-  int int8;
+  int int8;  // int8 expert weights (converted to fp16 on the way to the tensor cores)
+  int fp8;   // E4M3 expert weights and per-token E4M3 activations of the expert matmuls
 };
 
 moe_status_t check_cfg(const moe_config_t* c, int32_t T, Dims* d) {
   if (c == nullptr) return MOE_ERR_INVALID_ARG;
   if (T < 0) return MOE_ERR_INVALID_ARG;
   if (!(c->eps > 0.f) || !(c->eps < 1e30f)) return MOE_ERR_INVALID_ARG;
-  if (c->expert_wdtype != MOE_W_BF16 && c->expert_wdtype != MOE_W_INT8) return MOE_ERR_INVALID_ARG;
+  if (c->expert_wdtype != MOE_W_BF16 && c->expert_wdtype != MOE_W_INT8 &&
+      c->expert_wdtype != MOE_W_FP8_E4M3)
+    return MOE_ERR_INVALID_ARG;
   if (c->hidden < 128 || c->hidden > 6144 || c->hidden % 128) return MOE_ERR_UNSUPPORTED;
   if (c->expert_inter < 64 || c->expert_inter > 16384 || c->expert_inter % 64) return MOE_ERR_UNSUPPORTED;
   if (c->dense_inter < 64 || c->dense_inter > 16384 || c->dense_inter % 64) return MOE_ERR_UNSUPPORTED;
@@ -53,6 +56,7 @@ moe_status_t check_cfg(const moe_config_t* c, int32_t T, Dims* d) {
   d->D = c->dense_inter;
   d->eps = c->eps;
   d->int8 = c->expert_wdtype == MOE_W_INT8;
+  d->fp8 = c->expert_wdtype == MOE_W_FP8_E4M3;
   return MOE_OK;
 }
 
@@ -85,6 +89,7 @@ double expected_used_experts(const Dims& d) {
 struct Layout {
   size_t status, rcounters, counters, logits, bhist, bbase, topk_idx, topk_w, offsets, sorted, inv;
   size_t xn_moe, xn_dense, aperm, h, y, hd, dense, partials, wr_hi, wr_lo, sched, total;
+  size_t sx, h8, sh;  // fp8: token-row scales of the gathered rows, h in E4M3, h's scales
   size_t counters_bytes;
   int bn, split_gu, split_dgu, split_d, split_dd;
 };
@@ -95,7 +100,7 @@ Layout layout_of(const Dims& d) {
   Layout L{};
   const int64_t T = d.T, Tk = static_cast<int64_t>(d.T) * d.k;
   L.bn = choose_bn(d);
-  const int kw = d.int8 ? 128 : 64;  // K per pipeline step of the expert GEMMs
+  const int kw = (d.int8 || d.fp8) ? 128 : 64;  // K per pipeline step of the expert GEMMs
   // expected tiles of the two launches (experts and the dense MLP share each launch)
   const double u = expected_used_experts(d);
   const double dense_nt = static_cast<double>(ceil_div(T, L.bn));
@@ -147,6 +152,11 @@ Layout layout_of(const Dims& d) {
   L.wr_hi = take(wr_bytes);
   L.wr_lo = take(wr_bytes);
   L.sched = take(16);  // the GEMM launches' piece counters: [0..1] gate_up, [2..3] down
+  // fp8: the gathered rows' E4M3 codes share the aperm buffer; their scales, h in E4M3
+  // and h's row scales
+  L.sx = take(d.fp8 ? Tk * 4 : 0);
+  L.h8 = take(d.fp8 ? Tk * d.I : 0);
+  L.sh = take(d.fp8 ? Tk * 4 : 0);
   L.total = off;
   return L;
 }
@@ -251,7 +261,9 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
 struct GemmJob {
   // experts (problem 0), may be absent
   bool experts;
-  const uint16_t* a_rows;    // gathered xn_moe rows, [Tk][H]
+  const void* a_rows;        // gathered xn_moe rows, [Tk][H]: bf16, fp16 (int8 experts)
+                             // or E4M3 codes (fp8 experts)
+  const float* a_scales;     // fp8: the gathered rows' scales [Tk]
   const void* w_gate_up;
   const void* w_down;
   const float* s_gate_up;
@@ -272,6 +284,19 @@ struct GemmJob {
 // Records ev[i] on s when a stage-event array was given.
 bool mark(void* const* ev, int i, cudaStream_t s) {
   return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
+}
+
+// The routed tokens' rows in sorted order for the gate_up matmul: bf16 copies, fp16 copies
+// (int8 experts) or per-row E4M3 codes and scales (fp8 experts).
+moe_status_t gather_tokens(const Dims& d, const Layout& L, void* ws, const int* sorted,
+                           const uint16_t* xn_moe, cudaStream_t s, bool pdl) {
+  const int Tk = d.T * d.k;
+  if (d.fp8)
+    return cuda_status(launch_gather_quant_fp8(Tk, d.k, d.H, d.T, sorted, xn_moe,
+                                               at<uint8_t>(ws, L.aperm), at<float>(ws, L.sx),
+                                               s, pdl));
+  return cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe,
+                                        at<uint16_t>(ws, L.aperm), d.int8 != 0, s, pdl));
 }
 
 // The counters in the workspace start at zero (the caller zeroes a new workspace once)
@@ -323,14 +348,17 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
   if (j.experts) {
     GemmProblem& a = gu.prob[np];
     a = GemmProblem{};
-    // int8 steps cover 128 K (a ragged last step reads zeros past K through the maps)
-    const int kw = d.int8 ? 128 : 64;
+    // int8 and fp8 steps cover 128 K (a ragged last step reads zeros past K through the
+    // maps)
+    const int kw = (d.int8 || d.fp8) ? 128 : 64;
     a.kind = 0; a.groups = d.E; a.offsets = j.offsets; a.n_tokens = static_cast<int>(Tk);
     a.k_steps = (d.H + kw - 1) / kw; a.m_tiles = d.I / 64; a.w_rows_per_group = 2 * d.I; a.nw = d.I;
     a.split = std::min(L.split_gu, a.k_steps); a.map = np; a.out = h; a.out_ld = d.I;
     a.wscale = j.s_gate_up;
     a.w8 = d.int8;
     a.f16 = d.int8;  // int8 codes become fp16 (exact); the gathered rows and h are fp16
+    a.fp8 = d.fp8;   // E4M3 weights times E4M3 token rows, each row with its scale
+    a.xscale = d.fp8 ? j.a_scales : nullptr;
     GemmProblem& b = dn.prob[np];
     b = GemmProblem{};
     b.kind = 1; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = static_cast<int>(Tk);
@@ -338,10 +366,16 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
     b.split = std::min(L.split_d, b.k_steps); b.map = np; b.out = j.y; b.out_type = kOutF16;
     b.out_ld = d.H;
     b.wscale = j.s_down; b.w8 = d.int8; b.f16 = d.int8;
-    if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, d.int8) ||
-        !encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, bbox_gu) ||
-        !encode_a(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128, d.int8) ||
-        !encode_bf16(&mdn.b[np], h, Tk, d.I, bbox_dn))
+    b.fp8 = d.fp8;
+    b.xscale = d.fp8 ? at<float>(ws, L.sh) : nullptr;
+    // 8-bit weights (int8, E4M3) are byte tiles of 128 K; E4M3 token rows likewise
+    const bool w1 = d.int8 || d.fp8;
+    if (!encode_gate_up(&mgu.a[np], j.w_gate_up, d.E, d.I, d.H, w1) ||
+        !(d.fp8 ? encode_i8(&mgu.b[np], j.a_rows, Tk, d.H, bbox_gu)
+                : encode_bf16(&mgu.b[np], j.a_rows, Tk, d.H, bbox_gu)) ||
+        !encode_a(&mdn.a[np], j.w_down, static_cast<int64_t>(d.E) * d.H, d.I, 128, w1) ||
+        !(d.fp8 ? encode_i8(&mdn.b[np], at<uint8_t>(ws, L.h8), Tk, d.I, bbox_dn)
+                : encode_bf16(&mdn.b[np], h, Tk, d.I, bbox_dn)))
       return MOE_ERR_CUDA;
     ++np;
   }
@@ -374,6 +408,12 @@ moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& 
   // (programmatic dependent launch)
   moe_status_t st = cuda_status(launch_grouped_gemm(L.bn, mgu, gu, grid, s, !first_kernel));
   if (st != MOE_OK) return st;
+  // fp8 experts: h (bf16, sorted order) quantised per row for the down matmul
+  if (j.experts && d.fp8 &&
+      (st = cuda_status(launch_gather_quant_fp8(static_cast<int>(Tk), 1, d.I, static_cast<int>(Tk),
+                                                nullptr, h, at<uint8_t>(ws, L.h8),
+                                                at<float>(ws, L.sh), s, true))) != MOE_OK)
+    return st;
   if (!mark(ev, 4, s)) return MOE_ERR_CUDA;
   st = cuda_status(launch_grouped_gemm(L.bn, mdn, dn, grid, s, true));
   if (st != MOE_OK) return st;
@@ -427,10 +467,10 @@ moe_status_t run_router(const Dims& d, const Layout& L, void* ws, const RouteJob
                                       s));
 }
 
-bool w_ok(const moe_expert_weights_t* w, bool int8) {
+bool w_ok(const moe_expert_weights_t* w, bool scaled) {
   if (w == nullptr || w->w_gate_up == nullptr || w->w_down == nullptr) return false;
   if (!aligned16(w->w_gate_up) || !aligned16(w->w_down)) return false;
-  if (int8) return w->s_gate_up != nullptr && w->s_down != nullptr;
+  if (scaled) return w->s_gate_up != nullptr && w->s_down != nullptr;
   return w->s_gate_up == nullptr && w->s_down == nullptr;
 }
 
@@ -440,7 +480,7 @@ bool w_ok(const moe_expert_weights_t* w, bool int8) {
 
 extern "C" {
 
-int32_t moe_abi_version(void) { return 4; }
+int32_t moe_abi_version(void) { return 5; }
 
 int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T) {
   Dims d;
@@ -452,6 +492,7 @@ int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T) {
   const bool fused_sort = !tc && permute_blocks(Tk) == 0;
   int n = tc ? 2 : 1;                                     // router (prep + router)
   if (!fused_sort) n += permute_blocks(Tk) == 0 ? 1 : 3;  // permutation
+  if (d.fp8) n += 1;                                      // h quantised for the down matmul
   return n + 4;                                           // gather, gate_up, down, combine
 }
 
@@ -525,19 +566,16 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   for (const void* p : {(const void*)xn_moe, (const void*)topk_w, (const void*)expert_offsets,
                         (const void*)sorted_src, (const void*)inv_pos, (const void*)moe_out})
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (!w_ok(experts, d.int8)) return MOE_ERR_INVALID_ARG;
+  if (!w_ok(experts, d.int8 || d.fp8)) return MOE_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int Tk = d.T * d.k;
-  uint16_t* aperm = at<uint16_t>(ws, L.aperm);
   uint16_t* y = at<uint16_t>(ws, L.y);
-  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted_src, xn_moe, aperm,
-                                           d.int8 != 0, s))) != MOE_OK)
-    return st;
+  if ((st = gather_tokens(d, L, ws, sorted_src, xn_moe, s, false)) != MOE_OK) return st;
   GemmJob j{};
   j.experts = true;
-  j.a_rows = aperm;
+  j.a_rows = at<uint8_t>(ws, L.aperm);
+  j.a_scales = at<float>(ws, L.sx);
   j.w_gate_up = experts->w_gate_up;
   j.w_down = experts->w_down;
   j.s_gate_up = experts->s_gate_up;
@@ -590,7 +628,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   for (const void* p : {(const void*)moe_out, (const void*)w->logit_bias,
                         (const void*)w->g_post_moe, (const void*)w->g_post_dense})
     if (p != nullptr && !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (!w_ok(&w->experts, d.int8)) return MOE_ERR_INVALID_ARG;
+  if (!w_ok(&w->experts, d.int8 || d.fp8)) return MOE_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -621,14 +659,12 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
                                        at<int>(ws, L.bbase), s, true))) != MOE_OK)
     return st;
   if (!mark(ev, 2, s)) return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe, aperm, d.int8 != 0,
-                                           s, true))) !=
-      MOE_OK)
-    return st;
+  if ((st = gather_tokens(d, L, ws, sorted, xn_moe, s, true)) != MOE_OK) return st;
   if (!mark(ev, 3, s)) return MOE_ERR_CUDA;
   GemmJob j{};
   j.experts = true;
   j.a_rows = aperm;
+  j.a_scales = at<float>(ws, L.sx);
   j.w_gate_up = w->experts.w_gate_up;
   j.w_down = w->experts.w_down;
   j.s_gate_up = w->experts.s_gate_up;
@@ -661,6 +697,17 @@ moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, 
     return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(scales) & 3u) != 0) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_quantize_int8(w, rows, cols, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_quantize_fp8(const moe_bf16_t* w, int64_t rows, int32_t cols, uint8_t* q,
+                              float* scales, void* stream) {
+  if (rows < 0 || cols < 8 || cols > 65536 || cols % 8) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (rows > (int64_t(1) << 34)) return MOE_ERR_UNSUPPORTED;
+  if (w == nullptr || q == nullptr || scales == nullptr || !aligned16(w) || !aligned16(q))
+    return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scales) & 3u) != 0) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_fp8(w, rows, cols, q, scales, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_wait_selftest(void* ws, size_t ws_bytes, uint64_t timeout_ns, void* stream) {

@@ -174,6 +174,71 @@ __global__ void __launch_bounds__(32 * kGatherWarps) gather_rows_kernel(
   }
 }
 
+// The fp8 variant's activations (dynamic per-token E4M3 quantisation, the "Gemma 4 26B-A4B
+// IT" recipe page, "Quantized Variants"): row q of the matmul operand is source row r(q)
+// quantised with its own scale s = max|row| / 448 (fp32; 1 for an all-zero row), codes
+// E4M3(v / s) rounded to nearest even, saturating.  One warp per row, two passes over the
+// row (the second from cache).  r(q) = sorted_src[q] / k (the gather of the routed rows),
+// or q with sorted_src NULL (h, already in sorted order).
+__global__ void __launch_bounds__(32 * kGatherWarps) gather_quant_fp8_kernel(
+    int n, int k, int cols, int T, const int* __restrict__ sorted_src,
+    const uint16_t* __restrict__ src, uint8_t* __restrict__ dst, float* __restrict__ scales) {
+  const int nch = cols >> 3;
+  pdl_wait();
+  pdl_trigger();
+  const int q = static_cast<int>(blockIdx.x) * kGatherWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (q >= n) return;
+  int t = q;
+  if (sorted_src != nullptr) {
+    const int p = sorted_src[q];
+    t = (p >= 0 && p < n) ? p / k : -1;
+  }
+  const bool ok = t >= 0 && t < T;
+  const uint4* s = reinterpret_cast<const uint4*>(src + static_cast<size_t>(ok ? t : 0) * cols);
+  float amax = 0.f;
+  if (ok) {
+    for (int c0 = lane; c0 < nch; c0 += 32 * 4) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u;
+        v[u] = c < nch ? __ldg(s + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float f[8];
+        unpack8(v[u], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      }
+    }
+  }
+  amax = warp_max(amax);
+  const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  if (lane == 0) scales[q] = sc;
+  uint2* d = reinterpret_cast<uint2*>(dst + static_cast<size_t>(q) * cols);
+  for (int c = lane; c < nch; c += 32) {
+    uint32_t packed[2] = {0u, 0u};
+    if (ok) {
+      float f[8];
+      unpack8(__ldg(s + c), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        packed[i >> 2] |= static_cast<uint32_t>(e4m3_bits_sat(__fdiv_rn(f[i], sc))) << (8 * (i & 3));
+    }
+    d[c] = make_uint2(packed[0], packed[1]);
+  }
+}
+
+cudaError_t launch_gather_quant_fp8(int n, int k, int cols, int T, const int* sorted_src,
+                                    const uint16_t* src, uint8_t* dst, float* scales,
+                                    cudaStream_t s, bool pdl) {
+  const int blocks = (n + kGatherWarps - 1) / kGatherWarps;
+  return launch_k(gather_quant_fp8_kernel, dim3(static_cast<unsigned>(blocks)),
+                  dim3(32 * kGatherWarps), 0, s, pdl, n, k, cols, T, sorted_src, src, dst, scales);
+}
+
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
                                const uint16_t* src, uint16_t* dst, bool to_f16, cudaStream_t s,
                                bool pdl) {

@@ -304,17 +304,18 @@ def e4m3_round(v) -> np.ndarray:
     _, ex = np.frexp(np.where(a > 0, a, 1.0))       # a = f * 2^ex, f in [0.5, 1)
     spacing = np.where(a < 2.0 ** -6, 2.0 ** -9, 2.0 ** (ex - 1 - 3.0))
     q = np.rint(a / spacing) * spacing
-    return np.sign(v) * np.minimum(q, E4M3_MAX)
+    return np.copysign(np.minimum(q, E4M3_MAX), v)   # keeps the sign of a rounded zero
 
 
 def e4m3_encode(v) -> np.ndarray:
-    """Code (uint8) of E4M3 grid values (already rounded); -0 encodes as +0."""
+    """Code (uint8) of E4M3 grid values (already rounded).  The format has a signed zero:
+    a negative value that rounded to zero is -0, code 0x80."""
     tab = e4m3_decode_table()
     pos = tab[:127]                                   # codes 0..126: 0 .. 448, increasing
     v = np.asarray(v, dtype=np.float64)
     idx = np.searchsorted(pos, np.abs(v))
     assert np.all(pos[np.minimum(idx, 126)] == np.abs(v)), "not an E4M3 value"
-    return (idx + np.where(v < 0, 128, 0)).astype(np.uint8)
+    return (idx + np.where(np.signbit(v), 128, 0)).astype(np.uint8)
 
 
 def quantize_fp8_rows(v32: np.ndarray):

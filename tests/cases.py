@@ -23,6 +23,12 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 COS_MIN = 0.9999
 FRAC_BF16 = 2e-2
 FRAC_INT8 = 4e-2
+# fp8 experts: the oracle takes every E4M3 rounding decision from the same bf16 activation
+# the kernels quantise (xn_moe, h) in the same fp32 arithmetic, so the two sides differ by
+# fp32-vs-fp64 accumulation and the rare code that this moves across a rounding boundary
+# (one E4M3 step, 2^-3 relative, on one element of a 704- or 2816-long dot product): the
+# int8 bar holds with margin.
+FRAC_FP8 = 4e-2
 MIN_GAP = 1e-3
 
 

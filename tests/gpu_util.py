@@ -22,8 +22,8 @@ def bf16_np(t: torch.Tensor) -> np.ndarray:
     return oracle.bf16(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
 
 
-def config(shape: synth.Shape, int8: bool = False) -> mf.Config:
-    return mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps, int8)
+def config(shape: synth.Shape, int8: bool = False, fp8: bool = False) -> mf.Config:
+    return mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps, int8, fp8)
 
 
 _DEV_CACHE = cases._Lru(3)
@@ -120,4 +120,33 @@ def int8_experts(case: cases.Case):
                         q_down=host["w_down"], s_down=host["s_down"])
     res = (dev, ex, same)
     _INT8_CACHE.put(key, (case.p, res))
+    return res
+
+
+_FP8_CACHE = cases._Lru(2)
+
+
+def fp8_experts(case: cases.Case):
+    """Quantise the case's expert weights to E4M3 on the GPU (moe_quantize_fp8) and with
+    the oracle; return (device tensors, oracle.Experts in fp8 mode built from the oracle's
+    own codes and scales, whether the two quantisations are identical)."""
+    key = id(case.p)
+    if key in _FP8_CACHE and _FP8_CACHE[key][0] is case.p:
+        return _FP8_CACHE[key][1]
+    dev, host, same = {}, {}, True
+    for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down")):
+        w = case.p[name]
+        rows, cols = int(np.prod(w.shape[:-1])), w.shape[-1]
+        q = torch.empty(w.shape, dtype=torch.uint8, device="cuda")
+        s = torch.empty(w.shape[:-1], dtype=torch.float32, device="cuda")
+        mf.moe_quantize_fp8(to_dev(w).view(rows, cols), q.view(rows, cols), s.view(rows))
+        qo, so = oracle.quantize_fp8_per_channel(w)
+        same = same and np.array_equal(q.cpu().numpy(), qo) and \
+            np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+        dev[name], dev[sname] = q, s
+        host[name], host[sname] = qo, so
+    ex = oracle.Experts(q_gate_up=host["w_gate_up"], s_gate_up=host["s_gate_up"],
+                        q_down=host["w_down"], s_down=host["s_down"], fp8=True)
+    res = (dev, ex, same)
+    _FP8_CACHE.put(key, (case.p, res))
     return res

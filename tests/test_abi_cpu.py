@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 4
+    assert lib.moe_abi_version() == 5
     for s in range(6):
         assert mf.status_string(s)
     assert mf.status_string(99) == "unknown status"
@@ -74,6 +74,9 @@ def test_block_launch_count(lib):
         assert mf.moe_block_launch_count(CFG, T) == n, T
     for T, n in ((8, 5), (512, 7), (513, 9)):  # top-4: T*k = 2048 at T = 512
         assert mf.moe_block_launch_count(TINY, T) == n, T
+    FP8 = mf.Config(**{**CFG.__dict__, "fp8": True})  # + the quantisation of h
+    for T, n in ((8, 6), (2048, 10)):
+        assert mf.moe_block_launch_count(FP8, T) == n, T
     assert mf.moe_block_launch_count(CFG, 0) == 0
     assert mf.moe_block_launch_count(CFG, -1) == -1
     assert mf.moe_block_launch_count(mf.Config(**{**CFG.__dict__, "top_k": 17}), 8) == -1
@@ -143,6 +146,15 @@ def test_every_entry_point_validates(lib):
     assert lib.moe_quantize_int8(FAKE, 4, 12, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG
     assert lib.moe_quantize_int8(None, 4, 16, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG
     assert lib.moe_quantize_int8(FAKE, 0, 16, FAKE, FAKE, None) == mf.MOE_OK
+    assert lib.moe_quantize_fp8(FAKE, 4, 12, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_fp8(FAKE, 4, 16, FAKE, None, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_fp8(FAKE, 0, 16, FAKE, FAKE, None) == mf.MOE_OK
+    # fp8 experts need their row scales (like int8), and the config accepts the type
+    c8 = ctypes.byref(mf.Config(**{**CFG.__dict__, "fp8": True}).c())
+    assert lib.moe_ffn_forward(c8, 8, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(ew), FAKE,
+                               FAKE, mf.workspace_size(mf.Config(**{**CFG.__dict__, "fp8": True}), 8),
+                               None) == mf.MOE_ERR_INVALID_ARG
+    assert mf.workspace_size(mf.Config(**{**CFG.__dict__, "fp8": True}), 8) > 0
     assert lib.moe_check_device_status(None, 256, None) == mf.MOE_ERR_WORKSPACE
 
 

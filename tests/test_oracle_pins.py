@@ -350,8 +350,16 @@ def test_e4m3_rounding_matches_torch_and_closed_forms():
     mids = (pos[:-1] + pos[1:]) / 2                                # every exact tie
     v = np.concatenate([RNG.uniform(-440, 440, 4000), RNG.uniform(-0.05, 0.05, 4000),
                         mids, -mids, [0.0]]).astype(np.float32)
-    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).to(torch.float64).numpy()
-    assert np.array_equal(oracle.e4m3_round(v.astype(np.float64)), ref)
+    ref8 = torch.from_numpy(v).to(torch.float8_e4m3fn)
+    ref = ref8.to(torch.float64).numpy()
+    got = oracle.e4m3_round(v.astype(np.float64))
+    assert np.array_equal(got, ref)
+    # codes too, which also fixes the sign of values that round to zero (signed zero)
+    assert np.array_equal(oracle.e4m3_encode(got), ref8.view(torch.uint8).numpy())
+    tiny = np.array([-1e-9, -2.0 ** -11, 2.0 ** -11, -0.0, 0.0], dtype=np.float32)
+    t8 = torch.from_numpy(tiny).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert t8.tolist() == [0x80, 0x80, 0x00, 0x80, 0x00]
+    assert oracle.e4m3_encode(oracle.e4m3_round(tiny.astype(np.float64))).tolist() == t8.tolist()
     got = oracle.e4m3_round([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 449.0, 1e6, -1e6])
     assert got.tolist() == [1.0, 1.25, 0.0, 2.0 ** -8, 448.0, 448.0, -448.0]
     assert oracle.e4m3_encode(got[:4]).tolist() == [0x38, 0x3A, 0x00, 0x02]
