@@ -53,6 +53,14 @@ WORKLOADS = {
     "int8_T1024": dict(shape=synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112), layers=8,
                        int8=True, steps=500, warmup=20,
                        name="same layer with per-channel int8 experts, T=1024"),
+    "fp8_T8": dict(shape=synth.DECODE, layers=8, fp8=True, steps=3000, warmup=100,
+                   name="same layer with E4M3 experts and per-token E4M3 activations, T=8"),
+    "fp8_T64": dict(shape=synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                    fp8=True, steps=2000, warmup=100,
+                    name="same layer with E4M3 experts and per-token E4M3 activations, T=64"),
+    "fp8_T1024": dict(shape=synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                      fp8=True, steps=500, warmup=20,
+                      name="same layer with E4M3 experts and per-token E4M3 activations, T=1024"),
     "stack": dict(shape=synth.Shape(T=synth.STACK_T, H=2816, E=128, k=8, I=704, D=2112),
                   layers=synth.STACK_LAYERS, chain=True, steps=3, warmup=1,
                   name="stack of 30 distinct MoE-FFN layers, residual-chained, T=16384 (one 16K chunk)"),
@@ -165,9 +173,10 @@ class Clocks:
 def algorithmic(shape, used_experts: int, int8: bool = False):
     """Bytes that must move and FLOPs that must run for one block call.
 
-    Bytes: the weights of the experts that received a token (int8 codes plus fp32 row
-    scales for int8 experts), the dense MLP, the router and the norm vectors, plus x in
-    and out.  Intermediates are implementation traffic.
+    Bytes: the weights of the experts that received a token (int8 or E4M3 codes plus
+    fp32 row scales for 8-bit experts: `int8` means any 1-byte weight here), the dense
+    MLP, the router and the norm vectors, plus x in and out.  Intermediates are
+    implementation traffic.
     """
     H, E, k, I, D, T = shape.H, shape.E, shape.k, shape.I, shape.D, shape.T
     wb = 1 if int8 else 2
@@ -192,13 +201,15 @@ def _make_layers(mf, cfg, shape, wl, n, seed, device):
             with open(ZIPF_ALPHA_FILE) as f:
                 alpha = float(json.load(f)["alpha"])
             t["logit_bias"] = torch.from_numpy(synth.zipf_bias(seed, shape.E, alpha)).to(device)
-        if wl.get("int8"):
+        if wl.get("int8") or wl.get("fp8"):
             for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down")):
                 w = t.pop(name)
                 cols = w.shape[-1]
-                q = torch.empty(w.shape, dtype=torch.int8, device=device)
+                fp8 = bool(wl.get("fp8"))
+                q = torch.empty(w.shape, dtype=torch.uint8 if fp8 else torch.int8, device=device)
                 sc = torch.empty(w.shape[:-1], dtype=torch.float32, device=device)
-                mf.moe_quantize_int8(w.view(-1, cols), q.view(-1, cols), sc.view(-1))
+                quant = mf.moe_quantize_fp8 if fp8 else mf.moe_quantize_int8
+                quant(w.view(-1, cols), q.view(-1, cols), sc.view(-1))
                 t[name], t[sname] = q, sc
                 del w
         layers.append(t)
@@ -212,8 +223,9 @@ def run_ours(args, wl, rank, world, device):
     shape = wl["shape"]
     T = shape.T
     int8 = bool(wl.get("int8"))
+    fp8 = bool(wl.get("fp8"))
     chain = bool(wl.get("chain"))
-    cfg = mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps, int8)
+    cfg = mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps, int8, fp8)
     seed = 1234 + 7919 * rank
     nl = args.layers or wl["layers"]
     layers, alpha = _make_layers(mf, cfg, shape, wl, nl, seed, device)
@@ -333,7 +345,10 @@ def run_ours(args, wl, rank, world, device):
     pk = peaks()
     long_step = t_max / K > 10.0  # ms: a kernel inside a long step meets the sustained peak
     tc_peak = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
-    alg = [algorithmic(shape, u, int8) for u in used]
+    # an E4M3 contraction's peak: the measured bf16 peak times the nominal fp8:bf16 ratio
+    # (4.5 : 2.25 PFLOP/s dense); only the routed experts' matmuls run in fp8, so the
+    # gate_up launch's peak is the FLOP-weighted mix
+    alg = [algorithmic(shape, u, int8 or fp8) for u in used]
     gu_ms = sum(stages["gate_up"])
     gu_bytes = sum(a["gate_up_bytes"] for a in alg)
     gu_flops = sum(a["gate_up_flops"] for a in alg)
@@ -344,7 +359,12 @@ def run_ours(args, wl, rank, world, device):
     ms_step = t_max / K
     gu_t_hbm = gu_bytes / (pk["hbm_gbs"] * 1e9)
     gu_t_tc = gu_flops / (tc_peak * 1e12)
-    kern = "grouped_gemm_kernel (gate_up launch" + (", int8 converter variant)" if int8 else ")")
+    kern = "grouped_gemm_kernel (gate_up launch" + (", int8 converter variant)" if int8 else
+                                                      ", E4M3 experts)" if fp8 else ")")
+    if fp8:
+        f_exp = 2 * shape.k * 2 * shape.I * shape.H
+        f_den = 2 * 2 * shape.D * shape.H
+        tc_peak = round(tc_peak * (f_exp + f_den) / (f_exp / 2.0 + f_den), 1)
     if gu_t_tc > gu_t_hbm:
         roof = {"bound": "tensor", "achieved": round(gu_tf, 2), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(gu_tf / tc_peak, 4), "traffic": None,
@@ -352,7 +372,7 @@ def run_ours(args, wl, rank, world, device):
                 "peak_source": ("bf16_tflops_sustained" if long_step else "bf16_tflops")
                                + f" of {pk['source']} peaks"}
     else:
-        summary = {(8, False): "grouped_gemm_gate_up_decode_T8.md"}.get((T, int8))
+        summary = {(8, False): "grouped_gemm_gate_up_decode_T8.md"}.get((T, int8 or fp8))
         roof = {"bound": "hbm", "achieved": round(gu_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gu_gbs / pk["hbm_gbs"], 4),
                 "traffic": ncu_traffic(summary) if summary else None,
@@ -368,16 +388,19 @@ def run_ours(args, wl, rank, world, device):
     res = {
         "metric": METRIC, "value": round(world * T * K / (t_max * 1e-3), 1), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 (experts), bf16 (dense)" if fp8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the layer's shape)",
         "config": {"workload": wl["name"], "T": T, "H": shape.H, "E": shape.E, "top_k": shape.k,
                    "expert_inter": shape.I, "dense_inter": shape.D,
-                   "expert_weights": "int8 per-channel" if int8 else "bf16",
+                   "expert_weights": ("int8 per-channel" if int8 else
+                                      "E4M3 per-channel, E4M3 per-token activations" if fp8
+                                      else "bf16"),
                    "router_bias": ("zipf s=1.1, alpha=%.5f" % alpha) if wl.get("zipf") else "none",
                    "layers": nl, "chained": chain,
                    "l2": ("steps rotate over %d distinct layers (%.1f GB of weights) and distinct "
                           "inputs; no step's weights are L2-resident" %
-                          (nl, nl * 3 * shape.E * shape.I * shape.H * (1 if int8 else 2) / 1e9)),
+                          (nl, nl * 3 * shape.E * shape.I * shape.H * (1 if int8 or fp8 else 2) / 1e9)),
                    "parallelism": f"dp{world} (replicas, no collective)"},
         "roofline": roof,
         "block_roofline": block_roof,
@@ -467,6 +490,10 @@ def run_reference(args, wl, rank, world):
         qg, sg = oracle.quantize_int8_per_channel(p["w_gate_up"])
         qd, sd = oracle.quantize_int8_per_channel(p["w_down"])
         ex = oracle.Experts(q_gate_up=qg, s_gate_up=sg, q_down=qd, s_down=sd)
+    elif wl.get("fp8"):
+        qg, sg = oracle.quantize_fp8_per_channel(p["w_gate_up"])
+        qd, sd = oracle.quantize_fp8_per_channel(p["w_down"])
+        ex = oracle.Experts(q_gate_up=qg, s_gate_up=sg, q_down=qd, s_down=sd, fp8=True)
     else:
         ex = oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
     per_step = wl["layers"] if wl.get("chain") else 1

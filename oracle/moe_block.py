@@ -31,7 +31,7 @@ Readings taken where the pages leave a step open (each also listed in the design
   R8  gate_up rows 0..I-1 are the gate projection and rows I..2I-1 the up projection.
   R9  int8 experts: per output row s = max|w| / 127 (fp32), q = round-half-even(w / s)
       clamped to [-127, 127]; an all-zero row takes s = 1.
-  R10 fp8 experts ([P6]): E4M3 as the OCP 8-bit format defines it (1 sign, 4 exponent
+  R17 fp8 experts ([P6]): E4M3 as the OCP 8-bit format defines it (1 sign, 4 exponent
       bits of bias 7, 3 mantissa bits, subnormals, no infinities, largest finite 448).
       Weights per output row and activations per token row (the rows entering each
       expert matmul: the routed token's xn_moe, and h) take s = max|v| / 448 (fp32, an
@@ -176,7 +176,7 @@ class Experts:
 
 
 def expert_mlp(experts, u: np.ndarray, e: int) -> np.ndarray:
-    """Expert e's gated MLP on rows u; fp8 experts run it on quantised activations (R10).
+    """Expert e's gated MLP on rows u; fp8 experts run it on quantised activations (R17).
     `experts` is anything with gate_up(e) and down(e) (and optionally fp8)."""
     f = gated_mlp_fp8 if getattr(experts, "fp8", False) else gated_mlp
     return f(u, experts.gate_up(e), experts.down(e))
@@ -281,7 +281,7 @@ E4M3_MAX = 448.0
 
 
 def e4m3_decode_table() -> np.ndarray:
-    """Value of every E4M3 code 0..255, from the format's definition (R10): sign bit 7,
+    """Value of every E4M3 code 0..255, from the format's definition (R17): sign bit 7,
     exponent bits 6..3 (bias 7), mantissa bits 2..0; exponent 0 is subnormal
     (m/8 * 2^-6); code S.1111.111 is NaN."""
     c = np.arange(256)
@@ -294,7 +294,7 @@ def e4m3_decode_table() -> np.ndarray:
 
 
 def e4m3_round(v) -> np.ndarray:
-    """Round to the nearest E4M3 value, ties to even, saturating at +-448 (R10).
+    """Round to the nearest E4M3 value, ties to even, saturating at +-448 (R17).
 
     Normal binade [2^e, 2^(e+1)) has spacing 2^(e-3); below 2^-6 the spacing is 2^-9
     (subnormals).  np.rint rounds half to even on the integer multiple of the spacing,
@@ -319,7 +319,7 @@ def e4m3_encode(v) -> np.ndarray:
 
 
 def quantize_fp8_rows(v32: np.ndarray):
-    """Per-row E4M3 quantisation (R10) of fp32 values (rows = all axes but the last):
+    """Per-row E4M3 quantisation (R17) of fp32 values (rows = all axes but the last):
     s = max|v| / 448 in fp32 (1 for an all-zero row), codes of e4m3(fp32(v / s)).
     Returns (codes uint8, s fp32)."""
     v = np.asarray(v32, dtype=np.float32)
@@ -330,7 +330,7 @@ def quantize_fp8_rows(v32: np.ndarray):
 
 
 def quantize_fp8_per_channel(w_bits: np.ndarray):
-    """Per-output-row E4M3 quantisation of bf16 weights ([P6]; R10)."""
+    """Per-output-row E4M3 quantisation of bf16 weights ([P6]; R17)."""
     u = np.asarray(w_bits, dtype=np.uint16)
     return quantize_fp8_rows((u.astype(np.uint32) << np.uint32(16)).view(np.float32))
 
@@ -351,14 +351,14 @@ def bf16_round(v) -> np.ndarray:
 
 
 def fp8_activation(v) -> np.ndarray:
-    """An expert matmul's activation rows as the fp8 path uses them (R10): stored as
+    """An expert matmul's activation rows as the fp8 path uses them (R17): stored as
     bf16, quantised per row to E4M3, dequantised (float64)."""
     q, s = quantize_fp8_rows(bf16_round(v).astype(np.float32))
     return dequantize_fp8(q, s)
 
 
 def gated_mlp_fp8(u: np.ndarray, w_gate_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
-    """gated_mlp with both expert matmuls on fp8 activations (R10): the input rows and h
+    """gated_mlp with both expert matmuls on fp8 activations (R17): the input rows and h
     are quantised per row; the weights arrive already dequantised."""
     I = w_gate_up.shape[0] // 2
     uq = fp8_activation(u)

@@ -328,7 +328,7 @@ def test_int8_quantiser_pins():
 # ------------------------------------------------------------------ fp8 (E4M3)
 
 def test_e4m3_decode_table_matches_torch():
-    """R10: the format written out (sign, 4 exponent bits of bias 7, 3 mantissa bits,
+    """R17: the format written out (sign, 4 exponent bits of bias 7, 3 mantissa bits,
     subnormals, NaN at S.1111.111) equals the library's float8_e4m3fn decoding."""
     ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
     tab = oracle.e4m3_decode_table()
@@ -366,7 +366,7 @@ def test_e4m3_rounding_matches_torch_and_closed_forms():
 
 
 def test_fp8_quantiser_pins():
-    """R10: s = max|w| / 448; each value lands within half an E4M3 step (relative 2^-4,
+    """R17: s = max|w| / 448; each value lands within half an E4M3 step (relative 2^-4,
     or 2^-10 s absolute below the normal range) of w; the largest |w| of a row becomes
     +-448 exactly; an all-zero row takes s = 1 and code 0."""
     w = synth.normal_bf16(5, (98,), (6, 40), 0.02)
@@ -385,7 +385,7 @@ def test_fp8_quantiser_pins():
 
 
 def test_fp8_activation_scale_is_per_token():
-    """R10 and [P6] (dynamic per-token activation scales): the all-experts-dense form runs
+    """R17 and [P6] (dynamic per-token activation scales): the all-experts-dense form runs
     every token through every expert, the sparse form only the routed rows; the two agree
     only if a token's quantisation does not depend on which other rows share the matmul."""
     E, k, H, I, T = 6, 2, 32, 16, 9
