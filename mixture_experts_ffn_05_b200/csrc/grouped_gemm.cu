@@ -31,6 +31,8 @@
 // and the per-row scale multiplies the fp32 accumulator in the epilogue (it factors out
 // of the K sum, so this is exact).  Every wait is bounded; a wait that runs out records
 // a timeout in the status word and the CTA winds down.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -420,6 +422,11 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         // the other CTA the second half
         const int half = ((pc.n_valid + 15) & ~15) >> 1;
         const int brow = pc.b_row0 + pc.n * BN + (PAIR ? static_cast<int>(rank) * half : 0);
+        // a step covers 64 K (bf16), 128 K of int8 codes (two fp16 B sub-tiles) or 128 K of
+        // E4M3 codes (one B tile of 128-byte rows); the A tile is 16 KB in every case
+        const bool i8p = W8 && pr.w8;
+        const int kw = (i8p || pr.fp8) ? 128 : 64;
+        const int nb = i8p ? 2 : 1;
         for (int ks = pc.k0; ks < pc.k1; ++ks) {
           if (!waited && steps == C::kStages) release_b();  // the ring is full
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
@@ -428,11 +435,6 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
           }
           ++steps;
           uint8_t* sa = smem + stage * C::kStage;
-          // a step covers 64 K (bf16), 128 K of int8 codes (two fp16 B sub-tiles) or 128 K
-          // of E4M3 codes (one B tile of 128-byte rows); the A tile is 16 KB in every case
-          const bool i8p = W8 && pr.w8;
-          const int kw = (i8p || pr.fp8) ? 128 : 64;
-          const int nb = i8p ? 2 : 1;
           if (PAIR) {
             // both CTAs' bytes land on the leader's barrier; the leader expects them all
             const uint32_t fb = cluster_addr(&full[stage], 0);
@@ -505,61 +507,74 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         const uint32_t d = tmem_base + static_cast<uint32_t>(ab * BN);
         // int8 problems (W8): A comes from the TMEM buffer the converters filled
         const bool a_tmem = W8 && P.prob[pc.p].w8;
-        for (int ks = pc.k0; ks < pc.k1; ++ks) {
-          if (!mbar_wait(&full[stage], phase, tmo, abort_flag) ||
-              (a_tmem && !mbar_wait(&conv_full[cs], cph, tmo, abort_flag))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * C::kStage);
-          if (a_tmem) {
-            // a 128-K step: two 64-wide sub-steps; A sub-step `sub`, K slice kk sits in
-            // TMEM columns [32 sub + 8 kk, +8) of the buffer
-            const uint32_t ta = tmem_base + static_cast<uint32_t>(C::kTaCol + cs * 64);
-            for (int sub = 0; sub < 2; ++sub) {
-              const uint64_t bd = sdesc_k_sw128(sa + C::kABytes + sub * C::kBBytes);
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                umma_ta(d, ta + 32 * sub + 8 * kk, bd + 2 * kk, idesc,
-                        (ks > pc.k0 || sub > 0 || kk > 0) ? 1u : 0u);
+        // The k-step loop exists once per operand kind (bf16/fp16 from shared memory, E4M3
+        // from shared memory, int8-as-fp16 from TMEM), chosen per piece: this thread issues
+        // every MMA of the CTA, and a branch per MMA measured 25% at decode.
+        auto k_loop = [&](auto kind_tag) {
+          constexpr int kKind = decltype(kind_tag)::value;  // 0 f16 kinds, 1 E4M3, 2 TMEM A
+          for (int ks = pc.k0; ks < pc.k1; ++ks) {
+            if (!mbar_wait(&full[stage], phase, tmo, abort_flag) ||
+                (kKind == 2 && !mbar_wait(&conv_full[cs], cph, tmo, abort_flag))) {
+              ok = false;
+              return;
             }
-            umma_commit(&conv_empty[cs]);
-            if (++cs == C::kConv) {
-              cs = 0;
-              cph ^= 1u;
-            }
-          } else {
-            const uint64_t ad = sdesc_k_sw128(sa);
-            const uint64_t bd = sdesc_k_sw128(sa + C::kABytes);
-            // four MMAs per 128-byte row: K = 16 bf16 or K = 32 E4M3 each
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + stage * C::kStage);
+            if constexpr (kKind == 2) {
+              // a 128-K step: two 64-wide sub-steps; A sub-step `sub`, K slice kk sits in
+              // TMEM columns [32 sub + 8 kk, +8) of the buffer
+              const uint32_t ta = tmem_base + static_cast<uint32_t>(C::kTaCol + cs * 64);
+              for (int sub = 0; sub < 2; ++sub) {
+                const uint64_t bd = sdesc_k_sw128(sa + C::kABytes + sub * C::kBBytes);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (ks > pc.k0 || kk > 0) ? 1u : 0u;
-              if (f8) {
-                if (PAIR)
-                  umma_f8_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
-                else
-                  umma_f8(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
-              } else if (PAIR) {
-                umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
-              } else {
-                umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+                for (int kk = 0; kk < 4; ++kk)
+                  umma_ta(d, ta + 32 * sub + 8 * kk, bd + 2 * kk, idesc,
+                          (ks > pc.k0 || sub > 0 || kk > 0) ? 1u : 0u);
+              }
+              umma_commit(&conv_empty[cs]);
+              if (++cs == C::kConv) {
+                cs = 0;
+                cph ^= 1u;
+              }
+            } else {
+              const uint64_t ad = sdesc_k_sw128(sa);
+              const uint64_t bd = sdesc_k_sw128(sa + C::kABytes);
+              // four MMAs per 128-byte row: K = 16 bf16 or K = 32 E4M3 each
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (ks > pc.k0 || kk > 0) ? 1u : 0u;
+                if constexpr (kKind == 1) {
+                  if (PAIR)
+                    umma_f8_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+                  else
+                    umma_f8(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+                } else {
+                  if (PAIR)
+                    umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+                  else
+                    umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, acc);
+                }
               }
             }
+            if (PAIR) {
+              umma_commit_pair(smem_u32(&empty[stage]));
+              umma_commit_pair(peer_empty0 + stage * 8);
+            } else {
+              umma_commit(&empty[stage]);
+            }
+            issued = true;
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          if (PAIR) {
-            umma_commit_pair(smem_u32(&empty[stage]));
-            umma_commit_pair(peer_empty0 + stage * 8);
-          } else {
-            umma_commit(&empty[stage]);
-          }
-          issued = true;
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
+        };
+        if (W8 && a_tmem)
+          k_loop(std::integral_constant<int, 2>{});
+        else if (f8)
+          k_loop(std::integral_constant<int, 1>{});
+        else
+          k_loop(std::integral_constant<int, 0>{});
         if (!ok) break;
         if (PAIR) {
           umma_commit_pair(smem_u32(&acc_full[ab]));
