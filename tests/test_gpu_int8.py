@@ -22,7 +22,11 @@ SHAPES = {
     "int8_T1": synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112),
     "int8_T64": synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112),
     "int8_T1024": synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112),
+    # the interface limits: H = 6144, E = 256, k = 16, and I = D = 64, where a 128-K step
+    # of 8-bit weights is half past the end of K (zero-filled by the tensor maps)
+    "limits_T300": synth.Shape(T=300, H=6144, E=256, k=16, I=64, D=64),
 }
+ROUTER_STD = {"limits_T300": 0.3}  # wider router weights, so the gap filter finds rows
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -33,7 +37,7 @@ def _gpu():
 
 
 def _setup(name):
-    c = cases.make_case(SHAPES[name], seed=1234)
+    c = cases.make_case(SHAPES[name], seed=1234, router_std=ROUTER_STD.get(name))
     dev8, ex8, same = int8_experts(c)
     layer = dict(device_layer(c))
     layer.update(dev8)
