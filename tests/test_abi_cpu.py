@@ -163,3 +163,23 @@ def test_python_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(8, 512, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         mf.dense_mlp_forward(TINY, x, x, x, x, torch.zeros(16, dtype=torch.uint8))
+
+
+def test_python_binding_checks_expert_weight_types(lib):
+    """Each expert weight type takes its own element type (bf16, int8 codes, E4M3 codes
+    as uint8); a mismatch is refused before any pointer reaches the library."""
+    import torch
+    e16 = {"w_gate_up": torch.zeros(4, 2, dtype=torch.bfloat16),
+           "w_down": torch.zeros(4, 2, dtype=torch.bfloat16)}
+    e8 = {"w_gate_up": torch.zeros(4, 2, dtype=torch.int8),
+          "w_down": torch.zeros(4, 2, dtype=torch.int8)}
+    f8 = mf.Config(**{**TINY.__dict__, "fp8": True})
+    i8 = mf.Config(**{**TINY.__dict__, "int8": True})
+    for cfg, e in ((f8, e16), (f8, e8), (i8, e16), (TINY, e8)):
+        with pytest.raises(TypeError, match="must be"):
+            mf._experts(cfg, e)
+    # the right type passes the type check and then stops at the device check
+    u8 = {k: v.view(torch.uint8) for k, v in e8.items()}
+    with pytest.raises(ValueError, match="CUDA"):
+        mf._experts(f8, u8)
+    assert f8.c().expert_wdtype == mf.MOE_W_FP8 and i8.c().expert_wdtype == mf.MOE_W_INT8
