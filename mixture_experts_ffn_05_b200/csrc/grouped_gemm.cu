@@ -73,6 +73,12 @@ struct Cfg {
                                      : (BN <= 32 ? 8 : (BN <= 64 ? 7 : (BN <= 128 ? 6 : 4)));
   // W8: TMEM buffers for converted A tiles, 64 columns (128 K of fp16 pairs) each
   static constexpr int kConv = W8 ? 4 : 0;
+  // W8 with at least kConv ring stages: TMEM buffer j % kConv serves k-step j, and it is
+  // free once stage (j - kConv) % kStages has been released (its MMAs done), so the
+  // converters wait on that stage's empty barrier and the MMA warp commits once per
+  // k-step.  With fewer stages than buffers (BN = 256) a phase of that barrier could be
+  // passed twice before the wait, so that variant keeps a barrier of its own per buffer.
+  static constexpr bool kMergedRelease = W8 && kStages >= kConv;
   // TMEM accumulators: 4 for narrow tiles (the epilogue of a weight-streaming piece is
   // latency-bound and must not hold up the MMAs), 2 for wide ones (512 columns max, less
   // the converted A buffers of the W8 variant).
@@ -480,6 +486,8 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       uint32_t phase = 0;
       int cs = 0;
       uint32_t cph = 0;
+      uint32_t kj = 0;      // k-steps issued so far (kMergedRelease: buffer kj % kConv)
+      uint32_t cphm = 0;    // kMergedRelease: bit b = uses of buffer b so far, mod 2
       int ab = 0;
       uint32_t aph = 0;
       bool ok = true, issued = false;
@@ -512,9 +520,11 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
         // every MMA of the CTA, and a branch per MMA measured 25% at decode.
         auto k_loop = [&](auto kind_tag) {
           constexpr int kKind = decltype(kind_tag)::value;  // 0 f16 kinds, 1 E4M3, 2 TMEM A
-          for (int ks = pc.k0; ks < pc.k1; ++ks) {
+          for (int ks = pc.k0; ks < pc.k1; ++ks, ++kj) {
+            if (C::kMergedRelease) cs = static_cast<int>(kj % C::kConv);
+            const uint32_t cpar = C::kMergedRelease ? (cphm >> cs) & 1u : cph;
             if (!mbar_wait(&full[stage], phase, tmo, abort_flag) ||
-                (kKind == 2 && !mbar_wait(&conv_full[cs], cph, tmo, abort_flag))) {
+                (kKind == 2 && !mbar_wait(&conv_full[cs], cpar, tmo, abort_flag))) {
               ok = false;
               return;
             }
@@ -531,10 +541,14 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
                   umma_ta(d, ta + 32 * sub + 8 * kk, bd + 2 * kk, idesc,
                           (ks > pc.k0 || sub > 0 || kk > 0) ? 1u : 0u);
               }
-              umma_commit(&conv_empty[cs]);
-              if (++cs == C::kConv) {
-                cs = 0;
-                cph ^= 1u;
+              if (C::kMergedRelease) {
+                cphm ^= 1u << cs;  // the stage's release below also frees the buffer
+              } else {
+                umma_commit(&conv_empty[cs]);
+                if (++cs == C::kConv) {
+                  cs = 0;
+                  cph ^= 1u;
+                }
               }
             } else {
               const uint64_t ad = sdesc_k_sw128(sa);
@@ -609,6 +623,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
     uint32_t phase = 0;
     int cs = 0;
     uint32_t cph = 0;
+    uint32_t kj = 0;  // k-steps seen so far, in the MMA warp's order
     bool ok = true;
     int n_popped = 0;
     for (int piece = first_item; ok; piece += item_stride) {
@@ -626,13 +641,26 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
       const Piece pc = decode_piece<BN>(piece, P, pre, b0, ng, nent);
       const bool i8 = P.prob[pc.p].w8 != 0;
       const int q = warp & 3;  // TMEM lane quarter
-      for (int ks = pc.k0; ks < pc.k1; ++ks) {
+      for (int ks = pc.k0; ks < pc.k1; ++ks, ++kj) {
+        if (C::kMergedRelease) cs = static_cast<int>(kj % C::kConv);
         int good = 1;
-        if (lane == 0)
-          good = (mbar_wait(&full[stage], phase, tmo, abort_flag) &&
-                  (!i8 || mbar_wait(&conv_empty[cs], cph ^ 1u, tmo, abort_flag)))
-                     ? 1
-                     : 0;
+        if (lane == 0) {
+          bool free_buf = true;
+          if (i8) {
+            if (C::kMergedRelease) {
+              // the MMAs of k-step kj - kConv, the buffer's last user, are done once that
+              // step's stage has been released
+              if (kj >= static_cast<uint32_t>(C::kConv)) {
+                const uint32_t jp = kj - C::kConv;
+                free_buf = mbar_wait(&empty[jp % C::kStages], (jp / C::kStages) & 1u, tmo,
+                                     abort_flag);
+              }
+            } else {
+              free_buf = mbar_wait(&conv_empty[cs], cph ^ 1u, tmo, abort_flag);
+            }
+          }
+          good = (mbar_wait(&full[stage], phase, tmo, abort_flag) && free_buf) ? 1 : 0;
+        }
         good = __shfl_sync(0xffffffffu, good, 0);
         if (!good) {
           ok = false;
@@ -656,7 +684,7 @@ __global__ void __launch_bounds__((Cfg<BN, W8, PAIR>::kThreads), 1)
           stage = 0;
           phase ^= 1u;
         }
-        if (i8 && ++cs == C::kConv) {
+        if (!C::kMergedRelease && i8 && ++cs == C::kConv) {
           cs = 0;
           cph ^= 1u;
         }
