@@ -336,6 +336,9 @@ def test_e4m3_decode_table_matches_torch():
     ok = ~np.isnan(ref)
     assert np.array_equal(tab[ok], ref[ok])
     assert tab[0x7E] == 448.0 and tab[0x01] == 2.0 ** -9 and tab[0x08] == 2.0 ** -6
+    # every code but the two NaNs decodes and encodes back to itself (0x80 is -0)
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    assert np.array_equal(oracle.e4m3_encode(tab[codes]), codes)
 
 
 def test_e4m3_rounding_matches_torch_and_closed_forms():
