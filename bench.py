@@ -88,12 +88,41 @@ GEMM_SOURCES = [os.path.join(ROOT, "mixture_experts_ffn_05_b200", "csrc", f)
                 for f in ("grouped_gemm.cu", "common.cuh")]
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without its comments and blank lines (string and character literals,
+    such as inline PTX, are kept as they are)."""
+    out = []
+    i, n = 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def kernel_sha() -> str:
+    """Hash of the GEMM kernel's code: its sources without comments, so that the ncu
+    counters recorded for a kernel stay attached to it across comment edits and are
+    dropped as soon as any code changes."""
     import hashlib
     h = hashlib.sha256()
     for f in GEMM_SOURCES:
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f) as fh:
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()
 
 

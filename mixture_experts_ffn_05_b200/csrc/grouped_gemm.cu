@@ -2,7 +2,7 @@
 //
 // Used for both halves of every expert MLP and of the shared dense MLP:
 //   gate_up (kind 0): h[pos][i] = gelu_tanh(g) * u, g/u = xn[pos] . W_gate_up[e][i or I+i]
-//   down    (kind 1): Y[pos][o] = h[pos] . W_down[e][o]   (bf16 or fp32)
+//   down    (kind 1): Y[pos][o] = h[pos] . W_down[e][o]   (fp16, bf16 or fp32)
 // pos is the token row in sorted (expert-major) order; the routing weights are applied
 // where the slots of a token are summed (combine.cu).  (ONNX export card, "Truthful graph
 // contracts", "Mixture of Experts" and "MoE topology" rows; Inferentia2 card, "How it
@@ -13,7 +13,7 @@
 // batch puts a handful of tokens on each expert, so N is small and the kernel is a
 // weight stream; a prefill batch fills N up to 256.  A gate_up tile holds 64 features as
 // 8 gate rows, the 8 matching up rows, the next 8 gate rows, ... (one 5-D TMA box), so
-// the gate and up accumulators of a feature land in TMEM lanes l and l^8 of one warp.
+// the gate and up rows of a feature are 8 TMEM lanes apart.
 //
 // Work list: for each problem (experts, then the optional dense MLP), for each group,
 // for each M tile (PAIR: pair of M tiles), for each N tile of BN tokens, `split` pieces
@@ -22,15 +22,18 @@
 // stores its fp32 partial tile; the last piece to arrive (an atomic counter) sums all
 // partials in piece order, so the result does not depend on arrival order or schedule.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads into a ring of shared-memory
-// stages, warp 1 issues tcgen05.mma into one of 2-4 TMEM accumulators, and two groups of
-// four warps (2-5 and 6-9) take alternate pieces, read the accumulator back (tcgen05.ld)
-// and run the epilogue while later pieces are being multiplied.  With int8 expert
-// weights (the int8 build of the Inferentia2 card: per-channel symmetric INT8 experts),
-// warps 10-13 convert each raw int8 tile to bf16 in shared memory inside the mainloop,
-// and the per-row scale multiplies the fp32 accumulator in the epilogue (it factors out
-// of the K sum, so this is exact).  Every wait is bounded; a wait that runs out records
-// a timeout in the status word and the CTA winds down.
+// Warp roles (320 threads; 448 with the int8 converters): warp 0 issues TMA loads into a
+// ring of shared-memory stages, warp 1 issues every tcgen05.mma of the CTA into one of
+// 1-4 TMEM accumulators, and two groups of four warps (2-5 and 6-9) read the
+// accumulator back (tcgen05.ld) and run the epilogue while later
+// pieces are being multiplied (wide tiles: both groups, alternate column chunks; BN = 16:
+// alternate pieces).  Operand kinds per problem: bf16 (kind::f16); E4M3 codes with a
+// scale per weight row and per token row (kind::f8f6f4, the FP8-dynamic variant of the
+// "Gemma 4 26B-A4B IT" recipe page); int8 weights with per-channel scales (the int8 build
+// of the Inferentia2 card), which warps 10-13 convert to fp16 in tensor memory, exactly,
+// for MMAs that take A from TMEM.  Row scales multiply the fp32 accumulator in the
+// epilogue (they factor out of the K sum).  Every wait is bounded; a wait that runs out
+// records a timeout in the status word and the CTA winds down.
 #include <type_traits>
 
 #include "common.cuh"
