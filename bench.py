@@ -467,6 +467,9 @@ def _blas_threads():
     return os.cpu_count() or 1
 
 
+REF_BUDGET_S = 120.0  # the reference arm's timed region, about
+
+
 def _oracle_rows(shape):
     return shape.T if shape.T <= 64 else 64
 
@@ -526,9 +529,19 @@ def run_reference(args, wl, rank, world):
     else:
         ex = oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
     per_step = wl["layers"] if wl.get("chain") else 1
+    # Each step is one oracle call on a bounded sample of the step's token rows, sized
+    # from a timed calibration call so that the K timed steps take about REF_BUDGET_S
+    # (at least one row per step): any --steps stays within a few minutes.
     rows = _oracle_rows(shape)
-    xs = [synth.torch_x(shape, 1234, i, "cpu")[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
-          for i in range(args.warmup + args.steps)]
+
+    def host_x(i, n):
+        return synth.torch_x(shape, 1234, i, "cpu")[:n].contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    tc = time.perf_counter()
+    oracle.block_forward(host_x(0, rows), p, ex, shape.k, shape.eps, bias)
+    per_row = (time.perf_counter() - tc) / rows
+    rows = max(1, min(rows, int(REF_BUDGET_S / (args.steps * per_row))))
+    xs = [host_x(i, rows) for i in range(args.warmup + args.steps)]
     for i in range(args.warmup):
         oracle.block_forward(xs[i], p, ex, shape.k, shape.eps, bias)
     t0 = time.perf_counter()
