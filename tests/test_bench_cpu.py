@@ -1,0 +1,30 @@
+"""The benchmark's work model on the CPU: the algorithmic bytes and FLOPs behind every
+roofline fraction, against the layer's sizes written out by hand."""
+import synth
+
+import bench
+
+SHAPE = synth.Shape(T=8, H=2816, E=128, k=8, I=704, D=2112)
+
+
+def test_flops_per_token_of_the_layer():
+    # 2 k 3 I H (routed experts) + 2 3 D H (dense MLP) + 2 E H (router) per token
+    a = bench.algorithmic(SHAPE, used_experts=50)
+    per_token = a["flops"] / SHAPE.T
+    assert per_token == 2 * 8 * 3 * 704 * 2816 + 2 * 3 * 2112 * 2816 + 2 * 128 * 2816
+    assert abs(per_token / 1e6 - 131.56) < 0.01
+
+
+def test_bytes_count_the_used_experts_and_the_weight_type():
+    H, E, I, D, T = 2816, 128, 704, 2112, 8
+    fixed = 3 * D * H * 2 + E * H * 2 + 6 * H * 2 + E * 2 + 2 * T * H * 2
+    for u in (1, 54, 128):
+        assert bench.algorithmic(SHAPE, u)["bytes"] == u * 3 * I * H * 2 + fixed
+        # 8-bit experts (int8 or E4M3): one byte per weight plus an fp32 scale per row
+        assert bench.algorithmic(SHAPE, u, True)["bytes"] == \
+            u * (3 * I * H + (2 * I + H) * 4) + fixed
+    # the gate_up launch alone: its weights, token rows in, h out
+    g = bench.algorithmic(SHAPE, 54)
+    assert g["gate_up_bytes"] == (54 * 2 * I * H * 2 + 2 * D * H * 2 + (T * 8 + T) * H * 2
+                                  + (T * 8 * I + T * D) * 2)
+    assert g["gate_up_flops"] == T * (2 * 8 * 2 * I * H + 2 * 2 * D * H)
