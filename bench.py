@@ -180,21 +180,28 @@ class Clocks:
         except Exception:
             self.proc.kill()
             return None
-        rows = []
-        for line in out.splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) != 8:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), parts[4:]))
-            except ValueError:
-                continue
-        if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        return parse_clock_samples(out)
+
+
+def parse_clock_samples(text: str):
+    """Clock record of nvidia-smi samples (`Clocks.FIELDS`, csv, no header, no units):
+    median SM clock, the largest max clock, and every throttle reason seen Active in any
+    sample; None without a usable sample."""
+    rows = []
+    for line in text.splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) != 8:
+            continue
+        try:
+            rows.append((float(parts[0]), float(parts[1]), parts[4:]))
+        except ValueError:
+            continue
+    if not rows:
+        return None
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+    return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+            "reasons": reasons, "samples": len(rows)}
 
 
 # ---------------------------------------------------------------------------- work model

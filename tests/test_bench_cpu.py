@@ -28,3 +28,19 @@ def test_bytes_count_the_used_experts_and_the_weight_type():
     assert g["gate_up_bytes"] == (54 * 2 * I * H * 2 + 2 * D * H * 2 + (T * 8 + T) * H * 2
                                   + (T * 8 * I + T * D) * 2)
     assert g["gate_up_flops"] == T * (2 * 8 * 2 * I * H + 2 * 2 * D * H)
+
+
+def test_clock_record_keeps_every_throttle_reason():
+    """A throttle reason seen Active in any sample is reported (a run with hw or thermal
+    slowdown must be recognisable); the SM clock is the median; bad lines are skipped."""
+    txt = "\n".join([
+        "1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "1500, 1965, 998.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "1400, 1965, 999.0, 0x8, Active, Not Active, Not Active, Active",
+        "garbage line",
+        "N/A, 1965, 1.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ])
+    r = bench.parse_clock_samples(txt)
+    assert r == {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0,
+                 "reasons": ["hw_slowdown", "sw_power_cap"], "samples": 3}
+    assert bench.parse_clock_samples("") is None
