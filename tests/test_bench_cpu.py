@@ -44,3 +44,17 @@ def test_clock_record_keeps_every_throttle_reason():
     assert r == {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0,
                  "reasons": ["hw_slowdown", "sw_power_cap"], "samples": 3}
     assert bench.parse_clock_samples("") is None
+
+
+def test_traffic_record_follows_the_kernel_code(tmp_path, monkeypatch):
+    """The ncu DRAM traffic of a summary is used only while the GEMM's code (comments
+    aside) still hashes to the value recorded with it."""
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    (tmp_path / "k.md").write_text(
+        "notes\n\n    traffic_bytes_per_launch: 123456\n"
+        f"    source_sha256: {bench.kernel_sha()}\n")
+    assert bench.ncu_traffic("k.md") == 123456
+    (tmp_path / "s.md").write_text(
+        "    traffic_bytes_per_launch: 123456\n    source_sha256: " + "0" * 64 + "\n")
+    assert bench.ncu_traffic("s.md") is None
+    assert bench.ncu_traffic("missing.md") is None
