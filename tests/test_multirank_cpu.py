@@ -40,3 +40,27 @@ def test_max_over_two_ranks():
 def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(2.0, 1, torch.device("cpu")) == 2.0
+
+
+def test_reference_arm_under_torchrun_prints_one_line():
+    """bench.py --impl reference launched the way the driver launches N > 1 (torchrun, two
+    ranks): rank 0 alone times the oracle and prints one JSON line, every rank exits 0."""
+    import json
+    import os
+    import socket
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--steps", "1", "--warmup", "0", "--workload", "decode"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["n_gpus"] == 2
