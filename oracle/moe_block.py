@@ -31,6 +31,14 @@ Readings taken where the pages leave a step open (each also listed in the design
   R8  gate_up rows 0..I-1 are the gate projection and rows I..2I-1 the up projection.
   R9  int8 experts: per output row s = max|w| / 127 (fp32), q = round-half-even(w / s)
       clamped to [-127, 127]; an all-zero row takes s = 1.
+  R18 NVFP4 experts ([P6] variant list: "NVFP4 (4-bit) quantized weights", the format
+      named, not defined): weight-only; E2M1 values (1 sign, 2 exponent bits of bias 1,
+      1 mantissa bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6) with one E4M3 scale per 16 consecutive
+      weights of a row and one fp32 scale per weight matrix.  Quantiser (a reading):
+      t = max|W| / (448 * 6) in fp32 (1 for an all-zero matrix); block scale
+      b = E4M3(max|block| / 6 / t); codes E2M1(w / (b t)), nearest, ties to even,
+      saturating at +-6 (a block whose scale rounds to zero gets zero codes).  The weight
+      is q * b * t.
   R17 fp8 experts ([P6]): E4M3 as the OCP 8-bit format defines it (1 sign, 4 exponent
       bits of bias 7, 3 mantissa bits, subnormals, no infinities, largest finite 448).
       Weights per output row and activations per token row (the rows entering each
@@ -364,6 +372,69 @@ def gated_mlp_fp8(u: np.ndarray, w_gate_up: np.ndarray, w_down: np.ndarray) -> n
     uq = fp8_activation(u)
     h = gelu_tanh(uq @ w_gate_up[:I].T) * (uq @ w_gate_up[I:].T)
     return fp8_activation(h) @ w_down.T
+
+
+# ----------------------------------------------------------------------------- NVFP4
+
+E2M1_MAX = 6.0
+NVFP4_BLOCK = 16
+
+
+def e2m1_decode_table() -> np.ndarray:
+    """Value of every E2M1 code 0..15 (R18): sign bit 3, exponent bits 2..1 (bias 1),
+    mantissa bit 0; exponent 0 is subnormal (m/2)."""
+    c = np.arange(16)
+    sign = np.where(c & 8, -1.0, 1.0)
+    e = (c >> 1) & 3
+    m = (c & 1).astype(np.float64)
+    mag = np.where(e == 0, m / 2.0, (1.0 + m / 2.0) * 2.0 ** (e - 1.0))
+    return sign * mag
+
+
+def e2m1_round(v) -> np.ndarray:
+    """Round to the nearest E2M1 value, ties to the even mantissa, saturating at +-6: the
+    binade [2^e, 2^(e+1)) has spacing 2^(e-1), below 1 the spacing is 0.5."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    spacing = np.where(a < 1.0, 0.5, 2.0 ** (ex - 1 - 1.0))
+    q = np.rint(a / spacing) * spacing
+    return np.copysign(np.minimum(q, E2M1_MAX), v)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """Code (uint8, low 4 bits) of E2M1 values; -0 is code 8."""
+    pos = e2m1_decode_table()[:8]
+    v = np.asarray(v, dtype=np.float64)
+    idx = np.searchsorted(pos, np.abs(v))
+    assert np.all(pos[np.minimum(idx, 7)] == np.abs(v)), "not an E2M1 value"
+    return (idx + np.where(np.signbit(v), 8, 0)).astype(np.uint8)
+
+
+def quantize_nvfp4(w_bits: np.ndarray):
+    """R18 quantiser of one bf16 weight matrix [rows][K] (K a multiple of 16), in fp32:
+    returns (E2M1 codes uint8 [rows][K], E4M3 block-scale codes uint8 [rows][K/16],
+    fp32 tensor scale)."""
+    u = np.asarray(w_bits, dtype=np.uint16)
+    w = (u.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    amax = np.float32(np.max(np.abs(w)))
+    t = np.float32(amax / np.float32(E4M3_MAX * E2M1_MAX)) if amax > 0 else np.float32(1.0)
+    blocks = w.reshape(*w.shape[:-1], -1, NVFP4_BLOCK)
+    bmax = np.max(np.abs(blocks), axis=-1)
+    b = e4m3_round((bmax / np.float32(E2M1_MAX) / t).astype(np.float32).astype(np.float64))
+    bs = (b.astype(np.float32) * t).astype(np.float32)            # fp32 b * t
+    with np.errstate(divide="ignore", invalid="ignore"):
+        quot = np.where(bs[..., None] > 0, blocks / bs[..., None], 0.0).astype(np.float32)
+    q = e2m1_encode(e2m1_round(quot.astype(np.float64))).reshape(w.shape)
+    return q, e4m3_encode(b), t
+
+
+def dequantize_nvfp4(q: np.ndarray, bcodes: np.ndarray, t) -> np.ndarray:
+    """q * b * t in float64 (R18)."""
+    vals = e2m1_decode_table()[np.asarray(q, dtype=np.uint8)]
+    b = e4m3_decode_table()[np.asarray(bcodes, dtype=np.uint8)]
+    blocks = vals.reshape(*vals.shape[:-1], -1, NVFP4_BLOCK) * b[..., None]
+    return blocks.reshape(vals.shape) * float(t)
 
 
 # ----------------------------------------------------------------------------- gaps

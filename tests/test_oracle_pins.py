@@ -409,6 +409,58 @@ def test_fp8_activation_scale_is_per_token():
     assert 1e-3 < rel < 0.2
 
 
+# ------------------------------------------------------------------ NVFP4 (E2M1 + E4M3 blocks)
+
+def test_e2m1_table_and_rounding_by_brute_force():
+    """R18: the E2M1 values written out from the format (0, 0.5, 1, 1.5, 2, 3, 4, 6 and
+    their negatives), and rounding equal to a brute-force nearest-value search that breaks
+    ties towards the code with an even mantissa bit, saturating at 6."""
+    tab = oracle.e2m1_decode_table()
+    assert tab[:8].tolist() == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert np.array_equal(tab[8:], -tab[:8])
+    grid = tab[:8]
+
+    def brute(v):
+        a = min(abs(v), 6.0)
+        d = np.abs(grid - a)
+        best = np.flatnonzero(d == d.min())
+        pick = best[0] if len(best) == 1 else [c for c in best if c % 2 == 0][0]
+        return np.copysign(grid[pick], v)
+
+    pos = grid
+    v = np.concatenate([RNG.uniform(-8, 8, 3000), (pos[:-1] + pos[1:]) / 2,
+                        -(pos[:-1] + pos[1:]) / 2, [0.0, 6.0, 6.5, 1e9]])
+    assert np.array_equal(oracle.e2m1_round(v), np.array([brute(x) for x in v]))
+    codes = np.arange(16, dtype=np.uint8)
+    assert np.array_equal(oracle.e2m1_encode(tab[codes]), codes)
+
+
+def test_nvfp4_quantiser_pins():
+    """R18: the tensor scale maps the matrix max to 448 * 6; every block scale is an E4M3
+    value and makes the block's max land within rounding of 6; each weight is within half
+    an E2M1 step (times b t) of its dequantised value; zero blocks and an all-zero matrix
+    give zero codes."""
+    w = synth.normal_bf16(9, (5,), (6, 64), 0.02)
+    w[2, :16] = 0                                    # one all-zero block
+    q, bc, t = oracle.quantize_nvfp4(w)
+    wf = synth.bf16_bits_to_f32(w).astype(np.float64)
+    assert t == np.float32(np.abs(wf).max() / (448 * 6))
+    b = oracle.e4m3_decode_table()[bc]
+    assert np.all(np.isfinite(b)) and np.all(b >= 0)
+    deq = oracle.dequantize_nvfp4(q, bc, t)
+    bt = np.repeat(b, 16, axis=-1) * float(t)
+    # half the E2M1 step at |w| (0.25 below 2, else 2^(floor(log2)-2)), scaled, plus
+    # the saturation excess where rounding the block scale down pushed w / (b t) above 6
+    a = np.abs(wf) / np.where(bt > 0, bt, 1)
+    step = np.where(a < 1, 0.5, 2.0 ** (np.floor(np.log2(np.maximum(a, 1))) - 1))
+    bound = step / 2 * bt + np.maximum(np.abs(wf) - 6 * bt, 0)
+    assert np.all(np.abs(deq - wf) <= bound * (1 + 1e-6) + 1e-30)
+    assert np.all(q[2, :16] == 0) and bc[2, 0] == 0
+    z = np.zeros((2, 32), dtype=np.uint16)
+    qz, bz, tz = oracle.quantize_nvfp4(z)
+    assert tz == 1.0 and np.all(qz == 0) and np.all(bz == 0)
+
+
 # ------------------------------------------------------------------ the bar discriminates
 
 def test_fp16_accumulation_fails_the_bar():
