@@ -160,14 +160,19 @@ class Experts:
     """
 
     def __init__(self, w_gate_up=None, w_down=None, q_gate_up=None, s_gate_up=None,
-                 q_down=None, s_down=None, fp8: bool = False):
+                 q_down=None, s_down=None, fp8: bool = False, nvfp4=None):
         self.fp8 = fp8                     # q_* are E4M3 codes (uint8) and the activations
         self.int8 = q_gate_up is not None and not fp8   # of both matmuls are quantised
+        # NVFP4 (R18): {"gate_up": [(codes, block scales, tensor scale)] per expert,
+        # "down": [...]}, weight-only
+        self.nvfp4 = nvfp4
         self.w_gate_up, self.w_down = w_gate_up, w_down
         self.q_gate_up, self.s_gate_up = q_gate_up, s_gate_up
         self.q_down, self.s_down = q_down, s_down
 
     def gate_up(self, e: int) -> np.ndarray:
+        if self.nvfp4 is not None:
+            return dequantize_nvfp4(*self.nvfp4["gate_up"][e])
         if self.fp8:
             return dequantize_fp8(self.q_gate_up[e], self.s_gate_up[e])
         if self.int8:
@@ -175,6 +180,8 @@ class Experts:
         return bf16(self.w_gate_up[e])
 
     def down(self, e: int) -> np.ndarray:
+        if self.nvfp4 is not None:
+            return dequantize_nvfp4(*self.nvfp4["down"][e])
         if self.fp8:
             return dequantize_fp8(self.q_down[e], self.s_down[e])
         if self.int8:

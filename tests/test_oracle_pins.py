@@ -461,6 +461,26 @@ def test_nvfp4_quantiser_pins():
     assert tz == 1.0 and np.all(qz == 0) and np.all(bz == 0)
 
 
+def test_nvfp4_experts_in_the_block():
+    """R18 through the whole block: each expert matrix carries its own tensor scale; the
+    block runs on the dequantised weights (activations untouched), so its MoE branch stays
+    close to the bf16 one (4-bit weights: a few percent) and the all-experts-dense
+    identity holds exactly."""
+    c = cases.make_case(synth.TINY, seed=1234)
+    p, E = c.p, c.shape.E
+    nv = {"gate_up": [oracle.quantize_nvfp4(p["w_gate_up"][e]) for e in range(E)],
+          "down": [oracle.quantize_nvfp4(p["w_down"][e]) for e in range(E)]}
+    ex = oracle.Experts(nvfp4=nv)
+    o4 = oracle.block_forward(c.x, p, ex, c.shape.k, c.shape.eps, c.bias)
+    o16 = oracle.block_forward(c.x, p, cases.bf16_experts(p), c.shape.k, c.shape.eps, c.bias)
+    rel = np.abs(o4["moe"] - o16["moe"]).max() / np.abs(o16["moe"]).max()
+    assert 1e-3 < rel < 0.3
+    assert np.array_equal(o4["topk_idx"], o16["topk_idx"])      # the router is untouched
+    dense = oracle.block_forward(c.x, p, ex, c.shape.k, c.shape.eps, c.bias,
+                                 all_experts_dense=True)
+    np.testing.assert_allclose(dense["moe"], o4["moe"], rtol=1e-10, atol=1e-12)
+
+
 # ------------------------------------------------------------------ the bar discriminates
 
 def test_fp16_accumulation_fails_the_bar():
