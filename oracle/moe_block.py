@@ -18,7 +18,7 @@ Sources (page title, section):
   [P6] "Gemma 4 26B-A4B IT" (inference recipe), section "Quantized Variants" and its
        variant list: FP8 (E4M3) weights with dynamic per-token activation quantization.
 
-Readings taken where the pages leave a step open (each also listed in the design notes):
+Readings taken where the pages leave a step open:
   R1  RMSNorm multiplies by the stored gain as-is, eps inside the square root.
   R2  "four feed-forward layernorms" = a pre and a post norm on each branch, followed
       by the post_ff norm of the sum; a post norm given as None is skipped.

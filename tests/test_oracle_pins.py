@@ -409,6 +409,115 @@ def test_fp8_activation_scale_is_per_token():
     assert 1e-3 < rel < 0.2
 
 
+def _bf16_truncating(v):
+    """A deliberately wrong bf16 rounding (drops the low 16 bits), to show the pin below
+    tells it apart."""
+    u = np.asarray(v, dtype=np.float64).astype(np.float32).view(np.uint32)
+    return (u & np.uint32(0xFFFF0000)).view(np.float32).astype(np.float64)
+
+
+def _bf16_ties_away(v):
+    """A deliberately wrong bf16 rounding (nearest, ties away from zero)."""
+    u = np.asarray(v, dtype=np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x8000) >> 16).astype(np.uint32) << np.uint32(16)
+    return r.view(np.float32).astype(np.float64)
+
+
+def test_bf16_round_matches_torch():
+    """The bf16 storage of an activation (R10, R17) equals the library's fp32 -> bfloat16
+    conversion (round to nearest, ties to even) on random values of every magnitude,
+    exact ties with an even and with an odd kept bit, fp32 subnormals, values next to
+    the largest finite bf16 (which round up to infinity past it) and signed zeros.  The
+    inputs tell a truncating and a ties-away rounding apart from the right one."""
+    mant = RNG.integers(0, 1 << 23, 3000, dtype=np.uint32)
+    expo = RNG.integers(1, 254, 3000, dtype=np.uint32)
+    sign = RNG.integers(0, 2, 3000, dtype=np.uint32) << np.uint32(31)
+    rnd = (sign | (expo << np.uint32(23)) | mant).view(np.float32)
+    hi = RNG.integers(0, 1 << 16, 200, dtype=np.uint32) << np.uint32(16)
+    ties = (hi | np.uint32(0x8000)) & np.uint32(0x7F7FFFFF)      # low half exactly 0x8000
+    ties = ties[(ties >> np.uint32(23)) > 0].view(np.float32)
+    sub = (RNG.integers(1, 1 << 23, 200, dtype=np.uint32)).view(np.float32)   # subnormals
+    big = np.array([0x7F7F0000, 0x7F7F7FFF, 0x7F7F8000, 0x7F7FFFFF, 0x7F7E8000,
+                    0xFF7F8000], dtype=np.uint32).view(np.float32)
+    special = np.array([0.0, -0.0, 1.0, -1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8],
+                       dtype=np.float32)
+    v = np.concatenate([rnd, ties, -ties, sub, -sub, big, special])
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    got = oracle.bf16_round(v.astype(np.float64))
+    assert np.array_equal(got, ref) and np.array_equal(np.signbit(got), np.signbit(ref))
+    # closed forms: 1 + 2^-8 is the tie between 1 and 1 + 2^-7 (even: 1); 1 + 3 * 2^-8
+    # is the tie between 1 + 2^-7 and 1 + 2^-6 (even: 1 + 2^-6)
+    assert oracle.bf16_round([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8]).tolist() == \
+        [1.0, 1.0 + 2.0 ** -6]
+    assert np.isinf(oracle.bf16_round([3.4e38])[0])
+    # the pin discriminates: both wrong roundings differ from the library somewhere
+    for wrong in (_bf16_truncating, _bf16_ties_away):
+        assert not np.array_equal(wrong(v.astype(np.float64)), ref)
+
+
+def test_fp8_activation_closed_form_rows():
+    """R17 on hand-built rows whose scales and E4M3 codes are known: row 0 has max 7, so
+    s = 7/448 = 2^-6 and the quotients are v * 64; row 1 has max 14 (s = 2^-5, v * 32),
+    so a per-row scale gives each row its own grid.  Expected values, worked by hand:
+      row 0: 7 -> 448 (code 0x7E); 3.5 -> 224; -1.75 -> -112; 17/64 -> 17 is the tie
+      between 16 and 18 on the spacing-2 binade [16, 32), even mantissa: 16 (code 0x58:
+      exponent field 4 + 7, mantissa 0) -> 0.25;
+      19/64 -> tie between 18 and 20, even: 20 -> 20/64; 3 * 2^-16 -> 3 * 2^-10 is the
+      tie between the subnormals 2^-9 and 2 * 2^-9, even: 2^-8 -> 2^-14;
+      1 + 2^-9 -> stored as bf16 first: the tie between 1 and 1 + 2^-7 rounds to 1,
+      then 64 -> 1.0; 0 -> 0.
+      row 1: 14 -> 448; -14 -> -448; 0.5 -> 16 -> 0.5; 5/32 -> 5 (exact in [4, 8) with
+      spacing 0.5) -> 5/32."""
+    r0 = [7.0, 3.5, -1.75, 17 / 64, 19 / 64, 3 * 2.0 ** -16, 1.0 + 2.0 ** -9, 0.0]
+    r1 = [14.0, -14.0, 0.5, 5 / 32, 0.0, 0.0, 0.0, 0.0]
+    got = oracle.fp8_activation(np.array([r0, r1]))
+    want0 = [7.0, 3.5, -1.75, 0.25, 20 / 64, 2.0 ** -14, 1.0, 0.0]
+    want1 = [14.0, -14.0, 0.5, 5 / 32, 0.0, 0.0, 0.0, 0.0]
+    assert got.tolist() == [want0, want1]
+    q, s = oracle.quantize_fp8_rows(oracle.bf16_round(np.array([r0, r1])).astype(np.float32))
+    assert s.tolist() == [2.0 ** -6, 2.0 ** -5]
+    assert q[0, 0] == 0x7E and q[1, 1] == 0xFE and q[0, 3] == 0x58 and q[0, 5] == 0x02
+
+
+def test_gated_mlp_fp8_matches_torch_float8():
+    """R17: the fp8 gated MLP against the same steps written with the library's own
+    pieces: bfloat16 storage, per-row scales max|row| / 448 in fp32, float8_e4m3fn
+    rounding, float64 matmuls and torch's gelu(tanh).  The rows' quotients never exceed
+    448 (where the library's conversion, unlike the kernels', does not saturate)."""
+    T, H, I = 7, 48, 24
+    u = RNG.standard_normal((T, H)) * 1.3
+    wgu = RNG.standard_normal((2 * I, H)) * 0.2
+    wd = RNG.standard_normal((H, I)) * 0.2
+
+    def q8(v):
+        b = torch.from_numpy(v).to(torch.bfloat16).to(torch.float32)
+        s = b.abs().amax(dim=1, keepdim=True) / 448.0
+        s = torch.where(s > 0, s, torch.ones_like(s))
+        return (b / s).to(torch.float8_e4m3fn).to(torch.float64) * s.to(torch.float64)
+
+    uq = q8(u)
+    g = uq @ torch.from_numpy(wgu[:I]).T
+    v = uq @ torch.from_numpy(wgu[I:]).T
+    h = F.gelu(g, approximate="tanh") * v
+    ref = (q8(h.numpy()) @ torch.from_numpy(wd).T).numpy()
+    got = oracle.gated_mlp_fp8(u, wgu, wd)
+    np.testing.assert_allclose(got, ref, rtol=1e-9, atol=1e-12)
+
+
+def test_topk_gaps_hand_computed():
+    """The gap filter's measure on hand-computed rows: the smallest adjacent gap among the
+    k + 1 largest logits, the (k+1)-th included and everything past it ignored.
+      [0.5, 0.1, 0.9, 0.45, -1.0], k = 2: sorted 0.9, 0.5, 0.45 -> gaps 0.4, 0.05 -> 0.05
+        (the gap between the k-th and the (k+1)-th, which decides the selected set);
+      [1.0, 0.8, 0.5, 0.49], k = 2: top three 1.0, 0.8, 0.5 -> 0.2 (0.01 lies past them);
+      [0.3, 0.3, 0.1, 0.0], k = 1: a tie at the top -> 0;
+      [2.0, -1.0, 0.5], k = 3 (k = E): all three -> min(1.5, 1.5) = 1.5."""
+    g = oracle.topk_gaps(np.array([[0.5, 0.1, 0.9, 0.45, -1.0], [1.0, 0.8, 0.5, 0.49, -5.0]]), 2)
+    np.testing.assert_allclose(g, [0.05, 0.2], rtol=0, atol=1e-15)
+    assert oracle.topk_gaps(np.array([[0.3, 0.3, 0.1, 0.0]]), 1).tolist() == [0.0]
+    assert oracle.topk_gaps(np.array([[2.0, -1.0, 0.5]]), 3).tolist() == [1.5]
+
+
 # ------------------------------------------------------------------ NVFP4 (E2M1 + E4M3 blocks)
 
 def test_e2m1_table_and_rounding_by_brute_force():
