@@ -39,6 +39,9 @@ UNIT = "tokens/s"
 WORKLOADS = {
     "decode": dict(shape=synth.DECODE, layers=8, steps=3000, warmup=100,
                    name="Gemma-4-26B-A4B-shaped MoE-FFN layer, decode T=8 (bf16 experts)"),
+    "decode_T1": dict(shape=synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                      steps=3000, warmup=100,
+                      name="Gemma-4-26B-A4B-shaped MoE-FFN layer, decode T=1 (bf16 experts)"),
     "decode_T64": dict(shape=synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112), layers=8,
                        steps=2000, warmup=100,
                        name="Gemma-4-26B-A4B-shaped MoE-FFN layer, T=64 (bf16 experts)"),
@@ -66,6 +69,15 @@ WORKLOADS = {
                   name="stack of 30 distinct MoE-FFN layers, residual-chained, T=16384 (one 16K chunk)"),
 }
 ZIPF_ALPHA_FILE = os.path.join(ROOT, "tests", "golden", "zipf_alpha.json")
+
+# The default run measures the headline workload (decode, T=8) with the requested
+# --steps/--warmup, then, on one GPU, every other workload with these step counts (each
+# a few seconds of GPU time; the stack's steps are 30 chained layers each), so that one
+# run of a few minutes carries every configuration.
+SWEEP = {"decode_T1": (2000, 50), "decode_T64": (1000, 50), "prefill": (200, 10),
+         "int8_T1": (2000, 50), "int8_T64": (1000, 50), "int8_T1024": (200, 10),
+         "fp8_T8": (1000, 50), "fp8_T64": (1000, 50), "fp8_T1024": (200, 10),
+         "stack": (3, 2)}
 
 
 def peaks():
@@ -229,6 +241,29 @@ def algorithmic(shape, used_experts: int, int8: bool = False):
 
 # ---------------------------------------------------------------------------- our arm
 
+def workload_config(wl, world, nl, alpha):
+    """The `config` object of a workload's JSON line (both arms print the same one)."""
+    shape = wl["shape"]
+    int8, fp8 = bool(wl.get("int8")), bool(wl.get("fp8"))
+    return {"workload": wl["name"], "T": shape.T, "H": shape.H, "E": shape.E, "top_k": shape.k,
+            "expert_inter": shape.I, "dense_inter": shape.D,
+            "expert_weights": ("int8 per-channel" if int8 else
+                               "E4M3 per-channel, E4M3 per-token activations" if fp8 else "bf16"),
+            "router_bias": ("zipf s=1.1, alpha=%.5f" % alpha) if wl.get("zipf") else "none",
+            "layers": nl, "chained": bool(wl.get("chain")),
+            "l2": ("steps rotate over %d distinct layers (%.1f GB of weights) and distinct "
+                   "inputs; no step's weights are L2-resident" %
+                   (nl, nl * 3 * shape.E * shape.I * shape.H * (1 if int8 or fp8 else 2) / 1e9)),
+            "parallelism": f"dp{world} (replicas, no collective)"}
+
+
+def zipf_alpha(wl):
+    if not wl.get("zipf"):
+        return None
+    with open(ZIPF_ALPHA_FILE) as f:
+        return float(json.load(f)["alpha"])
+
+
 def _make_layers(mf, cfg, shape, wl, n, seed, device):
     layers, alpha = [], None
     for l in range(n):
@@ -253,7 +288,9 @@ def _make_layers(mf, cfg, shape, wl, n, seed, device):
     return layers, alpha
 
 
-def run_ours(args, wl, rank, world, device):
+def run_ours(args, wl, rank, world, device, K=None, W=None, headline=True):
+    """One workload: K timed steps after W warm-up steps.  The headline adds the
+    end-to-end run, the launch count and the CPU baseline."""
     import mixture_experts_ffn_05_b200 as mf
     mf.lib()  # fails loudly without the built CUDA library
     shape = wl["shape"]
@@ -266,7 +303,8 @@ def run_ours(args, wl, rank, world, device):
     nl = args.layers or wl["layers"]
     layers, alpha = _make_layers(mf, cfg, shape, wl, nl, seed, device)
     bws = [mf.BlockWeights(cfg, t) for t in layers]
-    W, K = args.warmup, args.steps
+    W = args.warmup if W is None else W
+    K = args.steps if K is None else K
     xs = [synth.torch_x(shape, seed, i, device) for i in range(W + K)]
     out = torch.empty(T, shape.H, dtype=torch.bfloat16, device=device)
     bufs = [torch.empty_like(out), torch.empty_like(out)]
@@ -347,8 +385,20 @@ def run_ours(args, wl, rank, world, device):
             for j, n in enumerate(stages):
                 stages[n].append(ev[j].elapsed_time(ev[j + 1]))
     t_max = max_over_ranks(t_ms, world, device)
+    te = None
+    if headline:
+        te = _e2e(mf, shape, xs, step, W, K, world, device, ws, stream)
+    res = _report(mf, wl, shape, cfg, used, stages, t_max, K, W, world, nl, alpha, chain, int8,
+                  fp8, clk, calls, te, headline)
+    if headline and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(shape, layers[0], xs[W], wl, alpha, nl if chain else 1)
+    return res
 
-    # ---- end to end through the public API, host buffers, copies inside the timed region
+
+def _e2e(mf, shape, xs, step, W, K, world, device, ws, stream):
+    """The same steps end to end through the public API: pinned host input copied in and
+    the output copied out inside the timed region.  Returns the slowest rank's ms."""
+    T = shape.T
     x_host = torch.empty(W + K, T, shape.H, dtype=torch.bfloat16, pin_memory=True)
     for i in range(W + K):
         x_host[i].copy_(xs[i])
@@ -376,7 +426,12 @@ def run_ours(args, wl, rank, world, device):
     te = max_over_ranks(f0.elapsed_time(f1), world, device)
     if mf.moe_check_device_status(ws) != mf.MOE_OK:
         raise RuntimeError("device status after the end-to-end region")
+    return te
 
+
+def _report(mf, wl, shape, cfg, used, stages, t_max, K, W, world, nl, alpha, chain, int8, fp8,
+            clk, calls, te, headline):
+    T = shape.T
     # ---- roofline of the dominant kernel (the gate_up grouped GEMM) and of the block
     pk = peaks()
     long_step = t_max / K > 10.0  # ms: a kernel inside a long step meets the sustained peak
@@ -421,23 +476,23 @@ def run_ours(args, wl, rank, world, device):
                   "binding_frac": round(max(t_hbm, t_tc) / (ms_step * 1e-3), 4),
                   "mean_used_experts": round(sum(used) / len(used), 2)}
     launches_per_call = mf.moe_block_launch_count(cfg, T)  # the library's own count
+    ncalls = len(calls(0))
+    if not headline:
+        return {"workload": wl["name"], "steps": K, "warmup": W, "ms_per_step": round(ms_step, 5),
+                "value": round(world * T * K / (t_max * 1e-3), 1), "unit": UNIT,
+                "dtype": "e4m3 x e4m3 (experts), bf16 (dense)" if fp8 else
+                         ("int8 weights, fp16 activations (experts), bf16 (dense)" if int8 else "bf16"),
+                "config": workload_config(wl, world, nl, alpha),
+                "roofline": roof, "block_roofline": block_roof,
+                "stages_ms": {n: round(statistics.mean(v), 5) for n, v in stages.items()},
+                "gpu_launches_per_step": launches_per_call * ncalls, "clocks": clk}
     res = {
         "metric": METRIC, "value": round(world * T * K / (t_max * 1e-3), 1), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 x e4m3 (experts), bf16 (dense)" if fp8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the layer's shape)",
-        "config": {"workload": wl["name"], "T": T, "H": shape.H, "E": shape.E, "top_k": shape.k,
-                   "expert_inter": shape.I, "dense_inter": shape.D,
-                   "expert_weights": ("int8 per-channel" if int8 else
-                                      "E4M3 per-channel, E4M3 per-token activations" if fp8
-                                      else "bf16"),
-                   "router_bias": ("zipf s=1.1, alpha=%.5f" % alpha) if wl.get("zipf") else "none",
-                   "layers": nl, "chained": chain,
-                   "l2": ("steps rotate over %d distinct layers (%.1f GB of weights) and distinct "
-                          "inputs; no step's weights are L2-resident" %
-                          (nl, nl * 3 * shape.E * shape.I * shape.H * (1 if int8 or fp8 else 2) / 1e9)),
-                   "parallelism": f"dp{world} (replicas, no collective)"},
+        "config": workload_config(wl, world, nl, alpha),
         "roofline": roof,
         "block_roofline": block_roof,
         "stages_ms": {n: round(statistics.mean(v), 5) for n, v in stages.items()},
@@ -446,8 +501,6 @@ def run_ours(args, wl, rank, world, device):
         "gpu_launches": launches_per_call * ncalls * K,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(shape, layers[0], xs[W], wl, alpha, nl if chain else 1)
     return res
 
 
@@ -519,10 +572,7 @@ def run_reference(args, wl, rank, world):
     import oracle
     shape = wl["shape"]
     layer = synth.torch_layer(shape, 1234, 0, "cpu")
-    alpha = None
-    if wl.get("zipf"):
-        with open(ZIPF_ALPHA_FILE) as f:
-            alpha = float(json.load(f)["alpha"])
+    alpha = zipf_alpha(wl)
     p = _host_layer(layer)
     bias = synth.zipf_bias(1234, shape.E, alpha) if wl.get("zipf") else None
     if wl.get("int8"):
@@ -556,13 +606,14 @@ def run_reference(args, wl, rank, world):
         oracle.block_forward(xs[args.warmup + i], p, ex, shape.k, shape.eps, bias)
     el = time.perf_counter() - t0
     v = round(args.steps * rows / el / per_step, 3)
-    sample = f"{args.steps} timed oracle block calls of {rows} tokens each ({wl['name']})" + (
+    sample = (f"{args.steps} timed oracle block calls of {rows} of the {shape.T} tokens of a "
+              f"step each ({wl['name']}; layer 0)") + (
         f"; one layer per call, rate divided by {per_step} layers" if per_step > 1 else "")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)",
-            "config": {"workload": wl["name"], "T": shape.T, "rows_per_step": rows},
+            "config": workload_config(wl, world, args.layers or wl["layers"], alpha),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -576,11 +627,14 @@ def main():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default=None,
+                    help="one workload only (default: the decode headline, then every other "
+                         "workload on one GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None, help="layer copies to rotate over")
     args = ap.parse_args()
-    wl = WORKLOADS[args.workload]
+    sweep = args.workload is None
+    wl = WORKLOADS[args.workload or "decode"]
     if args.impl == "reference":
         args.steps = args.steps if args.steps is not None else 10
         args.warmup = args.warmup if args.warmup is not None else 3
@@ -605,6 +659,14 @@ def main():
                                              device_id=device)
     try:
         res = run_ours(args, wl, rank, world, device)
+        if sweep and world == 1:
+            # every other workload, each with its own step counts; its weights are freed
+            # before the next one is built
+            res["workloads"] = {}
+            for name, (k, w) in SWEEP.items():
+                torch.cuda.empty_cache()
+                res["workloads"][name] = run_ours(args, WORKLOADS[name], rank, world, device,
+                                                  K=k, W=w, headline=False)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

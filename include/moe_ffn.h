@@ -167,8 +167,10 @@ moe_status_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk
  *   process exits.  Nothing is allocated or freed by this call.
  *   Limits: T*k <= MOE_PERMUTE_NOALLOC_MAX_PAIRS (2^20); larger batches return
  *   MOE_ERR_UNSUPPORTED before anything is launched (use moe_permute with a workspace).
- *   The first call on a device looks up the scratch array's device address (once per
- *   device, with that device current); make that first call before any stream capture.
+ *   Every call looks up the scratch array's address in the calling thread's current
+ *   context (an allocation-free lookup), so a device reset or another context on the
+ *   same device never leaves a stale address behind.  The first call in a context may
+ *   load the library's device code there: make it before any stream capture.
  *   Every call shares the one scratch array: calls whose kernels overlap on the GPU (on
  *   different streams, or from several threads) race and must be serialised by the
  *   caller.  Each call fully writes the scratch it reads, so nothing carries over. */

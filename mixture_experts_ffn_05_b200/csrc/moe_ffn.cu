@@ -739,8 +739,10 @@ moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream) {
 // For callers that can hand the library no scratch memory (see moe_permute_noalloc in
 // include/moe_ffn.h).  The multi-block counting sort needs per-block histograms and
 // per-block bases (2 x 256 blocks x 256 experts ints); they live in this fixed device
-// array instead of a caller workspace.  Its host-side name is only a handle: the
-// device address is looked up once per device with cudaGetSymbolAddress and cached.
+// array instead of a caller workspace.  Its host-side name is only a handle: the device
+// address is looked up on every call with cudaGetSymbolAddress (an allocation-free
+// lookup), in the context current at the call, so that no address outlives a device
+// reset or belongs to another context of the same device.
 
 namespace {
 
@@ -750,20 +752,11 @@ static_assert(kNoAllocInts * 4 == MOE_PERMUTE_NOALLOC_SCRATCH_BYTES, "scratch si
 
 static __device__ __align__(256) int g_permute_scratch[kNoAllocInts];
 
-std::mutex g_scratch_mu;
-int* g_scratch_ptr[64] = {};
-
-// Device address of the scratch array on the current device (NULL on failure).
+// Device address of the scratch array in the current context (NULL on failure).
 int* permute_scratch() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
-    g_scratch_ptr[dev] = static_cast<int*>(p);
-  }
-  return g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
 }
 
 }  // namespace

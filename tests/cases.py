@@ -48,8 +48,11 @@ def check_bar(got: np.ndarray, ref: np.ndarray, frac: float, what: str = "") -> 
     err = np.abs(got - ref)
     allow = frac * rms + half_ulp_bf16(ref)
     ratio = err / np.maximum(allow, 1e-300)
+    # the same error against the bare bar (frac * rms, without the output format's half
+    # ulp), reported so that the margin to it stays visible
+    bare = err / np.maximum(frac * rms, 1e-300)
     worst = {"min_cos": float(cos.min()), "max_err_over_allow": float(ratio.max()),
-             "max_abs_err": float(err.max())}
+             "max_err_over_bare_bar": float(bare.max()), "max_abs_err": float(err.max())}
     assert cos.min() >= COS_MIN, f"{what}: cosine {cos.min():.7f} < {COS_MIN} ({worst})"
     assert ratio.max() <= 1.0, f"{what}: max-abs error over the bar ({worst})"
     return worst

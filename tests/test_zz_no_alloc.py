@@ -4,8 +4,9 @@ Some callers cannot give the library any scratch memory: plugin hosts that hand 
 operation only its input and output buffers, or processes whose device memory is
 already held by another framework's caching allocator.  For them the library sorts with
 its own fixed device array.  These tests check, through the C interface, that it
-returns exactly what moe_permute (with a workspace) returns, on two calls in a row with
-different routing, so nothing left in the shared array by one call leaks into the next.
+returns exactly what the oracle's permutation and moe_permute (with a workspace) return,
+on two calls in a row with different routing, so nothing left in the shared array by
+one call leaks into the next.
 This file is collected last so that a run stopping at the first failure has already run
 every other test.
 """
@@ -16,6 +17,7 @@ import pytest
 import torch
 
 import mixture_experts_ffn_05_b200 as mf
+import oracle
 from tests.gpu_util import run_permute, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -46,16 +48,20 @@ def _noalloc(cfg, idx):
     return out
 
 
-# (2048, 8) and (40000, 16) take the multi-block sort, which uses the scratch array;
-# (8, 8) takes the single-block sort.
-@pytest.mark.parametrize("T,k,E", [(2048, 8, 128), (8, 8, 128), (40000, 16, 256)])
-def test_noalloc_equals_workspace_permutation_twice(T, k, E):
+# More than 2048 pairs take the multi-block sort, which uses the scratch array: 2049
+# pairs is the first such size, (2048, 8) and (40000, 16) larger ones; (8, 8) takes the
+# single-block sort.
+@pytest.mark.parametrize("T,k,E", [(2048, 8, 128), (8, 8, 128), (2049, 1, 16), (40000, 16, 256)])
+def test_noalloc_equals_oracle_and_workspace_permutation_twice(T, k, E):
     cfg = mf.Config(512, E, k, 64, 64)
     for seed in (1, 2):  # two calls in a row, different routing
-        idx = to_dev(_ids(T, k, E, seed), torch.int32)
-        ref = run_permute(cfg, idx)
+        ids = _ids(T, k, E, seed)
+        idx = to_dev(ids, torch.int32)
         got = _noalloc(cfg, idx)
+        want = dict(zip(("offsets", "sorted_src", "inv_pos"), oracle.permute(ids, E)))
+        ref = run_permute(cfg, idx)
         for name in ("offsets", "sorted_src", "inv_pos"):
+            assert np.array_equal(got[name].cpu().numpy(), want[name]), (name, seed, "oracle")
             assert torch.equal(got[name], ref[name][: got[name].numel()]), (name, seed)
 
 
