@@ -64,6 +64,15 @@ WORKLOADS = {
     "fp8_T1024": dict(shape=synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112), layers=8,
                       fp8=True, steps=500, warmup=20,
                       name="same layer with E4M3 experts and per-token E4M3 activations, T=1024"),
+    "nvfp4_T1": dict(shape=synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                     nvfp4=True, steps=3000, warmup=100,
+                     name="same layer with NVFP4 experts (weight-only), T=1"),
+    "nvfp4_T64": dict(shape=synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                      nvfp4=True, steps=2000, warmup=100,
+                      name="same layer with NVFP4 experts (weight-only), T=64"),
+    "nvfp4_T1024": dict(shape=synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112), layers=8,
+                        nvfp4=True, steps=500, warmup=20,
+                        name="same layer with NVFP4 experts (weight-only), T=1024"),
     "stack": dict(shape=synth.Shape(T=synth.STACK_T, H=2816, E=128, k=8, I=704, D=2112),
                   layers=synth.STACK_LAYERS, chain=True, steps=3, warmup=1,
                   name="stack of 30 distinct MoE-FFN layers, residual-chained, T=16384 (one 16K chunk)"),
@@ -77,6 +86,7 @@ ZIPF_ALPHA_FILE = os.path.join(ROOT, "tests", "golden", "zipf_alpha.json")
 SWEEP = {"decode_T1": (2000, 50), "decode_T64": (1000, 50), "prefill": (200, 10),
          "int8_T1": (2000, 50), "int8_T64": (1000, 50), "int8_T1024": (200, 10),
          "fp8_T8": (1000, 50), "fp8_T64": (1000, 50), "fp8_T1024": (200, 10),
+         "nvfp4_T1": (2000, 50), "nvfp4_T64": (1000, 50), "nvfp4_T1024": (200, 10),
          "stack": (3, 2)}
 
 
@@ -218,22 +228,28 @@ def parse_clock_samples(text: str):
 
 # ---------------------------------------------------------------------------- work model
 
-def algorithmic(shape, used_experts: int, int8: bool = False):
+def algorithmic(shape, used_experts: int, int8: bool = False, nvfp4: bool = False):
     """Bytes that must move and FLOPs that must run for one block call.
 
     Bytes: the weights of the experts that received a token (int8 or E4M3 codes plus
-    fp32 row scales for 8-bit experts: `int8` means any 1-byte weight here), the dense
-    MLP, the router and the norm vectors, plus x in and out.  Intermediates are
+    fp32 row scales for 8-bit experts: `int8` means any 1-byte weight here; NVFP4: half a
+    byte per weight, one E4M3 block scale per 16 weights, an fp32 scale per matrix), the
+    dense MLP, the router and the norm vectors, plus x in and out.  Intermediates are
     implementation traffic.
     """
     H, E, k, I, D, T = shape.H, shape.E, shape.k, shape.I, shape.D, shape.T
-    wb = 1 if int8 else 2
-    b_experts = used_experts * (3 * I * H * wb + ((2 * I + H) * 4 if int8 else 0))
+    if nvfp4:
+        wb = 0.5 + 1.0 / 16
+        sc_gu, sc_all = 4, 8
+    else:
+        wb = 1 if int8 else 2
+        sc_gu, sc_all = (2 * I * 4, (2 * I + H) * 4) if int8 else (0, 0)
+    b_experts = used_experts * (3 * I * H * wb + sc_all)
     b_dense = 3 * D * H * 2
     b = b_experts + b_dense + E * H * 2 + 6 * H * 2 + E * 2 + 2 * T * H * 2
     flops = T * (2 * k * 3 * I * H + 2 * 3 * D * H + 2 * E * H)
     # the gate_up launch alone: its weights, its token rows in, h out
-    b_gate_up = (used_experts * (2 * I * H * wb + (2 * I * 4 if int8 else 0)) + 2 * D * H * 2
+    b_gate_up = (used_experts * (2 * I * H * wb + sc_gu) + 2 * D * H * 2
                  + (T * k + T) * H * 2 + (T * k * I + T * D) * 2)
     f_gate_up = T * (2 * k * 2 * I * H + 2 * 2 * D * H)
     return {"bytes": b, "flops": flops, "gate_up_bytes": b_gate_up, "gate_up_flops": f_gate_up}
@@ -244,16 +260,19 @@ def algorithmic(shape, used_experts: int, int8: bool = False):
 def workload_config(wl, world, nl, alpha):
     """The `config` object of a workload's JSON line (both arms print the same one)."""
     shape = wl["shape"]
-    int8, fp8 = bool(wl.get("int8")), bool(wl.get("fp8"))
+    int8, fp8, nvfp4 = bool(wl.get("int8")), bool(wl.get("fp8")), bool(wl.get("nvfp4"))
+    wbytes = 0.5 + 1.0 / 16 if nvfp4 else (1 if int8 or fp8 else 2)
     return {"workload": wl["name"], "T": shape.T, "H": shape.H, "E": shape.E, "top_k": shape.k,
             "expert_inter": shape.I, "dense_inter": shape.D,
             "expert_weights": ("int8 per-channel" if int8 else
-                               "E4M3 per-channel, E4M3 per-token activations" if fp8 else "bf16"),
+                               "E4M3 per-channel, E4M3 per-token activations" if fp8 else
+                               "NVFP4 (E2M1, E4M3 per 16, fp32 per matrix), weight-only" if nvfp4
+                               else "bf16"),
             "router_bias": ("zipf s=1.1, alpha=%.5f" % alpha) if wl.get("zipf") else "none",
             "layers": nl, "chained": bool(wl.get("chain")),
             "l2": ("steps rotate over %d distinct layers (%.1f GB of weights) and distinct "
                    "inputs; no step's weights are L2-resident" %
-                   (nl, nl * 3 * shape.E * shape.I * shape.H * (1 if int8 or fp8 else 2) / 1e9)),
+                   (nl, nl * 3 * shape.E * shape.I * shape.H * wbytes / 1e9)),
             "parallelism": f"dp{world} (replicas, no collective)"}
 
 
@@ -272,7 +291,18 @@ def _make_layers(mf, cfg, shape, wl, n, seed, device):
             with open(ZIPF_ALPHA_FILE) as f:
                 alpha = float(json.load(f)["alpha"])
             t["logit_bias"] = torch.from_numpy(synth.zipf_bias(seed, shape.E, alpha)).to(device)
-        if wl.get("int8") or wl.get("fp8"):
+        if wl.get("nvfp4"):
+            for name, bname, sname in (("w_gate_up", "b_gate_up", "s_gate_up"),
+                                       ("w_down", "b_down", "s_down")):
+                w = t.pop(name)
+                E_, rows, cols = w.shape
+                q = torch.empty(E_, rows, cols // 2, dtype=torch.uint8, device=device)
+                bs = torch.empty(E_, rows, cols // 16, dtype=torch.uint8, device=device)
+                ts = torch.empty(E_, dtype=torch.float32, device=device)
+                mf.moe_quantize_nvfp4(w, q, bs, ts)
+                t[name], t[bname], t[sname] = q, bs, ts
+                del w
+        elif wl.get("int8") or wl.get("fp8"):
             for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down")):
                 w = t.pop(name)
                 cols = w.shape[-1]
@@ -297,8 +327,9 @@ def run_ours(args, wl, rank, world, device, K=None, W=None, headline=True):
     T = shape.T
     int8 = bool(wl.get("int8"))
     fp8 = bool(wl.get("fp8"))
+    nvfp4 = bool(wl.get("nvfp4"))
     chain = bool(wl.get("chain"))
-    cfg = mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps, int8, fp8)
+    cfg = mf.Config(shape.H, shape.E, shape.k, shape.I, shape.D, shape.eps, int8, fp8, nvfp4)
     seed = 1234 + 7919 * rank
     nl = args.layers or wl["layers"]
     layers, alpha = _make_layers(mf, cfg, shape, wl, nl, seed, device)
@@ -389,7 +420,7 @@ def run_ours(args, wl, rank, world, device, K=None, W=None, headline=True):
     if headline:
         te = _e2e(mf, shape, xs, step, W, K, world, device, ws, stream)
     res = _report(mf, wl, shape, cfg, used, stages, t_max, K, W, world, nl, alpha, chain, int8,
-                  fp8, clk, calls, te, headline)
+                  fp8, nvfp4, clk, calls, te, headline)
     if headline and rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(shape, layers[0], xs[W], wl, alpha, nl if chain else 1)
     return res
@@ -430,7 +461,7 @@ def _e2e(mf, shape, xs, step, W, K, world, device, ws, stream):
 
 
 def _report(mf, wl, shape, cfg, used, stages, t_max, K, W, world, nl, alpha, chain, int8, fp8,
-            clk, calls, te, headline):
+            nvfp4, clk, calls, te, headline):
     T = shape.T
     # ---- roofline of the dominant kernel (the gate_up grouped GEMM) and of the block
     pk = peaks()
@@ -439,7 +470,7 @@ def _report(mf, wl, shape, cfg, used, stages, t_max, K, W, world, nl, alpha, cha
     # an E4M3 contraction's peak: the measured bf16 peak times the nominal fp8:bf16 ratio
     # (4.5 : 2.25 PFLOP/s dense); only the routed experts' matmuls run in fp8, so the
     # gate_up launch's peak is the FLOP-weighted mix
-    alg = [algorithmic(shape, u, int8 or fp8) for u in used]
+    alg = [algorithmic(shape, u, int8 or fp8, nvfp4) for u in used]
     gu_ms = sum(stages["gate_up"])
     gu_bytes = sum(a["gate_up_bytes"] for a in alg)
     gu_flops = sum(a["gate_up_flops"] for a in alg)
@@ -450,8 +481,11 @@ def _report(mf, wl, shape, cfg, used, stages, t_max, K, W, world, nl, alpha, cha
     ms_step = t_max / K
     gu_t_hbm = gu_bytes / (pk["hbm_gbs"] * 1e9)
     gu_t_tc = gu_flops / (tc_peak * 1e12)
-    kern = "grouped_gemm_kernel (gate_up launch" + (", int8 converter variant)" if int8 else
-                                                      ", E4M3 experts)" if fp8 else ")")
+    streaming = nvfp4 or (int8 and T <= 256)  # the library's choice of GEMM kernel
+    kern = ("stream_gemm_kernel (gate_up launch, " + ("NVFP4" if nvfp4 else "int8") +
+            " weights widened in registers)" if streaming else
+            "grouped_gemm_kernel (gate_up launch" + (", int8 converter variant)" if int8 else
+                                                      ", E4M3 experts)" if fp8 else ")"))
     if fp8:
         f_exp = 2 * shape.k * 2 * shape.I * shape.H
         f_den = 2 * 2 * shape.D * shape.H
@@ -481,7 +515,9 @@ def _report(mf, wl, shape, cfg, used, stages, t_max, K, W, world, nl, alpha, cha
         return {"workload": wl["name"], "steps": K, "warmup": W, "ms_per_step": round(ms_step, 5),
                 "value": round(world * T * K / (t_max * 1e-3), 1), "unit": UNIT,
                 "dtype": "e4m3 x e4m3 (experts), bf16 (dense)" if fp8 else
-                         ("int8 weights, fp16 activations (experts), bf16 (dense)" if int8 else "bf16"),
+                         ("int8 weights, fp16 activations (experts), bf16 (dense)" if int8 else
+                          "nvfp4 weights, fp16 activations (experts), bf16 (dense)" if nvfp4 else
+                          "bf16"),
                 "config": workload_config(wl, world, nl, alpha),
                 "roofline": roof, "block_roofline": block_roof,
                 "stages_ms": {n: round(statistics.mean(v), 5) for n, v in stages.items()},
@@ -583,6 +619,10 @@ def run_reference(args, wl, rank, world):
         qg, sg = oracle.quantize_fp8_per_channel(p["w_gate_up"])
         qd, sd = oracle.quantize_fp8_per_channel(p["w_down"])
         ex = oracle.Experts(q_gate_up=qg, s_gate_up=sg, q_down=qd, s_down=sd, fp8=True)
+    elif wl.get("nvfp4"):
+        ex = oracle.Experts(nvfp4={
+            part: [oracle.quantize_nvfp4(p[name][e]) for e in range(shape.E)]
+            for part, name in (("gate_up", "w_gate_up"), ("down", "w_down"))})
     else:
         ex = oracle.Experts(w_gate_up=p["w_gate_up"], w_down=p["w_down"])
     per_step = wl["layers"] if wl.get("chain") else 1

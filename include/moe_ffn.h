@@ -72,8 +72,10 @@ typedef enum {
 typedef enum {
   MOE_W_BF16 = 0,    /* expert weights in bf16 */
   MOE_W_INT8 = 1,    /* expert weights int8, one fp32 scale per output row */
-  MOE_W_FP8_E4M3 = 2 /* expert weights E4M3, one fp32 scale per output row; the expert
-                        matmuls' activations are quantised to E4M3 per token row */
+  MOE_W_FP8_E4M3 = 2, /* expert weights E4M3, one fp32 scale per output row; the expert
+                         matmuls' activations are quantised to E4M3 per token row */
+  MOE_W_NVFP4 = 3     /* expert weights NVFP4: E2M1 codes, an E4M3 scale per 16 weights of a
+                         row and an fp32 scale per matrix; weight-only */
 } moe_wdtype_t;
 
 /* Sizes of one layer. */
@@ -100,12 +102,26 @@ typedef struct {
  *                      dynamic per-token activation quantisation): each expert matmul's
  *                      input rows (a routed token's xn_moe, its h) are quantised with
  *                      their own scale max|row| / 448, codes rounded to nearest even and
- *                      saturating; the products accumulate in fp32. */
+ *                      saturating; the products accumulate in fp32.
+ *   nvfp4 (MOE_W_NVFP4): "NVFP4 (4-bit) quantized weights" ("Gemma 4 26B-A4B IT" recipe
+ *                      page, variant list), weight-only: the weight is q * b * t with q an
+ *                      E2M1 value (0, 0.5, 1, 1.5, 2, 3, 4, 6 and negatives; code = sign << 3
+ *                      | index), b an E4M3 scale per 16 consecutive weights of a row and t an
+ *                      fp32 scale per matrix (see moe_quantize_nvfp4):
+ *                        w_gate_up [E][2I][H/2] bytes, w_down [E][H][I/2]: codes packed 8 to a
+ *                          little-endian 32-bit word, nibbles 0-3 = elements 0, 2, 4, 6 of the
+ *                          word's 8 consecutive weights, nibbles 4-7 = elements 1, 3, 5, 7;
+ *                        b_gate_up [E][2I][H/16], b_down [E][H][I/16]: E4M3 codes;
+ *                        s_gate_up [E], s_down [E]: t of each expert's two matrices.
+ *                      Activations stay 16-bit (fp16 inside the expert matmuls, as for int8).
+ *   b_gate_up and b_down must be NULL for the other formats. */
 typedef struct {
   const void* w_gate_up;
   const void* w_down;
   const float* s_gate_up;
   const float* s_down;
+  const uint8_t* b_gate_up;  /* nvfp4 block scales, else NULL */
+  const uint8_t* b_down;
 } moe_expert_weights_t;
 
 /* All weights of one block. */
@@ -231,6 +247,24 @@ moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, 
 moe_status_t moe_quantize_fp8(const moe_bf16_t* w, int64_t rows, int32_t cols, uint8_t* q,
                               float* scales, void* stream);
 
+/* NVFP4 quantisation of `matrices` bf16 weight matrices of [rows][cols] each, weight-only
+ * ("Gemma 4 26B-A4B IT" recipe page, variant list: "NVFP4 (4-bit) quantized weights"; the
+ * format is named there, not defined: this is the public NVFP4 format, quantised as
+ * follows), computed in fp32:
+ *   t = max|W| / (448 * 6) over the matrix (t = 1 for an all-zero matrix);
+ *   per block of 16 consecutive weights of a row: b = E4M3(max|block| / 6 / t), rounded to
+ *   nearest even, saturating at 448;
+ *   codes: E2M1(w / (b * t)) rounded to nearest, ties to the even code, saturating at +-6;
+ *   a block whose scale is 0 gets code 0 throughout.
+ * Outputs (layouts as in moe_expert_weights_t): q [matrices][rows][cols/2] packed codes,
+ * block_scales [matrices][rows][cols/16] E4M3 codes, tensor_scales [matrices] fp32 t.
+ * cols a multiple of 16 (16..65536), rows >= 1, matrices >= 0; w 16-byte aligned, q
+ * 8-byte aligned, tensor_scales 4-byte aligned.  tensor_scales is also used as scratch
+ * (it is cleared and filled by the call). */
+moe_status_t moe_quantize_nvfp4(const moe_bf16_t* w, int64_t matrices, int64_t rows,
+                                int32_t cols, uint8_t* q, uint8_t* block_scales,
+                                float* tensor_scales, void* stream);
+
 /* Waits for `stream`, then reads and clears the device status word in `ws`.
  * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, or MOE_ERR_CUDA if the stream failed. */
 moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, void* stream);
@@ -258,7 +292,8 @@ const char* moe_status_string(moe_status_t status);
 
 /* Version of this interface (increases when a signature or a calling contract changes;
  * 2: the workspace is zeroed once by the caller, MOE_BLOCK_EVENTS is 7;
- * 3: moe_wait_selftest; 4: moe_block_launch_count; 5: MOE_W_FP8_E4M3, moe_quantize_fp8). */
+ * 3: moe_wait_selftest; 4: moe_block_launch_count; 5: MOE_W_FP8_E4M3, moe_quantize_fp8;
+ * 6: MOE_W_NVFP4, moe_quantize_nvfp4, block-scale fields in moe_expert_weights_t). */
 int32_t moe_abi_version(void);
 
 #ifdef __cplusplus

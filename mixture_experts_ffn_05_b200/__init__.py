@@ -27,11 +27,13 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_W_BF16 = 0
 MOE_W_INT8 = 1
 MOE_W_FP8 = 2
+MOE_W_NVFP4 = 3
 
 # Entry points of include/moe_ffn.h (the CPU tests check the header declares exactly these).
 ENTRY_POINTS = ("moe_workspace_size", "moe_router", "moe_permute", "moe_permute_noalloc",
                 "moe_ffn_forward", "dense_mlp_forward", "moe_block_forward",
-                "moe_quantize_int8", "moe_quantize_fp8", "moe_check_device_status",
+                "moe_quantize_int8", "moe_quantize_fp8", "moe_quantize_nvfp4",
+                "moe_check_device_status",
                 "moe_wait_selftest",
                 "moe_block_launch_count", "moe_status_string", "moe_abi_version")
 PERMUTE_NOALLOC_MAX_PAIRS = 1 << 20
@@ -52,7 +54,8 @@ class CConfig(ctypes.Structure):
 
 class CExpertWeights(ctypes.Structure):
     _fields_ = [("w_gate_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
-                ("s_gate_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p)]
+                ("s_gate_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
+                ("b_gate_up", ctypes.c_void_p), ("b_down", ctypes.c_void_p)]
 
 
 class CBlockWeights(ctypes.Structure):
@@ -78,6 +81,7 @@ _SIG = {
                                  _P, _P, _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "moe_quantize_int8": (_I32, [_P, ctypes.c_int64, _I32, _P, _P, _P]),
     "moe_quantize_fp8": (_I32, [_P, ctypes.c_int64, _I32, _P, _P, _P]),
+    "moe_quantize_nvfp4": (_I32, [_P, ctypes.c_int64, ctypes.c_int64, _I32, _P, _P, _P, _P]),
     "moe_check_device_status": (_I32, [_P, ctypes.c_size_t, _P]),
     "moe_wait_selftest": (_I32, [_P, ctypes.c_size_t, ctypes.c_uint64, _P]),
     "moe_block_launch_count": (_I32, [ctypes.POINTER(CConfig), _I32]),
@@ -123,9 +127,11 @@ class Config:
     eps: float = 1e-6
     int8: bool = False
     fp8: bool = False   # E4M3 expert weights, per-token E4M3 activations
+    nvfp4: bool = False  # NVFP4 expert weights (packed E2M1 codes, E4M3 block scales)
 
     def c(self) -> CConfig:
-        wd = MOE_W_FP8 if self.fp8 else (MOE_W_INT8 if self.int8 else MOE_W_BF16)
+        wd = (MOE_W_NVFP4 if self.nvfp4 else MOE_W_FP8 if self.fp8 else
+              (MOE_W_INT8 if self.int8 else MOE_W_BF16))
         return CConfig(self.hidden, self.num_experts, self.top_k, self.expert_inter,
                        self.dense_inter, self.eps, wd)
 
@@ -204,10 +210,12 @@ def moe_permute_noalloc(cfg, topk_idx, expert_offsets, sorted_src, inv_pos, stre
 
 
 def _experts(cfg, e: dict) -> CExpertWeights:
-    wt = torch.uint8 if cfg.fp8 else (torch.int8 if cfg.int8 else BF16)
+    wt = torch.uint8 if (cfg.fp8 or cfg.nvfp4) else (torch.int8 if cfg.int8 else BF16)
     return CExpertWeights(_ptr(e["w_gate_up"], wt, "w_gate_up"), _ptr(e["w_down"], wt, "w_down"),
                           _ptr(e.get("s_gate_up"), torch.float32, "s_gate_up", True),
-                          _ptr(e.get("s_down"), torch.float32, "s_down", True))
+                          _ptr(e.get("s_down"), torch.float32, "s_down", True),
+                          _ptr(e.get("b_gate_up"), torch.uint8, "b_gate_up", True),
+                          _ptr(e.get("b_down"), torch.uint8, "b_down", True))
 
 
 def moe_ffn_forward(cfg, xn_moe, topk_w, expert_offsets, sorted_src, inv_pos, experts: dict,
@@ -293,6 +301,21 @@ def moe_quantize_fp8(w, q, scales, stream=None):
     st = lib().moe_quantize_fp8(_ptr(w, BF16, "w"), rows, cols, _ptr(q, torch.uint8, "q"),
                                 _ptr(scales, torch.float32, "scales"), _stream(stream))
     _check("moe_quantize_fp8", st)
+
+
+def moe_quantize_nvfp4(w, q, block_scales, tensor_scales, stream=None):
+    """NVFP4 codes of bf16 weight matrices w [matrices][rows][cols] (or [rows][cols]):
+    q [.., rows, cols // 2] uint8 packed codes, block_scales [.., rows, cols // 16] uint8
+    E4M3 codes, tensor_scales [matrices] fp32."""
+    cols = w.shape[-1]
+    rows = w.shape[-2]
+    matrices = w.numel() // (rows * cols)
+    st = lib().moe_quantize_nvfp4(_ptr(w, BF16, "w"), matrices, rows, cols,
+                                  _ptr(q, torch.uint8, "q"),
+                                  _ptr(block_scales, torch.uint8, "block_scales"),
+                                  _ptr(tensor_scales, torch.float32, "tensor_scales"),
+                                  _stream(stream))
+    _check("moe_quantize_nvfp4", st)
 
 
 def moe_wait_selftest(ws, timeout_ns: int, stream=None) -> None:

@@ -16,8 +16,8 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = ["router.cu", "router_tc.cu", "permute.cu", "grouped_gemm.cu", "combine.cu", "quant.cu",
-           "health.cu", "moe_ffn.cu"]
+SOURCES = ["router.cu", "router_tc.cu", "permute.cu", "grouped_gemm.cu", "stream_gemm.cu",
+           "combine.cu", "quant.cu", "health.cu", "moe_ffn.cu"]
 LIB = os.path.join(PKG, "libmoeffn.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

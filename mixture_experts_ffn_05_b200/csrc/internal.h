@@ -145,6 +145,42 @@ cudaError_t launch_combine_moe(int T, int H, int k, const uint16_t* y, const int
                                const int* sorted_src, const float* topk_w, uint16_t* moe_out,
                                cudaStream_t s, bool pdl = false);
 cudaError_t launch_wait_selftest(unsigned* status, uint64_t timeout_ns, cudaStream_t s);
+
+// The weight-streaming grouped GEMM of small batches (stream_gemm.cu): the same gate_up and
+// down problems as GemmProblem, with the weights dequantised in registers.
+constexpr int kStreamBf16 = 0, kStreamInt8 = 1, kStreamNvfp4 = 2;
+struct StreamProblem {
+  int kind;              // 0 gate_up (writes h = gelu_tanh(gate) * up), 1 down
+  int wtype;             // kStreamBf16 (bf16 B), kStreamInt8 or kStreamNvfp4 (fp16 B)
+  int groups;            // experts, or 1 for the dense MLP
+  const int* offsets;    // [groups+1] token segments of b; NULL = one group of n_tokens
+  int n_tokens;          // rows of b and of the output
+  int K;                 // reduction length, a multiple of 64
+  int rows;              // weight rows per group (gate_up: 2F), a multiple of 16
+  int F;                 // gate_up: features (first up row)
+  const void* w;         // [groups][rows][K] bf16 / int8, or [groups][rows][K/2] packed E2M1
+  const float* wscale;   // int8: [groups][rows] row scales; nvfp4: [groups] matrix scales
+  const uint8_t* bscale; // nvfp4: [groups][rows][K/16] E4M3 block scales
+  const uint16_t* b;     // [n_tokens][K] token rows (bf16, or fp16 for int8 / nvfp4)
+  void* out;             // gate_up: h [n_tokens][out_ld]; down: [n_tokens][out_ld]
+  int out_type;          // kOutBf16, kOutF16 (gate_up: h's format) or kOutF32 (down)
+  int out_ld;
+  int split;             // pieces per tile along K (1 .. stream_items(K, wtype))
+};
+struct StreamParams {
+  StreamProblem prob[2];
+  int nprob;
+  float* partials;       // split-K partial tiles, [piece][64][8] fp32 (split > 1)
+  unsigned* counters;    // split-K arrival counters, one per (tile, chunk); zero between launches
+  unsigned* sched;       // [2] piece counter and finished CTAs, zero between launches;
+                         // launches that may overlap need their own
+};
+// Tiles of 64 weight rows against chunks of 8 tokens; K in items of 128 bytes of a row.
+constexpr int kStreamTileRows = 64, kStreamChunk = 8;
+int stream_items(int K, int wtype);
+// CTAs of one launch (a persistent grid of every CTA that fits at once).
+int stream_gemm_ctas(int sms);
+cudaError_t launch_stream_gemm(const StreamParams& p, int sms, cudaStream_t s, bool pdl);
 // dst[q] = E4M3 codes of row r(q) of src divided by scales[q] = max|row| / 448 (1 for an
 // all-zero row), r(q) = sorted_src[q] / k, or q when sorted_src is NULL; a source row
 // outside [0, T) gives a zero row.  cols a multiple of 8.
@@ -155,5 +191,10 @@ cudaError_t launch_quantize_fp8(const uint16_t* w, int64_t rows, int cols, uint8
                                 float* scales, cudaStream_t s);
 cudaError_t launch_quantize_int8(const uint16_t* w, int64_t rows, int cols, int8_t* q,
                                  float* scales, cudaStream_t s);
+// matrices x [rows][cols] bf16 -> packed E2M1 codes [.][rows][cols/2], E4M3 block scales
+// [.][rows][cols/16], fp32 matrix scales [matrices]; cols a multiple of 16.
+cudaError_t launch_quantize_nvfp4(const uint16_t* w, int64_t matrices, int64_t rows, int cols,
+                                  uint8_t* q, uint8_t* bscale, float* tensor_scale,
+                                  cudaStream_t s);
 
 }  // namespace moe

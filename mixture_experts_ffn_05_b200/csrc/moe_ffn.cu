@@ -29,6 +29,7 @@ struct Dims {
   float eps;
   int int8;  // int8 expert weights (converted to fp16 on the way to the tensor cores)
   int fp8;   // E4M3 expert weights and per-token E4M3 activations of the expert matmuls
+  int nvfp4; // NVFP4 expert weights (weight-only; fp16 activations like int8)
 };
 
 moe_status_t check_cfg(const moe_config_t* c, int32_t T, Dims* d) {
@@ -36,7 +37,7 @@ moe_status_t check_cfg(const moe_config_t* c, int32_t T, Dims* d) {
   if (T < 0) return MOE_ERR_INVALID_ARG;
   if (!(c->eps > 0.f) || !(c->eps < 1e30f)) return MOE_ERR_INVALID_ARG;
   if (c->expert_wdtype != MOE_W_BF16 && c->expert_wdtype != MOE_W_INT8 &&
-      c->expert_wdtype != MOE_W_FP8_E4M3)
+      c->expert_wdtype != MOE_W_FP8_E4M3 && c->expert_wdtype != MOE_W_NVFP4)
     return MOE_ERR_INVALID_ARG;
   if (c->hidden < 128 || c->hidden > 6144 || c->hidden % 128) return MOE_ERR_UNSUPPORTED;
   if (c->expert_inter < 64 || c->expert_inter > 16384 || c->expert_inter % 64) return MOE_ERR_UNSUPPORTED;
@@ -57,6 +58,7 @@ moe_status_t check_cfg(const moe_config_t* c, int32_t T, Dims* d) {
   d->eps = c->eps;
   d->int8 = c->expert_wdtype == MOE_W_INT8;
   d->fp8 = c->expert_wdtype == MOE_W_FP8_E4M3;
+  d->nvfp4 = c->expert_wdtype == MOE_W_NVFP4;
   return MOE_OK;
 }
 
@@ -79,11 +81,61 @@ int choose_split(int k_steps, int bn, double tiles) {
   return std::max(1, std::min(std::min(k_steps, 4), (k_steps + 10) / 11));
 }
 
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
 // Expected number of experts that receive at least one of T*k uniformly routed pairs
 // (fewer when the routing is skewed, which only makes splitting more useful).
 double expected_used_experts(const Dims& d) {
   const double pairs = static_cast<double>(d.T) * d.k;
   return d.E * (1.0 - std::pow(1.0 - 1.0 / d.E, pairs));
+}
+
+// Batches up to this many tokens with 8-bit integer expert weights run the expert and
+// dense GEMMs on the weight-streaming kernel (stream_gemm.cu), which widens the codes in
+// registers; larger ones on the tensor-memory kernel with converter warps.  NVFP4 expert
+// weights always take the weight-streaming kernel.
+constexpr int kStreamMaxT = 256;
+
+bool stream_path(const Dims& d) { return d.nvfp4 || (d.int8 && d.T <= kStreamMaxT); }
+
+// K pieces of the weight-streaming kernel's tiles: enough pieces for about three per CTA
+// of the launch (five CTAs per SM assumed), each piece at least four K items long.
+constexpr int kStreamAssumedCtas = 5 * kAssumedSms;
+
+int stream_split(double units, int items) {
+  if (units <= 0) return 1;
+  const int want = static_cast<int>(std::ceil(3.0 * kStreamAssumedCtas / units));
+  return std::max(1, std::min(want, items / 4));
+}
+
+struct StreamSplits {
+  int gu_e, gu_d, dn_e, dn_d;  // gate_up experts / dense, down experts / dense
+  int64_t units, pieces;       // upper bounds over the two launches
+};
+
+StreamSplits stream_splits(const Dims& d) {
+  StreamSplits ss{};
+  const int64_t T = d.T, Tk = static_cast<int64_t>(d.T) * d.k;
+  const double u = expected_used_experts(d);
+  const double dense_chunks = static_cast<double>(ceil_div(T, kStreamChunk));
+  const double exp_chunks = u * std::max(1.0, static_cast<double>(Tk) / std::max(u, 1.0) / kStreamChunk);
+  const int tiles_gu_e = 2 * d.I / kStreamTileRows, tiles_gu_d = 2 * d.D / kStreamTileRows;
+  const int tiles_dn = d.H / kStreamTileRows;
+  const double units_gu = exp_chunks * tiles_gu_e + dense_chunks * tiles_gu_d;
+  const double units_dn = (exp_chunks + dense_chunks) * tiles_dn;
+  const int wt = d.nvfp4 ? kStreamNvfp4 : d.int8 ? kStreamInt8 : kStreamBf16;
+  ss.gu_e = stream_split(units_gu, stream_items(d.H, wt));
+  ss.gu_d = stream_split(units_gu, stream_items(d.H, kStreamBf16));
+  ss.dn_e = stream_split(units_dn, stream_items(d.I, wt));
+  ss.dn_d = stream_split(units_dn, stream_items(d.D, kStreamBf16));
+  // upper bounds: every non-empty expert has a partial chunk
+  const int64_t ch_e = std::min<int64_t>(d.E, Tk) + ceil_div(Tk, kStreamChunk);
+  const int64_t ch_d = ceil_div(T, kStreamChunk);
+  const int64_t u_gu = ch_e * tiles_gu_e + ch_d * tiles_gu_d, u_dn = (ch_e + ch_d) * tiles_dn;
+  ss.units = std::max(u_gu, u_dn);
+  ss.pieces = std::max(ch_e * tiles_gu_e * ss.gu_e + ch_d * tiles_gu_d * ss.gu_d,
+                       ch_e * tiles_dn * ss.dn_e + ch_d * tiles_dn * ss.dn_d);
+  return ss;
 }
 
 struct Layout {
@@ -92,9 +144,8 @@ struct Layout {
   size_t sx, h8, sh;  // fp8: token-row scales of the gathered rows, h in E4M3, h's scales
   size_t counters_bytes;
   int bn, split_gu, split_dgu, split_d, split_dd;
+  StreamSplits ss;    // the weight-streaming kernel's splits (stream_path only)
 };
-
-int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 Layout layout_of(const Dims& d) {
   Layout L{};
@@ -115,8 +166,18 @@ Layout layout_of(const Dims& d) {
   const int64_t ntl_d = ceil_div(T, L.bn);
   const int64_t pieces_gu = (d.I / 64) * ntl_e * L.split_gu + (d.D / 64) * ntl_d * L.split_dgu;
   const int64_t pieces_dn = (d.H / 128) * ntl_e * L.split_d + (d.H / 128) * ntl_d * L.split_dd;
-  const int64_t pieces = std::max(pieces_gu, pieces_dn);
-  const bool any_split = L.split_gu > 1 || L.split_dgu > 1 || L.split_d > 1 || L.split_dd > 1;
+  int64_t pieces = std::max(pieces_gu, pieces_dn);
+  bool any_split = L.split_gu > 1 || L.split_dgu > 1 || L.split_d > 1 || L.split_dd > 1;
+  int64_t partial_bytes = any_split ? pieces * L.bn * 128 * 4 : 0;
+  if (stream_path(d)) {
+    // the weight-streaming kernel: one counter per (tile, chunk), [64][8] fp32 per piece
+    L.ss = stream_splits(d);
+    pieces = std::max(pieces, L.ss.units);
+    const bool ssplit = L.ss.gu_e > 1 || L.ss.gu_d > 1 || L.ss.dn_e > 1 || L.ss.dn_d > 1;
+    if (ssplit)
+      partial_bytes = std::max<int64_t>(partial_bytes, L.ss.pieces * kStreamTileRows * kStreamChunk * 4);
+    any_split = any_split || ssplit;
+  }
   const int nb = permute_blocks(static_cast<int>(Tk));
 
   size_t off = 0;
@@ -146,7 +207,7 @@ Layout layout_of(const Dims& d) {
   L.y = take(Tk * d.H * 2);
   L.hd = take(T * d.D * 2);
   L.dense = take(T * d.H * 4);
-  L.partials = take(any_split ? static_cast<size_t>(pieces) * L.bn * 128 * 4 : 0);
+  L.partials = take(static_cast<size_t>(partial_bytes));
   // the tensor-core router's two-term split of the scaled router weights
   const size_t wr_bytes = router_uses_tc(d.T) ? static_cast<size_t>(d.E) * d.H * 2 : 0;
   L.wr_hi = take(wr_bytes);
@@ -268,6 +329,8 @@ struct GemmJob {
   const void* w_down;
   const float* s_gate_up;
   const float* s_down;
+  const uint8_t* b_gate_up;  // nvfp4 block scales
+  const uint8_t* b_down;
   const int* offsets;
   const int* sorted_src;
   const float* topk_w;
@@ -296,7 +359,58 @@ moe_status_t gather_tokens(const Dims& d, const Layout& L, void* ws, const int* 
                                                at<uint8_t>(ws, L.aperm), at<float>(ws, L.sx),
                                                s, pdl));
   return cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe,
-                                        at<uint16_t>(ws, L.aperm), d.int8 != 0, s, pdl));
+                                        at<uint16_t>(ws, L.aperm), d.int8 || d.nvfp4, s, pdl));
+}
+
+// The two GEMM launches on the weight-streaming kernel.
+moe_status_t run_stream_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& j,
+                              cudaStream_t s, bool first_kernel, void* const* ev) {
+  const int Tk = d.T * d.k;
+  const int sms = sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  uint16_t* h = at<uint16_t>(ws, L.h);
+  uint16_t* hd = at<uint16_t>(ws, L.hd);
+  StreamParams gu{}, dn{};
+  for (StreamParams* P : {&gu, &dn}) {
+    P->partials = at<float>(ws, L.partials);
+    P->counters = at<unsigned>(ws, L.counters);
+  }
+  gu.sched = at<unsigned>(ws, L.sched);
+  dn.sched = at<unsigned>(ws, L.sched) + 2;  // the down launch may start before gate_up ends
+  int np = 0;
+  if (j.experts) {
+    const int wt = d.nvfp4 ? kStreamNvfp4 : kStreamInt8;
+    StreamProblem& a = gu.prob[np];
+    a.kind = 0; a.wtype = wt; a.groups = d.E; a.offsets = j.offsets; a.n_tokens = Tk;
+    a.K = d.H; a.rows = 2 * d.I; a.F = d.I; a.w = j.w_gate_up; a.wscale = j.s_gate_up;
+    a.bscale = j.b_gate_up;
+    a.b = static_cast<const uint16_t*>(j.a_rows); a.out = h; a.out_type = kOutF16; a.out_ld = d.I;
+    a.split = L.ss.gu_e;
+    StreamProblem& b = dn.prob[np];
+    b.kind = 1; b.wtype = wt; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = Tk;
+    b.K = d.I; b.rows = d.H; b.F = d.H; b.w = j.w_down; b.wscale = j.s_down; b.bscale = j.b_down;
+    b.b = h; b.out = j.y; b.out_type = kOutF16; b.out_ld = d.H;
+    b.split = L.ss.dn_e;
+    ++np;
+  }
+  if (j.dense) {
+    StreamProblem& a = gu.prob[np];
+    a.kind = 0; a.wtype = kStreamBf16; a.groups = 1; a.offsets = nullptr; a.n_tokens = d.T;
+    a.K = d.H; a.rows = 2 * d.D; a.F = d.D; a.w = j.w_dgu; a.b = j.xn_dense; a.out = hd;
+    a.out_type = kOutBf16; a.out_ld = d.D; a.split = L.ss.gu_d;
+    StreamProblem& b = dn.prob[np];
+    b.kind = 1; b.wtype = kStreamBf16; b.groups = 1; b.offsets = nullptr; b.n_tokens = d.T;
+    b.K = d.D; b.rows = d.H; b.F = d.H; b.w = j.w_dd; b.b = hd; b.out = j.dense_out;
+    b.out_type = j.dense_f32 ? kOutF32 : kOutBf16; b.out_ld = d.H; b.split = L.ss.dn_d;
+    ++np;
+  }
+  gu.nprob = dn.nprob = np;
+  moe_status_t st = cuda_status(launch_stream_gemm(gu, sms, s, !first_kernel));
+  if (st != MOE_OK) return st;
+  if (!mark(ev, 4, s)) return MOE_ERR_CUDA;
+  st = cuda_status(launch_stream_gemm(dn, sms, s, true));
+  if (st != MOE_OK) return st;
+  return mark(ev, 5, s) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // The counters in the workspace start at zero (the caller zeroes a new workspace once)
@@ -305,6 +419,7 @@ moe_status_t gather_tokens(const Dims& d, const Layout& L, void* ws, const int* 
 // launch on whatever the stream ran before).
 moe_status_t run_gemms(const Dims& d, const Layout& L, void* ws, const GemmJob& j,
                        cudaStream_t s, bool first_kernel, void* const* ev = nullptr) {
+  if (stream_path(d)) return run_stream_gemms(d, L, ws, j, s, first_kernel, ev);
   const int64_t Tk = static_cast<int64_t>(d.T) * d.k;
   const int grid = sm_count();
   if (grid <= 0) return MOE_ERR_CUDA;
@@ -467,10 +582,17 @@ moe_status_t run_router(const Dims& d, const Layout& L, void* ws, const RouteJob
                                       s));
 }
 
-bool w_ok(const moe_expert_weights_t* w, bool scaled) {
+bool w_ok(const moe_expert_weights_t* w, const Dims& d) {
   if (w == nullptr || w->w_gate_up == nullptr || w->w_down == nullptr) return false;
   if (!aligned16(w->w_gate_up) || !aligned16(w->w_down)) return false;
-  if (scaled) return w->s_gate_up != nullptr && w->s_down != nullptr;
+  if (d.nvfp4) {
+    // block scales are copied four bytes at a time, the matrix scales read one by one
+    return w->s_gate_up != nullptr && w->s_down != nullptr && w->b_gate_up != nullptr &&
+           w->b_down != nullptr && (reinterpret_cast<uintptr_t>(w->b_gate_up) & 3u) == 0 &&
+           (reinterpret_cast<uintptr_t>(w->b_down) & 3u) == 0;
+  }
+  if (w->b_gate_up != nullptr || w->b_down != nullptr) return false;
+  if (d.int8 || d.fp8) return w->s_gate_up != nullptr && w->s_down != nullptr;
   return w->s_gate_up == nullptr && w->s_down == nullptr;
 }
 
@@ -480,7 +602,7 @@ bool w_ok(const moe_expert_weights_t* w, bool scaled) {
 
 extern "C" {
 
-int32_t moe_abi_version(void) { return 5; }
+int32_t moe_abi_version(void) { return 6; }
 
 int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T) {
   Dims d;
@@ -566,7 +688,7 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   for (const void* p : {(const void*)xn_moe, (const void*)topk_w, (const void*)expert_offsets,
                         (const void*)sorted_src, (const void*)inv_pos, (const void*)moe_out})
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (!w_ok(experts, d.int8 || d.fp8)) return MOE_ERR_INVALID_ARG;
+  if (!w_ok(experts, d)) return MOE_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -580,6 +702,8 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   j.w_down = experts->w_down;
   j.s_gate_up = experts->s_gate_up;
   j.s_down = experts->s_down;
+  j.b_gate_up = experts->b_gate_up;
+  j.b_down = experts->b_down;
   j.offsets = expert_offsets;
   j.sorted_src = sorted_src;
   j.topk_w = topk_w;
@@ -628,7 +752,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   for (const void* p : {(const void*)moe_out, (const void*)w->logit_bias,
                         (const void*)w->g_post_moe, (const void*)w->g_post_dense})
     if (p != nullptr && !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (!w_ok(&w->experts, d.int8 || d.fp8)) return MOE_ERR_INVALID_ARG;
+  if (!w_ok(&w->experts, d)) return MOE_ERR_INVALID_ARG;
   Layout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -669,6 +793,8 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
   j.w_down = w->experts.w_down;
   j.s_gate_up = w->experts.s_gate_up;
   j.s_down = w->experts.s_down;
+  j.b_gate_up = w->experts.b_gate_up;
+  j.b_down = w->experts.b_down;
   j.offsets = offsets;
   j.sorted_src = sorted;
   j.topk_w = topk_w;
@@ -708,6 +834,20 @@ moe_status_t moe_quantize_fp8(const moe_bf16_t* w, int64_t rows, int32_t cols, u
     return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(scales) & 3u) != 0) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_quantize_fp8(w, rows, cols, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_quantize_nvfp4(const moe_bf16_t* w, int64_t matrices, int64_t rows,
+                                int32_t cols, uint8_t* q, uint8_t* block_scales,
+                                float* tensor_scales, void* stream) {
+  if (matrices < 0 || rows < 1 || cols < 16 || cols > 65536 || cols % 16) return MOE_ERR_INVALID_ARG;
+  if (matrices == 0) return MOE_OK;
+  if (matrices > (int64_t(1) << 24) || matrices * rows > (int64_t(1) << 34)) return MOE_ERR_UNSUPPORTED;
+  if (w == nullptr || q == nullptr || block_scales == nullptr || tensor_scales == nullptr ||
+      !aligned16(w) || (reinterpret_cast<uintptr_t>(q) & 7u) != 0 ||
+      (reinterpret_cast<uintptr_t>(tensor_scales) & 3u) != 0)
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_nvfp4(w, matrices, rows, cols, q, block_scales, tensor_scales,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_wait_selftest(void* ws, size_t ws_bytes, uint64_t timeout_ns, void* stream) {

@@ -82,6 +82,125 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(int64_t rows, int col
   }
 }
 
+// NVFP4 quantisation of bf16 weight matrices (the "NVFP4 (4-bit) quantized weights" of the
+// "Gemma 4 26B-A4B IT" recipe page's variant list), weight-only, in fp32:
+//   t = max|W| / (448 * 6) over the whole matrix (t = 1 for an all-zero matrix)
+//   per block of 16 consecutive elements of a row: b = E4M3(max|block| / 6 / t), rounded to
+//   nearest even and saturating; codes E2M1(w / (b t)), nearest, ties to even, saturating
+//   at +-6 (a block whose scale is zero gets code 0 throughout).
+// E2M1 values: 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives; code = sign << 3 | index.
+// Packed 8 codes to a 32-bit word: nibbles 0-3 hold elements 0, 2, 4, 6 of the word's 8,
+// nibbles 4-7 elements 1, 3, 5, 7 (the order the weight-streaming kernel widens them in).
+
+// Pass 1: tensor_amax[m] = max |w| over matrix m, as float bits (zeroed beforehand; the
+// bits of non-negative floats order like the floats).
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(int64_t per_matrix_chunks,
+                                                         int64_t total_chunks,
+                                                         const uint16_t* __restrict__ w,
+                                                         unsigned* __restrict__ amax_bits) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  float a = 0.f;
+  int64_t m = -1;
+  if (i < total_chunks) {
+    m = i / per_matrix_chunks;
+    float f[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(w) + i), f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(f[j]));
+  }
+  // a warp's chunks may straddle two matrices: combine only lanes of the same matrix
+  const int64_t m0 = __shfl_sync(0xffffffffu, m, 0);
+  const bool uniform = __all_sync(0xffffffffu, m == m0);
+  if (uniform) {
+    a = warp_max(a);
+    if ((threadIdx.x & 31) == 0 && m0 >= 0) atomicMax(amax_bits + m0, __float_as_uint(a));
+  } else if (m >= 0) {
+    atomicMax(amax_bits + m, __float_as_uint(a));
+  }
+}
+
+// E2M1 magnitude index of a >= 0 (round to nearest, ties to the even index, saturating).
+__device__ __forceinline__ uint32_t e2m1_index(float a) {
+  return static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
+         static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
+         static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
+         static_cast<uint32_t>(a > 5.0f);
+}
+
+// Pass 2: one thread per block of 16 elements: its E4M3 scale and 16 packed codes.
+__global__ void __launch_bounds__(256) nvfp4_quant_kernel(int64_t blocks_per_matrix,
+                                                          int64_t total_blocks,
+                                                          const uint16_t* __restrict__ w,
+                                                          const float* __restrict__ amax,
+                                                          uint8_t* __restrict__ q,
+                                                          uint8_t* __restrict__ bscale) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= total_blocks) return;
+  const float am = amax[i / blocks_per_matrix];
+  const float t = am > 0.f ? __fdiv_rn(am, 2688.0f) : 1.0f;
+  const uint4* src = reinterpret_cast<const uint4*>(w) + 2 * i;
+  float f[16];
+  {
+    float lo[8], hi[8];
+    unpack8(__ldg(src), lo);
+    unpack8(__ldg(src + 1), hi);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      f[j] = lo[j];
+      f[8 + j] = hi[j];
+    }
+  }
+  float bmax = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(f[j]));
+  const uint8_t bcode = e4m3_bits_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), t));
+  const __half bh = __nv_cvt_fp8_to_halfraw(bcode, __NV_E4M3);  // exact
+  const float bval = __half2float(bh);
+  const float bs = __fmul_rn(bval, t);
+  uint32_t code[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float quot = bs > 0.f ? __fdiv_rn(f[j], bs) : 0.f;
+    code[j] = (signbit(quot) ? 8u : 0u) | e2m1_index(fabsf(quot));
+  }
+  uint32_t word[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t* c = code + 8 * h;
+    word[h] = c[0] | (c[2] << 4) | (c[4] << 8) | (c[6] << 12) | (c[1] << 16) | (c[3] << 20) |
+              (c[5] << 24) | (c[7] << 28);
+  }
+  reinterpret_cast<uint2*>(q)[i] = make_uint2(word[0], word[1]);
+  bscale[i] = bcode;
+}
+
+// Pass 3: the matrix scales from the maxima, in place: t = amax / 2688, 1 for a zero matrix.
+__global__ void __launch_bounds__(256) nvfp4_tscale_kernel(int64_t matrices, float* __restrict__ ts) {
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (m >= matrices) return;
+  const float am = ts[m];
+  ts[m] = am > 0.f ? __fdiv_rn(am, 2688.0f) : 1.0f;
+}
+
+cudaError_t launch_quantize_nvfp4(const uint16_t* w, int64_t matrices, int64_t rows, int cols,
+                                  uint8_t* q, uint8_t* bscale, float* tensor_scale,
+                                  cudaStream_t s) {
+  const int64_t per_matrix = rows * cols;
+  cudaError_t e = cudaMemsetAsync(tensor_scale, 0, static_cast<size_t>(matrices) * sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  const int64_t chunks = matrices * per_matrix / 8;
+  nvfp4_amax_kernel<<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, s>>>(
+      per_matrix / 8, chunks, w, reinterpret_cast<unsigned*>(tensor_scale));
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t blocks = matrices * per_matrix / 16;
+  nvfp4_quant_kernel<<<static_cast<unsigned>((blocks + 255) / 256), 256, 0, s>>>(
+      per_matrix / 16, blocks, w, tensor_scale, q, bscale);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  nvfp4_tscale_kernel<<<static_cast<unsigned>((matrices + 255) / 256), 256, 0, s>>>(matrices,
+                                                                                 tensor_scale);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_fp8(const uint16_t* w, int64_t rows, int cols, uint8_t* q,
                                 float* scales, cudaStream_t s) {
   const int64_t blocks = (rows + 7) / 8;

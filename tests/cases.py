@@ -29,6 +29,10 @@ FRAC_INT8 = 4e-2
 # (one E4M3 step, 2^-3 relative, on one element of a 704- or 2816-long dot product): the
 # int8 bar holds with margin.
 FRAC_FP8 = 4e-2
+# NVFP4 experts (weight-only, R18): the oracle multiplies the same dequantised weights
+# (q * b * t, exact in fp16 before t) as the kernels; the two sides differ by the fp16
+# activations and fp32-vs-fp64 accumulation, as for int8, so the bar of 8-bit weights holds.
+FRAC_NVFP4 = 4e-2
 MIN_GAP = 1e-3
 
 

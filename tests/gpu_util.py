@@ -150,3 +150,48 @@ def fp8_experts(case: cases.Case):
     res = (dev, ex, same)
     _FP8_CACHE.put(key, (case.p, res))
     return res
+
+
+def unpack_nvfp4(q: np.ndarray) -> np.ndarray:
+    """E2M1 codes (one per uint8, natural element order) from the library's packed layout:
+    each little-endian 32-bit word holds 8 consecutive elements, nibbles 0-3 elements 0, 2,
+    4, 6 and nibbles 4-7 elements 1, 3, 5, 7."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    words = q.reshape(*q.shape[:-1], -1, 4).view(np.uint32)[..., 0]   # [..., cols / 8]
+    nib = np.stack([(words >> np.uint32(4 * n)) & np.uint32(0xF) for n in range(8)], axis=-1)
+    order = [0, 4, 1, 5, 2, 6, 3, 7]  # element e sits in nibble order[e]
+    out = nib[..., order].astype(np.uint8)
+    return out.reshape(*q.shape[:-1], q.shape[-1] * 2)
+
+
+_NVFP4_CACHE = cases._Lru(2)
+
+
+def nvfp4_experts(case: cases.Case):
+    """Quantise the case's expert weights to NVFP4 on the GPU (moe_quantize_nvfp4, one
+    matrix per expert) and with the oracle; return (device tensors, oracle.Experts built
+    from the oracle's own codes and scales, whether the two quantisations are identical)."""
+    key = id(case.p)
+    if key in _NVFP4_CACHE and _NVFP4_CACHE[key][0] is case.p:
+        return _NVFP4_CACHE[key][1]
+    dev, host, same = {}, {}, True
+    for name, bname, sname, part in (("w_gate_up", "b_gate_up", "s_gate_up", "gate_up"),
+                                     ("w_down", "b_down", "s_down", "down")):
+        w = case.p[name]
+        E, rows, cols = w.shape
+        q = torch.empty(E, rows, cols // 2, dtype=torch.uint8, device="cuda")
+        b = torch.empty(E, rows, cols // 16, dtype=torch.uint8, device="cuda")
+        t = torch.empty(E, dtype=torch.float32, device="cuda")
+        mf.moe_quantize_nvfp4(to_dev(w), q, b, t)
+        qg, bg, tg = unpack_nvfp4(q.cpu().numpy()), b.cpu().numpy(), t.cpu().numpy()
+        ref = [oracle.quantize_nvfp4(w[e]) for e in range(E)]
+        for e in range(E):
+            qo, bo, to = ref[e]
+            same = same and np.array_equal(qg[e], qo) and np.array_equal(bg[e], bo) and \
+                np.float32(tg[e]).view(np.uint32) == np.float32(to).view(np.uint32)
+        dev[name], dev[bname], dev[sname] = q, b, t
+        host[part] = ref
+    ex = oracle.Experts(nvfp4=host)
+    res = (dev, ex, same)
+    _NVFP4_CACHE.put(key, (case.p, res))
+    return res

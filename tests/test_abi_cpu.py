@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 5
+    assert lib.moe_abi_version() == 6
     for s in range(6):
         assert mf.status_string(s)
     assert mf.status_string(99) == "unknown status"
@@ -155,6 +155,31 @@ def test_every_entry_point_validates(lib):
                                FAKE, mf.workspace_size(mf.Config(**{**CFG.__dict__, "fp8": True}), 8),
                                None) == mf.MOE_ERR_INVALID_ARG
     assert mf.workspace_size(mf.Config(**{**CFG.__dict__, "fp8": True}), 8) > 0
+    # nvfp4 experts need matrix scales and block scales (4-byte aligned); block scales are
+    # refused for the other formats
+    n4 = mf.Config(**{**CFG.__dict__, "nvfp4": True})
+    c4 = ctypes.byref(n4.c())
+    w4 = mf.workspace_size(n4, 8)
+    assert w4 > 0
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE)
+    for bad in (mf.CExpertWeights(FAKE, FAKE, FAKE, FAKE),
+                mf.CExpertWeights(FAKE, FAKE, FAKE, FAKE, FAKE + 2, FAKE),
+                mf.CExpertWeights(FAKE, FAKE, None, FAKE, FAKE, FAKE)):
+        assert lib.moe_ffn_forward(c4, 8, *args, ctypes.byref(bad), FAKE, FAKE, w4,
+                                   None) == mf.MOE_ERR_INVALID_ARG
+    good4 = mf.CExpertWeights(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert lib.moe_ffn_forward(c4, 0, *args, ctypes.byref(good4), FAKE, FAKE, w4, None) == mf.MOE_OK
+    i8c = ctypes.byref(mf.Config(**{**CFG.__dict__, "int8": True}).c())
+    assert lib.moe_ffn_forward(i8c, 8, *args, ctypes.byref(good4), FAKE, FAKE,
+                               mf.workspace_size(mf.Config(**{**CFG.__dict__, "int8": True}), 8),
+                               None) == mf.MOE_ERR_INVALID_ARG
+    assert mf.moe_block_launch_count(n4, 8) == mf.moe_block_launch_count(CFG, 8)
+    q4 = lib.moe_quantize_nvfp4
+    assert q4(FAKE, 2, 4, 24, FAKE, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG   # cols % 16
+    assert q4(FAKE, 2, 0, 32, FAKE, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG   # no rows
+    assert q4(FAKE, 2, 4, 32, FAKE, None, FAKE, None) == mf.MOE_ERR_INVALID_ARG
+    assert q4(FAKE, 2, 4, 32, FAKE + 4, FAKE, FAKE, None) == mf.MOE_ERR_INVALID_ARG  # q align
+    assert q4(FAKE, 0, 4, 32, FAKE, FAKE, FAKE, None) == mf.MOE_OK
     assert lib.moe_check_device_status(None, 256, None) == mf.MOE_ERR_WORKSPACE
 
 

@@ -25,8 +25,15 @@ SHAPES = {
     # the interface limits: H = 6144, E = 256, k = 16, and I = D = 64, where a 128-K step
     # of 8-bit weights is half past the end of K (zero-filled by the tensor maps)
     "limits_T300": synth.Shape(T=300, H=6144, E=256, k=16, I=64, D=64),
+    # the same limits on the weight-streaming kernel of small batches (one K step of the
+    # down matmul: three of its four warps have no steps)
+    "limits_T48": synth.Shape(T=48, H=6144, E=256, k=16, I=64, D=64),
+    # Zipf-skewed routing on the weight-streaming kernel: the busiest experts hold more than
+    # one 32-token chunk, and the dense MLP's 256 tokens are eight chunks
+    "int8_T256_zipf": synth.Shape(T=256, H=2816, E=128, k=8, I=704, D=2112),
 }
-ROUTER_STD = {"limits_T300": 0.3}  # wider router weights, so the gap filter finds rows
+ROUTER_STD = {"limits_T300": 0.3, "limits_T48": 0.3}  # wider router weights (gap filter)
+ZIPF = {"int8_T256_zipf"}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -37,7 +44,7 @@ def _gpu():
 
 
 def _setup(name):
-    c = cases.make_case(SHAPES[name], seed=1234, router_std=ROUTER_STD.get(name))
+    c = cases.make_case(SHAPES[name], seed=1234, zipf=name in ZIPF, router_std=ROUTER_STD.get(name))
     dev8, ex8, same = int8_experts(c)
     layer = dict(device_layer(c))
     layer.update(dev8)
