@@ -231,6 +231,27 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
                                moe_bf16_t* moe_out, void* ws, size_t ws_bytes, void* stream,
                                void* const* stage_events);
 
+/* Chunked prefill over a stack of blocks (the Tenstorrent card's "Configurable knobs":
+ * GEMMA4_CHUNKED_PREFILL, GEMMA4_PREFILL_CHUNK_SIZE 16384 "snapped to 1024, capped at
+ * 32768").  The blocks of one layer stack are chained through the residual (block l's `out`
+ * is block l+1's `x`); the block is row-independent, so a long prompt runs as consecutive
+ * chunks of at most moe_stack_chunk_tokens(chunk_tokens) tokens, every chunk through every
+ * layer, with a workspace sized for one chunk instead of the whole prompt.
+ *   moe_stack_chunk_tokens: the chunk length used for a requested one: rounded down to a
+ *     multiple of 1024, at least 1024, at most 32768.  Host function.
+ *   moe_stack_workspace_size: bytes of workspace for chunks of that length (0 if cfg is
+ *     invalid); 256-byte aligned, zeroed once before first use like the block workspace.
+ *   moe_stack_forward: x [T][H] -> out [T][H] through layers[0..n_layers-1] (host array of
+ *     weight structs; the device pointers inside as for moe_block_forward), chunk after
+ *     chunk on `stream`; x and out must not overlap.  n_layers >= 1.  Errors as for
+ *     moe_block_forward; the first failing call's status is returned. */
+int32_t moe_stack_chunk_tokens(int32_t chunk_tokens);
+size_t moe_stack_workspace_size(const moe_config_t* cfg, int32_t chunk_tokens);
+moe_status_t moe_stack_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
+                               const moe_block_weights_t* layers, int32_t n_layers,
+                               moe_bf16_t* out, int32_t chunk_tokens, void* ws,
+                               size_t ws_bytes, void* stream);
+
 /* Per-output-row symmetric int8 quantisation ("Gemma-4 26B-A4B (MoE, int8 experts)",
  * "How it works": per-channel symmetric INT8 expert weights).
  *   w [rows][cols] bf16 -> q [rows][cols] int8, scales [rows] fp32, computed in fp32:
@@ -293,7 +314,8 @@ const char* moe_status_string(moe_status_t status);
 /* Version of this interface (increases when a signature or a calling contract changes;
  * 2: the workspace is zeroed once by the caller, MOE_BLOCK_EVENTS is 7;
  * 3: moe_wait_selftest; 4: moe_block_launch_count; 5: MOE_W_FP8_E4M3, moe_quantize_fp8;
- * 6: MOE_W_NVFP4, moe_quantize_nvfp4, block-scale fields in moe_expert_weights_t). */
+ * 6: MOE_W_NVFP4, moe_quantize_nvfp4, block-scale fields in moe_expert_weights_t;
+ * 7: moe_stack_chunk_tokens, moe_stack_workspace_size, moe_stack_forward). */
 int32_t moe_abi_version(void);
 
 #ifdef __cplusplus

@@ -34,7 +34,8 @@ ENTRY_POINTS = ("moe_workspace_size", "moe_router", "moe_permute", "moe_permute_
                 "moe_ffn_forward", "dense_mlp_forward", "moe_block_forward",
                 "moe_quantize_int8", "moe_quantize_fp8", "moe_quantize_nvfp4",
                 "moe_check_device_status",
-                "moe_wait_selftest",
+                "moe_wait_selftest", "moe_stack_chunk_tokens", "moe_stack_workspace_size",
+                "moe_stack_forward",
                 "moe_block_launch_count", "moe_status_string", "moe_abi_version")
 PERMUTE_NOALLOC_MAX_PAIRS = 1 << 20
 
@@ -85,6 +86,10 @@ _SIG = {
     "moe_check_device_status": (_I32, [_P, ctypes.c_size_t, _P]),
     "moe_wait_selftest": (_I32, [_P, ctypes.c_size_t, ctypes.c_uint64, _P]),
     "moe_block_launch_count": (_I32, [ctypes.POINTER(CConfig), _I32]),
+    "moe_stack_chunk_tokens": (_I32, [_I32]),
+    "moe_stack_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(CConfig), _I32]),
+    "moe_stack_forward": (_I32, [ctypes.POINTER(CConfig), _I32, _P, ctypes.POINTER(CBlockWeights),
+                                 _I32, _P, _I32, _P, ctypes.c_size_t, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
     "moe_abi_version": (_I32, []),
 }
@@ -284,6 +289,29 @@ def moe_block_forward(cfg, x, weights: BlockWeights, out, ws, moe_out=None, stre
                                  _ptr(moe_out, BF16, "moe_out", True), _ptr(ws, torch.uint8, "ws"),
                                  ws.numel(), _stream(stream), ev)
     _check("moe_block_forward", st)
+
+
+def moe_stack_chunk_tokens(chunk_tokens: int) -> int:
+    """The chunk length moe_stack_forward uses for a requested one (host only)."""
+    return int(lib().moe_stack_chunk_tokens(int(chunk_tokens)))
+
+
+def stack_workspace(cfg: Config, chunk_tokens: int, device=None) -> torch.Tensor:
+    """A zeroed workspace for moe_stack_forward with chunks of chunk_tokens tokens."""
+    n = int(lib().moe_stack_workspace_size(ctypes.byref(cfg.c()), int(chunk_tokens)))
+    if n == 0:
+        raise MoeError("moe_stack_workspace_size", MOE_ERR_INVALID_ARG)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def moe_stack_forward(cfg, x, layers, out, ws, chunk_tokens: int = 16384, stream=None):
+    """x [T][H] through every BlockWeights of `layers` (residual chain), chunk by chunk."""
+    T = x.shape[0]
+    arr = (CBlockWeights * len(layers))(*[l.c for l in layers])
+    st = lib().moe_stack_forward(ctypes.byref(cfg.c()), T, _ptr(x, BF16, "x"), arr, len(layers),
+                                 _ptr(out, BF16, "out"), int(chunk_tokens),
+                                 _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check("moe_stack_forward", st)
 
 
 def moe_quantize_int8(w, q, scales, stream=None):

@@ -172,8 +172,6 @@ struct StreamParams {
   int nprob;
   float* partials;       // split-K partial tiles, [piece][64][8] fp32 (split > 1)
   unsigned* counters;    // split-K arrival counters, one per (tile, chunk); zero between launches
-  unsigned* sched;       // [2] piece counter and finished CTAs, zero between launches;
-                         // launches that may overlap need their own
 };
 // Tiles of 64 weight rows against chunks of 8 tokens; K in items of 128 bytes of a row.
 constexpr int kStreamTileRows = 64, kStreamChunk = 8;

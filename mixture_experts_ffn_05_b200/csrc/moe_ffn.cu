@@ -98,20 +98,20 @@ constexpr int kStreamMaxT = 256;
 
 bool stream_path(const Dims& d) { return d.nvfp4 || (d.int8 && d.T <= kStreamMaxT); }
 
-// K pieces of the weight-streaming kernel's tiles: enough pieces for about three per CTA
-// of the launch (five CTAs per SM assumed), each piece at least four K items long.
+// K pieces of the weight-streaming kernel's tiles.  Pieces are dealt round-robin, so the
+// pieces of both problems of a launch are sized to about the same bytes: about four per CTA
+// of the launch (five CTAs per SM assumed), at least 32 KB and four K items each.
 constexpr int kStreamAssumedCtas = 5 * kAssumedSms;
-
-int stream_split(double units, int items) {
-  if (units <= 0) return 1;
-  const int want = static_cast<int>(std::ceil(3.0 * kStreamAssumedCtas / units));
-  return std::max(1, std::min(want, items / 4));
-}
 
 struct StreamSplits {
   int gu_e, gu_d, dn_e, dn_d;  // gate_up experts / dense, down experts / dense
   int64_t units, pieces;       // upper bounds over the two launches
 };
+
+int stream_split(double tile_bytes, double target, int items) {
+  const int want = static_cast<int>(std::lround(tile_bytes / target));
+  return std::max(1, std::min(want, items / 4));
+}
 
 StreamSplits stream_splits(const Dims& d) {
   StreamSplits ss{};
@@ -121,13 +121,20 @@ StreamSplits stream_splits(const Dims& d) {
   const double exp_chunks = u * std::max(1.0, static_cast<double>(Tk) / std::max(u, 1.0) / kStreamChunk);
   const int tiles_gu_e = 2 * d.I / kStreamTileRows, tiles_gu_d = 2 * d.D / kStreamTileRows;
   const int tiles_dn = d.H / kStreamTileRows;
-  const double units_gu = exp_chunks * tiles_gu_e + dense_chunks * tiles_gu_d;
-  const double units_dn = (exp_chunks + dense_chunks) * tiles_dn;
   const int wt = d.nvfp4 ? kStreamNvfp4 : d.int8 ? kStreamInt8 : kStreamBf16;
-  ss.gu_e = stream_split(units_gu, stream_items(d.H, wt));
-  ss.gu_d = stream_split(units_gu, stream_items(d.H, kStreamBf16));
-  ss.dn_e = stream_split(units_dn, stream_items(d.I, wt));
-  ss.dn_d = stream_split(units_dn, stream_items(d.D, kStreamBf16));
+  // bytes of one tile (64 rows of the full K)
+  const double t_gu_e = 128.0 * kStreamTileRows * stream_items(d.H, wt);
+  const double t_gu_d = 128.0 * kStreamTileRows * stream_items(d.H, kStreamBf16);
+  const double t_dn_e = 128.0 * kStreamTileRows * stream_items(d.I, wt);
+  const double t_dn_d = 128.0 * kStreamTileRows * stream_items(d.D, kStreamBf16);
+  const double gu_bytes = exp_chunks * tiles_gu_e * t_gu_e + dense_chunks * tiles_gu_d * t_gu_d;
+  const double dn_bytes = (exp_chunks * t_dn_e + dense_chunks * t_dn_d) * tiles_dn;
+  const double tgt_gu = std::max(32.0 * 1024, gu_bytes / (4.0 * kStreamAssumedCtas));
+  const double tgt_dn = std::max(32.0 * 1024, dn_bytes / (4.0 * kStreamAssumedCtas));
+  ss.gu_e = stream_split(t_gu_e, tgt_gu, stream_items(d.H, wt));
+  ss.gu_d = stream_split(t_gu_d, tgt_gu, stream_items(d.H, kStreamBf16));
+  ss.dn_e = stream_split(t_dn_e, tgt_dn, stream_items(d.I, wt));
+  ss.dn_d = stream_split(t_dn_d, tgt_dn, stream_items(d.D, kStreamBf16));
   // upper bounds: every non-empty expert has a partial chunk
   const int64_t ch_e = std::min<int64_t>(d.E, Tk) + ceil_div(Tk, kStreamChunk);
   const int64_t ch_d = ceil_div(T, kStreamChunk);
@@ -375,8 +382,6 @@ moe_status_t run_stream_gemms(const Dims& d, const Layout& L, void* ws, const Ge
     P->partials = at<float>(ws, L.partials);
     P->counters = at<unsigned>(ws, L.counters);
   }
-  gu.sched = at<unsigned>(ws, L.sched);
-  dn.sched = at<unsigned>(ws, L.sched) + 2;  // the down launch may start before gate_up ends
   int np = 0;
   if (j.experts) {
     const int wt = d.nvfp4 ? kStreamNvfp4 : kStreamInt8;
@@ -602,7 +607,7 @@ bool w_ok(const moe_expert_weights_t* w, const Dims& d) {
 
 extern "C" {
 
-int32_t moe_abi_version(void) { return 6; }
+int32_t moe_abi_version(void) { return 7; }
 
 int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T) {
   Dims d;
@@ -812,6 +817,53 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
                                              true))) != MOE_OK)
     return st;
   return mark(ev, 6, s) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int32_t moe_stack_chunk_tokens(int32_t chunk_tokens) {
+  constexpr int32_t kSnap = 1024, kMax = 32768;
+  const int32_t c = chunk_tokens / kSnap * kSnap;
+  return std::min(kMax, std::max(kSnap, c));
+}
+
+size_t moe_stack_workspace_size(const moe_config_t* cfg, int32_t chunk_tokens) {
+  Dims d;
+  const int32_t c = moe_stack_chunk_tokens(chunk_tokens);
+  if (check_cfg(cfg, c, &d) != MOE_OK) return 0;
+  // the block's workspace, then two [chunk][H] bf16 buffers for the residual chain
+  const size_t block = align_up(layout_of(d).total, kAlign);
+  return block + 2 * align_up(static_cast<size_t>(c) * d.H * 2, kAlign);
+}
+
+moe_status_t moe_stack_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* x,
+                               const moe_block_weights_t* layers, int32_t n_layers,
+                               moe_bf16_t* out, int32_t chunk_tokens, void* ws,
+                               size_t ws_bytes, void* stream) {
+  Dims d;
+  const int32_t c = moe_stack_chunk_tokens(chunk_tokens);
+  moe_status_t st = check_cfg(cfg, c, &d);
+  if (st != MOE_OK) return st;
+  if (T < 0 || n_layers < 1 || layers == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || out == nullptr || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 ||
+      ws_bytes < moe_stack_workspace_size(cfg, chunk_tokens))
+    return MOE_ERR_WORKSPACE;
+  const size_t block = align_up(layout_of(d).total, kAlign);
+  const size_t buf = align_up(static_cast<size_t>(c) * d.H * 2, kAlign);
+  moe_bf16_t* ping[2] = {at<moe_bf16_t>(ws, block), at<moe_bf16_t>(ws, block + buf)};
+  for (int32_t t0 = 0; t0 < T; t0 += c) {
+    const int32_t n = std::min(c, T - t0);
+    const size_t row0 = static_cast<size_t>(t0) * d.H;
+    const moe_bf16_t* in = x + row0;
+    for (int32_t l = 0; l < n_layers; ++l) {
+      moe_bf16_t* dst = l == n_layers - 1 ? out + row0 : ping[l & 1];
+      // the block's own checks run on every call; its workspace is the first part of ws
+      st = moe_block_forward(cfg, n, in, &layers[l], dst, nullptr, ws, block, stream, nullptr);
+      if (st != MOE_OK) return st;
+      in = dst;
+    }
+  }
+  return MOE_OK;
 }
 
 moe_status_t moe_quantize_int8(const moe_bf16_t* w, int64_t rows, int32_t cols, int8_t* q,

@@ -17,7 +17,7 @@
 // Work: a tile of 64 weight rows of one group against a chunk of up to 8 of its tokens,
 // over a range of K (the tile's K is split into pieces when a launch has too few tiles to
 // keep every SM streaming; the last piece to finish adds the others' fp32 partial sums in
-// piece order, so results do not depend on timing).  CTAs take pieces from a counter.
+// piece order, so results do not depend on timing).  Pieces are dealt round-robin.
 // Inside a CTA, warp w multiplies tile rows 16w .. 16w + 15 (gate_up: 8 gate rows and the
 // 8 matching up rows; down: 16 output rows).
 //
@@ -467,23 +467,10 @@ __device__ __forceinline__ void finish_piece(const StreamParams& P, const Stream
   store_unit(pr, pc, warp, g, t, v);
 }
 
-// Pieces come from the launch's counter in increasing order.  s_q[k % 8] is this CTA's
-// k-th piece.  Thread 0 keeps one request in flight and publishes its result a piece later
-// (no barrier waits for an atomic's round trip); pieces k .. k + 3 are published before the
-// CTA starts piece k, enough for a copy cursor that runs at most three items ahead.
-struct Sched {
-  int* q;             // [8] this CTA's pieces, in order
-  unsigned* counter;  // the launch's piece counter
-  int pending;        // thread 0: the request in flight
-};
-
-// Every thread, once the CTA is done with piece k - 1: thread 0 publishes piece k + 3 and
-// requests the next.  Visible to all after the next barrier.
-__device__ __forceinline__ void sched_advance(Sched& sc, int k) {
-  if (threadIdx.x == 0) {
-    sc.q[(k + 3) & 7] = sc.pending;
-    sc.pending = static_cast<int>(atomicAdd(sc.counter, 1u));
-  }
+// Pieces are dealt round-robin over the launch: the CTA's k-th piece is blockIdx.x +
+// k * gridDim.x (the host sizes the pieces of both problems to about the same bytes).
+__device__ __forceinline__ int cta_piece(int k) {
+  return static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
 }
 
 // The copy side of the ring: walks this CTA's pieces of one problem item by item.
@@ -507,17 +494,15 @@ __device__ __forceinline__ void cursor_set(IssueCursor& c, int piece, const Stre
   }
 }
 
-// Issues the cursor's item and steps past it.  The move to the next piece waits for the
-// next issue: only then is that piece's id sure to be published (the cursor runs up to
-// S - 1 items ahead of the multiply-adds, and piece k + 3 is published when piece k
-// starts).
+// Issues the cursor's item and steps past it (moving to the CTA's next piece at the next
+// issue once the piece is exhausted).
 template <int WT>
 __device__ __forceinline__ void cursor_issue(IssueCursor& c, uint32_t st, const StreamParams& P,
-                                             const StreamProblem& pr, const Tables& tb,
-                                             const Sched& sc, int end, bool weights, bool tokens) {
+                                             const StreamProblem& pr, const Tables& tb, int end,
+                                             bool weights, bool tokens) {
   if (c.next) {
     ++c.k;
-    cursor_set<WT>(c, sc.q[c.k & 7], P, pr, tb, end);
+    cursor_set<WT>(c, cta_piece(c.k), P, pr, tb, end);
   }
   if (c.piece >= end) return;
   issue_item<WT>(st, c.cp, c.pc.it0 + c.item, weights, tokens);
@@ -530,8 +515,7 @@ __device__ __forceinline__ void cursor_issue(IssueCursor& c, uint32_t st, const 
 // Returns the index of the CTA's first piece not handled (of the next problem, or done).
 template <int WT>
 __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k, int end,
-                           const Tables& tb, Sched& sc, uint8_t* ring, bool& waited,
-                           volatile int* flag) {
+                           const Tables& tb, uint8_t* ring, bool& waited, volatile int* flag) {
   constexpr int S = Stage<WT>::kCount;
   constexpr int SB = Stage<WT>::kBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -539,32 +523,32 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
   const int steps_total = pr.K >> 6;
   IssueCursor ic;
   ic.k = k;
-  cursor_set<WT>(ic, sc.q[k & 7], P, pr, tb, end);
+  cursor_set<WT>(ic, cta_piece(k), P, pr, tb, end);
   // prologue: S - 1 items in flight.  Weight copies do not depend on the previous kernel;
   // before the first dependency wait they are issued ahead of the token copies.
   if (!waited) {
     IssueCursor wc = ic;
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q)
-      cursor_issue<WT>(wc, r0 + q * SB, P, pr, tb, sc, end, true, false);
+      cursor_issue<WT>(wc, r0 + q * SB, P, pr, tb, end, true, false);
     pdl_wait();
     waited = true;
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q) {
-      cursor_issue<WT>(ic, r0 + q * SB, P, pr, tb, sc, end, false, true);
+      cursor_issue<WT>(ic, r0 + q * SB, P, pr, tb, end, false, true);
       cp_async_commit();
     }
   } else {
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q) {
-      cursor_issue<WT>(ic, r0 + q * SB, P, pr, tb, sc, end, true, true);
+      cursor_issue<WT>(ic, r0 + q * SB, P, pr, tb, end, true, true);
       cp_async_commit();
     }
   }
   int consumed = 0;
 #pragma unroll 1
   for (;;) {
-    const int piece = sc.q[k & 7];
+    const int piece = cta_piece(k);
     if (piece >= end) break;
     const Piece pc = piece_of(piece, P, tb);
     const int n = pc.it1 - pc.it0;
@@ -573,7 +557,7 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
     for (int i = 0; i < n; ++i) {
       cp_async_wait<S - 2>();  // this thread's copies of the item being consumed have landed
       __syncthreads();         // everyone's have, and everyone is done with the item before
-      cursor_issue<WT>(ic, r0 + ((consumed + S - 1) % S) * SB, P, pr, tb, sc, end, true, true);
+      cursor_issue<WT>(ic, r0 + ((consumed + S - 1) % S) * SB, P, pr, tb, end, true, true);
       cp_async_commit();
       const int it = pc.it0 + i;
       const int nsteps = min(Geo<WT>::kSteps, steps_total - it * Geo<WT>::kSteps);
@@ -584,7 +568,7 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
 #pragma unroll
     for (int q = 0; q < 4; ++q) v[q] = a0[q] + a1[q];
     finish_piece(P, pr, pc, v, flag);
-    sched_advance(sc, ++k);
+    ++k;
   }
   cp_async_wait<0>();
   __syncthreads();  // the ring is free for the next problem
@@ -597,19 +581,11 @@ __global__ void __launch_bounds__(kStreamThreads, 5) stream_gemm_kernel(const St
   __shared__ int upre[kStreamMaxEntries + 1];
   __shared__ int b0s[kStreamMaxEntries];
   __shared__ int ngs[kStreamMaxEntries];
-  __shared__ int s_q[8];
   __shared__ int s_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G0 = P.prob[0].groups;
   const int nent = G0 + (P.nprob > 1 ? P.prob[1].groups : 0);
 
-  // the CTA's first four pieces, and the request for the fifth (the counter does not
-  // depend on the previous kernel)
-  Sched sc{s_q, P.sched, 0};
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < 4; ++i) s_q[i] = static_cast<int>(atomicAdd(sc.counter, 1u));
-    sc.pending = static_cast<int>(atomicAdd(sc.counter, 1u));
-  }
   // ---- the piece table (routing offsets come from kernels that completed before the
   // previous kernel on the stream started); pre/upre first hold the counts
   for (int i = threadIdx.x; i < nent; i += kStreamThreads) {
@@ -666,24 +642,13 @@ __global__ void __launch_bounds__(kStreamThreads, 5) stream_gemm_kernel(const St
     const StreamProblem& pr = P.prob[p];
     const int ue = p == 0 ? u1 : total;
     if (pr.wtype == kStreamInt8)
-      k = run_problem<kStreamInt8>(P, pr, k, ue, tb, sc, s_ring, waited, &s_flag);
+      k = run_problem<kStreamInt8>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
     else if (pr.wtype == kStreamNvfp4)
-      k = run_problem<kStreamNvfp4>(P, pr, k, ue, tb, sc, s_ring, waited, &s_flag);
+      k = run_problem<kStreamNvfp4>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
     else
-      k = run_problem<kStreamBf16>(P, pr, k, ue, tb, sc, s_ring, waited, &s_flag);
+      k = run_problem<kStreamBf16>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
   }
   if (!waited) pdl_wait();
-  // the last CTA to finish returns the piece counter to zero for the next launch (every
-  // CTA's requests, the one in flight included, are done before it counts itself)
-  if (threadIdx.x == 0) {
-    asm volatile("" ::"r"(sc.pending));  // the request in flight has returned
-    __threadfence();
-    if (atomicAdd(P.sched + 1, 1u) == gridDim.x - 1) {
-      P.sched[0] = 0u;
-      P.sched[1] = 0u;
-      __threadfence();
-    }
-  }
 }
 
 int stream_items(int K, int wtype) { return stream_items_of(K, wtype); }
@@ -697,7 +662,6 @@ cudaError_t launch_stream_gemm(const StreamParams& p, int sms, cudaStream_t s, b
     if (pr.split < 1 || pr.split > stream_items_of(pr.K, pr.wtype)) return cudaErrorInvalidValue;
     if (pr.split > 1 && (p.partials == nullptr || p.counters == nullptr)) return cudaErrorInvalidValue;
   }
-  if (p.sched == nullptr) return cudaErrorInvalidValue;
   const int ctas = stream_gemm_ctas(sms);
   if (ctas <= 0) return cudaErrorInvalidValue;
   return launch_k(stream_gemm_kernel, dim3(ctas), dim3(kStreamThreads), kStreamRingBytes, s, pdl, p);

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 6
+    assert lib.moe_abi_version() == 7
     for s in range(6):
         assert mf.status_string(s)
     assert mf.status_string(99) == "unknown status"
@@ -220,3 +220,21 @@ def test_kernel_hash_ignores_comments_only():
     assert bench.strip_comments(a) == bench.strip_comments(b)
     assert "// not a comment" in bench.strip_comments(a)
     assert bench.strip_comments(a) != bench.strip_comments(a.replace("x = 1", "x = 2"))
+
+
+def test_stack_chunk_length(lib):
+    """The chunked prefill's chunk length: a multiple of 1024, at least 1024, at most
+    32768 (the Tenstorrent card's GEMMA4_PREFILL_CHUNK_SIZE rule); the stack workspace
+    holds one chunk's block workspace and two residual buffers."""
+    f = mf.moe_stack_chunk_tokens
+    assert [f(v) for v in (16384, 16385, 17407, 1, 0, -5, 1024, 2047, 40000, 32768)] == \
+        [16384, 16384, 16384, 1024, 1024, 1024, 1024, 1024, 32768, 32768]
+    n = lib.moe_stack_workspace_size(ctypes.byref(CFG.c()), 16384)
+    assert n >= mf.workspace_size(CFG, 16384) + 2 * 16384 * 2816 * 2
+    assert lib.moe_stack_workspace_size(ctypes.byref(CFG.c()), 16384) == \
+        lib.moe_stack_workspace_size(ctypes.byref(CFG.c()), 17000)
+    c = ctypes.byref(CFG.c())
+    arr = (mf.CBlockWeights * 1)()
+    assert lib.moe_stack_forward(c, 8, FAKE, arr, 0, FAKE, 1024, FAKE, n, None) == mf.MOE_ERR_INVALID_ARG
+    assert lib.moe_stack_forward(c, 8, FAKE, arr, 1, FAKE, 1024, FAKE, 1, None) == mf.MOE_ERR_WORKSPACE
+    assert lib.moe_stack_forward(c, 0, FAKE, arr, 1, FAKE, 1024, FAKE, n, None) == mf.MOE_OK
