@@ -37,7 +37,7 @@
  *     only enqueues work on that stream and returns; results are ready when the
  *     stream reaches that point.  Calls on different streams must not share `ws`.
  *   - Size limits: H a multiple of 128 (128..6144), I and D multiples of 64
- *     (64..16384), 1 <= E <= 256, 1 <= k <= min(E, 16), 0 <= T, T*k < 2^31.
+ *     (128..16384), 1 <= E <= 256, 1 <= k <= min(E, 16), 0 <= T, T*k < 2^31.
  *     T = 0 returns MOE_OK at once (before any pointer is checked) and launches
  *     nothing.
  *   - Argument errors are found on the host before anything is launched and

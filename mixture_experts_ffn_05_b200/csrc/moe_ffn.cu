@@ -40,8 +40,10 @@ moe_status_t check_cfg(const moe_config_t* c, int32_t T, Dims* d) {
       c->expert_wdtype != MOE_W_FP8_E4M3 && c->expert_wdtype != MOE_W_NVFP4)
     return MOE_ERR_INVALID_ARG;
   if (c->hidden < 128 || c->hidden > 6144 || c->hidden % 128) return MOE_ERR_UNSUPPORTED;
-  if (c->expert_inter < 64 || c->expert_inter > 16384 || c->expert_inter % 64) return MOE_ERR_UNSUPPORTED;
-  if (c->dense_inter < 64 || c->dense_inter > 16384 || c->dense_inter % 64) return MOE_ERR_UNSUPPORTED;
+  // I, D >= 128: with a 64-wide dense intermediate the bf16 rounding of the GEMM operands
+  // alone can reach the accuracy bar at the largest H, E and k (an emulation over seeds)
+  if (c->expert_inter < 128 || c->expert_inter > 16384 || c->expert_inter % 64) return MOE_ERR_UNSUPPORTED;
+  if (c->dense_inter < 128 || c->dense_inter > 16384 || c->dense_inter % 64) return MOE_ERR_UNSUPPORTED;
   if (c->num_experts < 1 || c->num_experts > 256) return MOE_ERR_UNSUPPORTED;
   if (c->top_k < 1 || c->top_k > 16 || c->top_k > c->num_experts) return MOE_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(T) * c->top_k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;

