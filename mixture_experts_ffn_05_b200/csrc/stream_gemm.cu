@@ -275,25 +275,74 @@ __device__ __forceinline__ void plan_piece(CopyPlan& cp, const StreamProblem& pr
   cp.b_lim = pr.K;
 }
 
+// This thread's byte offsets inside a stage, fixed for the whole kernel (worked out once
+// so that no swizzle arithmetic runs per item): the chunks it reads for each K step of an
+// item (weight rows g and g + 8 of its warp's strip, token g) and the chunks it copies.
+template <int WT>
+struct Offs {
+  uint32_t a[Geo<WT>::kSteps][2][2];  // [step][row g, g + 8][first, second 16-byte chunk]
+  uint32_t b[Geo<WT>::kSteps][2];     // token g: the two chunks of a step
+  uint32_t bs[2];                     // nvfp4: block-scale bytes of rows g and g + 8 (+ 4h + t)
+  uint32_t cpa[4];                    // the 16-byte weight chunks it copies
+  uint32_t cpb[4];                    // the 16-byte token chunks it copies
+  uint32_t cpbs[2];                   // nvfp4: the block-scale words it copies
+};
+
+template <int WT>
+__device__ __forceinline__ Offs<WT> make_offs(int warp, int lane) {
+  using Gm = Geo<WT>;
+  Offs<WT> o;
+  const int g = lane >> 2, t = lane & 3, tid = threadIdx.x;
+  const int r0 = 16 * warp + g, r1 = r0 + 8;
+#pragma unroll
+  for (int h = 0; h < Gm::kSteps; ++h) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int r = rr ? r1 : r0;
+      if constexpr (WT == kStreamBf16) {
+        o.a[h][rr][0] = a_off(r, 2 * t, Gm::kASwz);
+        o.a[h][rr][1] = a_off(r, 2 * t + 1, Gm::kASwz);
+      } else if constexpr (WT == kStreamInt8) {
+        o.a[h][rr][0] = o.a[h][rr][1] = a_off(r, 4 * h + t, Gm::kASwz);
+      } else {  // 8 bytes: bytes [32h + 8t, +8) of the row
+        o.a[h][rr][0] = o.a[h][rr][1] = a_off(r, 2 * h + (t >> 1), Gm::kASwz) + 8 * (t & 1);
+      }
+    }
+    o.b[h][0] = Stage<WT>::kA + b_off(g, 8 * h + 2 * t, Gm::kBRow);
+    o.b[h][1] = Stage<WT>::kA + b_off(g, 8 * h + 2 * t + 1, Gm::kBRow);
+  }
+  o.bs[0] = Stage<WT>::kA + Stage<WT>::kB + r0 * 16 + t;
+  o.bs[1] = Stage<WT>::kA + Stage<WT>::kB + r1 * 16 + t;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) o.cpa[j] = a_off((tid >> 3) + 16 * j, tid & 7, Gm::kASwz);
+  constexpr int kChunks = Gm::kBRow / 16;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int q = tid + j * kStreamThreads;
+    o.cpb[j] = Stage<WT>::kA + b_off(q / kChunks, q % kChunks, Gm::kBRow);
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    o.cpbs[j] = Stage<WT>::kA + Stage<WT>::kB + ((tid >> 2) + 32 * j) * 16 + (tid & 3) * 4;
+  return o;
+}
+
 // Copies of item `it` of the planned piece into the stage at shared address `st`.
 template <int WT>
-__device__ __forceinline__ void issue_item(uint32_t st, const CopyPlan& cp, int it, bool weights,
-                                           bool tokens) {
+__device__ __forceinline__ void issue_item(uint32_t st, const CopyPlan& cp, const Offs<WT>& of,
+                                           int it, bool weights, bool tokens) {
   using Gm = Geo<WT>;
   const int tid = threadIdx.x;
   if (weights) {
     const bool ok = it * 128 < cp.a_lim;
-    const int c = tid & 7;
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      cp_async16(st + a_off((tid >> 3) + 16 * j, c, Gm::kASwz), ok ? cp.a[j] + it * 128 : cp.a[j],
-                 ok ? 16u : 0u);
+      cp_async16(st + of.cpa[j], ok ? cp.a[j] + it * 128 : cp.a[j], ok ? 16u : 0u);
     if constexpr (WT == kStreamNvfp4) {
       const bool okb = it * 16 < cp.bs_lim;
 #pragma unroll
       for (int j = 0; j < 2; ++j)
-        cp_async4(st + Stage<WT>::kA + Stage<WT>::kB + ((tid >> 2) + 32 * j) * 16 + (tid & 3) * 4,
-                  okb ? cp.bs[j] + it * 16 : cp.bs[j], okb ? 4u : 0u);
+        cp_async4(st + of.cpbs[j], okb ? cp.bs[j] + it * 16 : cp.bs[j], okb ? 4u : 0u);
     }
   }
   if (tokens) {
@@ -303,35 +352,31 @@ __device__ __forceinline__ void issue_item(uint32_t st, const CopyPlan& cp, int 
     for (int j = 0; j < (8 * kChunks + kStreamThreads - 1) / kStreamThreads; ++j) {
       const int q = tid + j * kStreamThreads;
       if (q < 8 * kChunks) {
-        const int tk = q / kChunks, ch = q % kChunks;
-        const bool ok = cp.b[j] != nullptr && k0 + ch * 8 < cp.b_lim;
+        const bool ok = cp.b[j] != nullptr && k0 + (q % kChunks) * 8 < cp.b_lim;
         const void* src = ok ? static_cast<const void*>(cp.b[j] + k0) : static_cast<const void*>(cp.a[0]);
-        cp_async16(st + Stage<WT>::kA + b_off(tk, ch, Gm::kBRow), src, ok ? 16u : 0u);
+        cp_async16(st + of.cpb[j], src, ok ? 16u : 0u);
       }
     }
   }
 }
 
-// The fp16/bf16 pairs of step h of the item for lane (g, t) of warp w: rows g (w[0..7])
-// and g + 8 (w[8..15]) of the warp's strip.
+// The fp16/bf16 pairs of step h of the item: rows g (w[0..7]) and g + 8 (w[8..15]) of the
+// warp's strip.
 template <int WT>
-__device__ __forceinline__ void widen(const uint8_t* st, int warp, int g, int t, int h,
+__device__ __forceinline__ void widen(const uint8_t* st, const Offs<WT>& of, int h,
                                       uint32_t (&w)[16]) {
-  using Gm = Geo<WT>;
-  const int r0 = 16 * warp + g, r1 = r0 + 8;
   if constexpr (WT == kStreamBf16) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
-      const int r = rr ? r1 : r0;
-      const uint4 a = *reinterpret_cast<const uint4*>(st + a_off(r, 2 * t, Gm::kASwz));
-      const uint4 b = *reinterpret_cast<const uint4*>(st + a_off(r, 2 * t + 1, Gm::kASwz));
+      const uint4 a = *reinterpret_cast<const uint4*>(st + of.a[h][rr][0]);
+      const uint4 b = *reinterpret_cast<const uint4*>(st + of.a[h][rr][1]);
       w[8 * rr + 0] = a.x; w[8 * rr + 1] = a.y; w[8 * rr + 2] = a.z; w[8 * rr + 3] = a.w;
       w[8 * rr + 4] = b.x; w[8 * rr + 5] = b.y; w[8 * rr + 6] = b.z; w[8 * rr + 7] = b.w;
     }
   } else if constexpr (WT == kStreamInt8) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
-      const uint4 v = *reinterpret_cast<const uint4*>(st + a_off(rr ? r1 : r0, 4 * h + t, Gm::kASwz));
+      const uint4 v = *reinterpret_cast<const uint4*>(st + of.a[h][rr][0]);
       const uint32_t q[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u,
                              v.w ^ 0x80808080u};
 #pragma unroll
@@ -341,14 +386,11 @@ __device__ __forceinline__ void widen(const uint8_t* st, int warp, int g, int t,
       }
     }
   } else {
-    // step h: bytes [32h + 8t, +8) of the row (16 codes), block 4h + t of the item
-    const uint8_t* bs = st + Stage<WT>::kA + Stage<WT>::kB;
+    // step h: 16 codes of each row, block 4h + t of the item
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
-      const int r = rr ? r1 : r0;
-      const uint2 v = *reinterpret_cast<const uint2*>(st + a_off(r, 2 * h + (t >> 1), Gm::kASwz) +
-                                                      8 * (t & 1));
-      const uint32_t b = e4m3_to_f16x2_both(bs[r * 16 + 4 * h + t]);
+      const uint2 v = *reinterpret_cast<const uint2*>(st + of.a[h][rr][0]);
+      const uint32_t b = e4m3_to_f16x2_both(st[of.bs[rr] + 4 * h]);
       const uint32_t words[2] = {v.x, v.y};
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -364,19 +406,17 @@ __device__ __forceinline__ void widen(const uint8_t* st, int warp, int g, int t,
 }
 
 template <int WT>
-__device__ __forceinline__ void consume_item(const uint8_t* st, int nsteps, int warp, int lane,
+__device__ __forceinline__ void consume_item(const uint8_t* st, const Offs<WT>& of, int nsteps,
                                              float (&a0)[4], float (&a1)[4]) {
   using Gm = Geo<WT>;
-  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int h = 0; h < Gm::kSteps; ++h) {
     if (h < nsteps) {
       uint32_t w[16];
-      widen<WT>(st, warp, g, t, h, w);
-      // token g, elements [64h + 16t, +16): chunks 8h + 2t, 8h + 2t + 1 of its row
-      const uint8_t* bb = st + Stage<WT>::kA;
-      const uint4 b0 = *reinterpret_cast<const uint4*>(bb + b_off(g, 8 * h + 2 * t, Gm::kBRow));
-      const uint4 b1 = *reinterpret_cast<const uint4*>(bb + b_off(g, 8 * h + 2 * t + 1, Gm::kBRow));
+      widen<WT>(st, of, h, w);
+      // token g, elements [64h + 16t, +16)
+      const uint4 b0 = *reinterpret_cast<const uint4*>(st + of.b[h][0]);
+      const uint4 b1 = *reinterpret_cast<const uint4*>(st + of.b[h][1]);
       const uint32_t b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
       float(&acc)[4] = (h & 1) ? a1 : a0;  // two chains: consecutive steps do not wait
 #pragma unroll
@@ -497,15 +537,16 @@ __device__ __forceinline__ void cursor_set(IssueCursor& c, int piece, const Stre
 // Issues the cursor's item and steps past it (moving to the CTA's next piece at the next
 // issue once the piece is exhausted).
 template <int WT>
-__device__ __forceinline__ void cursor_issue(IssueCursor& c, uint32_t st, const StreamParams& P,
-                                             const StreamProblem& pr, const Tables& tb, int end,
-                                             bool weights, bool tokens) {
+__device__ __forceinline__ void cursor_issue(IssueCursor& c, uint32_t st, const Offs<WT>& of,
+                                             const StreamParams& P, const StreamProblem& pr,
+                                             const Tables& tb, int end, bool weights,
+                                             bool tokens) {
   if (c.next) {
     ++c.k;
     cursor_set<WT>(c, cta_piece(c.k), P, pr, tb, end);
   }
   if (c.piece >= end) return;
-  issue_item<WT>(st, c.cp, c.pc.it0 + c.item, weights, tokens);
+  issue_item<WT>(st, c.cp, of, c.pc.it0 + c.item, weights, tokens);
   if (++c.item == c.pc.it1 - c.pc.it0) c.next = true;
 }
 
@@ -521,6 +562,7 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t r0 = smem_u32(ring);
   const int steps_total = pr.K >> 6;
+  const Offs<WT> of = make_offs<WT>(warp, lane);
   IssueCursor ic;
   ic.k = k;
   cursor_set<WT>(ic, cta_piece(k), P, pr, tb, end);
@@ -530,18 +572,18 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
     IssueCursor wc = ic;
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q)
-      cursor_issue<WT>(wc, r0 + q * SB, P, pr, tb, end, true, false);
+      cursor_issue<WT>(wc, r0 + q * SB, of, P, pr, tb, end, true, false);
     pdl_wait();
     waited = true;
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q) {
-      cursor_issue<WT>(ic, r0 + q * SB, P, pr, tb, end, false, true);
+      cursor_issue<WT>(ic, r0 + q * SB, of, P, pr, tb, end, false, true);
       cp_async_commit();
     }
   } else {
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q) {
-      cursor_issue<WT>(ic, r0 + q * SB, P, pr, tb, end, true, true);
+      cursor_issue<WT>(ic, r0 + q * SB, of, P, pr, tb, end, true, true);
       cp_async_commit();
     }
   }
@@ -557,11 +599,11 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
     for (int i = 0; i < n; ++i) {
       cp_async_wait<S - 2>();  // this thread's copies of the item being consumed have landed
       __syncthreads();         // everyone's have, and everyone is done with the item before
-      cursor_issue<WT>(ic, r0 + ((consumed + S - 1) % S) * SB, P, pr, tb, end, true, true);
+      cursor_issue<WT>(ic, r0 + ((consumed + S - 1) % S) * SB, of, P, pr, tb, end, true, true);
       cp_async_commit();
       const int it = pc.it0 + i;
       const int nsteps = min(Geo<WT>::kSteps, steps_total - it * Geo<WT>::kSteps);
-      consume_item<WT>(ring + (consumed % S) * SB, nsteps, warp, lane, a0, a1);
+      consume_item<WT>(ring + (consumed % S) * SB, of, nsteps, a0, a1);
       ++consumed;
     }
     float v[4];
