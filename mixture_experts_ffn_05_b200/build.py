@@ -31,7 +31,7 @@ def nvcc() -> str:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     srcs = [os.path.join(PKG, "csrc", s) for s in SOURCES]
-    deps = srcs + [os.path.join(PKG, "csrc", h) for h in ("common.cuh", "internal.h", "permute_impl.cuh")] + [
+    deps = srcs + [os.path.join(PKG, "csrc", h) for h in ("common.cuh", "internal.h", "permute_impl.cuh", "warp_mma.cuh")] + [
         os.path.join(ROOT, "include", "moe_ffn.h")]
     if not force and os.path.exists(LIB):
         t = os.path.getmtime(LIB)

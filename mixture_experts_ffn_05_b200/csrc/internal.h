@@ -166,16 +166,22 @@ struct StreamProblem {
   int out_type;          // kOutBf16, kOutF16 (gate_up: h's format) or kOutF32 (down)
   int out_ld;
   int split;             // pieces per tile along K (1 .. stream_items(K, wtype))
+  int nt;                // tokens per unit in n-tiles of 8 (1 .. stream_max_nt(wtype))
 };
 struct StreamParams {
   StreamProblem prob[2];
   int nprob;
-  float* partials;       // split-K partial tiles, [piece][64][8] fp32 (split > 1)
+  float* partials;       // split-K partial tiles, [piece][64][8 * nt] fp32, problem 0's first
   unsigned* counters;    // split-K arrival counters, one per (tile, chunk); zero between launches
 };
-// Tiles of 64 weight rows against chunks of 8 tokens; K in items of 128 bytes of a row.
+// Tiles of 64 weight rows against chunks of 8 * nt tokens; K in items of 128 bytes of a row.
 constexpr int kStreamTileRows = 64, kStreamChunk = 8;
 int stream_items(int K, int wtype);
+// The widest unit (n-tiles of 8 tokens) a weight format allows: 4 for bf16, 2 for int8,
+// 1 for NVFP4.
+constexpr int stream_max_nt(int wtype) {
+  return wtype == kStreamBf16 ? 4 : wtype == kStreamInt8 ? 2 : 1;
+}
 // CTAs of one launch (a persistent grid of every CTA that fits at once).
 int stream_gemm_ctas(int sms);
 cudaError_t launch_stream_gemm(const StreamParams& p, int sms, cudaStream_t s, bool pdl);

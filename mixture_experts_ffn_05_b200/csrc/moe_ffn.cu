@@ -75,12 +75,16 @@ int choose_bn(const Dims& d) {
 // K pieces per tile: only for the narrowest token tiles (weight-streaming batches), and
 // only when a launch has too few tiles to keep every SM streaming to the end (fewer than
 // kSplitTilesPerSm per SM); the partial sums cost more than the balance gains beyond.
+// Pieces keep about 22 k-steps (each piece costs a partial store and an arrival, and at
+// decode T = 8 pieces of 22 k-steps measured 6% faster for gate_up than pieces of 11),
+// unless that leaves fewer than three pieces per SM.
 constexpr int kSplitTilesPerSm = 8;
 constexpr int kAssumedSms = 148;  // a B200; only shifts the threshold if the GPU differs
 
 int choose_split(int k_steps, int bn, double tiles) {
   if (bn != 16 || tiles >= kSplitTilesPerSm * kAssumedSms) return 1;
-  return std::max(1, std::min(std::min(k_steps, 4), (k_steps + 10) / 11));
+  const int fill = static_cast<int>(std::ceil(3.0 * kAssumedSms / std::max(tiles, 1.0)));
+  return std::max(1, std::min(std::min(k_steps, 4), std::max((k_steps + 21) / 22, fill)));
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -106,8 +110,10 @@ bool stream_path(const Dims& d) { return d.nvfp4 || (d.int8 && d.T <= kStreamMax
 constexpr int kStreamAssumedCtas = 5 * kAssumedSms;
 
 struct StreamSplits {
-  int gu_e, gu_d, dn_e, dn_d;  // gate_up experts / dense, down experts / dense
+  int gu_e, gu_d, dn_e, dn_d;  // K pieces: gate_up experts / dense, down experts / dense
+  int nt_e, nt_d;              // token n-tiles of 8 per unit: experts / dense (both launches)
   int64_t units, pieces;       // upper bounds over the two launches
+  int64_t partial_floats;      // upper bound of the split-K partials of one launch
 };
 
 int stream_split(double tile_bytes, double target, int items) {
@@ -115,15 +121,28 @@ int stream_split(double tile_bytes, double target, int items) {
   return std::max(1, std::min(want, items / 4));
 }
 
+// Token n-tiles per unit for a group of about `mean` tokens: a weight tile is read once
+// per unit, so groups of many tokens take wide units (up to the ring's limit for the
+// weight format: three stages must fit).
+int stream_nt(double mean, int wtype) {
+  const int cap = stream_max_nt(wtype);
+  int nt = 1;
+  while (nt < cap && mean > kStreamChunk * nt) nt *= 2;
+  return nt;
+}
+
 StreamSplits stream_splits(const Dims& d) {
   StreamSplits ss{};
   const int64_t T = d.T, Tk = static_cast<int64_t>(d.T) * d.k;
   const double u = expected_used_experts(d);
-  const double dense_chunks = static_cast<double>(ceil_div(T, kStreamChunk));
-  const double exp_chunks = u * std::max(1.0, static_cast<double>(Tk) / std::max(u, 1.0) / kStreamChunk);
+  const int wt = d.nvfp4 ? kStreamNvfp4 : d.int8 ? kStreamInt8 : kStreamBf16;
+  ss.nt_e = stream_nt(static_cast<double>(Tk) / std::max(u, 1.0), wt);
+  ss.nt_d = stream_nt(static_cast<double>(T), kStreamBf16);
+  const int nc_e = kStreamChunk * ss.nt_e, nc_d = kStreamChunk * ss.nt_d;
+  const double dense_chunks = static_cast<double>(ceil_div(T, nc_d));
+  const double exp_chunks = u * std::max(1.0, static_cast<double>(Tk) / std::max(u, 1.0) / nc_e);
   const int tiles_gu_e = 2 * d.I / kStreamTileRows, tiles_gu_d = 2 * d.D / kStreamTileRows;
   const int tiles_dn = d.H / kStreamTileRows;
-  const int wt = d.nvfp4 ? kStreamNvfp4 : d.int8 ? kStreamInt8 : kStreamBf16;
   // bytes of one tile (64 rows of the full K)
   const double t_gu_e = 128.0 * kStreamTileRows * stream_items(d.H, wt);
   const double t_gu_d = 128.0 * kStreamTileRows * stream_items(d.H, kStreamBf16);
@@ -138,12 +157,16 @@ StreamSplits stream_splits(const Dims& d) {
   ss.dn_e = stream_split(t_dn_e, tgt_dn, stream_items(d.I, wt));
   ss.dn_d = stream_split(t_dn_d, tgt_dn, stream_items(d.D, kStreamBf16));
   // upper bounds: every non-empty expert has a partial chunk
-  const int64_t ch_e = std::min<int64_t>(d.E, Tk) + ceil_div(Tk, kStreamChunk);
-  const int64_t ch_d = ceil_div(T, kStreamChunk);
+  const int64_t ch_e = std::min<int64_t>(d.E, Tk) + ceil_div(Tk, nc_e);
+  const int64_t ch_d = ceil_div(T, nc_d);
   const int64_t u_gu = ch_e * tiles_gu_e + ch_d * tiles_gu_d, u_dn = (ch_e + ch_d) * tiles_dn;
   ss.units = std::max(u_gu, u_dn);
-  ss.pieces = std::max(ch_e * tiles_gu_e * ss.gu_e + ch_d * tiles_gu_d * ss.gu_d,
-                       ch_e * tiles_dn * ss.dn_e + ch_d * tiles_dn * ss.dn_d);
+  const int64_t p_gu_e = ch_e * tiles_gu_e * ss.gu_e, p_gu_d = ch_d * tiles_gu_d * ss.gu_d;
+  const int64_t p_dn_e = ch_e * tiles_dn * ss.dn_e, p_dn_d = ch_d * tiles_dn * ss.dn_d;
+  ss.pieces = std::max(p_gu_e + p_gu_d, p_dn_e + p_dn_d);
+  // partials: [piece][64 rows][8 * nt tokens] fp32, problem by problem
+  ss.partial_floats = kStreamTileRows * std::max(p_gu_e * nc_e + p_gu_d * nc_d,
+                                                 p_dn_e * nc_e + p_dn_d * nc_d);
   return ss;
 }
 
@@ -183,8 +206,7 @@ Layout layout_of(const Dims& d) {
     L.ss = stream_splits(d);
     pieces = std::max(pieces, L.ss.units);
     const bool ssplit = L.ss.gu_e > 1 || L.ss.gu_d > 1 || L.ss.dn_e > 1 || L.ss.dn_d > 1;
-    if (ssplit)
-      partial_bytes = std::max<int64_t>(partial_bytes, L.ss.pieces * kStreamTileRows * kStreamChunk * 4);
+    if (ssplit) partial_bytes = std::max<int64_t>(partial_bytes, L.ss.partial_floats * 4);
     any_split = any_split || ssplit;
   }
   const int nb = permute_blocks(static_cast<int>(Tk));
@@ -392,23 +414,24 @@ moe_status_t run_stream_gemms(const Dims& d, const Layout& L, void* ws, const Ge
     a.K = d.H; a.rows = 2 * d.I; a.F = d.I; a.w = j.w_gate_up; a.wscale = j.s_gate_up;
     a.bscale = j.b_gate_up;
     a.b = static_cast<const uint16_t*>(j.a_rows); a.out = h; a.out_type = kOutF16; a.out_ld = d.I;
-    a.split = L.ss.gu_e;
+    a.split = L.ss.gu_e; a.nt = L.ss.nt_e;
     StreamProblem& b = dn.prob[np];
     b.kind = 1; b.wtype = wt; b.groups = d.E; b.offsets = j.offsets; b.n_tokens = Tk;
     b.K = d.I; b.rows = d.H; b.F = d.H; b.w = j.w_down; b.wscale = j.s_down; b.bscale = j.b_down;
     b.b = h; b.out = j.y; b.out_type = kOutF16; b.out_ld = d.H;
-    b.split = L.ss.dn_e;
+    b.split = L.ss.dn_e; b.nt = L.ss.nt_e;
     ++np;
   }
   if (j.dense) {
     StreamProblem& a = gu.prob[np];
     a.kind = 0; a.wtype = kStreamBf16; a.groups = 1; a.offsets = nullptr; a.n_tokens = d.T;
     a.K = d.H; a.rows = 2 * d.D; a.F = d.D; a.w = j.w_dgu; a.b = j.xn_dense; a.out = hd;
-    a.out_type = kOutBf16; a.out_ld = d.D; a.split = L.ss.gu_d;
+    a.out_type = kOutBf16; a.out_ld = d.D; a.split = L.ss.gu_d; a.nt = L.ss.nt_d;
     StreamProblem& b = dn.prob[np];
     b.kind = 1; b.wtype = kStreamBf16; b.groups = 1; b.offsets = nullptr; b.n_tokens = d.T;
     b.K = d.D; b.rows = d.H; b.F = d.H; b.w = j.w_dd; b.b = hd; b.out = j.dense_out;
     b.out_type = j.dense_f32 ? kOutF32 : kOutBf16; b.out_ld = d.H; b.split = L.ss.dn_d;
+    b.nt = L.ss.nt_d;
     ++np;
   }
   gu.nprob = dn.nprob = np;

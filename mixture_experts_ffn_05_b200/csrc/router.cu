@@ -1,4 +1,5 @@
-// Router of the MoE block and the pre norms of both branches, in one launch.
+// Router of the MoE block and the pre norms of both branches, in one launch (batches of
+// up to 128 tokens; larger ones take the tensor-memory router, router_tc.cu).
 //
 // Follows the router of the ONNX export card ("Truthful graph contracts", Router row):
 // scale-free RMSNorm -> learned scale x hidden_size^-0.5 -> linear to E logits ->
@@ -6,23 +7,32 @@
 // the pre norms of the MoE and dense branches, so the kernel also writes
 // xn_moe = xhat * g_pre_moe and xn_dense = xhat * g_pre_dense.
 //
-// Grid (token blocks of 8, expert slices).  Every CTA stages its 8 tokens in shared
-// memory as z' = x * scale * H^-0.5 (fp32) in the same pass that sums x^2, and computes
-// the logits of its expert slice as (z' . W_r[e]) / rms(x): the norm factor is a
-// per-token scalar, so it can be applied after the dot product.  Each warp owns one
-// eighth of H for all experts of the slice, and the eight partial sums are added in
-// warp order.  The last CTA of a token block to finish (an
-// atomic counter) takes the top-k of its 8 tokens.  When asked, the last token block to
-// finish then runs the token-to-expert counting sort for the whole batch, so a decode
-// step routes and sorts in a single launch.  Counters reset themselves after use.
+// Grid (token blocks of 8, expert slices of EB <= 8), sized to about one CTA per SM.  A
+// CTA copies its W_r rows and the router scale into shared memory with bulk copies
+// before the dependency wait (weights do not come from an earlier kernel), then its
+// token rows.  The norm factor 1/rms(x) is a per-token scalar, so the logits are
+// rinv * (x . W'[e]) + b[e] with W' = scale * W_r * H^-0.5 formed in fp32.  The dot
+// products run on mma.sync (m16n8k16, bf16 operands, fp32 accumulation) with W' split
+// into two bf16 terms, W' = hi + lo + d, |d| <= 2^-16 |W'| (the split of the
+// tensor-memory router): A rows 0..7 hold hi of the slice's experts, rows 8..15 lo, B
+// the 8 tokens as they are, so every product is exact and the two halves of the
+// accumulator add up to the logit.  Warp w takes every 16th K step, and the 16 partial
+// sums are added in warp order; the same pass sums x^2 per token.  Every expert slice
+// writes its share of the columns of xn_moe and xn_dense.  The last slice of a token
+// block to finish (an acq_rel counter) takes the top-k of its 8 tokens; when asked, the
+// last token block then runs the token-to-expert counting sort for the whole batch, so
+// a decode step routes and sorts in one launch.  Counters reset themselves after use.
 #include "common.cuh"
 #include "internal.h"
+#include "warp_mma.cuh"
 #include "permute_impl.cuh"
 
 namespace moe {
 
-constexpr int kRT = 8;        // tokens per CTA
-constexpr int kRThreads = 256;
+constexpr int kRT = 8;          // tokens per CTA (the MMA's N)
+constexpr int kRThreads = 512;  // 16 warps
+constexpr int kRWarps = kRThreads / 32;
+constexpr int kRMaxEB = 8;      // experts per CTA (the MMA's M holds hi and lo of each)
 
 // Orderable 64-bit key of (logit, expert): a larger key is a larger logit, and for equal
 // logits a smaller expert id.  NaN sorts below every number.
@@ -41,23 +51,25 @@ __device__ __forceinline__ float key_logit(unsigned long long key) {
 
 // Top-k of one token's logits (ties to the lower expert id), then the softmax restricted
 // to the selected experts (the full-softmax denominator cancels in the renormalisation),
-// then per_expert_scale.  One warp: each lane sorts its (up to 8) candidates, then each
-// of the k rounds takes the warp maximum of the lanes' best remaining keys.
+// then per_expert_scale.  One warp: each lane sorts its KPL candidates (experts lane +
+// 32 i), then each of the k rounds takes the warp maximum of the lanes' best remaining
+// keys, high word first, then the low word among the lanes that share it.
+template <int KPL>
 __device__ void topk_one_token(int t, int E, int k, const float* logits, const uint16_t* pes,
                                int* __restrict__ topk_idx, float* __restrict__ topk_w,
                                int* s_ids = nullptr) {
   const int lane = threadIdx.x & 31;
-  unsigned long long key[8];
+  unsigned long long key[KPL];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < KPL; ++i) {
     const int e = lane + 32 * i;
     key[i] = (e < E) ? topk_key(__ldcg(logits + static_cast<size_t>(t) * E + e), e) : 0ull;
   }
-  // sort the lane's 8 keys in descending order (odd-even transposition, registers only)
+  // sort the lane's keys in descending order (odd-even transposition, registers only)
 #pragma unroll
-  for (int r = 0; r < 8; ++r)
+  for (int r = 0; r < KPL; ++r)
 #pragma unroll
-    for (int i = r & 1; i + 1 < 8; i += 2)
+    for (int i = r & 1; i + 1 < KPL; i += 2)
       if (key[i] < key[i + 1]) {
         const unsigned long long tmp = key[i];
         key[i] = key[i + 1];
@@ -65,16 +77,14 @@ __device__ void topk_one_token(int t, int E, int k, const float* logits, const u
       }
   unsigned long long mine = 0ull;  // lane j keeps the j-th selected key
   for (int j = 0; j < k; ++j) {
-    unsigned long long best = key[0];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-      best = other > best ? other : best;
-    }
+    const uint32_t hi = static_cast<uint32_t>(key[0] >> 32);
+    const uint32_t bh = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t bl = __reduce_max_sync(0xffffffffu, hi == bh ? static_cast<uint32_t>(key[0]) : 0u);
+    const unsigned long long best = (static_cast<unsigned long long>(bh) << 32) | bl;
     if (key[0] == best) {  // keys are unique: exactly one lane pops its head
 #pragma unroll
-      for (int i = 0; i < 7; ++i) key[i] = key[i + 1];
-      key[7] = 0ull;
+      for (int i = 0; i + 1 < KPL; ++i) key[i] = key[i + 1];
+      key[KPL - 1] = 0ull;
     }
     if (lane == j) mine = best;
   }
@@ -140,260 +150,207 @@ struct RouterArgs {
   float* topk_w;
   unsigned* counters;  // [token blocks + 1], zero on entry, zero again on exit
   unsigned* status;    // device status word (a bounded wait that ran out)
-  int stage_w;         // copy the slice's W_r rows to shared memory first
   // counting sort of all T*k pairs by the last token block (NULL = not here)
   int* offsets;
   int* sorted_src;
   int* inv_pos;
 };
 
-// Narrow expert slices (EB <= kStageEB) copy their W_r rows into shared memory with 1-D
-// bulk copies at the start, overlapping the pass over x.
-constexpr int kStageEB = 4;
+// Two floats rounded to bf16 (nearest even), the first in the low half.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 
 template <int EB>
-__global__ void __launch_bounds__(kRThreads) router_kernel(const RouterArgs a) {
-  extern __shared__ __align__(16) float z[];  // [kRT][H], then (narrow slices) W_r rows
-  __shared__ float part[8][EB * kRT];
+__global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a) {
+  extern __shared__ __align__(128) uint8_t r_smem[];  // x rows [8][H], W_r rows [EB][H], scale [H]
+  __shared__ float part[kRWarps][kRMaxEB][kRT];
+  __shared__ float ssp[kRWarps][kRT];
+  __shared__ float rinv[kRT];
   __shared__ int flag;
-  __shared__ __align__(8) uint64_t wbar;
+  __shared__ __align__(8) uint64_t bar;
   __shared__ uint16_t s_pes[kPermMaxE];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = threadIdx.x; e < a.E; e += kRThreads) s_pes[e] = a.pes[e];
+  __shared__ int s_ids[kRT * 16];
+  __shared__ PermuteSmem<kRThreads> ps;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
   const int H = a.H, E = a.E;
-  const int t0 = blockIdx.x * kRT;
-  const int nch = H >> 3;  // chunks of 8 values
-  const bool stage_w = a.stage_w != 0;
-  uint16_t* wsm = reinterpret_cast<uint16_t*>(z + kRT * H);  // [EB][H] bf16
-  if (stage_w && threadIdx.x == 0) {
-    // W_r is a weight (not produced by an earlier kernel), so it is fetched before the
-    // dependency wait
-    mbar_init(&wbar, 1);
+  const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * EB;
+  const int nt = min(kRT, a.T - t0);  // tokens of the block
+  const int ne = min(EB, E - e0);     // experts of the slice
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(r_smem);
+  uint16_t* wsm = xs + kRT * H;
+  uint16_t* ssc = wsm + EB * H;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
     mbar_fence_init();
-    mbar_arrive_expect_tx(&wbar, EB * H * 2);
-    for (int i = 0; i < EB; ++i) {
-      const int e = min(blockIdx.y * EB + i, E - 1);
-      bulk_load_1d(wsm + i * H, a.wr + static_cast<size_t>(e) * H, H * 2, &wbar);
-    }
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(ne + 1 + nt) * row_bytes);
+    for (int i = 0; i < ne; ++i)
+      bulk_load_1d(wsm + i * H, a.wr + static_cast<size_t>(e0 + i) * H, row_bytes, &bar);
+    bulk_load_1d(ssc, a.rscale, row_bytes, &bar);
+  }
+  for (int e = tid; e < E; e += kRThreads) s_pes[e] = a.pes[e];
+  // this slice's share of the pre-norm columns: chunks [cb, ce) of 8 values, for each token
+  const int nch = H >> 3;
+  const int cb = static_cast<int>(static_cast<int64_t>(blockIdx.y) * nch / gridDim.y);
+  const int ce = static_cast<int>(static_cast<int64_t>(blockIdx.y + 1) * nch / gridDim.y);
+  const int nc = ce - cb, npairs = nc * nt;
+  uint4 gm0 = make_uint4(0u, 0u, 0u, 0u), gd0 = gm0;  // the gains of the first pair, early
+  if (tid < npairs) {
+    gm0 = __ldg(reinterpret_cast<const uint4*>(a.gm) + cb + tid % nc);
+    gd0 = __ldg(reinterpret_cast<const uint4*>(a.gd) + cb + tid % nc);
   }
   pdl_wait();
   pdl_trigger();
+  if (tid == 0) {
+    for (int i = 0; i < nt; ++i)
+      bulk_load_1d(xs + i * H, a.x + static_cast<size_t>(t0 + i) * H, row_bytes, &bar);
+    flag = mbar_wait(&bar, 0, 2000000000ull, nullptr) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!flag) {  // the copies did not land in time: report it, leave the outputs alone
+    if (tid == 0) record_status(a.status, kStatusTimeout);
+    return;
+  }
 
-  // ---- one pass over the CTA's tokens: z' = x * scale * H^-0.5 (the norm factor
-  // 1/rms(x) is a per-token scalar, applied to the logits at the end) and sum(x^2)
-  __shared__ float rinv[kRT];
+  // ---- logits of the slice and sum(x^2): warp w takes K steps w, w + 16, ...; lane (g, t)
+  // takes elements [16 s + 4t, +4) of step s (a permutation of K applied to both operands)
   {
-    const int t = t0 + warp;
-    float* zt = z + warp * H;
-    if (t < a.T) {
-      const uint4* xr = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * H);
-      const uint4* sr = reinterpret_cast<const uint4*>(a.rscale);
-      float ss = 0.f;
-      for (int c0 = lane; c0 < nch; c0 += 32 * 4) {
-        uint4 vx[4], vs[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {  // 8 loads in flight per lane
-          const int c = min(c0 + 32 * u, nch - 1);
-          vx[u] = __ldg(xr + c);
-          vs[u] = __ldg(sr + c);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = c0 + 32 * u;
-          if (c < nch) {
-            float f[8], sc[8];
-            unpack8(vx[u], f);
-            unpack8(vs[u], sc);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
-            float4* zz = reinterpret_cast<float4*>(zt + c * 8);
-            zz[0] = make_float4(f[0] * sc[0] * a.inv_sqrt_h, f[1] * sc[1] * a.inv_sqrt_h,
-                                f[2] * sc[2] * a.inv_sqrt_h, f[3] * sc[3] * a.inv_sqrt_h);
-            zz[1] = make_float4(f[4] * sc[4] * a.inv_sqrt_h, f[5] * sc[5] * a.inv_sqrt_h,
-                                f[6] * sc[6] * a.inv_sqrt_h, f[7] * sc[7] * a.inv_sqrt_h);
-          }
-        }
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    float ss = 0.f;
+    const bool xok = g < nt, wok = g < ne;
+    const uint16_t* xr = xs + g * H + 4 * t;
+    const uint16_t* wr = wsm + g * H + 4 * t;
+    const uint16_t* sr = ssc + 4 * t;
+    const float ish = a.inv_sqrt_h;
+#pragma unroll 2
+    for (int st = warp; st < (H >> 4); st += kRWarps) {
+      const int k0 = st * 16;
+      uint2 xv = make_uint2(0u, 0u);
+      if (xok) xv = *reinterpret_cast<const uint2*>(xr + k0);
+      const float x0 = bf16lo(xv.x), x1 = bf16hi(xv.x), x2 = bf16lo(xv.y), x3 = bf16hi(xv.y);
+      ss = fmaf(x0, x0, ss);
+      ss = fmaf(x1, x1, ss);
+      ss = fmaf(x2, x2, ss);
+      ss = fmaf(x3, x3, ss);
+      uint32_t h01 = 0u, h23 = 0u, l01 = 0u, l23 = 0u;
+      if (wok) {
+        const uint2 wv = *reinterpret_cast<const uint2*>(wr + k0);
+        const uint2 sv = *reinterpret_cast<const uint2*>(sr + k0);
+        const float v0 = bf16lo(wv.x) * bf16lo(sv.x) * ish, v1 = bf16hi(wv.x) * bf16hi(sv.x) * ish;
+        const float v2 = bf16lo(wv.y) * bf16lo(sv.y) * ish, v3 = bf16hi(wv.y) * bf16hi(sv.y) * ish;
+        h01 = cvt_bf16x2(v0, v1);
+        h23 = cvt_bf16x2(v2, v3);
+        l01 = cvt_bf16x2(v0 - bf16lo(h01), v1 - bf16hi(h01));
+        l23 = cvt_bf16x2(v2 - bf16lo(h23), v3 - bf16hi(h23));
       }
-      ss = warp_sum(ss);
-      if (lane == 0) rinv[warp] = 1.0f / sqrtf(ss / static_cast<float>(H) + a.eps);
-    } else {
-      for (int i = lane; i < H; i += 32) zt[i] = 0.f;
-      if (lane == 0) rinv[warp] = 0.f;
+      mma16816<true>(c, h01, l01, h23, l23, xv.x, xv.y);
     }
+    // C rows g (hi) and g + 8 (lo) of expert g, columns (tokens) 2t and 2t + 1
+    if (g < EB) {
+      part[warp][g][2 * t] = c[0] + c[2];
+      part[warp][g][2 * t + 1] = c[1] + c[3];
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    if (t == 0) ssp[warp][g] = ss;
   }
   __syncthreads();
-
-  // ---- logits of the slice: warp w sums its eighth of H, 4 experts x 8 tokens at a time
-  const int e0 = blockIdx.y * EB;
-  const int cb = warp * nch / 8, ce = (warp + 1) * nch / 8;
-  if (stage_w) {
-    if (threadIdx.x == 0) flag = mbar_wait(&wbar, 0, 2000000000ull, nullptr) ? 1 : 0;
-    __syncthreads();
-    if (!flag) {  // the copy did not land in time: report it, leave the outputs alone
-      if (threadIdx.x == 0) record_status(a.status, kStatusTimeout);
-      return;
+  if (tid < EB * kRT) {
+    const int e = tid / kRT, tl = tid % kRT;
+    float sq = 0.f, dot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRWarps; ++w) {
+      sq += ssp[w][tl];
+      dot += part[w][e][tl];
     }
-  }
-#pragma unroll 1
-  for (int g = 0; g < EB / 4; ++g) {
-    float acc[4][kRT];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int t = 0; t < kRT; ++t) acc[i][t] = 0.f;
-    const uint4* wrow[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = min(e0 + 4 * g + i, E - 1);
-      wrow[i] = stage_w ? reinterpret_cast<const uint4*>(wsm + (4 * g + i) * H)
-                        : reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H);
-    }
-    for (int c0 = cb + lane; c0 < ce; c0 += 64) {
-      uint4 wv[2][4];
-#pragma unroll
-      for (int u = 0; u < 2; ++u)  // both chunks' weights in flight before any math
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = min(c0 + 32 * u, ce - 1);
-          wv[u][i] = stage_w ? wrow[i][c] : __ldg(wrow[i] + c);
-        }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = c0 + 32 * u;
-        if (c < ce) {
-          float w[4][8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) unpack8(wv[u][i], w[i]);
-#pragma unroll
-          for (int t = 0; t < kRT; ++t) {
-            const float4* zz = reinterpret_cast<const float4*>(z + t * H + c * 8);
-            const float4 z0 = zz[0], z1 = zz[1];
-            const float zv[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-              for (int q = 0; q < 8; ++q) acc[i][t] = fmaf(w[i][q], zv[q], acc[i][t]);
-          }
-        }
-      }
-    }
-    // transpose-reduce the 32 sums over the warp: after 5 halving steps (31 shuffles)
-    // lane l holds the full sum of value index l = i * 8 + t
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int t = 0; t < kRT; ++t) v[i * kRT + t] = acc[i][t];
-#pragma unroll
-    for (int w = 16; w >= 1; w >>= 1) {
-      const bool upper = (lane & w) != 0;
-#pragma unroll
-      for (int j = 0; j < w; ++j) {
-        const float send = upper ? v[j] : v[j + w];
-        const float keep = upper ? v[j + w] : v[j];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-      }
-    }
-    // lane l now holds value index l (the halving kept bit b of the index where bit b of
-    // the lane is set)
-    part[warp][4 * g * kRT + lane] = v[0];
+    const float r = 1.0f / sqrtf(sq / static_cast<float>(H) + a.eps);
+    if (e == 0) rinv[tl] = r;
+    if (e < ne && tl < nt)
+      a.logits[static_cast<size_t>(t0 + tl) * E + e0 + e] = dot * r + (a.bias ? a.bias[e0 + e] : 0.f);
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < EB * kRT; j += kRThreads) {
-    const int e = e0 + j / kRT, tl = j % kRT, t = t0 + tl;
-    if (e < E && t < a.T) {
-      float sm = 0.f;
+  // ---- the slice's share of the pre norms of both branches
+  for (int j = tid; j < npairs; j += kRThreads) {
+    const int c = cb + j % nc, tl = j / nc;
+    float f[8], gm[8], gd[8], o1[8], o2[8];
+    unpack8(*reinterpret_cast<const uint4*>(xs + tl * H + c * 8), f);
+    unpack8(j == tid ? gm0 : __ldg(reinterpret_cast<const uint4*>(a.gm) + c), gm);
+    unpack8(j == tid ? gd0 : __ldg(reinterpret_cast<const uint4*>(a.gd) + c), gd);
+    const float r = rinv[tl];
 #pragma unroll
-      for (int w = 0; w < 8; ++w) sm += part[w][j];
-      a.logits[static_cast<size_t>(t) * E + e] = sm * rinv[tl] + (a.bias ? a.bias[e] : 0.f);
+    for (int i = 0; i < 8; ++i) {
+      const float xh = f[i] * r;
+      o1[i] = xh * gm[i];
+      o2[i] = xh * gd[i];
     }
+    reinterpret_cast<uint4*>(a.xn_moe + static_cast<size_t>(t0 + tl) * H)[c] = pack8(o1);
+    reinterpret_cast<uint4*>(a.xn_dense + static_cast<size_t>(t0 + tl) * H)[c] = pack8(o2);
   }
 
-  // ---- the last slice of this token block takes the top-k
+  // ---- the last slice of this token block takes the top-k.  The barrier orders every
+  // thread's logits before the elected thread's atomic, whose acq_rel also acquires the
+  // other slices' logits for the last one.
   __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned old = atomicAdd(a.counters + blockIdx.x, 1u);
+  if (tid == 0) {
+    const unsigned old = atom_add_acq_rel_gpu(a.counters + blockIdx.x, 1u);
     flag = old == gridDim.y - 1;
-    if (flag) {
-      a.counters[blockIdx.x] = 0u;
-      __threadfence();
-    }
-  }
-  // ---- every expert slice writes its share of the pre norms of both branches:
-  // columns [y, y + gridDim.y, ...) in chunks of 8, for the CTA's tokens
-  {
-    const int t = t0 + warp;
-    if (t < a.T) {
-      const float r = rinv[warp];
-      const uint4* xr = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * H);
-      for (int c = blockIdx.y + gridDim.y * lane; c < nch; c += gridDim.y * 32) {
-        float f[8], gm[8], gd[8], o1[8], o2[8];
-        unpack8(__ldg(xr + c), f);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(a.gm) + c), gm);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(a.gd) + c), gd);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float xh = f[i] * r;
-          o1[i] = xh * gm[i];
-          o2[i] = xh * gd[i];
-        }
-        reinterpret_cast<uint4*>(a.xn_moe + static_cast<size_t>(t) * H)[c] = pack8(o1);
-        reinterpret_cast<uint4*>(a.xn_dense + static_cast<size_t>(t) * H)[c] = pack8(o2);
-      }
-    }
+    if (flag) a.counters[blockIdx.x] = 0u;
   }
   __syncthreads();
   if (!flag) return;
-  __shared__ int s_ids[kRT * 16];
   const bool small_sort = a.offsets != nullptr && gridDim.x == 1;  // every pair is here
-  if (t0 + warp < a.T)
-    topk_one_token(t0 + warp, E, a.k, a.logits, s_pes, a.topk_idx, a.topk_w,
-                   small_sort ? s_ids : nullptr);
+  if (warp < nt) {
+    if (E <= 128)
+      topk_one_token<4>(t0 + warp, E, a.k, a.logits, s_pes, a.topk_idx, a.topk_w,
+                        small_sort ? s_ids : nullptr);
+    else
+      topk_one_token<8>(t0 + warp, E, a.k, a.logits, s_pes, a.topk_idx, a.topk_w,
+                        small_sort ? s_ids : nullptr);
+  }
   if (a.offsets == nullptr) return;
   if (small_sort) {
-    __shared__ int s_wcnt[4][kPermMaxE];
-    __shared__ int s_tot[kPermMaxE];
-    __shared__ int s_off[kPermMaxE + 1];
     __syncthreads();
-    sort_small(a.T * a.k, E, s_ids, s_wcnt, s_tot, s_off, a.offsets, a.sorted_src, a.inv_pos);
+    sort_small(a.T * a.k, E, s_ids, ps.wcnt, ps.cnt, ps.off, a.offsets, a.sorted_src, a.inv_pos);
     return;
   }
 
   // ---- the last token block sorts every (token, slot) pair by expert
   __syncthreads();
-  if (gridDim.x > 1) {
-    if (threadIdx.x == 0) {
-      __threadfence();
-      const unsigned old = atomicAdd(a.counters + gridDim.x, 1u);
-      flag = old == gridDim.x - 1;
-      if (flag) {
-        a.counters[gridDim.x] = 0u;
-        __threadfence();
-      }
-    }
-    __syncthreads();
-    if (!flag) return;
+  if (tid == 0) {
+    const unsigned old = atom_add_acq_rel_gpu(a.counters + gridDim.x, 1u);
+    flag = old == gridDim.x - 1;
+    if (flag) a.counters[gridDim.x] = 0u;
   }
-  __shared__ PermuteSmem<kRThreads> ps;
+  __syncthreads();
+  if (!flag) return;
   permute_block<kRThreads>(a.T * a.k, E, a.topk_idx, a.offsets, a.sorted_src, a.inv_pos, ps);
+}
+
+// Dynamic shared memory of a CTA with EB experts.
+static size_t router_smem(int H, int EB) { return static_cast<size_t>(kRT + EB + 1) * H * 2; }
+
+// Experts per CTA: about one CTA per SM (token blocks x expert slices), within the
+// shared-memory budget.
+static int router_eb(int T, int H, int E) {
+  const int tb = (T + kRT - 1) / kRT;
+  int eb = 1;
+  while (eb < kRMaxEB && tb * ((E + eb - 1) / eb) > 160) eb *= 2;
+  while (eb > 1 && router_smem(H, eb) > 176 * 1024) eb /= 2;
+  return eb;
 }
 
 template <int EB>
 static cudaError_t launch_eb(const RouterArgs& a, cudaStream_t s, bool pdl) {
-  const size_t zbytes = static_cast<size_t>(kRT) * a.H * sizeof(float);
-  const size_t wbytes = static_cast<size_t>(EB) * a.H * 2;
-  RouterArgs b = a;
-  b.stage_w = (EB <= kStageEB && zbytes + wbytes <= 160 * 1024) ? 1 : 0;
-  const size_t smem = zbytes + (b.stage_w ? wbytes : 0);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(router_kernel<EB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
+  const size_t smem = router_smem(a.H, EB);
+  cudaError_t e = cudaFuncSetAttribute(router_kernel<EB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
   dim3 grid((a.T + kRT - 1) / kRT, (a.E + EB - 1) / EB);
-  return launch_k(router_kernel<EB>, grid, dim3(kRThreads), smem, s, pdl, b);
+  return launch_k(router_kernel<EB>, grid, dim3(kRThreads), smem, s, pdl, a);
 }
 
 int router_counters(int T) { return (T + kRT - 1) / kRT + 1; }
@@ -407,11 +364,13 @@ cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t*
                           int* sorted_src, int* inv_pos, cudaStream_t s, bool pdl) {
   RouterArgs a{T, H, E, k, eps, 1.0f / sqrtf(static_cast<float>(H)), x, router_scale, w_router,
                bias, per_expert_scale, g_pre_moe, g_pre_dense, xn_moe, xn_dense, logits,
-               topk_idx, topk_w, counters, status, 0, offsets, sorted_src, inv_pos};
-  // Narrow expert slices for small batches (more CTAs streaming W_r), wide ones for
-  // large batches (fewer redundant normalisations).
-  if (T <= 64) return launch_eb<4>(a, s, pdl);
-  return launch_eb<32>(a, s, pdl);
+               topk_idx, topk_w, counters, status, offsets, sorted_src, inv_pos};
+  switch (router_eb(T, H, E)) {
+    case 1: return launch_eb<1>(a, s, pdl);
+    case 2: return launch_eb<2>(a, s, pdl);
+    case 4: return launch_eb<4>(a, s, pdl);
+    default: return launch_eb<8>(a, s, pdl);
+  }
 }
 
 }  // namespace moe

@@ -9,7 +9,7 @@
 //     l[t,e] = rinv[t] * sum_h x[t,h] * W'[e,h] + bias[e],   W'[e,h] = s[h] W_r[e,h] / sqrt(H)
 // with rinv[t] = 1 / sqrt(mean_h x[t,h]^2 + eps).  x is bf16 and goes to the tensor cores
 // as it is.  W' is fp32; a preparation kernel splits it into two bf16 matrices,
-// W' = W'hi + W'lo + d with |d| <= 2^-18 |W'|, and the kernel accumulates x.W'hi and
+// W' = W'hi + W'lo + d with |d| <= 2^-16 |W'|, and the kernel accumulates x.W'hi and
 // x.W'lo into the same fp32 accumulator, so the logits carry the accuracy of an fp32 dot
 // product (every bf16 x bf16 product is exact in fp32).
 //

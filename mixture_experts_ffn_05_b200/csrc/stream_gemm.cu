@@ -14,7 +14,8 @@
 // waits per k-step.  Here the codes are widened to fp16 in registers and fed to mma.sync
 // (m16n8k16, fp32 accumulation), which at decode sizes has tensor throughput to spare.
 //
-// Work: a tile of 64 weight rows of one group against a chunk of up to 8 of its tokens,
+// Work: a tile of 64 weight rows of one group against a chunk of up to 8 nt of its tokens
+// (nt n-tiles of 8: groups of many tokens read each weight tile once per wide unit),
 // over a range of K (the tile's K is split into pieces when a launch has too few tiles to
 // keep every SM streaming; the last piece to finish adds the others' fp32 partial sums in
 // piece order, so results do not depend on timing).  Pieces are dealt round-robin.
@@ -46,6 +47,7 @@
 //     2^14 and the matrix scale multiply the fp32 sum.  Tokens are fp16.
 #include "common.cuh"
 #include "internal.h"
+#include "warp_mma.cuh"
 
 namespace moe {
 
@@ -56,25 +58,6 @@ constexpr int kStreamMaxEntries = 258;
 constexpr int kStreamRingBytes = 40 * 1024;
 
 // ---- operand widening helpers
-
-// D += A B (m16n8k16, fp32 accumulators), fp16 or bf16 operands.
-template <bool BF16>
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  if constexpr (BF16) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-  } else {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-  }
-}
 
 // Two int8 codes of a word of biased codes (q + 128) -> fp16x2 (see grouped_gemm.cu).
 __device__ __forceinline__ uint32_t s_i8x2_f16x2(uint32_t biased, uint32_t sel) {
@@ -150,10 +133,10 @@ struct Geo<kStreamNvfp4> {
   static constexpr int kBs = kStreamRows * 16;
   static constexpr int kASwz = 2;
 };
-template <int WT>
+template <int WT, int NT>
 struct Stage {
   static constexpr int kA = kStreamRows * 128;
-  static constexpr int kB = 8 * Geo<WT>::kBRow;
+  static constexpr int kB = 8 * NT * Geo<WT>::kBRow;
   static constexpr int kBytes = kA + kB + Geo<WT>::kBs;
   static constexpr int kCount = kStreamRingBytes / kBytes;
   static_assert(kCount >= 3, "ring too small");
@@ -172,7 +155,7 @@ struct Piece {
   int tok0, n_valid;      // token rows of the chunk
   int it0, it1;           // K items of the piece
   int unit;               // (tile, chunk) index for the split-K counters
-  int first_piece;        // piece id of split 0 of this unit
+  int64_t part0;          // float offset of split 0's partial tile of this unit
 };
 
 struct Tables {
@@ -205,18 +188,23 @@ __device__ __forceinline__ Piece piece_of(int piece, const StreamParams& P, cons
   const StreamProblem& pr = P.prob[pc.p];
   const int local = piece - tb.pre[i];
   const int tiles = pr.rows / kStreamRows;
-  const int split = pr.split;
+  const int split = pr.split, nc = kStreamChunk * pr.nt;
   pc.s = local % split;
   const int ul = local / split;          // unit within the entry: chunk-major
   pc.m = ul % tiles;
   pc.c = ul / tiles;
-  pc.tok0 = tb.b0s[i] + pc.c * 8;
-  pc.n_valid = min(8, tb.ngs[i] - pc.c * 8);
+  pc.tok0 = tb.b0s[i] + pc.c * nc;
+  pc.n_valid = min(nc, tb.ngs[i] - pc.c * nc);
   const int items = stream_items_of(pr.K, pr.wtype);
   pc.it0 = pc.s * items / split;
   pc.it1 = (pc.s + 1) * items / split;
   pc.unit = tb.upre[i] + ul;
-  pc.first_piece = piece - pc.s;
+  // partial tiles [piece][64][nc] fp32, problem 0's pieces first
+  const int first = piece - pc.s;
+  const int p0end = tb.pre[tb.G0];
+  pc.part0 = pc.p == 0 ? static_cast<int64_t>(first) * kStreamRows * nc
+                       : static_cast<int64_t>(p0end) * kStreamRows * kStreamChunk * P.prob[0].nt +
+                             static_cast<int64_t>(first - p0end) * kStreamRows * nc;
   return pc;
 }
 
@@ -241,7 +229,7 @@ struct CopyPlan {
   int b_lim;             // elements of a token row
 };
 
-template <int WT>
+template <int WT, int NT>
 __device__ __forceinline__ void plan_piece(CopyPlan& cp, const StreamProblem& pr, const Piece& pc) {
   using Gm = Geo<WT>;
   const int tid = threadIdx.x;
@@ -268,7 +256,7 @@ __device__ __forceinline__ void plan_piece(CopyPlan& cp, const StreamProblem& pr
   for (int j = 0; j < 4; ++j) {
     const int q = tid + j * kStreamThreads;
     const int tk = q / kChunks, ch = q % kChunks;
-    cp.b[j] = (q < 8 * kChunks && tk < pc.n_valid)
+    cp.b[j] = (q < 8 * NT * kChunks && tk < pc.n_valid)
                   ? pr.b + static_cast<size_t>(pc.tok0 + tk) * pr.K + ch * 8
                   : nullptr;
   }
@@ -288,7 +276,7 @@ struct Offs {
   uint32_t cpbs[2];                   // nvfp4: the block-scale words it copies
 };
 
-template <int WT>
+template <int WT, int NT>
 __device__ __forceinline__ Offs<WT> make_offs(int warp, int lane) {
   using Gm = Geo<WT>;
   Offs<WT> o;
@@ -308,27 +296,27 @@ __device__ __forceinline__ Offs<WT> make_offs(int warp, int lane) {
         o.a[h][rr][0] = o.a[h][rr][1] = a_off(r, 2 * h + (t >> 1), Gm::kASwz) + 8 * (t & 1);
       }
     }
-    o.b[h][0] = Stage<WT>::kA + b_off(g, 8 * h + 2 * t, Gm::kBRow);
-    o.b[h][1] = Stage<WT>::kA + b_off(g, 8 * h + 2 * t + 1, Gm::kBRow);
+    o.b[h][0] = Stage<WT, NT>::kA + b_off(g, 8 * h + 2 * t, Gm::kBRow);
+    o.b[h][1] = Stage<WT, NT>::kA + b_off(g, 8 * h + 2 * t + 1, Gm::kBRow);
   }
-  o.bs[0] = Stage<WT>::kA + Stage<WT>::kB + r0 * 16 + t;
-  o.bs[1] = Stage<WT>::kA + Stage<WT>::kB + r1 * 16 + t;
+  o.bs[0] = Stage<WT, NT>::kA + Stage<WT, NT>::kB + r0 * 16 + t;
+  o.bs[1] = Stage<WT, NT>::kA + Stage<WT, NT>::kB + r1 * 16 + t;
 #pragma unroll
   for (int j = 0; j < 4; ++j) o.cpa[j] = a_off((tid >> 3) + 16 * j, tid & 7, Gm::kASwz);
   constexpr int kChunks = Gm::kBRow / 16;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int q = tid + j * kStreamThreads;
-    o.cpb[j] = Stage<WT>::kA + b_off(q / kChunks, q % kChunks, Gm::kBRow);
+    o.cpb[j] = Stage<WT, NT>::kA + b_off(q / kChunks, q % kChunks, Gm::kBRow);
   }
 #pragma unroll
   for (int j = 0; j < 2; ++j)
-    o.cpbs[j] = Stage<WT>::kA + Stage<WT>::kB + ((tid >> 2) + 32 * j) * 16 + (tid & 3) * 4;
+    o.cpbs[j] = Stage<WT, NT>::kA + Stage<WT, NT>::kB + ((tid >> 2) + 32 * j) * 16 + (tid & 3) * 4;
   return o;
 }
 
 // Copies of item `it` of the planned piece into the stage at shared address `st`.
-template <int WT>
+template <int WT, int NT>
 __device__ __forceinline__ void issue_item(uint32_t st, const CopyPlan& cp, const Offs<WT>& of,
                                            int it, bool weights, bool tokens) {
   using Gm = Geo<WT>;
@@ -349,9 +337,9 @@ __device__ __forceinline__ void issue_item(uint32_t st, const CopyPlan& cp, cons
     constexpr int kChunks = Gm::kBRow / 16;
     const int k0 = it * 64 * Gm::kSteps;
 #pragma unroll
-    for (int j = 0; j < (8 * kChunks + kStreamThreads - 1) / kStreamThreads; ++j) {
+    for (int j = 0; j < (8 * NT * kChunks + kStreamThreads - 1) / kStreamThreads; ++j) {
       const int q = tid + j * kStreamThreads;
-      if (q < 8 * kChunks) {
+      if (q < 8 * NT * kChunks) {
         const bool ok = cp.b[j] != nullptr && k0 + (q % kChunks) * 8 < cp.b_lim;
         const void* src = ok ? static_cast<const void*>(cp.b[j] + k0) : static_cast<const void*>(cp.a[0]);
         cp_async16(st + of.cpb[j], src, ok ? 16u : 0u);
@@ -405,32 +393,38 @@ __device__ __forceinline__ void widen(const uint8_t* st, const Offs<WT>& of, int
   }
 }
 
-template <int WT>
+// One item against the unit's NT n-tiles: the weights are widened once per step and feed
+// every n-tile (token g + 8n of the chunk).  With one n-tile, consecutive steps alternate
+// between two accumulator sets, so that an MMA does not wait for the previous one.
+template <int WT, int NT>
 __device__ __forceinline__ void consume_item(const uint8_t* st, const Offs<WT>& of, int nsteps,
-                                             float (&a0)[4], float (&a1)[4]) {
+                                             float (&acc)[NT + (NT == 1)][4]) {
   using Gm = Geo<WT>;
 #pragma unroll
   for (int h = 0; h < Gm::kSteps; ++h) {
     if (h < nsteps) {
       uint32_t w[16];
       widen<WT>(st, of, h, w);
-      // token g, elements [64h + 16t, +16)
-      const uint4 b0 = *reinterpret_cast<const uint4*>(st + of.b[h][0]);
-      const uint4 b1 = *reinterpret_cast<const uint4*>(st + of.b[h][1]);
-      const uint32_t b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-      float(&acc)[4] = (h & 1) ? a1 : a0;  // two chains: consecutive steps do not wait
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        mma16816<WT == kStreamBf16>(acc, w[2 * j], w[8 + 2 * j], w[2 * j + 1], w[8 + 2 * j + 1],
-                                    b[2 * j], b[2 * j + 1]);
+      for (int n = 0; n < NT; ++n) {
+        // token g + 8n, elements [64h + 16t, +16)
+        const uint4 b0 = *reinterpret_cast<const uint4*>(st + of.b[h][0] + n * 8 * Gm::kBRow);
+        const uint4 b1 = *reinterpret_cast<const uint4*>(st + of.b[h][1] + n * 8 * Gm::kBRow);
+        const uint32_t b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        float(&c)[4] = acc[NT == 1 ? (h & 1) : n];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma16816<WT == kStreamBf16>(c, w[2 * j], w[8 + 2 * j], w[2 * j + 1], w[8 + 2 * j + 1],
+                                      b[2 * j], b[2 * j + 1]);
+      }
     }
   }
 }
 
-// The epilogue of one unit from its (full-K) sums v: lane (g, t) of warp w holds rows g and
-// g + 8 of strip w for tokens 2t and 2t + 1 of the chunk.
+// The epilogue of n-tile n of one unit from its (full-K) sums v: lane (g, t) of warp w
+// holds rows g and g + 8 of strip w for tokens 8n + 2t and 8n + 2t + 1 of the chunk.
 __device__ __forceinline__ void store_unit(const StreamProblem& pr, const Piece& pc, int warp,
-                                           int g, int t, const float (&v)[4]) {
+                                           int g, int t, int n, const float (&v)[4]) {
   const int r0 = 16 * warp + g;
   const int wr0 = weight_row(pr, pc.m, r0), wr1 = weight_row(pr, pc.m, r0 + 8);
   const size_t grow = static_cast<size_t>(pc.gg) * pr.rows;
@@ -444,7 +438,7 @@ __device__ __forceinline__ void store_unit(const StreamProblem& pr, const Piece&
   }
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
-    const int col = 2 * t + q;
+    const int col = 8 * n + 2 * t + q;
     if (col >= pc.n_valid) continue;
     const size_t pos = static_cast<size_t>(pc.tok0 + col);
     if (pr.kind == 0) {  // row r0: gate of feature wr0, row r0 + 8: its up row
@@ -468,19 +462,25 @@ __device__ __forceinline__ void store_unit(const StreamProblem& pr, const Piece&
   }
 }
 
-// The end of one piece: its partial sum, or (unsplit tiles, and the last piece of a split
-// tile) the full sum and the epilogue.  All threads of the CTA.
+// The end of one piece: its partial sums, or (unsplit tiles, and the last piece of a split
+// tile) the full sums and the epilogue.  All threads of the CTA.
+template <int NT>
 __device__ __forceinline__ void finish_piece(const StreamParams& P, const StreamProblem& pr,
-                                             const Piece& pc, float (&v)[4], volatile int* flag) {
+                                             const Piece& pc, float (&v)[NT][4], volatile int* flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
+  constexpr int NC = kStreamChunk * NT;
   if (pr.split > 1) {
-    // partial tile [64 rows][8 tokens] fp32: lane (g, t) of warp w writes rows 16w + g and
-    // 16w + g + 8, tokens 2t and 2t + 1
-    float* part = P.partials + static_cast<size_t>(pc.first_piece + pc.s) * (kStreamRows * 8);
+    // partial tile [64 rows][NC tokens] fp32: lane (g, t) of warp w writes rows 16w + g and
+    // 16w + g + 8, tokens 8n + 2t and 8n + 2t + 1
+    float* part = P.partials + pc.part0 + static_cast<int64_t>(pc.s) * (kStreamRows * NC);
     const int r = 16 * warp + g;
-    __stcg(reinterpret_cast<float2*>(part + r * 8 + 2 * t), make_float2(v[0], v[1]));
-    __stcg(reinterpret_cast<float2*>(part + (r + 8) * 8 + 2 * t), make_float2(v[2], v[3]));
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      __stcg(reinterpret_cast<float2*>(part + r * NC + 8 * n + 2 * t), make_float2(v[n][0], v[n][1]));
+      __stcg(reinterpret_cast<float2*>(part + (r + 8) * NC + 8 * n + 2 * t),
+             make_float2(v[n][2], v[n][3]));
+    }
     // one release for the CTA: the barrier orders every thread's partial before the
     // elected thread's atomic, whose acq_rel also acquires the other pieces' partials
     __syncthreads();
@@ -496,15 +496,21 @@ __device__ __forceinline__ void finish_piece(const StreamParams& P, const Stream
     if (!last) return;
     // the last piece: every piece's partial, added in piece order
 #pragma unroll
-    for (int q = 0; q < 4; ++q) v[q] = 0.f;
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[n][q] = 0.f;
     for (int s2 = 0; s2 < pr.split; ++s2) {
-      const float* pp = P.partials + static_cast<size_t>(pc.first_piece + s2) * (kStreamRows * 8);
-      const float2 x = __ldcg(reinterpret_cast<const float2*>(pp + r * 8 + 2 * t));
-      const float2 y = __ldcg(reinterpret_cast<const float2*>(pp + (r + 8) * 8 + 2 * t));
-      v[0] += x.x; v[1] += x.y; v[2] += y.x; v[3] += y.y;
+      const float* pp = P.partials + pc.part0 + static_cast<int64_t>(s2) * (kStreamRows * NC);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(pp + r * NC + 8 * n + 2 * t));
+        const float2 y = __ldcg(reinterpret_cast<const float2*>(pp + (r + 8) * NC + 8 * n + 2 * t));
+        v[n][0] += x.x; v[n][1] += x.y; v[n][2] += y.x; v[n][3] += y.y;
+      }
     }
   }
-  store_unit(pr, pc, warp, g, t, v);
+#pragma unroll
+  for (int n = 0; n < NT; ++n) store_unit(pr, pc, warp, g, t, n, v[n]);
 }
 
 // Pieces are dealt round-robin over the launch: the CTA's k-th piece is blockIdx.x +
@@ -522,7 +528,7 @@ struct IssueCursor {
   CopyPlan cp;
 };
 
-template <int WT>
+template <int WT, int NT>
 __device__ __forceinline__ void cursor_set(IssueCursor& c, int piece, const StreamParams& P,
                                            const StreamProblem& pr, const Tables& tb, int end) {
   c.piece = piece;
@@ -530,23 +536,23 @@ __device__ __forceinline__ void cursor_set(IssueCursor& c, int piece, const Stre
   c.next = false;
   if (piece < end) {
     c.pc = piece_of(piece, P, tb);
-    plan_piece<WT>(c.cp, pr, c.pc);
+    plan_piece<WT, NT>(c.cp, pr, c.pc);
   }
 }
 
 // Issues the cursor's item and steps past it (moving to the CTA's next piece at the next
 // issue once the piece is exhausted).
-template <int WT>
+template <int WT, int NT>
 __device__ __forceinline__ void cursor_issue(IssueCursor& c, uint32_t st, const Offs<WT>& of,
                                              const StreamParams& P, const StreamProblem& pr,
                                              const Tables& tb, int end, bool weights,
                                              bool tokens) {
   if (c.next) {
     ++c.k;
-    cursor_set<WT>(c, cta_piece(c.k), P, pr, tb, end);
+    cursor_set<WT, NT>(c, cta_piece(c.k), P, pr, tb, end);
   }
   if (c.piece >= end) return;
-  issue_item<WT>(st, c.cp, of, c.pc.it0 + c.item, weights, tokens);
+  issue_item<WT, NT>(st, c.cp, of, c.pc.it0 + c.item, weights, tokens);
   if (++c.item == c.pc.it1 - c.pc.it0) c.next = true;
 }
 
@@ -554,36 +560,36 @@ __device__ __forceinline__ void cursor_issue(IssueCursor& c, uint32_t st, const 
 // one ring that runs S - 1 items ahead continuously, across piece boundaries: the next
 // piece's first copies are in flight while a piece's partial sums are exchanged and stored.
 // Returns the index of the CTA's first piece not handled (of the next problem, or done).
-template <int WT>
+template <int WT, int NT>
 __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k, int end,
                            const Tables& tb, uint8_t* ring, bool& waited, volatile int* flag) {
-  constexpr int S = Stage<WT>::kCount;
-  constexpr int SB = Stage<WT>::kBytes;
+  constexpr int S = Stage<WT, NT>::kCount;
+  constexpr int SB = Stage<WT, NT>::kBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t r0 = smem_u32(ring);
   const int steps_total = pr.K >> 6;
-  const Offs<WT> of = make_offs<WT>(warp, lane);
+  const Offs<WT> of = make_offs<WT, NT>(warp, lane);
   IssueCursor ic;
   ic.k = k;
-  cursor_set<WT>(ic, cta_piece(k), P, pr, tb, end);
+  cursor_set<WT, NT>(ic, cta_piece(k), P, pr, tb, end);
   // prologue: S - 1 items in flight.  Weight copies do not depend on the previous kernel;
   // before the first dependency wait they are issued ahead of the token copies.
   if (!waited) {
     IssueCursor wc = ic;
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q)
-      cursor_issue<WT>(wc, r0 + q * SB, of, P, pr, tb, end, true, false);
+      cursor_issue<WT, NT>(wc, r0 + q * SB, of, P, pr, tb, end, true, false);
     pdl_wait();
     waited = true;
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q) {
-      cursor_issue<WT>(ic, r0 + q * SB, of, P, pr, tb, end, false, true);
+      cursor_issue<WT, NT>(ic, r0 + q * SB, of, P, pr, tb, end, false, true);
       cp_async_commit();
     }
   } else {
 #pragma unroll 1
     for (int q = 0; q < S - 1; ++q) {
-      cursor_issue<WT>(ic, r0 + q * SB, of, P, pr, tb, end, true, true);
+      cursor_issue<WT, NT>(ic, r0 + q * SB, of, P, pr, tb, end, true, true);
       cp_async_commit();
     }
   }
@@ -594,22 +600,28 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
     if (piece >= end) break;
     const Piece pc = piece_of(piece, P, tb);
     const int n = pc.it1 - pc.it0;
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[NT + (NT == 1)][4];
+#pragma unroll
+    for (int n = 0; n < NT + (NT == 1); ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
 #pragma unroll 1
     for (int i = 0; i < n; ++i) {
       cp_async_wait<S - 2>();  // this thread's copies of the item being consumed have landed
       __syncthreads();         // everyone's have, and everyone is done with the item before
-      cursor_issue<WT>(ic, r0 + ((consumed + S - 1) % S) * SB, of, P, pr, tb, end, true, true);
+      cursor_issue<WT, NT>(ic, r0 + ((consumed + S - 1) % S) * SB, of, P, pr, tb, end, true, true);
       cp_async_commit();
       const int it = pc.it0 + i;
       const int nsteps = min(Geo<WT>::kSteps, steps_total - it * Geo<WT>::kSteps);
-      consume_item<WT>(ring + (consumed % S) * SB, of, nsteps, a0, a1);
+      consume_item<WT, NT>(ring + (consumed % S) * SB, of, nsteps, acc);
       ++consumed;
     }
-    float v[4];
+    float v[NT][4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) v[q] = a0[q] + a1[q];
-    finish_piece(P, pr, pc, v, flag);
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[n][q] = NT == 1 ? acc[0][q] + acc[NT == 1 ? 1 : 0][q] : acc[n][q];
+    finish_piece<NT>(P, pr, pc, v, flag);
     ++k;
   }
   cp_async_wait<0>();
@@ -644,7 +656,8 @@ __global__ void __launch_bounds__(kStreamThreads, 5) stream_gemm_kernel(const St
     }
     b0s[i] = s0;
     ngs[i] = n;
-    const int units = (pr.rows / kStreamRows) * ((n + 7) / 8);
+    const int nc = kStreamChunk * pr.nt;
+    const int units = (pr.rows / kStreamRows) * ((n + nc - 1) / nc);
     upre[i] = units;
     pre[i] = units * pr.split;
   }
@@ -683,12 +696,21 @@ __global__ void __launch_bounds__(kStreamThreads, 5) stream_gemm_kernel(const St
     if (p >= P.nprob) break;
     const StreamProblem& pr = P.prob[p];
     const int ue = p == 0 ? u1 : total;
-    if (pr.wtype == kStreamInt8)
-      k = run_problem<kStreamInt8>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
-    else if (pr.wtype == kStreamNvfp4)
-      k = run_problem<kStreamNvfp4>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
-    else
-      k = run_problem<kStreamBf16>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
+    if (pr.wtype == kStreamInt8) {
+      if (pr.nt == 2)
+        k = run_problem<kStreamInt8, 2>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
+      else
+        k = run_problem<kStreamInt8, 1>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
+    } else if (pr.wtype == kStreamNvfp4) {
+      k = run_problem<kStreamNvfp4, 1>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
+    } else {
+      if (pr.nt == 4)
+        k = run_problem<kStreamBf16, 4>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
+      else if (pr.nt == 2)
+        k = run_problem<kStreamBf16, 2>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
+      else
+        k = run_problem<kStreamBf16, 1>(P, pr, k, ue, tb, s_ring, waited, &s_flag);
+    }
   }
   if (!waited) pdl_wait();
 }
@@ -702,6 +724,8 @@ cudaError_t launch_stream_gemm(const StreamParams& p, int sms, cudaStream_t s, b
     if (pr.wtype == kStreamNvfp4 && pr.bscale == nullptr) return cudaErrorInvalidValue;
     if (pr.wtype != kStreamBf16 && pr.wscale == nullptr) return cudaErrorInvalidValue;
     if (pr.split < 1 || pr.split > stream_items_of(pr.K, pr.wtype)) return cudaErrorInvalidValue;
+    if (pr.nt != 1 && pr.nt != 2 && pr.nt != 4) return cudaErrorInvalidValue;
+    if (pr.nt > stream_max_nt(pr.wtype)) return cudaErrorInvalidValue;
     if (pr.split > 1 && (p.partials == nullptr || p.counters == nullptr)) return cudaErrorInvalidValue;
   }
   const int ctas = stream_gemm_ctas(sms);

@@ -39,7 +39,6 @@ SHAPES = {
     "limits_T300": (synth.Shape(T=300, H=6144, E=256, k=16, I=128, D=128), False),
 }
 FAST = ["tiny", "tiny_T37", "tiny_T1", "decode_T8", "decode_T1", "decode_T64"]
-TC_ROUTER_MIN_T = 128  # larger batches take the tensor-core router
 
 
 def _case(name):
@@ -65,16 +64,14 @@ def test_router(name):
     o = oracle_block(c)
     assert np.array_equal(r["topk_idx"].cpu().numpy(), o["topk_idx"])
     got_w = r["topk_w"].cpu().numpy().astype(np.float64)
-    rtol = np.full((c.shape.T, 1), 2e-6)
-    if c.shape.T > TC_ROUTER_MIN_T:
-        # The tensor-core router adds 2H/16 products of 16 terms into one fp32 accumulator;
-        # each addition may lose up to one unit in the last place of the accumulator
-        # (nothing promises round-to-nearest inside the tensor core), so a logit may be off
-        # by steps * 2^-23 * max|l - b| and a weight, exp(l_j - l_0) / sum, by four times
-        # that, relatively.
-        lraw = np.abs(o["logits"] - (0.0 if c.bias is None else c.bias[None, :]))
-        steps = 2 * c.shape.H / 16
-        rtol = rtol + 4 * steps * 2.0 ** -23 * lraw.max(axis=1, keepdims=True)
+    # Both routers take the logits from tensor-core sums of the two-term split of W'
+    # (2H/16 products of 16 terms into one fp32 accumulator); each addition may lose up to
+    # one unit in the last place of the accumulator (nothing promises round-to-nearest
+    # inside the tensor core), so a logit may be off by steps * 2^-23 * max|l - b| and a
+    # weight, exp(l_j - l_0) / sum, by four times that, relatively.
+    lraw = np.abs(o["logits"] - (0.0 if c.bias is None else c.bias[None, :]))
+    steps = 2 * c.shape.H / 16
+    rtol = 2e-6 + 4 * steps * 2.0 ** -23 * lraw.max(axis=1, keepdims=True)
     err = np.abs(got_w - o["topk_w"]) / np.abs(o["topk_w"])
     assert np.all(err <= rtol), f"topk_w: worst {err.max():.3g} over {rtol.max():.3g}"
     for nm in ("xn_moe", "xn_dense"):
@@ -93,7 +90,7 @@ def test_permute_bit_exact(T, k, E):
     # skewed ids: some experts empty, some hot
     p = rng.zipf(1.3, size=(T, k)) % E
     idx = p.astype(np.int32)
-    cfg = mf.Config(512, E, k, 64, 64)
+    cfg = mf.Config(512, E, k, 128, 128)
     got = run_permute(cfg, to_dev(idx, torch.int32))
     offs, src, inv = oracle.permute(idx, E)
     n = T * k
@@ -104,7 +101,7 @@ def test_permute_bit_exact(T, k, E):
 
 def test_permute_drops_invalid_ids():
     idx = np.array([[3, -1], [16, 3], [0, 2]], dtype=np.int32)  # E = 16: -1 and 16 invalid
-    cfg = mf.Config(512, 16, 2, 64, 64)
+    cfg = mf.Config(512, 16, 2, 128, 128)
     got = run_permute(cfg, to_dev(idx, torch.int32))
     flat = idx.reshape(-1)
     valid = np.nonzero((flat >= 0) & (flat < 16))[0]
@@ -172,6 +169,31 @@ def test_block_at_the_limits_over_seeds(seed):
     w1 = cases.check_bar(bf16_np(out), o["out"], cases.FRAC_BF16, f"out limits seed {seed}")
     w2 = cases.check_bar(bf16_np(moe), o["moe"], cases.FRAC_BF16, f"moe_out limits seed {seed}")
     print("limits seed", seed, w1, w2)
+
+
+def test_block_extreme_skew_T16384():
+    """Every token of a 16384-token batch routed to the same 8 experts (a logit offset of
+    43..50 on experts 0..7, far above the logits' spread): 16384 tokens per expert, 64
+    tiles of 256 tokens each, 120 experts with no token.  The ids must be exactly 0..7 in
+    offset order for every token, and sampled rows (first, last, and spread over the
+    batch) must meet the bar against the oracle block."""
+    shape = synth.Shape(T=16384, H=2816, E=128, k=8, I=704, D=2112)
+    base = cases.make_case(synth.DECODE, seed=1234)          # the layer's weights
+    bias = np.zeros(shape.E, dtype=np.float32)
+    bias[:8] = 50.0 - np.arange(8, dtype=np.float32)
+    x = synth.x_rows(4242, shape.H, shape.T)
+    c = cases.Case(shape, x, base.p, bias, 4242)
+    cfg = config(shape)
+    layer = device_layer(c)
+    T = shape.T
+    xd = to_dev(x)
+    r = run_router(cfg, c, layer, x=xd)
+    assert torch.equal(r["topk_idx"].cpu(), torch.arange(8, dtype=torch.int32).repeat(T, 1))
+    out, moe = run_block(cfg, c, layer, x=xd)
+    rows = np.unique(np.concatenate([[0, 1, T - 1], np.linspace(0, T - 1, 61).astype(int)]))
+    o = oracle.block_forward(x[rows], c.p, cases.bf16_experts(c.p), shape.k, shape.eps, bias)
+    cases.check_bar(bf16_np(out)[rows], o["out"], cases.FRAC_BF16, "out, extreme skew")
+    cases.check_bar(bf16_np(moe)[rows], o["moe"], cases.FRAC_BF16, "moe_out, extreme skew")
 
 
 def test_block_without_branch_post_norms():

@@ -53,7 +53,7 @@ def _noalloc(cfg, idx):
 # single-block sort.
 @pytest.mark.parametrize("T,k,E", [(2048, 8, 128), (8, 8, 128), (2049, 1, 16), (40000, 16, 256)])
 def test_noalloc_equals_oracle_and_workspace_permutation_twice(T, k, E):
-    cfg = mf.Config(512, E, k, 64, 64)
+    cfg = mf.Config(512, E, k, 128, 128)
     for seed in (1, 2):  # two calls in a row, different routing
         ids = _ids(T, k, E, seed)
         idx = to_dev(ids, torch.int32)
@@ -66,7 +66,7 @@ def test_noalloc_equals_oracle_and_workspace_permutation_twice(T, k, E):
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
-    cfg = mf.Config(512, 128, 8, 64, 64)
+    cfg = mf.Config(512, 128, 8, 128, 128)
     T = mf.PERMUTE_NOALLOC_MAX_PAIRS // 8 + 1
     fake = 1 << 20  # never dereferenced: the size check comes first
     st = mf.lib().moe_permute_noalloc(ctypes.byref(cfg.c()), T, fake, fake, fake, fake, None)
