@@ -165,7 +165,9 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
 
 template <int EB>
 __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a) {
-  extern __shared__ __align__(128) uint8_t r_smem[];  // x rows [8][H], W_r rows [EB][H], scale [H]
+  // x rows [8], W_r rows [EB] and the scale row, each padded by 32 bytes so that the eight
+  // rows read by the lanes of one phase start in distinct banks
+  extern __shared__ __align__(128) uint8_t r_smem[];
   __shared__ float part[kRWarps][kRMaxEB][kRT];
   __shared__ float ssp[kRWarps][kRT];
   __shared__ float rinv[kRT];
@@ -181,15 +183,16 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
   const int nt = min(kRT, a.T - t0);  // tokens of the block
   const int ne = min(EB, E - e0);     // experts of the slice
   const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
+  const int RS = H + 16;  // padded row stride in elements
   uint16_t* xs = reinterpret_cast<uint16_t*>(r_smem);
-  uint16_t* wsm = xs + kRT * H;
-  uint16_t* ssc = wsm + EB * H;
+  uint16_t* wsm = xs + kRT * RS;
+  uint16_t* ssc = wsm + EB * RS;
   if (tid == 0) {
     mbar_init(&bar, 1);
     mbar_fence_init();
     mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(ne + 1 + nt) * row_bytes);
     for (int i = 0; i < ne; ++i)
-      bulk_load_1d(wsm + i * H, a.wr + static_cast<size_t>(e0 + i) * H, row_bytes, &bar);
+      bulk_load_1d(wsm + i * RS, a.wr + static_cast<size_t>(e0 + i) * H, row_bytes, &bar);
     bulk_load_1d(ssc, a.rscale, row_bytes, &bar);
   }
   for (int e = tid; e < E; e += kRThreads) s_pes[e] = a.pes[e];
@@ -207,7 +210,7 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
   pdl_trigger();
   if (tid == 0) {
     for (int i = 0; i < nt; ++i)
-      bulk_load_1d(xs + i * H, a.x + static_cast<size_t>(t0 + i) * H, row_bytes, &bar);
+      bulk_load_1d(xs + i * RS, a.x + static_cast<size_t>(t0 + i) * H, row_bytes, &bar);
     flag = mbar_wait(&bar, 0, 2000000000ull, nullptr) ? 1 : 0;
   }
   __syncthreads();
@@ -222,8 +225,8 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     float ss = 0.f;
     const bool xok = g < nt, wok = g < ne;
-    const uint16_t* xr = xs + g * H + 4 * t;
-    const uint16_t* wr = wsm + g * H + 4 * t;
+    const uint16_t* xr = xs + g * RS + 4 * t;
+    const uint16_t* wr = wsm + g * RS + 4 * t;
     const uint16_t* sr = ssc + 4 * t;
     const float ish = a.inv_sqrt_h;
 #pragma unroll 2
@@ -272,12 +275,17 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
     if (e < ne && tl < nt)
       a.logits[static_cast<size_t>(t0 + tl) * E + e0 + e] = dot * r + (a.bias ? a.bias[e0 + e] : 0.f);
   }
+  // ---- the last slice of this token block takes the top-k.  The barrier orders every
+  // thread's logits before the elected thread's atomic, whose acq_rel also acquires the
+  // other slices' logits for the last one; the pre norms are written while it is in flight.
   __syncthreads();
+  unsigned old = 0;
+  if (tid == 0) old = atom_add_acq_rel_gpu(a.counters + blockIdx.x, 1u);
   // ---- the slice's share of the pre norms of both branches
   for (int j = tid; j < npairs; j += kRThreads) {
     const int c = cb + j % nc, tl = j / nc;
     float f[8], gm[8], gd[8], o1[8], o2[8];
-    unpack8(*reinterpret_cast<const uint4*>(xs + tl * H + c * 8), f);
+    unpack8(*reinterpret_cast<const uint4*>(xs + tl * RS + c * 8), f);
     unpack8(j == tid ? gm0 : __ldg(reinterpret_cast<const uint4*>(a.gm) + c), gm);
     unpack8(j == tid ? gd0 : __ldg(reinterpret_cast<const uint4*>(a.gd) + c), gd);
     const float r = rinv[tl];
@@ -290,13 +298,7 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
     reinterpret_cast<uint4*>(a.xn_moe + static_cast<size_t>(t0 + tl) * H)[c] = pack8(o1);
     reinterpret_cast<uint4*>(a.xn_dense + static_cast<size_t>(t0 + tl) * H)[c] = pack8(o2);
   }
-
-  // ---- the last slice of this token block takes the top-k.  The barrier orders every
-  // thread's logits before the elected thread's atomic, whose acq_rel also acquires the
-  // other slices' logits for the last one.
-  __syncthreads();
   if (tid == 0) {
-    const unsigned old = atom_add_acq_rel_gpu(a.counters + blockIdx.x, 1u);
     flag = old == gridDim.y - 1;
     if (flag) a.counters[blockIdx.x] = 0u;
   }
@@ -331,7 +333,7 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
 }
 
 // Dynamic shared memory of a CTA with EB experts.
-static size_t router_smem(int H, int EB) { return static_cast<size_t>(kRT + EB + 1) * H * 2; }
+static size_t router_smem(int H, int EB) { return static_cast<size_t>(kRT + EB + 1) * (H + 16) * 2; }
 
 // Experts per CTA: about one CTA per SM (token blocks x expert slices), within the
 // shared-memory budget.
