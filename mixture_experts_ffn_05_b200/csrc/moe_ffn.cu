@@ -75,16 +75,16 @@ int choose_bn(const Dims& d) {
 // K pieces per tile: only for the narrowest token tiles (weight-streaming batches), and
 // only when a launch has too few tiles to keep every SM streaming to the end (fewer than
 // kSplitTilesPerSm per SM); the partial sums cost more than the balance gains beyond.
-// Pieces keep about 22 k-steps (each piece costs a partial store and an arrival, and at
-// decode T = 8 pieces of 22 k-steps measured 6% faster for gate_up than pieces of 11),
-// unless that leaves fewer than three pieces per SM.
+// Pieces keep about 22 k-steps (each piece costs a partial store and an arrival: at
+// decode T = 8 the gate_up launch measured 6% faster with pieces of 22 k-steps than of
+// 11), or about 11 when a launch has fewer than two tiles per SM (T = 1).
 constexpr int kSplitTilesPerSm = 8;
 constexpr int kAssumedSms = 148;  // a B200; only shifts the threshold if the GPU differs
 
 int choose_split(int k_steps, int bn, double tiles) {
   if (bn != 16 || tiles >= kSplitTilesPerSm * kAssumedSms) return 1;
-  const int fill = static_cast<int>(std::ceil(3.0 * kAssumedSms / std::max(tiles, 1.0)));
-  return std::max(1, std::min(std::min(k_steps, 4), std::max((k_steps + 21) / 22, fill)));
+  const int per = tiles < 2 * kAssumedSms ? 11 : 22;
+  return std::max(1, std::min(std::min(k_steps, 4), (k_steps + per - 1) / per));
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

@@ -421,21 +421,30 @@ __device__ __forceinline__ void consume_item(const uint8_t* st, const Offs<WT>& 
   }
 }
 
+// The scales of this lane's two output rows (g and g + 8 of its warp's strip): int8 one
+// per row, nvfp4 the matrix scale times 2^14, bf16 none.  Loaded when a piece starts, so
+// that the epilogue does not wait for them.
+__device__ __forceinline__ float2 row_scales(const StreamProblem& pr, const Piece& pc) {
+  const int warp = threadIdx.x >> 5, g = (threadIdx.x & 31) >> 2;
+  const int r0 = 16 * warp + g;
+  const size_t grow = static_cast<size_t>(pc.gg) * pr.rows;
+  if (pr.wtype == kStreamInt8)
+    return make_float2(__ldg(pr.wscale + grow + weight_row(pr, pc.m, r0)),
+                       __ldg(pr.wscale + grow + weight_row(pr, pc.m, r0 + 8)));
+  if (pr.wtype == kStreamNvfp4) {
+    const float s = __ldg(pr.wscale + pc.gg) * 16384.0f;
+    return make_float2(s, s);
+  }
+  return make_float2(1.f, 1.f);
+}
+
 // The epilogue of n-tile n of one unit from its (full-K) sums v: lane (g, t) of warp w
 // holds rows g and g + 8 of strip w for tokens 8n + 2t and 8n + 2t + 1 of the chunk.
 __device__ __forceinline__ void store_unit(const StreamProblem& pr, const Piece& pc, int warp,
-                                           int g, int t, int n, const float (&v)[4]) {
+                                           int g, int t, int n, const float (&v)[4], float2 sc) {
   const int r0 = 16 * warp + g;
   const int wr0 = weight_row(pr, pc.m, r0), wr1 = weight_row(pr, pc.m, r0 + 8);
-  const size_t grow = static_cast<size_t>(pc.gg) * pr.rows;
-  // row scales: int8 per row; nvfp4 the matrix scale times 2^14; bf16 none
-  float s0 = 1.f, s1 = 1.f;
-  if (pr.wtype == kStreamInt8) {
-    s0 = pr.wscale[grow + wr0];
-    s1 = pr.wscale[grow + wr1];
-  } else if (pr.wtype == kStreamNvfp4) {
-    s0 = s1 = pr.wscale[pc.gg] * 16384.0f;
-  }
+  const float s0 = sc.x, s1 = sc.y;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int col = 8 * n + 2 * t + q;
@@ -466,7 +475,8 @@ __device__ __forceinline__ void store_unit(const StreamProblem& pr, const Piece&
 // tile) the full sums and the epilogue.  All threads of the CTA.
 template <int NT>
 __device__ __forceinline__ void finish_piece(const StreamParams& P, const StreamProblem& pr,
-                                             const Piece& pc, float (&v)[NT][4], volatile int* flag) {
+                                             const Piece& pc, float (&v)[NT][4], float2 sc,
+                                             volatile int* flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   constexpr int NC = kStreamChunk * NT;
@@ -510,7 +520,7 @@ __device__ __forceinline__ void finish_piece(const StreamParams& P, const Stream
     }
   }
 #pragma unroll
-  for (int n = 0; n < NT; ++n) store_unit(pr, pc, warp, g, t, n, v[n]);
+  for (int n = 0; n < NT; ++n) store_unit(pr, pc, warp, g, t, n, v[n], sc);
 }
 
 // Pieces are dealt round-robin over the launch: the CTA's k-th piece is blockIdx.x +
@@ -599,6 +609,7 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
     const int piece = cta_piece(k);
     if (piece >= end) break;
     const Piece pc = piece_of(piece, P, tb);
+    const float2 sc = row_scales(pr, pc);
     const int n = pc.it1 - pc.it0;
     float acc[NT + (NT == 1)][4];
 #pragma unroll
@@ -621,7 +632,7 @@ __device__ int run_problem(const StreamParams& P, const StreamProblem& pr, int k
     for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int q = 0; q < 4; ++q) v[n][q] = NT == 1 ? acc[0][q] + acc[NT == 1 ? 1 : 0][q] : acc[n][q];
-    finish_piece<NT>(P, pr, pc, v, flag);
+    finish_piece<NT>(P, pr, pc, v, sc, flag);
     ++k;
   }
   cp_async_wait<0>();
