@@ -119,10 +119,12 @@ cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int*
                            int* inv_pos, int* block_hist, int* block_base, cudaStream_t s,
                            bool pdl = false);
 int permute_blocks(int n);  // blocks of the multi-block path, <= 256 (0 = single-block path)
-// to_f16: write the rows as fp16 (the operand type of int8 experts) instead of bf16.
+// dst[q] = src row sorted_src[q] / k for the n sorted positions; to_f16: write the rows
+// as fp16 (the operand type of int8 experts) instead of bf16.  With inv_pos (the inverse
+// permutation) large batches are written token by token.
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
-                               const uint16_t* src, uint16_t* dst, bool to_f16, cudaStream_t s,
-                               bool pdl = false);
+                               const int* inv_pos, const uint16_t* src, uint16_t* dst,
+                               bool to_f16, cudaStream_t s, bool pdl = false);
 // A launch may run on CTA pairs (GemmParams::pairs) when its weights are bf16 and its
 // token tiles are 128 or 256 wide; its B maps then take boxes of bn / 2 rows (each CTA
 // loads half of a tile's token rows), and the grid is even.  A pair takes two M tiles:

@@ -383,13 +383,13 @@ bool mark(void* const* ev, int i, cudaStream_t s) {
 // The routed tokens' rows in sorted order for the gate_up matmul: bf16 copies, fp16 copies
 // (int8 experts) or per-row E4M3 codes and scales (fp8 experts).
 moe_status_t gather_tokens(const Dims& d, const Layout& L, void* ws, const int* sorted,
-                           const uint16_t* xn_moe, cudaStream_t s, bool pdl) {
+                           const int* inv, const uint16_t* xn_moe, cudaStream_t s, bool pdl) {
   const int Tk = d.T * d.k;
   if (d.fp8)
     return cuda_status(launch_gather_quant_fp8(Tk, d.k, d.H, d.T, sorted, xn_moe,
                                                at<uint8_t>(ws, L.aperm), at<float>(ws, L.sx),
                                                s, pdl));
-  return cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, xn_moe,
+  return cuda_status(launch_gather_rows(Tk, d.k, d.H, d.T, sorted, inv, xn_moe,
                                         at<uint16_t>(ws, L.aperm), d.int8 || d.nvfp4, s, pdl));
 }
 
@@ -723,7 +723,7 @@ moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint16_t* y = at<uint16_t>(ws, L.y);
-  if ((st = gather_tokens(d, L, ws, sorted_src, xn_moe, s, false)) != MOE_OK) return st;
+  if ((st = gather_tokens(d, L, ws, sorted_src, inv_pos, xn_moe, s, false)) != MOE_OK) return st;
   GemmJob j{};
   j.experts = true;
   j.a_rows = at<uint8_t>(ws, L.aperm);
@@ -813,7 +813,7 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
                                        at<int>(ws, L.bbase), s, true))) != MOE_OK)
     return st;
   if (!mark(ev, 2, s)) return MOE_ERR_CUDA;
-  if ((st = gather_tokens(d, L, ws, sorted, xn_moe, s, true)) != MOE_OK) return st;
+  if ((st = gather_tokens(d, L, ws, sorted, inv, xn_moe, s, true)) != MOE_OK) return st;
   if (!mark(ev, 3, s)) return MOE_ERR_CUDA;
   GemmJob j{};
   j.experts = true;

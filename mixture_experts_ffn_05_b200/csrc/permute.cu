@@ -129,6 +129,9 @@ cudaError_t launch_permute(int n, int E, const int* topk_idx, int* offsets, int*
 // 4 KB of loads in flight.  A pair index outside [0, T*k) yields a zero row (never an
 // out-of-bounds read).
 constexpr int kGatherWarps = 8;
+// From this many pairs on, the rows are written token by token (each source row read
+// once); below, pair by pair (more warps for a small batch).
+constexpr int kScatterMinPairs = 4096;
 
 // bf16 -> fp16 of 8 values (exact for |v| in the fp16 normal range; smaller values keep
 // fp16 subnormal precision, 2^-24 absolute).
@@ -170,6 +173,51 @@ __global__ void __launch_bounds__(32 * kGatherWarps) gather_rows_kernel(
     for (int u = 0; u < 8; ++u) {
       const int c = c0 + 32 * u;
       if (c < nch) d[c] = F16 ? bf16x8_to_f16x8(v[u]) : v[u];
+    }
+  }
+}
+
+// The same rows written token by token: warp t reads row t of src once and writes it to the
+// sorted position of each of its k pairs (pos = inv_pos[t k + j], taken only where
+// sorted_src[pos] names the pair back, so that dropped pairs write nothing).  For large
+// batches: each source row is read once instead of k times, from HBM once it no longer
+// sits in L2.  Every row the matmuls read (the positions below the pair count) is written.
+template <bool F16>
+__global__ void __launch_bounds__(32 * kGatherWarps) scatter_rows_kernel(
+    int T, int k, int H, int n, const int* __restrict__ inv_pos,
+    const int* __restrict__ sorted_src, const uint16_t* __restrict__ src,
+    uint16_t* __restrict__ dst) {
+  const int nch = H >> 3;
+  pdl_wait();
+  pdl_trigger();
+  const int t = static_cast<int>(blockIdx.x) * kGatherWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  // lane j < k: the destination of pair (t, j), or -1
+  int pos = -1;
+  if (lane < k) {
+    const int p = t * k + lane;
+    const int q = __ldg(inv_pos + p);
+    if (q >= 0 && q < n && __ldg(sorted_src + q) == p) pos = q;
+  }
+  const uint4* srow = reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * H);
+  for (int c0 = lane; c0 < nch; c0 += 32 * 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + 32 * u;
+      v[u] = c < nch ? __ldg(srow + c) : make_uint4(0u, 0u, 0u, 0u);
+      if (F16) v[u] = bf16x8_to_f16x8(v[u]);
+    }
+    for (int j = 0; j < k; ++j) {
+      const int q = __shfl_sync(0xffffffffu, pos, j);
+      if (q < 0) continue;
+      uint4* d = reinterpret_cast<uint4*>(dst + static_cast<size_t>(q) * H);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < nch) d[c] = v[u];
+      }
     }
   }
 }
@@ -240,8 +288,17 @@ cudaError_t launch_gather_quant_fp8(int n, int k, int cols, int T, const int* so
 }
 
 cudaError_t launch_gather_rows(int n, int k, int H, int T, const int* sorted_src,
-                               const uint16_t* src, uint16_t* dst, bool to_f16, cudaStream_t s,
-                               bool pdl) {
+                               const int* inv_pos, const uint16_t* src, uint16_t* dst,
+                               bool to_f16, cudaStream_t s, bool pdl) {
+  if (inv_pos != nullptr && n >= kScatterMinPairs && k <= 32) {
+    const int tb = (T + kGatherWarps - 1) / kGatherWarps;
+    return to_f16 ? launch_k(scatter_rows_kernel<true>, dim3(static_cast<unsigned>(tb)),
+                             dim3(32 * kGatherWarps), 0, s, pdl, T, k, H, n, inv_pos, sorted_src,
+                             src, dst)
+                  : launch_k(scatter_rows_kernel<false>, dim3(static_cast<unsigned>(tb)),
+                             dim3(32 * kGatherWarps), 0, s, pdl, T, k, H, n, inv_pos, sorted_src,
+                             src, dst);
+  }
   const int blocks = (n + kGatherWarps - 1) / kGatherWarps;
   return to_f16 ? launch_k(gather_rows_kernel<true>, dim3(static_cast<unsigned>(blocks)),
                            dim3(32 * kGatherWarps), 0, s, pdl, n, k, H, T, sorted_src, src, dst)
