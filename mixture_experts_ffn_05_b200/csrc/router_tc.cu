@@ -10,8 +10,9 @@
 // with rinv[t] = 1 / sqrt(mean_h x[t,h]^2 + eps).  x is bf16 and goes to the tensor cores
 // as it is.  W' is fp32; a preparation kernel splits it into two bf16 matrices,
 // W' = W'hi + W'lo + d with |d| <= 2^-16 |W'|, and the kernel accumulates x.W'hi and
-// x.W'lo into the same fp32 accumulator, so the logits carry the accuracy of an fp32 dot
-// product (every bf16 x bf16 product is exact in fp32).
+// x.W'lo in fp32 (one MMA of N = 2 ne over both, each into its own accumulator columns,
+// added when read), so the logits carry the accuracy of an fp32 dot product (every bf16 x
+// bf16 product is exact in fp32).
 //
 // One CTA per 128 tokens (the 128 TMEM lanes) and slice of the experts (the N dimension:
 // all E experts when the batch has enough token tiles to fill the GPU, else E/2, E/4 or
@@ -19,11 +20,13 @@
 // Warp roles:
 //   0      TMA producer: per 64-wide K step the x tile and the W'hi, W'lo tiles
 //          (phase 1), then the x tiles again, several per ring stage (phase 2);
-//   1      MMA issuer (two MMAs per 16 K) and TMEM owner;
+//   1      MMA issuer (one MMA per 16 K over W'hi and W'lo, two for slices wider than
+//          128 experts) and TMEM owner;
 //   2..5   sums of x^2 of one token row per thread, read from the x tiles of phase 1;
 //          afterwards the top-k of the same row from its TMEM lane (one expert slice),
 //          or the row's logits of the slice to global memory (several slices: the last
-//          CTA of a token tile to finish then takes the top-k of its 128 tokens);
+//          CTA of a token tile to finish then takes the top-k of its 128 tokens, one
+//          warp per token);
 //   6..13  phase 2: xn_moe = x * rinv * g_pre_moe and xn_dense = x * rinv * g_pre_dense,
 //          for the CTA's share of the columns (its slice of the 64-wide K steps).
 // Every wait is bounded.
@@ -147,6 +150,58 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
   return __all_sync(0xffffffffu, ok);
 }
 
+// Top-k of one row of E <= 32 KPL logits in shared memory by one warp (ties to the lower
+// expert id): lane i holds experts i, i + 32, ...; each of the k rounds takes the warp
+// maximum of the lanes' best remaining 64-bit keys (ordered logit, then the inverted
+// expert id), high word first, then the low word among the lanes that share it.  Then
+// the weights as TopK::write computes them.
+template <int KPL>
+__device__ __forceinline__ void topk_row_warp(const float* row, int E, int k, int t,
+                                              const uint16_t* pes, int* topk_idx,
+                                              float* topk_w) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long key[KPL];
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? (static_cast<unsigned long long>(order_key(row[e])) << 32) |
+                         (0xFFFFFFFFu - static_cast<uint32_t>(e))
+                   : 0ull;
+  }
+#pragma unroll
+  for (int r = 0; r < KPL; ++r)
+#pragma unroll
+    for (int i = r & 1; i + 1 < KPL; i += 2)
+      if (key[i] < key[i + 1]) {
+        const unsigned long long tmp = key[i];
+        key[i] = key[i + 1];
+        key[i + 1] = tmp;
+      }
+  unsigned long long mine = 0ull;  // lane j keeps the j-th selected key
+  for (int j = 0; j < k; ++j) {
+    const uint32_t hi = static_cast<uint32_t>(key[0] >> 32);
+    const uint32_t bh = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t bl = __reduce_max_sync(0xffffffffu, hi == bh ? static_cast<uint32_t>(key[0]) : 0u);
+    const unsigned long long best = (static_cast<unsigned long long>(bh) << 32) | bl;
+    if (key[0] == best) {
+#pragma unroll
+      for (int i = 0; i + 1 < KPL; ++i) key[i] = key[i + 1];
+      key[KPL - 1] = 0ull;
+    }
+    if (lane == j) mine = best;
+  }
+  const float top = key_value(static_cast<uint32_t>(__shfl_sync(0xffffffffu, mine, 0) >> 32));
+  const int my_e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(mine));
+  const float ex = lane < k ? expf(key_value(static_cast<uint32_t>(mine >> 32)) - top) : 0.f;
+  float sum = 0.f;  // in slot order
+  for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);
+  if (lane < k) {
+    topk_idx[static_cast<size_t>(t) * k + lane] = my_e;
+    topk_w[static_cast<size_t>(t) * k + lane] =
+        ex / sum * __uint_as_float(static_cast<uint32_t>(pes[my_e]) << 16);
+  }
+}
+
 template <int KMAX>
 __global__ void __launch_bounds__(kTcThreads, 1)
     router_tc_kernel(const __grid_constant__ RouterTcMaps maps, const RouterTcArgs a) {
@@ -175,7 +230,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int ks1 = static_cast<int>(blockIdx.y + 1) * KS / a.slices;
   const int J2 = (ks1 - ks0 + a.tiles_per_stage - 1) / a.tiles_per_stage;
   const uint32_t b_bytes = static_cast<uint32_t>(a.ne) * 128u;
-  const uint32_t tmem_cols = a.ne <= 32 ? 32u : a.ne <= 64 ? 64u : a.ne <= 128 ? 128u : 256u;
+  // W'hi and W'lo rows sit back to back in a stage, so with 2 ne <= 256 one MMA of N = 2 ne
+  // multiplies both: accumulator columns [0, ne) hold x.W'hi, [ne, 2 ne) x.W'lo (two
+  // independent sums, added when read).  Wider slices take two MMAs into one accumulator.
+  const bool merged = 2 * a.ne <= 256;
+  const int acc_cols = merged ? 2 * a.ne : a.ne;
+  const uint32_t tmem_cols = acc_cols <= 32 ? 32u : acc_cols <= 64 ? 64u : acc_cols <= 128 ? 128u : 256u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -254,7 +314,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, a.ne);
+      const uint32_t idesc = idesc_bf16_f32(128, acc_cols);
       bool ok = true;
       int done = 0;
       for (int j = 0; j < KS; ++j) {
@@ -265,11 +325,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_after();
         const uint32_t sa = smem_u32(ring + static_cast<size_t>(s) * a.stage_bytes);
+        // one 32-byte K slice per MMA: descriptors advance by 2 (16-byte units)
+        const uint64_t ad = sdesc_k_sw128(sa);
+        const uint64_t bh = sdesc_k_sw128(sa + kTcTile);
+        if (merged) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = sdesc_k_sw128(sa + kk * 32);
-          umma_bf16(tmem, ad, sdesc_k_sw128(sa + kTcTile + kk * 32), idesc, (j | kk) != 0);
-          umma_bf16(tmem, ad, sdesc_k_sw128(sa + kTcTile + b_bytes + kk * 32), idesc, 1u);
+          for (int kk = 0; kk < 4; ++kk) umma_bf16(tmem, ad + 2 * kk, bh + 2 * kk, idesc, (j | kk) != 0);
+        } else {
+          const uint64_t bl = sdesc_k_sw128(sa + kTcTile + b_bytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            umma_bf16(tmem, ad + 2 * kk, bh + 2 * kk, idesc, (j | kk) != 0);
+            umma_bf16(tmem, ad + 2 * kk, bl + 2 * kk, idesc, 1u);
+          }
         }
         umma_commit(&empty1[s]);
         done = j + 1;
@@ -332,6 +400,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < a.ne; c += 16) {
           float v[16];
           tmem_ld16(lane_base + c, v);
+          if (merged) {
+            float w[16];
+            tmem_ld16(lane_base + a.ne + c, w);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] += w[i];
+          }
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             if (c + i < a.E) tk.push(v[i] * rinv + s_bias[c + i], c + i);
@@ -342,6 +416,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < a.ne; c += 16) {
           float v[16];
           tmem_ld16(lane_base + c, v);
+          if (merged) {
+            float w[16];
+            tmem_ld16(lane_base + a.ne + c, w);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] += w[i];
+          }
           if (t < a.T) {
             float* lr = a.logits + static_cast<size_t>(t) * a.E + e0 + c;
 #pragma unroll
@@ -444,14 +524,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int i = threadIdx.x; i < n; i += kTcThreads) sl[(i / a.E) * ld + i % a.E] = __ldcg(src + i);
   }
   __syncthreads();
-  if (threadIdx.x < 64 || threadIdx.x >= 64 + kTcTokens) return;
-  const int r = static_cast<int>(threadIdx.x) - 64;
-  if (r >= rows) return;
-  TopK<KMAX> tk;
-  tk.init();
-  const float* lr = sl + r * ld;
-  for (int e = 0; e < a.E; ++e) tk.push(lr[e], e);
-  tk.write(t0 + r, a.k, s_pes, a.topk_idx, a.topk_w);
+  // one warp per row (a thread per row took ~15 us for the 128 rows of a tile)
+  for (int r = warp; r < rows; r += kTcThreads / 32) {
+    if (a.E <= 128)
+      topk_row_warp<4>(sl + r * ld, a.E, a.k, t0 + r, s_pes, a.topk_idx, a.topk_w);
+    else
+      topk_row_warp<8>(sl + r * ld, a.E, a.k, t0 + r, s_pes, a.topk_idx, a.topk_w);
+  }
 }
 
 // W'hi, W'lo = the two-term bf16 split of s[h] * W_r[e,h] / sqrt(H); one thread per 8.

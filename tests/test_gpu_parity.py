@@ -65,10 +65,11 @@ def test_router(name):
     assert np.array_equal(r["topk_idx"].cpu().numpy(), o["topk_idx"])
     got_w = r["topk_w"].cpu().numpy().astype(np.float64)
     # Both routers take the logits from tensor-core sums of the two-term split of W'
-    # (2H/16 products of 16 terms into one fp32 accumulator); each addition may lose up to
-    # one unit in the last place of the accumulator (nothing promises round-to-nearest
-    # inside the tensor core), so a logit may be off by steps * 2^-23 * max|l - b| and a
-    # weight, exp(l_j - l_0) / sum, by four times that, relatively.
+    # (2H/16 products of 16 terms, added into fp32 accumulators: one, or one per term and
+    # then the two sums); each addition may lose up to one unit in the last place of the
+    # accumulator (nothing promises round-to-nearest inside the tensor core), so a logit
+    # may be off by steps * 2^-23 * max|l - b| and a weight, exp(l_j - l_0) / sum, by four
+    # times that, relatively.
     lraw = np.abs(o["logits"] - (0.0 if c.bias is None else c.bias[None, :]))
     steps = 2 * c.shape.H / 16
     rtol = 2e-6 + 4 * steps * 2.0 ** -23 * lraw.max(axis=1, keepdims=True)
