@@ -201,8 +201,10 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int32_t T, const int32
  *   xn_moe [T][H] bf16; topk_w [T][k] fp32; expert_offsets, sorted_src, inv_pos as
  *   produced by moe_permute.
  *   moe_out [T][H] bf16 = sum_j topk_w[t][j] * MLP_{e(t,j)}(xn_moe[t]), the branch
- *   output before its post norm.  Accumulation is fp32; h and the weighted expert
- *   outputs are stored as bf16 between the two GEMMs. */
+ *   output before its post norm.  Accumulation is fp32; between the steps h is stored
+ *   as bf16 (fp16 with int8 or NVFP4 experts, E4M3 codes with a row scale with fp8
+ *   experts) and each pair's unweighted expert output as fp16; the weighted sum over the
+ *   slots is taken in fp32, in slot order. */
 moe_status_t moe_ffn_forward(const moe_config_t* cfg, int32_t T, const moe_bf16_t* xn_moe,
                              const float* topk_w, const int32_t* expert_offsets,
                              const int32_t* sorted_src, const int32_t* inv_pos,
