@@ -584,9 +584,9 @@ struct RouteJob {
 };
 
 // The router step, launched as the first kernel of the entry point: the tensor-core
-// router for large batches, the CUDA-core one (router.cu) for small ones.  Only the
-// CUDA-core router sorts the pairs in the same launch (r.offsets); the caller asks for
-// it for batches of the CUDA-core router.
+// router for large batches, the small-batch one (router.cu) for small ones.  Only the
+// small-batch router sorts the pairs in the same launch (r.offsets); the caller asks for
+// it for batches of the small-batch router.
 moe_status_t run_router(const Dims& d, const Layout& L, void* ws, const RouteJob& r,
                         cudaStream_t s) {
   unsigned* counters = at<unsigned>(ws, L.rcounters);

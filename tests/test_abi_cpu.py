@@ -67,7 +67,7 @@ def test_workspace_size(lib):
 
 def test_block_launch_count(lib):
     # router 1 (2 above T = 128: weight prep + tensor-core router); permutation 0 when the
-    # CUDA-core router sorts (T*k <= 2048), 1 (T*k <= 2048), else 3; gather, gate_up,
+    # small-batch router sorts (T*k <= 2048), 1 (T*k <= 2048), else 3; gather, gate_up,
     # down, combine 1 each
     for T, n in ((1, 5), (8, 5), (64, 5), (128, 5), (129, 7), (256, 7), (257, 9), (2048, 9),
                  (16384, 9)):

@@ -28,7 +28,7 @@ SHAPES = {
     "decode_T8": (synth.DECODE, False),
     "decode_T1": (synth.Shape(T=1, H=2816, E=128, k=8, I=704, D=2112), False),
     "decode_T64": (synth.Shape(T=64, H=2816, E=128, k=8, I=704, D=2112), False),
-    # the largest batch of the CUDA-core router (16 token blocks, the multi-block sort)
+    # the largest batch of the small-batch router (16 token blocks, the multi-block sort)
     "decode_T128": (synth.Shape(T=128, H=2816, E=128, k=8, I=704, D=2112), False),
     "prefill_T2048_zipf": (synth.PREFILL, True),
     "limits": (synth.Shape(T=5, H=6144, E=256, k=16, I=128, D=128), False),
