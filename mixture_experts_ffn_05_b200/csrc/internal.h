@@ -84,7 +84,9 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 // Launchers.  All return cudaSuccess or the launch error.
 // Router + pre norms + top-k in one launch; when offsets != NULL (and T*k fits the
-// single-block sort, see permute_blocks) also the token-to-expert counting sort.
+// single-block sort, see permute_blocks) also the token-to-expert counting sort, and with
+// aperm != NULL (a single token block, T <= 8) the gather of the routed rows of xn_moe in
+// sorted order into aperm (fp16 when aperm_f16).
 // counters: router_counters(T) words, zero on entry (left zero on exit).
 cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t* x,
                           const uint16_t* router_scale, const uint16_t* w_router,
@@ -92,7 +94,8 @@ cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t*
                           const uint16_t* g_pre_moe, const uint16_t* g_pre_dense,
                           uint16_t* xn_moe, uint16_t* xn_dense, float* logits, int* topk_idx,
                           float* topk_w, unsigned* counters, unsigned* status, int* offsets,
-                          int* sorted_src, int* inv_pos, cudaStream_t s, bool pdl = false);
+                          int* sorted_src, int* inv_pos, uint16_t* aperm, bool aperm_f16,
+                          cudaStream_t s, bool pdl = false);
 int router_counters(int T);
 
 // The tensor-core router (router_tc.cu) serves batches of more than kRouterTcMinT

@@ -104,6 +104,19 @@ constexpr int kStreamMaxT = 256;
 
 bool stream_path(const Dims& d) { return d.nvfp4 || (d.int8 && d.T <= kStreamMaxT); }
 
+// Batches of at most this many (token, slot) pairs in one token block of the small-batch
+// router have their routed rows gathered by the router's last CTA, after its sort, instead
+// of by a launch of its own (a few rows: less than the launch and its kernel boundary;
+// bf16 T = 1 step 52.7 -> 50.8 us).  With int8 or NVFP4 experts it measured slower (T = 1
+// +4% and +7%: the weight-streaming GEMM's weight requests, issued before its dependency
+// wait, then overlap only the router's tail), and fp8 rows are quantised on the way, so
+// those keep the separate gather.
+constexpr int kRouterGatherMaxPairs = 32;
+
+bool router_gathers(const Dims& d) {
+  return d.T <= 8 && d.T * d.k <= kRouterGatherMaxPairs && !d.fp8 && !d.int8 && !d.nvfp4;
+}
+
 // K pieces of the weight-streaming kernel's tiles.  Pieces are dealt round-robin, so the
 // pieces of both problems of a launch are sized to about the same bytes: about four per CTA
 // of the launch (five CTAs per SM assumed), at least 32 KB and four K items each.
@@ -581,6 +594,8 @@ struct RouteJob {
   int* offsets;  // with sorted_src and inv_pos: sort the pairs in the same launch; or NULL
   int* sorted_src;
   int* inv_pos;
+  uint16_t* aperm;  // with the sort: gather the routed rows there too (router_gathers); or NULL
+  bool aperm_f16;
 };
 
 // The router step, launched as the first kernel of the entry point: the tensor-core
@@ -596,11 +611,12 @@ moe_status_t run_router(const Dims& d, const Layout& L, void* ws, const RouteJob
                                      r.logit_bias, r.per_expert_scale, r.g_pre_moe,
                                      r.g_pre_dense, r.xn_moe, r.xn_dense,
                                      at<float>(ws, L.logits), r.topk_idx, r.topk_w, counters,
-                                     status, r.offsets, r.sorted_src, r.inv_pos, s));
+                                     status, r.offsets, r.sorted_src, r.inv_pos, r.aperm,
+                                     r.aperm_f16, s));
   uint16_t* whi = at<uint16_t>(ws, L.wr_hi);
   uint16_t* wlo = at<uint16_t>(ws, L.wr_lo);
   const int ne = (d.E + 15) / 16 * 16 / router_tc_slices(d.T, d.E);  // experts per CTA
-  if (r.offsets != nullptr) return MOE_ERR_INVALID_ARG;  // no fused sort on this path
+  if (r.offsets != nullptr || r.aperm != nullptr) return MOE_ERR_INVALID_ARG;  // not on this path
   RouterTcMaps m;
   if (!encode_bf16(&m.x, r.x, d.T, d.H, 128) || !encode_bf16(&m.whi, whi, d.E, d.H, ne) ||
       !encode_bf16(&m.wlo, wlo, d.E, d.H, ne))
@@ -645,7 +661,8 @@ int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T) {
   int n = tc ? 2 : 1;                                     // router (prep + router)
   if (!fused_sort) n += permute_blocks(Tk) == 0 ? 1 : 3;  // permutation
   if (d.fp8) n += 1;                                      // h quantised for the down matmul
-  return n + 4;                                           // gather, gate_up, down, combine
+  if (!(fused_sort && router_gathers(d))) n += 1;         // gather
+  return n + 3;                                           // gate_up, down, combine
 }
 
 const char* moe_status_string(moe_status_t s) {
@@ -803,9 +820,11 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
       if (ev[i] == nullptr) return MOE_ERR_INVALID_ARG;
   if (!mark(ev, 0, s)) return MOE_ERR_CUDA;
   const bool fused_sort = !router_uses_tc(d.T) && permute_blocks(Tk) == 0;
+  const bool rgather = fused_sort && router_gathers(d);
   const RouteJob r{x, w->router_scale, w->w_router, w->logit_bias, w->per_expert_scale,
                    w->g_pre_moe, w->g_pre_dense, topk_idx, topk_w, xn_moe, xn_dense,
-                   fused_sort ? offsets : nullptr, sorted, inv};
+                   fused_sort ? offsets : nullptr, sorted, inv,
+                   rgather ? aperm : nullptr, false};
   if ((st = run_router(d, L, ws, r, s)) != MOE_OK) return st;
   if (!mark(ev, 1, s)) return MOE_ERR_CUDA;
   if (!fused_sort &&
@@ -813,7 +832,8 @@ moe_status_t moe_block_forward(const moe_config_t* cfg, int32_t T, const moe_bf1
                                        at<int>(ws, L.bbase), s, true))) != MOE_OK)
     return st;
   if (!mark(ev, 2, s)) return MOE_ERR_CUDA;
-  if ((st = gather_tokens(d, L, ws, sorted, inv, xn_moe, s, true)) != MOE_OK) return st;
+  if (!rgather && (st = gather_tokens(d, L, ws, sorted, inv, xn_moe, s, true)) != MOE_OK)
+    return st;
   if (!mark(ev, 3, s)) return MOE_ERR_CUDA;
   GemmJob j{};
   j.experts = true;

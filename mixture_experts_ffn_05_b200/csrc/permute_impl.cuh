@@ -12,6 +12,20 @@ namespace moe {
 
 constexpr int kPermMaxE = 256;
 
+// bf16 -> fp16 of 8 values (exact for |v| in the fp16 normal range; smaller values keep
+// fp16 subnormal precision, 2^-24 absolute).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& u) {
+  float f[8];
+  unpack8(u, f);
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+    o[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 template <int NT>
 struct PermuteSmem {
   int cnt[kPermMaxE];

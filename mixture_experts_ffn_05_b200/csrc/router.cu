@@ -154,6 +154,10 @@ struct RouterArgs {
   int* offsets;
   int* sorted_src;
   int* inv_pos;
+  // with the sort of a single token block: the routed rows of xn_moe in sorted order
+  // (fp16 when aperm_f16), or NULL
+  uint16_t* aperm;
+  int aperm_f16;
 };
 
 // Two floats rounded to bf16 (nearest even), the first in the low half.
@@ -175,6 +179,7 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
   __shared__ __align__(8) uint64_t bar;
   __shared__ uint16_t s_pes[kPermMaxE];
   __shared__ int s_ids[kRT * 16];
+  __shared__ int s_tok[kRT * 16];  // router gather: the token of each sorted position
   __shared__ PermuteSmem<kRThreads> ps;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -317,6 +322,37 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
   if (small_sort) {
     __syncthreads();
     sort_small(a.T * a.k, E, s_ids, ps.wcnt, ps.cnt, ps.off, a.offsets, a.sorted_src, a.inv_pos);
+    if (a.aperm != nullptr) {
+      // the gather of the routed rows, for a batch this small cheaper here than as a launch
+      // of its own: the other slices' xn_moe columns were acquired with the counter.  The
+      // token of each sorted position goes to shared memory first, then every thread
+      // requests all of its chunks before storing any (one round trip).
+      const int n = a.T * a.k, nch = H >> 3;
+      __syncthreads();  // sorted_src is written
+      if (tid < n) s_tok[tid] = __ldcg(a.sorted_src + tid) / a.k;
+      __syncthreads();
+      constexpr int U = 6;
+      for (int i0 = tid; i0 < n * nch; i0 += kRThreads * U) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int i = i0 + u * kRThreads;
+          if (i < n * nch) {
+            const int q = i / nch, c = i - q * nch;
+            v[u] = __ldcg(reinterpret_cast<const uint4*>(a.xn_moe + static_cast<size_t>(s_tok[q]) * H) + c);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int i = i0 + u * kRThreads;
+          if (i < n * nch) {
+            const int q = i / nch, c = i - q * nch;
+            reinterpret_cast<uint4*>(a.aperm + static_cast<size_t>(q) * H)[c] =
+                a.aperm_f16 ? bf16x8_to_f16x8(v[u]) : v[u];
+          }
+        }
+      }
+    }
     return;
   }
 
@@ -363,10 +399,13 @@ cudaError_t launch_router(int T, int H, int E, int k, float eps, const uint16_t*
                           const uint16_t* g_pre_moe, const uint16_t* g_pre_dense,
                           uint16_t* xn_moe, uint16_t* xn_dense, float* logits, int* topk_idx,
                           float* topk_w, unsigned* counters, unsigned* status, int* offsets,
-                          int* sorted_src, int* inv_pos, cudaStream_t s, bool pdl) {
+                          int* sorted_src, int* inv_pos, uint16_t* aperm, bool aperm_f16,
+                          cudaStream_t s, bool pdl) {
+  if (aperm != nullptr && (offsets == nullptr || T > kRT)) return cudaErrorInvalidValue;
   RouterArgs a{T, H, E, k, eps, 1.0f / sqrtf(static_cast<float>(H)), x, router_scale, w_router,
                bias, per_expert_scale, g_pre_moe, g_pre_dense, xn_moe, xn_dense, logits,
-               topk_idx, topk_w, counters, status, offsets, sorted_src, inv_pos};
+               topk_idx, topk_w, counters, status, offsets, sorted_src, inv_pos, aperm,
+               aperm_f16 ? 1 : 0};
   switch (router_eb(T, H, E)) {
     case 1: return launch_eb<1>(a, s, pdl);
     case 2: return launch_eb<2>(a, s, pdl);

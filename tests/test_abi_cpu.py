@@ -67,16 +67,19 @@ def test_workspace_size(lib):
 
 def test_block_launch_count(lib):
     # router 1 (2 above T = 128: weight prep + tensor-core router); permutation 0 when the
-    # small-batch router sorts (T*k <= 2048), 1 (T*k <= 2048), else 3; gather, gate_up,
+    # small-batch router sorts (T*k <= 2048), 1 (T*k <= 2048), else 3; gather 1, or 0 when
+    # the small-batch router also gathers (T <= 8 and T*k <= 32, bf16 experts); gate_up,
     # down, combine 1 each
-    for T, n in ((1, 5), (8, 5), (64, 5), (128, 5), (129, 7), (256, 7), (257, 9), (2048, 9),
-                 (16384, 9)):
+    for T, n in ((1, 4), (4, 4), (5, 5), (8, 5), (64, 5), (128, 5), (129, 7), (256, 7),
+                 (257, 9), (2048, 9), (16384, 9)):
         assert mf.moe_block_launch_count(CFG, T) == n, T
-    for T, n in ((8, 5), (512, 7), (513, 9)):  # top-4: T*k = 2048 at T = 512
+    for T, n in ((8, 4), (9, 5), (512, 7), (513, 9)):  # top-4: T*k = 2048 at T = 512
         assert mf.moe_block_launch_count(TINY, T) == n, T
     FP8 = mf.Config(**{**CFG.__dict__, "fp8": True})  # + the quantisation of h
-    for T, n in ((8, 6), (2048, 10)):
+    for T, n in ((1, 6), (8, 6), (2048, 10)):
         assert mf.moe_block_launch_count(FP8, T) == n, T
+    for flag in ("int8", "nvfp4"):  # these keep the separate gather
+        assert mf.moe_block_launch_count(mf.Config(**{**CFG.__dict__, flag: True}), 1) == 5
     assert mf.moe_block_launch_count(CFG, 0) == 0
     assert mf.moe_block_launch_count(CFG, -1) == -1
     assert mf.moe_block_launch_count(mf.Config(**{**CFG.__dict__, "top_k": 17}), 8) == -1
