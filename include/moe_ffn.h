@@ -305,8 +305,9 @@ moe_status_t moe_wait_selftest(void* ws, size_t ws_bytes, uint64_t timeout_ns, v
 /* Number of kernels that one moe_block_forward(cfg, T, ...) launches (host-only, no
  * GPU needed): the router (1, or 2 for the tensor-core router of T > 128: weight prep and
  * router), the permutation (0 when the router sorts in the same launch, else 1 or 3),
- * the row gather, the gate_up and down GEMMs and the combine (1 each), and for
- * MOE_W_FP8_E4M3 the quantisation of h between the GEMMs.  0 for T = 0;
+ * the row gather (0 when the router also gathers: bf16 experts, T <= 8 and T*k <= 32),
+ * the gate_up and down GEMMs and the combine (1 each), and for MOE_W_FP8_E4M3 the
+ * quantisation of h between the GEMMs.  0 for T = 0;
  * -1 when cfg or T is invalid (the arguments moe_block_forward would reject). */
 int32_t moe_block_launch_count(const moe_config_t* cfg, int32_t T);
 
