@@ -1,5 +1,5 @@
-"""Expert parallelism on the host: two gloo ranks, each with its own tokens and half of the
-experts, exchange routed rows with mixture_experts_ffn_05_b200.ep and must reproduce, bit
+"""Expert parallelism on the host: two (or four) gloo ranks, each with its own tokens and
+its share of the experts, exchange routed rows with mixture_experts_ffn_05_b200.ep and must reproduce, bit
 for bit, the MoE branch that one rank holding every expert computes for the same tokens.
 The expert arithmetic is the oracle's (fp64, one row at a time, so that a row's result
 does not depend on which rows share its matmul), on both sides of the comparison."""
@@ -87,8 +87,8 @@ def _rank(rank, world, port, bias, results):
         dist.destroy_process_group()
 
 
-def _run(bias):
-    world, port = 2, _free_port()
+def _run(bias, world=2):
+    port = _free_port()
     mgr = mp.get_context("spawn").Manager()
     results = mgr.dict()
     mp.start_processes(_rank, args=(world, port, bias, results), nprocs=world, join=True,
@@ -102,6 +102,15 @@ def test_two_ranks_reproduce_the_single_rank_branch():
         same, remote, err = res[rank]
         assert same, (rank, err)
     assert res[0][1] > 0 and res[1][1] > 0  # rows really crossed ranks both ways
+
+
+def test_four_ranks_reproduce_the_single_rank_branch():
+    """Four ranks of two experts each: every rank's rows scatter over three peers."""
+    res = _run(None, world=4)
+    for rank in range(4):
+        same, remote, err = res[rank]
+        assert same, (rank, err)
+    assert sum(res[r][1] for r in range(4)) > 0
 
 
 def test_one_sided_exchange():
