@@ -1,6 +1,7 @@
 """Expert parallelism on the host: two (or four) gloo ranks, each with its own tokens and
-its share of the experts, exchange routed rows with mixture_experts_ffn_05_b200.ep and must reproduce, bit
-for bit, the MoE branch that one rank holding every expert computes for the same tokens.
+its share of the experts, exchange routed rows with mixture_experts_ffn_05_b200.ep and
+must reproduce, bit for bit, the MoE branch that one rank holding every expert computes
+for the same tokens.
 The expert arithmetic is the oracle's (fp64, one row at a time, so that a row's result
 does not depend on which rows share its matmul), on both sides of the comparison."""
 import os
