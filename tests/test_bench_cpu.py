@@ -23,6 +23,13 @@ def test_bytes_count_the_used_experts_and_the_weight_type():
         # 8-bit experts (int8 or E4M3): one byte per weight plus an fp32 scale per row
         assert bench.algorithmic(SHAPE, u, True)["bytes"] == \
             u * (3 * I * H + (2 * I + H) * 4) + fixed
+        # NVFP4 experts: half a byte per weight, an E4M3 scale per 16 weights, an fp32
+        # scale per matrix (two matrices per expert)
+        assert bench.algorithmic(SHAPE, u, nvfp4=True)["bytes"] == \
+            u * (3 * I * H * (0.5 + 1 / 16) + 2 * 4) + fixed
+    assert bench.algorithmic(SHAPE, 54, nvfp4=True)["gate_up_bytes"] == \
+        (54 * (2 * I * H * (0.5 + 1 / 16) + 4) + 2 * D * H * 2 + (T * 8 + T) * H * 2
+         + (T * 8 * I + T * D) * 2)
     # the gate_up launch alone: its weights, token rows in, h out
     g = bench.algorithmic(SHAPE, 54)
     assert g["gate_up_bytes"] == (54 * 2 * I * H * 2 + 2 * D * H * 2 + (T * 8 + T) * H * 2
