@@ -114,6 +114,19 @@ def test_four_ranks_reproduce_the_single_rank_branch():
     assert sum(res[r][1] for r in range(4)) > 0
 
 
+def test_four_ranks_all_pairs_to_one_owner():
+    """Every pair routed to the experts of rank 3 (a logit offset on experts 6 and 7): rank
+    3 receives all 4 x T x k rows, the others none, and every rank still reproduces its
+    branch (the receive buffers are sized from the exchanged counts)."""
+    bias = np.array([0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 50.0, 49.0])
+    res = _run(bias, world=4)
+    for rank in range(4):
+        assert res[rank][0], (rank, res[rank][2])
+    assert res[3][1] == 0  # rank 3 sends nothing away
+    for rank in range(3):
+        assert res[rank][1] == SHAPE.T * SHAPE.k  # every pair of the others crosses
+
+
 def test_one_sided_exchange():
     """A logit offset sends every pair to experts 0..3 (rank 0's): rank 1 receives nothing
     (zero-size splits) and still gets every result back."""
